@@ -1,0 +1,483 @@
+"""Benchmark of the MTLA decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one call of mtla_decode_attn with the merge fused: every sequence
+merges its new token into the compressed cache and attends all ceil(t/s)
+rows.  Workload: B=32 sequences, H=8, d_h=64, r=256, d_R=32, s=2, 4096
+processed tokens in even sequences (the new token opens row 2049) and 4095 in
+odd ones (row 2048 is completed in place); cache rows, queries and the new
+token ~ N(0,1), bf16 storage.  Sixteen independent replicas of that state
+(~600 MB, more than the 126 MB L2) are visited in turn, so every step streams
+its cache from HBM; each replica's state really advances (t grows by one per
+visit, so the caches grow by ~2% over a default run) and the algorithmic
+bytes are counted from the exact lengths of every step.
+
+Metric: decode query-steps per second (sequences x steps / s) and the decode
+kernel's achieved HBM GB/s against the measured copy bandwidth.  With
+--gpus N (one process per GPU, torchrun), every rank runs its own B=32
+workload (independent sequences: no collective on the data path); the time
+is the max over ranks and value counts all ranks' query-steps.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import mtla_synth as synth  # noqa: E402
+
+METRIC = "MTLA decode query-steps/sec and achieved HBM GB/s (% of roofline) on 1 B200"
+UNIT = "query-steps/s"
+WORKLOAD = ("decode step bf16 with fused merge: B=32, H=8, d_h=64, r=256, d_R=32, s=2, "
+            "4096/4095 processed tokens (2049/2048 cache rows)")
+ROW_BYTES = 288 * 2
+N_REPLICAS = 16
+E2E_STEPS = 500
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_tc_b32_s2.md")
+KERNEL_SOURCES = ["temporally_compressed_latent_b200/csrc/decode_tc.cu",
+                  "temporally_compressed_latent_b200/csrc/kernels.cuh",
+                  "temporally_compressed_latent_b200/csrc/mtla_common.cuh"]
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def profiled_traffic():
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    if not os.path.exists(PROFILE_SUMMARY):
+        return None
+    vals = {}
+    for ln in open(PROFILE_SUMMARY):
+        if ln.startswith("- ") and ":" in ln:
+            k, v = ln[2:].split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_sha") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch_full_size"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML, read only)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._period = period_s
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self._h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        except Exception:  # noqa: BLE001 - clocks are reported as unavailable
+            self._nv = None
+
+    _NAMES = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+              0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+              0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = self._reasons_fn(self._h)
+                for bit, name in self._NAMES.items():
+                    if mask & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._nv is not None:
+            self._t.join()
+
+    def report(self):
+        if self._nv is None or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+class Replica:
+    def __init__(self, case, torch, mtla, glue, capacity_extra, J_max, dev):
+        d = case.dims
+        B = case.B
+        self.B = B
+        L0 = [len(r) for r in case.rows]
+        cap = max(L0) + capacity_extra
+        self.cap = cap
+        self.cache_rows = B * cap
+        host_buf = np.zeros((B, cap, d.D), dtype=np.float32)
+        for b, r in enumerate(case.rows):
+            host_buf[b, :len(r)] = r
+        self.cache = torch.from_numpy(host_buf).to(dev).to(torch.bfloat16).reshape(B * cap, d.D)
+        del host_buf
+        self.offset = (torch.arange(B, dtype=torch.int64, device=dev) * cap).contiguous()
+        self.capacity = torch.full((B,), cap, dtype=torch.int64, device=dev)
+        self.t0 = case.t_prev.copy()
+        self.t = torch.tensor(case.t_prev, dtype=torch.int32, device=dev)
+        self.cache_len = torch.zeros(B, dtype=torch.int32, device=dev)
+        bf = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(dev).to(torch.bfloat16)
+        self.q_abs, self.q_rope = bf(case.q_abs), bf(case.q_rope)
+        self.c_new, self.kR_new = bf(case.c_new), bf(case.kR_new)
+        self.out = torch.empty(B, d.H, d.r, dtype=torch.float32, device=dev)
+        self.lse = torch.empty(B, d.H, dtype=torch.float32, device=dev)
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import temporally_compressed_latent_b200 as mtla
+    from temporally_compressed_latent_b200 import glue
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    case = synth.decode_uniform(B=32, seed=2)
+    d = case.dims
+    B = case.B
+    W, K = args.warmup, args.steps
+    visits = math.ceil((W + K + E2E_STEPS + 8) / N_REPLICAS) + 1
+    extra = visits // d.s + 4
+    J_max = synth.ceil_div(int(case.t_prev.max()) + visits + 8, d.s) + 1
+    W_c = torch.from_numpy(case.lin["W_c"]).to(dev)
+    b_c = torch.from_numpy(case.lin["b_c"]).to(dev)
+    P = glue.pe_table(J_max, torch.from_numpy(case.lin["W_p"]).to(dev), torch.from_numpy(case.lin["b_p"]).to(dev))
+    md = mtla.dims(d.H, d.d_h, d.r, d.d_R, d.s, "bf16")
+    reps = [Replica(case, torch, mtla, glue, extra, J_max, dev) for _ in range(N_REPLICAS)]
+    ws_bytes = mtla.mtla_workspace_bytes(md, B)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(rep, st):
+        merge = {"c_new": rep.c_new, "kR_new": rep.kR_new, "W_c": W_c, "b_c": b_c, "P": P, "J_max": J_max}
+        mtla.mtla_decode_attn(md, B, rep.q_abs, rep.q_rope, merge, rep.cache, rep.cache_rows, d.D, rep.offset,
+                              rep.capacity, rep.t, rep.cache_len, rep.out, rep.lse, ws, ws_bytes, err, stream=st)
+
+    # algorithmic bytes of every step, from the exact lengths the state goes through
+    visit = [0] * N_REPLICAS
+
+    def step_bytes(i):
+        rep_i = i % N_REPLICAS
+        v = visit[rep_i]
+        visit[rep_i] += 1
+        t = case.t_prev + v + 1
+        rows = int(sum(synth.ceil_div(int(x), d.s) for x in t))
+        return (rows * ROW_BYTES + B * ROW_BYTES + B * d.H * d.D * 2 + B * d.D * 2 + B * d.H * d.r * 4 +
+                B * d.H * 4 + d.r * d.D * 4 + d.D * 4 + B * d.D * 4)
+
+    bytes_per_step = [step_bytes(i) for i in range(W + K)]
+    timed_bytes = bytes_per_step[W:]
+
+    # capture W warm-up steps and K timed steps as two CUDA graphs (launch cost
+    # of a ~6 us kernel must not be Python's); replica i % 8 at step i
+    torch.cuda.synchronize()
+    # one call per replica outside capture without a merge (no state change):
+    # sets the kernel's attributes and checks the arguments before capture
+    for rp in reps:
+        mtla.mtla_decode_attn(md, B, rp.q_abs, rp.q_rope, None, rp.cache, rp.cache_rows, d.D, rp.offset,
+                              rp.capacity, rp.t, rp.cache_len, rp.out, rp.lse, ws, ws_bytes, err, stream=stream)
+    torch.cuda.synchronize()
+    g_warm, g_timed = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_warm, stream=stream, capture_error_mode="thread_local"):
+        for i in range(W):
+            step(reps[i % N_REPLICAS], torch.cuda.current_stream())
+    with torch.cuda.graph(g_timed, stream=stream, capture_error_mode="thread_local"):
+        for i in range(W, W + K):
+            step(reps[i % N_REPLICAS], torch.cuda.current_stream())
+    torch.cuda.synchronize()
+
+    with torch.cuda.stream(stream):
+        g_warm.replay()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            g_timed.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    dev_err = int(err.item())
+    if dev_err:
+        raise RuntimeError(f"device error bits {dev_err} during the timed steps")
+    ms_max = ms
+    if dist:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_max = float(tt.item())
+    ms_step = ms_max / K
+    value = world * B * K / (ms_max / 1e3)
+
+    hbm_peak, _, _, peak_kind = measured_peaks()
+    achieved_gbs = (sum(timed_bytes) / K) / (ms / K / 1e3) / 1e9
+    traffic = profiled_traffic()
+
+    # end to end through the public API with host buffers: per step, H2D of the
+    # step's inputs from pinned memory, the call, D2H of the result, and a sync
+    e2e = run_e2e(torch, mtla, md, case, reps, W_c, b_c, P, J_max, ws, ws_bytes, err, stream, dev, K, W)
+
+    prefill = None
+    if not args.no_prefill and rank == 0:
+        prefill = run_prefill(torch, mtla, glue, dev)
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    res = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded N(0,1) cache rows, queries and new tokens)",
+        "config": {"workload": WORKLOAD, "B_per_gpu": B, "H": d.H, "d_h": d.d_h, "r": d.r, "d_R": d.d_R,
+                   "s": d.s, "parallelism": f"independent sequences per GPU x{world}",
+                   "l2": f"inputs larger than L2: {N_REPLICAS} rotating cache replicas "
+                         f"(~{N_REPLICAS * 37.8:.0f} MB > 126 MB L2)",
+                   "timing": "CUDA graph of K steps, CUDA events on the launching stream"},
+        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved_gbs / hbm_peak, "traffic": traffic,
+                     "kernel": "mtla::dtc::decode_tc_kernel", "peak_kind": f"{peak_kind} copy bandwidth",
+                     "algorithmic_bytes_per_launch": sum(timed_bytes) / K},
+        "gpu_launches": K,
+        "e2e": e2e,
+        "clocks": clk.report(),
+    }
+    if prefill:
+        res["prefill"] = prefill
+    if args.cpu_baseline and world == 1:
+        res["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    return res
+
+
+def run_e2e(torch, mtla, md, case, reps, W_c, b_c, P, J_max, ws, ws_bytes, err, stream, dev, K, W):
+    B = case.B
+    d = case.dims
+    pin = lambda shape, dt: torch.empty(shape, dtype=dt, pin_memory=True)
+    h_qa, h_qr = pin((B, d.H, d.r), torch.bfloat16), pin((B, d.H, d.d_R), torch.bfloat16)
+    h_c, h_k = pin((B, d.r), torch.bfloat16), pin((B, d.d_R), torch.bfloat16)
+    h_out = pin((B, d.H, d.r), torch.float32)
+    h_qa.copy_(torch.from_numpy(case.q_abs).to(torch.bfloat16))
+    h_qr.copy_(torch.from_numpy(case.q_rope).to(torch.bfloat16))
+    h_c.copy_(torch.from_numpy(case.c_new).to(torch.bfloat16))
+    h_k.copy_(torch.from_numpy(case.kR_new).to(torch.bfloat16))
+    n = min(K, E2E_STEPS)
+    h2d = (h_qa.numel() + h_qr.numel() + h_c.numel() + h_k.numel()) * 2
+    d2h = h_out.numel() * 4
+
+    def one(i):
+        rep = reps[i % N_REPLICAS]
+        rep.q_abs.copy_(h_qa, non_blocking=True)
+        rep.q_rope.copy_(h_qr, non_blocking=True)
+        rep.c_new.copy_(h_c, non_blocking=True)
+        rep.kR_new.copy_(h_k, non_blocking=True)
+        merge = {"c_new": rep.c_new, "kR_new": rep.kR_new, "W_c": W_c, "b_c": b_c, "P": P, "J_max": J_max}
+        mtla.mtla_decode_attn(md, B, rep.q_abs, rep.q_rope, merge, rep.cache, rep.cache_rows, d.D, rep.offset,
+                              rep.capacity, rep.t, rep.cache_len, rep.out, rep.lse, ws, ws_bytes, err,
+                              stream=torch.cuda.current_stream())
+        h_out.copy_(rep.out, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+
+    # the replicas may run out of spare rows: e2e reuses at most n steps
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            one(i)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(n):
+            one(3 + i)
+        e1.record()
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    return {"value": B * n / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": n, "ms_per_step": ms / n}
+
+
+def run_prefill(torch, mtla, glue, dev):
+    """Companion measurement: the masked parallel forward, B=8, T=4096, s=2."""
+    mc = synth.prefill_model()
+    d = mc.dims
+    W = {k: torch.from_numpy(v).to(dev) for k, v in mc.W.items()}
+    qa, qr, c, kR = (t.to(torch.bfloat16).contiguous() for t in glue.project(torch.from_numpy(mc.x).to(dev), W))
+    B, T = c.shape[0], c.shape[1]
+    J = synth.ceil_div(T, d.s) + 1
+    P = glue.pe_table(J, torch.from_numpy(mc.lin["W_p"]).to(dev), torch.from_numpy(mc.lin["b_p"]).to(dev))
+    W_c = torch.from_numpy(mc.lin["W_c"]).to(dev)
+    b_c = torch.from_numpy(mc.lin["b_c"]).to(dev)
+    cp = torch.empty(B, T, d.D, dtype=torch.bfloat16, device=dev)
+    cache = torch.empty(B, J - 1, d.D, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(B, T, d.H, d.r, dtype=torch.bfloat16, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    md = mtla.dims(d.H, d.d_h, d.r, d.d_R, d.s, "bf16")
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def call():
+        mtla.mtla_prefill_masked_attn(md, B, T, qa, qr, c, kR, W_c, b_c, P, J, cp, cache, out, err)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(5):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        call()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    pairs = B * d.H * sum(math.ceil(m / d.s) for m in range(1, T + 1))
+    flops = pairs * (2 * d.D + 2 * d.r)
+    _, tflops_peak, _, kind = measured_peaks()
+    return {"workload": "masked prefill bf16: B=8, T=4096, d=512, H=8, d_h=64, r=256, d_R=32, s=2",
+            "ms": ms, "unmasked_tflops": flops / (ms / 1e3) / 1e12, "peak_tflops": tflops_peak,
+            "frac": flops / (ms / 1e3) / 1e12 / tflops_peak, "peak_kind": f"{kind} cuBLAS bf16 (burst)",
+            "note": "both kernels (running merge + attention) inside the timed call; L2 flushed before each"}
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host cores (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+def cpu_baseline(seconds: float):
+    import oracle
+    from threadpoolctl import threadpool_limits
+    case = synth.decode_uniform(B=32, seed=2)
+    d = case.dims
+    P = oracle.pe_table(synth.ceil_div(int(case.t_prev.max()) + 1, d.s) + 1, case.lin["W_p"], case.lin["b_p"])
+    done = 0
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < seconds:
+            b = done % case.B
+            oracle.decode_step(case.rows[b], int(case.t_prev[b]), d.s, case.c_new[b], case.kR_new[b],
+                               case.q_abs[b], case.q_rope[b], case.lin["W_c"], case.lin["b_c"], P, d.d_h)
+            done += 1
+        el = time.perf_counter() - t0
+    return {"value": done / el, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{done} sequence-steps of the B=32 workload (cycling over its sequences) in {el:.1f} s, "
+                      "numpy float64, one thread"}
+
+
+def run_reference(args, rank, world):
+    """The oracle, as it stands, on the host cores: each step is a bounded
+    sample of the B=32 decode step (one sequence's merge + attention, cycling
+    over the 32 sequences); W untimed steps, then K timed ones."""
+    if rank != 0:
+        return None
+    import oracle
+    from threadpoolctl import threadpool_limits
+    W, K = args.warmup, args.steps
+    case = synth.decode_uniform(B=32, seed=2)
+    d = case.dims
+    P = oracle.pe_table(synth.ceil_div(int(case.t_prev.max()) + 1, d.s) + 1, case.lin["W_p"], case.lin["b_p"])
+
+    def one(i):
+        b = i % case.B
+        oracle.decode_step(case.rows[b], int(case.t_prev[b]), d.s, case.c_new[b], case.kR_new[b], case.q_abs[b],
+                           case.q_rope[b], case.lin["W_c"], case.lin["b_c"], P, d.d_h)
+
+    with threadpool_limits(limits=1):
+        for i in range(W):
+            one(i)
+        t0 = time.perf_counter()
+        for i in range(K):
+            one(W + i)
+        el = time.perf_counter() - t0
+    value = K / el
+    cb = {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+          "sample": f"{K} timed steps, each one sequence of the B=32 workload (merge + attention over "
+                    f"2048/2049 rows), numpy float64, one thread, {el:.1f} s"}
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": el / K * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1))",
+            "config": {"workload": WORKLOAD, "B_per_gpu": 32,
+                       "step": "one sequence of the B=32 step (bounded sample)"},
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=500)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--cpu-baseline", dest="cpu_baseline", action="store_true", default=True)
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", str(args.gpus)))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+    else:
+        res = run_ours(args, rank, world, local_rank)
+    if res is not None:
+        print(json.dumps(res))
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,184 @@
+/*
+ * mtla.h — C ABI of the MTLA hot-path library (libmtla.so), sm_100a.
+ *
+ * Multi-head Temporal Latent Attention (Deng & Woodland, NeurIPS 2025) keeps a
+ * KV cache compressed twice: in feature width (a latent c of width r plus a
+ * decoupled-RoPE key of width d_R) and in time (every s adjacent steps are
+ * merged by a sigmoid-gated hyper-network).  This library runs the inference
+ * hot path (merge/append + absorbed decode attention) and the parallel
+ * training/prefill forward under the stride-aware causal mask.
+ *
+ * Sources (page title, section):
+ *   [merge]   MTLA paper notes, "Key designs: hyper-network temporal merging":
+ *             w_i = Sigmoid(Linear(c_i) ⊙ Linear(pe_j)), c_hat_j = sum_i w_i ⊙ c_i,
+ *             the cache holds ceil(T/s) rows.
+ *   [mask]    MTLA paper notes, "Key designs: stride-aware causal mask": query m
+ *             sees column n of C_hat' iff n == m, or n < m and n mod s == 0.
+ *   [rope]    MTLA paper notes, "Key designs: decoupled RoPE with temporal
+ *             compression": Y = softmax((X W_Q W_K^T C_hat^T + Q^R K_hat^R^T)
+ *             / sqrt(d_h)) C_hat (W_V W_O).
+ *   [fig2]    arXiv 2505.13544 abstract page, Figure 2: (a) incremental
+ *             inference attends a temporary c_hat'_j at steps 1, 3, 5 (s = 2);
+ *             (c) training with the stride-aware mask.
+ *
+ * Conventions for every call
+ *   - Time is 1-indexed as on the pages: token t of a sequence belongs to group
+ *     j(t) = ceil(t/s); token t opens a new cache row iff (t-1) mod s == 0 and is
+ *     added in place to the tail row otherwise.
+ *   - A cache row is [c_hat (r) | k_hat^R (d_R)], D = r + d_R elements, stored
+ *     in the cache dtype; consecutive rows are row_stride elements apart.
+ *     Sequence b owns rows [seq_offset[b], seq_offset[b] + seq_capacity[b]) of a
+ *     buffer of cache_rows rows ("paged contiguous" cache).
+ *   - Softmax scale is 1/sqrt(d_h) ([rope]); values are the latent part only.
+ *   - All pointers except `dims`, `merge` and the host outputs of
+ *     mtla_debug_stride_mask are DEVICE pointers.  The caller owns every
+ *     buffer; the library allocates no memory and never synchronises.  Every
+ *     call is asynchronous on `stream` (a cudaStream_t, NULL = legacy stream).
+ *   - Argument errors are reported synchronously, before any launch, as the
+ *     returned status.  Conditions only the device can see are OR-ed into
+ *     *dev_err (MTLA_DEVERR_* bits); the kernels then skip the offending work
+ *     and never trap.  dev_err is never cleared by the library.
+ *   - bf16 tensors must be 16-byte aligned and row strides multiples of 8
+ *     elements; fp32 tensors 16-byte aligned.
+ */
+#ifndef MTLA_H
+#define MTLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MTLA_OK = 0,
+  MTLA_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, bad size or stride */
+  MTLA_ERR_UNSUPPORTED = 2,   /* dims or dtype this build has no kernel for    */
+  MTLA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required    */
+  MTLA_ERR_CUDA = 4           /* a CUDA runtime/driver call failed             */
+} mtla_status;
+
+typedef enum { MTLA_F32 = 0, MTLA_BF16 = 1 } mtla_dtype;
+
+/* Problem dimensions: H heads of width d_h (sets the 1/sqrt(d_h) scale),
+ * latent width r, RoPE width d_R, temporal stride s >= 1, cache dtype. */
+typedef struct {
+  int32_t H, d_h, r, d_R, s;
+  int32_t dtype; /* mtla_dtype */
+} mtla_dims;
+
+/* Hyper-network merge inputs for ONE new token per sequence ([merge]).
+ * Linear(c_t) = c_t W_c + b_c maps width r to D so that one gate covers
+ * [c_t ; k^R_t]; Linear(pe_j) is precomputed by the caller as row j-1 of P. */
+typedef struct {
+  const void *c_new;   /* [B, r]    cache dtype: the new latents c_t            */
+  const void *kR_new;  /* [B, d_R]  cache dtype: the new RoPE keys, rotated      */
+  const float *W_c;    /* [r, D]    row-major                                    */
+  const float *b_c;    /* [D]                                                    */
+  const float *P;      /* [J_max, D] row j-1 = Linear(pe_j) for group j          */
+  int32_t J_max;       /* rows of P; a token with j(t) > J_max sets PE_RANGE     */
+} mtla_merge_args;
+
+/* device error bits (OR-ed into *dev_err) */
+#define MTLA_DEVERR_PE_RANGE 1   /* j(t) > J_max: merge skipped                   */
+#define MTLA_DEVERR_CAPACITY 2   /* ceil(t/s) > seq_capacity, or the sequence's   */
+                                 /* rows run past cache_rows: work clamped        */
+#define MTLA_DEVERR_EMPTY    4   /* attention over an empty cache (t == 0)        */
+#define MTLA_DEVERR_TIMEOUT  8   /* an internal bounded wait gave up              */
+
+/*
+ * mtla_merge_append — fold one new token per sequence into the cache ([merge],
+ * [fig2](a)).  For each b: t = t_processed[b] + 1, j = ceil(t/s),
+ * w = sigmoid((c_t W_c + b_c) ⊙ P[j-1]); the row j-1 of sequence b becomes
+ * w ⊙ [c_t ; k^R_t] if (t-1) mod s == 0, else row += w ⊙ [c_t ; k^R_t]
+ * (fp32 arithmetic, stored in the cache dtype).  Then t_processed[b] = t and,
+ * if cache_len != NULL, cache_len[b] = j.
+ *   cache           [cache_rows, row_stride] cache dtype, updated in place
+ *   seq_offset, seq_capacity [B] int64, t_processed [B] int32 (in/out),
+ *   cache_len [B] int32 (out, nullable), dev_err int32 (in/out).
+ */
+mtla_status mtla_merge_append(const mtla_dims *dims, int32_t B, const mtla_merge_args *merge,
+                              void *cache, int64_t cache_rows, int64_t row_stride,
+                              const int64_t *seq_offset, const int64_t *seq_capacity,
+                              int32_t *t_processed, int32_t *cache_len, int32_t *dev_err,
+                              void *stream);
+
+/*
+ * mtla_decode_attn — one incremental decode step ([rope], [fig2](a)).
+ * If merge != NULL the new token is first merged exactly as mtla_merge_append
+ * does, in the same launch, and t_processed advances by one; if merge == NULL
+ * the cache is read as it stands (t_processed unchanged).  Then for every
+ * sequence b and head h, over the L = ceil(t/s) cached rows (the partial tail
+ * included):
+ *   score_j = (q_abs[b,h] · c_hat_j + q_rope[b,h] · k_hat^R_j) / sqrt(d_h),
+ *   out[b,h,:] = sum_j softmax(score)_j c_hat_j,  lse[b,h] = ln sum_j e^score_j.
+ *   q_abs [B, H, r], q_rope [B, H, d_R]   cache dtype
+ *   out   [B, H, r] fp32;  lse [B, H] fp32 (nullable)
+ *   workspace: mtla_workspace_bytes(dims, B, MTLA_WS_DECODE) bytes, zeroed
+ *              by the caller ONCE before first use; every call leaves it zeroed
+ *              again, so one workspace serves calls that run one after another
+ *              on a stream (not calls that overlap).
+ * Kernels: bf16 with (H, r, d_R) = (8, 256, 32) and B <= 2048 runs the
+ * split-L tensor-core kernel (workspace required); any other supported dims
+ * run a one-block-per-sequence kernel (workspace unused, may be NULL).
+ * Supported dims everywhere: H <= 16, r <= 512, r + d_R <= 576, r and d_R
+ * multiples of 8 (bf16) or 4 (fp32); otherwise MTLA_ERR_UNSUPPORTED.
+ */
+mtla_status mtla_decode_attn(const mtla_dims *dims, int32_t B,
+                             const void *q_abs, const void *q_rope,
+                             const mtla_merge_args *merge,
+                             void *cache, int64_t cache_rows, int64_t row_stride,
+                             const int64_t *seq_offset, const int64_t *seq_capacity,
+                             int32_t *t_processed, int32_t *cache_len,
+                             float *out, float *lse,
+                             void *workspace, size_t workspace_bytes,
+                             int32_t *dev_err, void *stream);
+
+/*
+ * mtla_prefill_masked_attn — the parallel (training / prefill) forward of B
+ * sequences of T tokens, t = 1..T ([mask], [fig2](c)).
+ *   1. c_partial[b, n] = C_hat'_n = sum_{i=(j(n)-1)s+1}^{n} w_i ⊙ [c_i ; k^R_i],
+ *      w_i = sigmoid((c_i W_c + b_c) ⊙ P[j(i)-1])  (the running merge);
+ *   2. out[b, m, h] = sum_{n visible} softmax(score)_n c_hat'_n with the
+ *      stride-aware mask (n == m, or n < m and n mod s == 0) and the score of
+ *      mtla_decode_attn against row n of C_hat'.
+ *   3. if cache_out != NULL: cache_out[b, g-1] = C_hat'_{min(g s, T)},
+ *      g = 1..ceil(T/s) — the decode cache after the prompt.
+ *   If out == NULL only steps 1 and 3 run (building a cache from a prompt);
+ *   q_abs and q_rope may then be NULL.
+ *   q_abs [B, T, H, r], q_rope [B, T, H, d_R], c [B, T, r], kR [B, T, d_R]
+ *   (cache dtype, contiguous); W_c, b_c, P, J_max as in mtla_merge_args
+ *   (J_max >= ceil(T/s)); c_partial [B, T, D], cache_out [B, ceil(T/s), D],
+ *   out [B, T, H, r] all cache dtype, contiguous, written by the call.
+ * Kernels: bf16 with (H, r, d_R) = (8, 256, 32) runs the tcgen05/TMEM
+ * tensor-core kernel; other supported dims run a SIMT kernel.
+ */
+mtla_status mtla_prefill_masked_attn(const mtla_dims *dims, int32_t B, int32_t T,
+                                     const void *q_abs, const void *q_rope,
+                                     const void *c, const void *kR,
+                                     const float *W_c, const float *b_c,
+                                     const float *P, int32_t J_max,
+                                     void *c_partial, void *cache_out, void *out,
+                                     int32_t *dev_err, void *stream);
+
+#define MTLA_WS_DECODE 0
+
+/* Bytes of workspace a call needs (0 if none).  Queries the current device. */
+size_t mtla_workspace_bytes(const mtla_dims *dims, int32_t B, int32_t which);
+
+/* Static text for a status code. */
+const char *mtla_status_string(mtla_status status);
+
+/* The kernels' own visibility predicate ([mask]) written to host_out[T*T]
+ * (row m-1, column n-1, 1 = visible).  Host only; no GPU needed. */
+mtla_status mtla_debug_stride_mask(int32_t s, int32_t T, uint8_t *host_out);
+
+/* The kernels' own cache-length rule: rows after t processed tokens. */
+int64_t mtla_cache_length(int64_t t, int32_t s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MTLA_H */

@@ -1,0 +1,30 @@
+"""MTLA hot path on B200: Python binding of the C ABI in ``include/mtla.h``.
+
+Multi-head Temporal Latent Attention keeps a KV cache compressed in feature
+width (MLA-style latents plus decoupled-RoPE keys) and in time (a sigmoid
+hyper-network merges every s adjacent steps).  Every step of the hot path runs
+in the CUDA library ``libmtla.so``; this package only marshals arguments
+(torch tensors -> device pointers, the current CUDA stream) and turns error
+statuses into exceptions.  Importing it fails if the library is not built.
+"""
+from ._abi import (  # noqa: F401
+    DEVERR_CAPACITY,
+    DEVERR_EMPTY,
+    DEVERR_PE_RANGE,
+    DEVERR_TIMEOUT,
+    LIB_PATH,
+    MTLA_BF16,
+    MTLA_F32,
+    WS_DECODE,
+    MtlaError,
+    dims,
+    exported_symbols,
+    lib,
+    mtla_cache_length,
+    mtla_debug_stride_mask,
+    mtla_decode_attn,
+    mtla_merge_append,
+    mtla_prefill_masked_attn,
+    mtla_status_string,
+    mtla_workspace_bytes,
+)

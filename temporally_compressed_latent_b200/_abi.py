@@ -1,0 +1,144 @@
+"""ctypes binding of libmtla.so: the C ABI of include/mtla.h, same names.
+
+Arguments are torch tensors (their device pointer is passed), plain integers
+(taken as raw pointers) or None (NULL).  Nothing here computes any part of the
+method; every call goes straight to the library, asynchronously on the current
+CUDA stream unless ``stream`` is given.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmtla.so")
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "mtla.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is not built; run `python temporally_compressed_latent_b200/build_lib.py` "
+        "(the MTLA hot path has no fallback)")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+MTLA_F32, MTLA_BF16 = 0, 1
+WS_DECODE = 0
+DEVERR_PE_RANGE, DEVERR_CAPACITY, DEVERR_EMPTY, DEVERR_TIMEOUT = 1, 2, 4, 8
+_c = ctypes
+
+
+class _Dims(_c.Structure):
+    _fields_ = [("H", _c.c_int32), ("d_h", _c.c_int32), ("r", _c.c_int32), ("d_R", _c.c_int32),
+                ("s", _c.c_int32), ("dtype", _c.c_int32)]
+
+
+class _Merge(_c.Structure):
+    _fields_ = [("c_new", _c.c_void_p), ("kR_new", _c.c_void_p), ("W_c", _c.c_void_p), ("b_c", _c.c_void_p),
+                ("P", _c.c_void_p), ("J_max", _c.c_int32)]
+
+
+_P = _c.c_void_p
+_I32, _I64, _SZ = _c.c_int32, _c.c_int64, _c.c_size_t
+_DIMS_P, _MERGE_P = _c.POINTER(_Dims), _c.POINTER(_Merge)
+
+lib.mtla_merge_append.restype = _c.c_int
+lib.mtla_merge_append.argtypes = [_DIMS_P, _I32, _MERGE_P, _P, _I64, _I64, _P, _P, _P, _P, _P, _P]
+lib.mtla_decode_attn.restype = _c.c_int
+lib.mtla_decode_attn.argtypes = [_DIMS_P, _I32, _P, _P, _MERGE_P, _P, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ,
+                                 _P, _P]
+lib.mtla_prefill_masked_attn.restype = _c.c_int
+lib.mtla_prefill_masked_attn.argtypes = [_DIMS_P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P, _P]
+lib.mtla_workspace_bytes.restype = _SZ
+lib.mtla_workspace_bytes.argtypes = [_DIMS_P, _I32, _I32]
+lib.mtla_status_string.restype = _c.c_char_p
+lib.mtla_status_string.argtypes = [_c.c_int]
+lib.mtla_debug_stride_mask.restype = _c.c_int
+lib.mtla_debug_stride_mask.argtypes = [_I32, _I32, _P]
+lib.mtla_cache_length.restype = _I64
+lib.mtla_cache_length.argtypes = [_I64, _I32]
+
+
+class MtlaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {mtla_status_string(status)} (status {status})")
+
+
+def mtla_status_string(status: int) -> str:
+    return lib.mtla_status_string(int(status)).decode()
+
+
+def dims(H: int, d_h: int, r: int, d_R: int, s: int, dtype) -> _Dims:
+    if isinstance(dtype, str):
+        dtype = {"f32": MTLA_F32, "bf16": MTLA_BF16}[dtype]
+    return _Dims(H, d_h, r, d_R, s, int(dtype))
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def _merge(m):
+    if m is None:
+        return None
+    return _c.byref(_Merge(_ptr(m["c_new"]), _ptr(m["kR_new"]), _ptr(m["W_c"]), _ptr(m["b_c"]), _ptr(m["P"]),
+                           int(m["J_max"])))
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise MtlaError(status, where)
+
+
+def mtla_merge_append(d, B, merge, cache, cache_rows, row_stride, seq_offset, seq_capacity, t_processed,
+                      cache_len, dev_err, stream=None):
+    _check(lib.mtla_merge_append(_c.byref(d), B, _merge(merge), _ptr(cache), cache_rows, row_stride,
+                                 _ptr(seq_offset), _ptr(seq_capacity), _ptr(t_processed), _ptr(cache_len),
+                                 _ptr(dev_err), _stream(stream)), "mtla_merge_append")
+
+
+def mtla_decode_attn(d, B, q_abs, q_rope, merge, cache, cache_rows, row_stride, seq_offset, seq_capacity,
+                     t_processed, cache_len, out, lse, workspace, workspace_bytes, dev_err, stream=None):
+    _check(lib.mtla_decode_attn(_c.byref(d), B, _ptr(q_abs), _ptr(q_rope), _merge(merge), _ptr(cache), cache_rows,
+                                row_stride, _ptr(seq_offset), _ptr(seq_capacity), _ptr(t_processed),
+                                _ptr(cache_len), _ptr(out), _ptr(lse), _ptr(workspace), workspace_bytes,
+                                _ptr(dev_err), _stream(stream)), "mtla_decode_attn")
+
+
+def mtla_prefill_masked_attn(d, B, T, q_abs, q_rope, c, kR, W_c, b_c, P, J_max, c_partial, cache_out, out,
+                             dev_err, stream=None):
+    _check(lib.mtla_prefill_masked_attn(_c.byref(d), B, T, _ptr(q_abs), _ptr(q_rope), _ptr(c), _ptr(kR),
+                                        _ptr(W_c), _ptr(b_c), _ptr(P), J_max, _ptr(c_partial), _ptr(cache_out),
+                                        _ptr(out), _ptr(dev_err), _stream(stream)), "mtla_prefill_masked_attn")
+
+
+def mtla_workspace_bytes(d, B, which=WS_DECODE) -> int:
+    return int(lib.mtla_workspace_bytes(_c.byref(d), B, which))
+
+
+def mtla_debug_stride_mask(s: int, T: int):
+    import numpy as np
+    out = np.zeros((T, T), dtype=np.uint8)
+    _check(lib.mtla_debug_stride_mask(s, T, out.ctypes.data if T else None), "mtla_debug_stride_mask")
+    return out
+
+
+def mtla_cache_length(t: int, s: int) -> int:
+    return int(lib.mtla_cache_length(t, s))
+
+
+def exported_symbols():
+    """Function names declared in include/mtla.h (the ABI's entry points)."""
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w]+\s*\*?\s*(mtla_\w+)\s*\(", text, flags=re.M)))

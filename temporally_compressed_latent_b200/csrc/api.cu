@@ -1,0 +1,283 @@
+// C ABI of the MTLA library: argument checks, kernel selection, launches.
+// See include/mtla.h for the contract of every entry point.
+#include <math.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "kernels.cuh"
+
+namespace {
+
+using namespace mtla;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t elem_size(int dtype) { return dtype == MTLA_BF16 ? 2 : 4; }
+
+mtla_status check_dims(const mtla_dims* d) {
+  if (!d) return MTLA_ERR_INVALID_ARG;
+  if (d->H < 1 || d->d_h < 1 || d->r < 1 || d->d_R < 0 || d->s < 1) return MTLA_ERR_INVALID_ARG;
+  if (d->dtype != MTLA_F32 && d->dtype != MTLA_BF16) return MTLA_ERR_INVALID_ARG;
+  // limits of the generic kernels (register tiles sized for these)
+  if (d->H > 16 || d->r > 512 || d->r + d->d_R > 576) return MTLA_ERR_UNSUPPORTED;
+  if (d->dtype == MTLA_BF16 && ((d->r % 8) || (d->d_R % 8))) return MTLA_ERR_UNSUPPORTED;
+  if (d->dtype == MTLA_F32 && ((d->r % 4) || (d->d_R % 4))) return MTLA_ERR_UNSUPPORTED;
+  return MTLA_OK;
+}
+
+bool tc_decode_dims(const mtla_dims* d, int B) {
+  return d->dtype == MTLA_BF16 && d->H == dtc::H && d->r == dtc::R && d->d_R == dtc::DR && B <= dtc::MAXB;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point, so the
+// library needs no link-time dependency on libcuda.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D view of a bf16 cache: {32 elements, 9 chunks of 32, cache_rows rows}.
+bool encode_cache_map(CUtensorMap* map, void* cache, int64_t cache_rows, int64_t row_stride, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {32, (cuuint64_t)(dtc::D / 32), (cuuint64_t)cache_rows};
+  const cuuint64_t strides[2] = {64, (cuuint64_t)row_stride * 2};
+  const cuuint32_t box[3] = {32, (cuuint32_t)(dtc::D / 32), box_rows};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, cache, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct CacheMaps {
+  void* ptr = nullptr;
+  int64_t rows = -1, stride = -1;
+  CUtensorMap m64, m8;
+};
+
+mtla_status seq_args(const mtla_dims* d, void* cache, int64_t cache_rows, int64_t row_stride,
+                     const int64_t* seq_offset, const int64_t* seq_capacity, int32_t* t_processed,
+                     int32_t* cache_len, int32_t* dev_err, SeqArgs* a) {
+  if (!cache || !seq_offset || !seq_capacity || !t_processed || !dev_err) return MTLA_ERR_INVALID_ARG;
+  if (!aligned16(cache) || !aligned16(seq_offset) || !aligned16(seq_capacity)) return MTLA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(t_processed) & 3) || (cache_len && (reinterpret_cast<uintptr_t>(cache_len) & 3)) ||
+      (reinterpret_cast<uintptr_t>(dev_err) & 3))
+    return MTLA_ERR_INVALID_ARG;
+  const int D = d->r + d->d_R;
+  if (cache_rows < 0 || cache_rows >= (int64_t(1) << 31) || row_stride < D) return MTLA_ERR_INVALID_ARG;
+  if ((row_stride * (int64_t)elem_size(d->dtype)) % 16) return MTLA_ERR_INVALID_ARG;
+  a->cache = cache;
+  a->cache_rows = cache_rows;
+  a->row_stride = row_stride;
+  a->seq_offset = seq_offset;
+  a->seq_capacity = seq_capacity;
+  a->t_processed = t_processed;
+  a->cache_len = cache_len;
+  a->dev_err = dev_err;
+  a->r = d->r;
+  a->d_R = d->d_R;
+  a->s = d->s;
+  return MTLA_OK;
+}
+
+mtla_status merge_args(const mtla_merge_args* m, MergeArgsDev* md) {
+  if (!m || !m->c_new || !m->kR_new || !m->W_c || !m->b_c || !m->P || m->J_max < 1) return MTLA_ERR_INVALID_ARG;
+  if (!aligned16(m->c_new) || !aligned16(m->kR_new) || !aligned16(m->W_c) || !aligned16(m->b_c) ||
+      !aligned16(m->P))
+    return MTLA_ERR_INVALID_ARG;
+  md->c_new = m->c_new;
+  md->kR_new = m->kR_new;
+  md->W_c = m->W_c;
+  md->b_c = m->b_c;
+  md->P = m->P;
+  md->J_max = m->J_max;
+  return MTLA_OK;
+}
+
+mtla_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MTLA_OK : MTLA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* mtla_status_string(mtla_status st) {
+  switch (st) {
+    case MTLA_OK: return "ok";
+    case MTLA_ERR_INVALID_ARG: return "invalid argument";
+    case MTLA_ERR_UNSUPPORTED: return "unsupported dimensions or dtype";
+    case MTLA_ERR_WORKSPACE: return "workspace missing or too small";
+    case MTLA_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+int64_t mtla_cache_length(int64_t t, int32_t s) {
+  if (t <= 0 || s < 1) return 0;
+  return group_of(t, s);
+}
+
+mtla_status mtla_debug_stride_mask(int32_t s, int32_t T, uint8_t* host_out) {
+  if (s < 1 || T < 0 || (T > 0 && !host_out)) return MTLA_ERR_INVALID_ARG;
+  for (int64_t m = 1; m <= T; ++m)
+    for (int64_t n = 1; n <= T; ++n) host_out[(m - 1) * T + (n - 1)] = stride_visible(m, n, s) ? 1 : 0;
+  return MTLA_OK;
+}
+
+size_t mtla_workspace_bytes(const mtla_dims* dims, int32_t B, int32_t which) {
+  if (check_dims(dims) != MTLA_OK || B < 0) return 0;
+  if (which == MTLA_WS_DECODE && tc_decode_dims(dims, B)) {
+    const int g = sm_count();
+    return g > 0 ? dtc::workspace_bytes(B, g) : 0;
+  }
+  return 0;
+}
+
+mtla_status mtla_merge_append(const mtla_dims* dims, int32_t B, const mtla_merge_args* merge, void* cache,
+                              int64_t cache_rows, int64_t row_stride, const int64_t* seq_offset,
+                              const int64_t* seq_capacity, int32_t* t_processed, int32_t* cache_len,
+                              int32_t* dev_err, void* stream) {
+  mtla_status st = check_dims(dims);
+  if (st != MTLA_OK) return st;
+  if (B < 0) return MTLA_ERR_INVALID_ARG;
+  SeqArgs a;
+  MergeArgsDev m;
+  if ((st = seq_args(dims, cache, cache_rows, row_stride, seq_offset, seq_capacity, t_processed, cache_len, dev_err,
+                     &a)) != MTLA_OK)
+    return st;
+  if ((st = merge_args(merge, &m)) != MTLA_OK) return st;
+  if (B == 0) return MTLA_OK;
+  return from_cuda(launch_merge_append(a, m, B, dims->dtype, static_cast<cudaStream_t>(stream)));
+}
+
+mtla_status mtla_decode_attn(const mtla_dims* dims, int32_t B, const void* q_abs, const void* q_rope,
+                             const mtla_merge_args* merge, void* cache, int64_t cache_rows, int64_t row_stride,
+                             const int64_t* seq_offset, const int64_t* seq_capacity, int32_t* t_processed,
+                             int32_t* cache_len, float* out, float* lse, void* workspace, size_t workspace_bytes,
+                             int32_t* dev_err, void* stream) {
+  mtla_status st = check_dims(dims);
+  if (st != MTLA_OK) return st;
+  if (B < 0) return MTLA_ERR_INVALID_ARG;
+  SeqArgs a;
+  MergeArgsDev m = {};
+  if ((st = seq_args(dims, cache, cache_rows, row_stride, seq_offset, seq_capacity, t_processed, cache_len, dev_err,
+                     &a)) != MTLA_OK)
+    return st;
+  if (merge && (st = merge_args(merge, &m)) != MTLA_OK) return st;
+  if (!q_abs || !q_rope || !out || !aligned16(q_abs) || !aligned16(q_rope) || !aligned16(out) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3)))
+    return MTLA_ERR_INVALID_ARG;
+  if (B == 0) return MTLA_OK;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  DecodeOut o;
+  o.q_abs = q_abs;
+  o.q_rope = q_rope;
+  o.out = out;
+  o.lse = lse;
+  o.scale = (float)(1.0 / sqrt((double)dims->d_h));
+  o.H = dims->H;
+
+  if (!tc_decode_dims(dims, B))
+    return from_cuda(launch_decode_simt(a, m, merge != nullptr, o, B, dims->dtype, cs));
+
+  const int grid = sm_count();
+  if (grid <= 0) return MTLA_ERR_CUDA;
+  const size_t need = dtc::workspace_bytes(B, grid);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return MTLA_ERR_WORKSPACE;
+
+  thread_local CacheMaps maps;
+  if (maps.ptr != cache || maps.rows != cache_rows || maps.stride != row_stride) {
+    if (!encode_cache_map(&maps.m64, cache, cache_rows, row_stride, dtc::UNIT) ||
+        !encode_cache_map(&maps.m8, cache, cache_rows, row_stride, dtc::SUB)) {
+      maps.ptr = nullptr;
+      return MTLA_ERR_CUDA;
+    }
+    maps.ptr = cache;
+    maps.rows = cache_rows;
+    maps.stride = row_stride;
+  }
+  dtc::Params p;
+  p.a = a;
+  p.m = m;
+  p.o = o;
+  p.with_merge = merge != nullptr;
+  p.B = B;
+  p.merge_cost = dtc::MERGE_COST;
+  p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->d_h));
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  size_t off = 0;
+  p.tickets = reinterpret_cast<int32_t*>(ws + off);
+  p.done = p.tickets + B;
+  off += ((size_t)B + 1) * 4;
+  off = (off + 255) & ~(size_t)255;
+  p.ws_ml = reinterpret_cast<float*>(ws + off);
+  off += (size_t)2 * grid * dtc::H * 2 * 4;
+  off = (off + 255) & ~(size_t)255;
+  p.ws_o = reinterpret_cast<float*>(ws + off);
+  return from_cuda(launch_decode_tc(p, maps.m64, maps.m8, grid, cs));
+}
+
+mtla_status mtla_prefill_masked_attn(const mtla_dims* dims, int32_t B, int32_t T, const void* q_abs,
+                                     const void* q_rope, const void* c, const void* kR, const float* W_c,
+                                     const float* b_c, const float* P, int32_t J_max, void* c_partial,
+                                     void* cache_out, void* out, int32_t* dev_err, void* stream) {
+  mtla_status st = check_dims(dims);
+  if (st != MTLA_OK) return st;
+  if (B < 0 || T < 0) return MTLA_ERR_INVALID_ARG;
+  if (!c || !kR || !W_c || !b_c || !P || !c_partial || !dev_err) return MTLA_ERR_INVALID_ARG;
+  if (out && (!q_abs || !q_rope)) return MTLA_ERR_INVALID_ARG;
+  const void* ptrs[] = {c, kR, W_c, b_c, P, c_partial};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return MTLA_ERR_INVALID_ARG;
+  if (out && (!aligned16(out) || !aligned16(q_abs) || !aligned16(q_rope))) return MTLA_ERR_INVALID_ARG;
+  if (cache_out && !aligned16(cache_out)) return MTLA_ERR_INVALID_ARG;
+  if (B == 0 || T == 0) return MTLA_OK;
+  if ((int64_t)J_max < cdiv(T, dims->s)) return MTLA_ERR_INVALID_ARG;
+  if ((int64_t)B * T >= (int64_t(1) << 31)) return MTLA_ERR_UNSUPPORTED;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  PrefillArgs p;
+  p.q_abs = q_abs;
+  p.q_rope = q_rope;
+  p.c = c;
+  p.kR = kR;
+  p.W_c = W_c;
+  p.b_c = b_c;
+  p.P = P;
+  p.c_partial = c_partial;
+  p.cache_out = cache_out;
+  p.out = out;
+  p.dev_err = dev_err;
+  p.T = T;
+  p.groups_per_block = 1;
+  p.H = dims->H;
+  p.r = dims->r;
+  p.d_R = dims->d_R;
+  p.s = dims->s;
+  p.scale = (float)(1.0 / sqrt((double)dims->d_h));
+  p.J_max = J_max;
+  cudaError_t e = launch_partial_merge(p, B, dims->dtype, cs);
+  if (e != cudaSuccess) return MTLA_ERR_CUDA;
+  if (!out) return MTLA_OK;
+  return from_cuda(launch_prefill_simt(p, B, dims->dtype, cs));
+}
+
+}  // extern "C"

@@ -1,0 +1,101 @@
+// Argument blocks and launchers shared by the MTLA kernels and the C ABI.
+#pragma once
+
+#include "mtla_common.cuh"
+
+namespace mtla {
+
+// Cache and per-sequence state (device pointers).
+struct SeqArgs {
+  void* cache;
+  int64_t cache_rows;
+  int64_t row_stride;  // elements
+  const int64_t* seq_offset;
+  const int64_t* seq_capacity;
+  int32_t* t_processed;
+  int32_t* cache_len;
+  int32_t* dev_err;
+  int r, d_R, s;
+};
+
+// Hyper-network merge inputs of one new token per sequence.
+struct MergeArgsDev {
+  const void* c_new;
+  const void* kR_new;
+  const float* W_c;
+  const float* b_c;
+  const float* P;
+  int32_t J_max;
+};
+
+struct DecodeOut {
+  const void* q_abs;
+  const void* q_rope;
+  float* out;
+  float* lse;
+  float scale;  // 1/sqrt(d_h)
+  int H;
+};
+
+struct PrefillArgs {
+  const void* q_abs;
+  const void* q_rope;
+  const void* c;
+  const void* kR;
+  const float* W_c;
+  const float* b_c;
+  const float* P;
+  void* c_partial;
+  void* cache_out;
+  void* out;
+  int32_t* dev_err;
+  int64_t T;
+  int64_t groups_per_block;
+  int H, r, d_R, s;
+  float scale;
+  int32_t J_max;
+};
+
+// Split-L tensor-core decode (bf16, H = 8, r = 256, d_R = 32).
+namespace dtc {
+constexpr int H = 8, R = 256, DR = 32, D = R + DR;
+constexpr int UNIT = 64;                 // rows per full TMA box
+constexpr int SUB = 8;                   // rows per box of a ragged last unit
+constexpr int ROWB = D * 2;              // bytes per cache row (576)
+constexpr int STAGE = UNIT * ROWB;       // 36864 bytes per pipeline stage
+constexpr int NS = 4;                    // pipeline depth
+constexpr int NCW = 4;                   // consumer warps
+constexpr int NT = 32 * (NCW + 1);       // + 1 producer warp
+constexpr int WC_ROWS = STAGE / (D * 4); // W_c rows per stage (32)
+constexpr int N_WC = R / WC_ROWS;        // W_c stages per merge (8)
+constexpr int MAXB = 2048;
+constexpr int OSTR = 260;                // head stride of the combine buffer (floats)
+constexpr int MERGE_COST = 128;          // partition weight of one merge, in rows
+
+struct Params {
+  SeqArgs a;
+  MergeArgsDev m;
+  DecodeOut o;
+  int with_merge;
+  int B;
+  int merge_cost;
+  float scale_log2;     // log2(e) / sqrt(d_h)
+  int32_t* tickets;     // [B]
+  int32_t* done;        // [1]
+  float* ws_ml;         // [2 * grid][H][2]
+  float* ws_o;          // [2 * grid][H][R]
+};
+
+size_t smem_bytes();
+size_t workspace_bytes(int B, int grid);
+}  // namespace dtc
+
+cudaError_t launch_merge_append(const SeqArgs& a, const MergeArgsDev& m, int B, int dtype, cudaStream_t st);
+cudaError_t launch_decode_simt(const SeqArgs& a, const MergeArgsDev& m, bool with_merge, const DecodeOut& o,
+                               int B, int dtype, cudaStream_t st);
+cudaError_t launch_decode_tc(const dtc::Params& p, const CUtensorMap& map64, const CUtensorMap& map8, int grid,
+                             cudaStream_t st);
+cudaError_t launch_partial_merge(const PrefillArgs& p, int B, int dtype, cudaStream_t st);
+cudaError_t launch_prefill_simt(const PrefillArgs& p, int B, int dtype, cudaStream_t st);
+
+}  // namespace mtla
