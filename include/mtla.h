@@ -119,7 +119,7 @@ mtla_status mtla_merge_append(const mtla_dims *dims, int32_t B, const mtla_merge
  *              by the caller ONCE before first use; every call leaves it zeroed
  *              again, so one workspace serves calls that run one after another
  *              on a stream (not calls that overlap).
- * Kernels: bf16 with (H, r, d_R) = (8, 256, 32) and B <= 2048 runs the
+ * Kernels: bf16 with (H, r, d_R) = (8, 256, 32) and B <= 1024 runs the
  * split-L tensor-core kernel (workspace required); any other supported dims
  * run a one-block-per-sequence kernel (workspace unused, may be NULL).
  * Supported dims everywhere: H <= 16, r <= 512, r + d_R <= 576, r and d_R

@@ -30,11 +30,15 @@ bool tc_decode_dims(const mtla_dims* d, int B) {
   return d->dtype == MTLA_BF16 && d->H == dtc::H && d->r == dtc::R && d->d_R == dtc::DR && B <= dtc::MAXB;
 }
 
-int sm_count() {
-  int dev = 0, n = 0;
+// persistent grid of the tensor-core decode on the current device, cached per device
+int decode_grid() {
+  static int cached[64] = {0};
+  int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  return n;
+  if (dev < 64 && cached[dev] > 0) return cached[dev];
+  const int g = dtc::grid_size();
+  if (dev < 64 && g > 0) cached[dev] = g;
+  return g;
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point, so the
@@ -146,7 +150,7 @@ mtla_status mtla_debug_stride_mask(int32_t s, int32_t T, uint8_t* host_out) {
 size_t mtla_workspace_bytes(const mtla_dims* dims, int32_t B, int32_t which) {
   if (check_dims(dims) != MTLA_OK || B < 0) return 0;
   if (which == MTLA_WS_DECODE && tc_decode_dims(dims, B)) {
-    const int g = sm_count();
+    const int g = decode_grid();
     return g > 0 ? dtc::workspace_bytes(B, g) : 0;
   }
   return 0;
@@ -199,7 +203,7 @@ mtla_status mtla_decode_attn(const mtla_dims* dims, int32_t B, const void* q_abs
   if (!tc_decode_dims(dims, B))
     return from_cuda(launch_decode_simt(a, m, merge != nullptr, o, B, dims->dtype, cs));
 
-  const int grid = sm_count();
+  const int grid = decode_grid();
   if (grid <= 0) return MTLA_ERR_CUDA;
   const size_t need = dtc::workspace_bytes(B, grid);
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return MTLA_ERR_WORKSPACE;
@@ -227,7 +231,11 @@ mtla_status mtla_decode_attn(const mtla_dims* dims, int32_t B, const void* q_abs
   size_t off = 0;
   p.tickets = reinterpret_cast<int32_t*>(ws + off);
   p.done = p.tickets + B;
-  off += ((size_t)B + 1) * 4;
+  p.gate_done = p.tickets + B + 1;
+  off += ((size_t)B + 2) * 4;
+  off = (off + 255) & ~(size_t)255;
+  p.gates = reinterpret_cast<float*>(ws + off);
+  off += (size_t)B * dtc::D * 4;
   off = (off + 255) & ~(size_t)255;
   p.ws_ml = reinterpret_cast<float*>(ws + off);
   off += (size_t)2 * grid * dtc::H * 2 * 4;

@@ -10,7 +10,7 @@
 // Design (B200):
 //  * The H heads share one latent cache, so every cache row (576 B) is read
 //    from HBM exactly once for all heads.  The rows of all sequences are cut
-//    into equal shares for a persistent grid of one block per SM (split-L,
+//    into equal shares for a persistent grid of two blocks per SM (split-L,
 //    balanced to the row; a merge counts as MERGE_COST rows).
 //  * One producer warp streams 64-row tiles HBM -> shared memory with 3-D TMA
 //    boxes {32 elements, 9 chunks, 64 rows} and 64-byte swizzle (a ragged last
@@ -22,37 +22,57 @@
 //    value-MMA operand with one in-register 8x8 transpose (movmatrix).  Each
 //    warp keeps its own online-softmax state, so no block barrier is needed
 //    per tile.
-//  * The merge of a new token is done by the block owning that sequence's
-//    tail row: W_c (fp32) streams through the same pipeline (8 stages), the
-//    gate and the updated row are computed in fp32, written to the cache in
-//    bf16 and patched into the tile before it is used.
+//  * The merge of the new tokens is spread over the whole grid: the gate
+//    pre-activations Linear(c_t) = c_t W_c + b_c of all B tokens are cut into
+//    channel-major slices, one per block, computed while the block's first
+//    tiles are in flight (each block reads about one column of W_c).  The
+//    block owning a sequence's tail row waits (bounded) for all slices, then
+//    forms the gate, the gated entry and the updated row in fp32, writes it to
+//    the cache in bf16 and patches it into the tile before the tile is used.
+//  * Launched with programmatic dependent launch: the next call's blocks are
+//    scheduled while this call's last blocks finish and wait for it before
+//    touching memory.
 //  * Partial results of sequences split between blocks go to the workspace;
 //    the last block to finish a sequence (atomic ticket) combines them.  No
 //    block ever waits for another.  The last block of the grid advances
-//    t_processed and resets the counters.
+//    t_processed and resets the counters.  Every block's share and first
+//    sequence are tabulated once in shared memory, so the bookkeeping in the
+//    loops needs no integer division.
 #include "kernels.cuh"
 
 namespace mtla {
 namespace dtc {
 
-size_t smem_bytes() {
-  size_t b = 0;
-  b += (size_t)NS * STAGE;                 // stages
-  b += (size_t)NCW * H * OSTR * 4;         // combine O
-  b += (size_t)NCW * H * 2 * 4;            // combine m, l
-  b += (size_t)(MAXB + 1) * 8;             // cost prefix (int64)
-  b += (size_t)MAXB * 4;                   // rows + flags per sequence
-  b += 128 * 8;                            // scan scratch (int64)
-  b += (size_t)R * 4;                      // c_new in fp32
-  b += (size_t)D * 2;                      // merged tail row (bf16)
-  b += 2 * NS * 8;                         // mbarriers
-  b += 16;                                 // flags
-  return b + 1024;                         // alignment slack
-}
+// every region starts on a 128-byte boundary (the tail row is read with
+// 16-byte vector loads, the mbarriers need 8)
+constexpr size_t kAlign = 128;
+__host__ __device__ constexpr size_t rup(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+constexpr int kCombHeads = 4;  // heads per pass of the block combine
+constexpr int QSTR = D / 2 + 4;  // words per query row in shared memory (148: conflict-free)
+static_assert(17 * H * 2 <= NCW * kCombHeads * OSTR, "combine scratch must fit the combine buffer");
+static_assert((size_t)H * QSTR * 4 <= (size_t)NCW * kCombHeads * OSTR * 4, "query buffer must fit the combine buffer");
+constexpr size_t kOffComb = rup((size_t)NS * STAGE);
+constexpr size_t kOffCombMl = kOffComb + rup((size_t)NCW * kCombHeads * OSTR * 4);
+constexpr size_t kOffPrefix = kOffCombMl + rup((size_t)NCW * H * 2 * 4);
+constexpr size_t kOffMeta = kOffPrefix + rup((size_t)(MAXB + 1) * 8);
+constexpr size_t kOffScan = kOffMeta + rup((size_t)MAXB * 4);
+constexpr size_t kOffLo = kOffScan + rup(128 * 8);
+constexpr size_t kOffFs = kOffLo + rup((size_t)(MAXG + 1) * 8);
+constexpr size_t kOffSlots = kOffFs + rup((size_t)MAXG * 4);
+constexpr size_t kOffC = kOffSlots + rup((size_t)MAXG * 4);
+constexpr size_t kOffTail = kOffC + rup((size_t)R * 4);
+constexpr size_t kOffBar = kOffTail + rup((size_t)D * 2);
+constexpr size_t kOffFlags = kOffBar + rup(2 * NS * 8);
+constexpr size_t kSmemUsed = kOffFlags + rup(16);
+static_assert(kOffTail % 16 == 0 && kOffBar % 8 == 0, "shared-memory regions must stay aligned");
+
+size_t smem_bytes() { return kSmemUsed + 1024; }  // + slack to align the base to 1024
 
 size_t workspace_bytes(int B, int grid) {
   size_t b = 0;
-  b += ((size_t)B + 1) * 4;
+  b += ((size_t)B + 2) * 4;
+  b = (b + 255) & ~(size_t)255;
+  b += (size_t)B * D * 4;
   b = (b + 255) & ~(size_t)255;
   b += (size_t)2 * grid * H * 2 * 4;
   b = (b + 255) & ~(size_t)255;
@@ -60,9 +80,10 @@ size_t workspace_bytes(int B, int grid) {
   return b;
 }
 
-// byte address in a swizzled tile of row `row`, 16-byte chunk `ch` (0..35)
-__device__ __forceinline__ uint32_t swz(uint32_t tile, int row, int ch) {
-  const uint32_t seg = tile + (uint32_t)row * ROWB + (uint32_t)(ch >> 2) * 64u;
+// byte offset, inside a swizzled tile, of row `row`, 16-byte chunk `ch` (0..35):
+// TMA's 64-byte swizzle XORs chunk bits [4:5] with address bits [7:8]
+__host__ __device__ __forceinline__ uint32_t swz_off(int row, int ch) {
+  const uint32_t seg = (uint32_t)row * ROWB + (uint32_t)(ch >> 2) * 64u;
   return seg + ((((uint32_t)ch & 3u) ^ ((seg >> 7) & 3u)) << 4);
 }
 
@@ -75,6 +96,9 @@ struct Smem {
   int64_t* prefix;
   uint32_t* meta;     // rows (bits 0..29) | merge ok (bit 30)
   int64_t* scan;
+  int64_t* lo;        // [G + 1] first cost position of each block's share
+  int32_t* fs;        // [G] first sequence with rows in each block's share
+  int32_t* slots;     // [G] workspace slots of the sequence being combined
   float* c_sm;
   __nv_bfloat16* tail_sm;
   uint64_t* full_bar;
@@ -86,26 +110,19 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   Smem s;
   uint8_t* p = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
   s.stages = p;
-  p += NS * STAGE;
-  s.comb_o = reinterpret_cast<float*>(p);
-  p += NCW * H * OSTR * 4;
-  s.comb_ml = reinterpret_cast<float*>(p);
-  p += NCW * H * 2 * 4;
-  s.prefix = reinterpret_cast<int64_t*>(p);
-  p += (MAXB + 1) * 8;
-  s.meta = reinterpret_cast<uint32_t*>(p);
-  p += MAXB * 4;
-  s.scan = reinterpret_cast<int64_t*>(p);
-  p += 128 * 8;
-  s.c_sm = reinterpret_cast<float*>(p);
-  p += R * 4;
-  s.tail_sm = reinterpret_cast<__nv_bfloat16*>(p);
-  p += D * 2;
-  s.full_bar = reinterpret_cast<uint64_t*>(p);
-  p += NS * 8;
-  s.empty_bar = reinterpret_cast<uint64_t*>(p);
-  p += NS * 8;
-  s.flags = reinterpret_cast<int32_t*>(p);
+  s.comb_o = reinterpret_cast<float*>(p + kOffComb);
+  s.comb_ml = reinterpret_cast<float*>(p + kOffCombMl);
+  s.prefix = reinterpret_cast<int64_t*>(p + kOffPrefix);
+  s.meta = reinterpret_cast<uint32_t*>(p + kOffMeta);
+  s.scan = reinterpret_cast<int64_t*>(p + kOffScan);
+  s.lo = reinterpret_cast<int64_t*>(p + kOffLo);
+  s.fs = reinterpret_cast<int32_t*>(p + kOffFs);
+  s.slots = reinterpret_cast<int32_t*>(p + kOffSlots);
+  s.c_sm = reinterpret_cast<float*>(p + kOffC);
+  s.tail_sm = reinterpret_cast<__nv_bfloat16*>(p + kOffTail);
+  s.full_bar = reinterpret_cast<uint64_t*>(p + kOffBar);
+  s.empty_bar = s.full_bar + NS;
+  s.flags = reinterpret_cast<int32_t*>(p + kOffFlags);
   return s;
 }
 
@@ -119,27 +136,19 @@ __device__ __forceinline__ int upper_bound_i64(const int64_t* a, int n, int64_t 
   return lo;
 }
 
-struct Part {
-  const int64_t* prefix;
-  const uint32_t* meta;
-  int B;
-  int G;
-  int64_t C;
-  __device__ __forceinline__ int64_t lo(int c) const { return (int64_t)c * C / G; }
-  __device__ __forceinline__ int64_t rows(int b) const { return (int64_t)(meta[b] & (kMetaMergeOk - 1)); }
-  // block whose share holds cost position pos
-  __device__ __forceinline__ int owner(int64_t pos) const { return (int)(((pos + 1) * G - 1) / C); }
-  // first sequence with rows inside block c's share (B if none)
-  __device__ __forceinline__ int first_seq(int c) const {
-    const int64_t x = lo(c);
-    int b = upper_bound_i64(prefix, B + 1, x) - 1;
-    if (b < 0) b = 0;
-    if (b < B && x - prefix[b] >= rows(b)) ++b;
-    return b;
-  }
-};
+constexpr uint32_t kSpinLimit = 1u << 22;  // x 64 ns sleeps: gives up after ~0.3 s
 
-__global__ void __launch_bounds__(NT, 1)
+__device__ __forceinline__ int ld_acquire_gpu(const int32_t* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ int64_t rows_of(const uint32_t* meta, int b) {
+  return (int64_t)(meta[b] & (kMetaMergeOk - 1));
+}
+
+__global__ void __launch_bounds__(NT, 2)
 decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constant__ CUtensorMap map8,
                  const Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -147,6 +156,23 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int B = p.B, s = p.a.s, G = gridDim.x, cta = blockIdx.x;
   const bool with_merge = p.with_merge != 0;
+  const int64_t mcost = with_merge ? p.merge_cost : 0;
+
+  // let the next launch on the stream be scheduled as soon as blocks retire;
+  // then wait for the previous launch before reading anything it may write
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (tid == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&sm.full_bar[i], 1);
+      mbar_init(&sm.empty_bar[i], NCW);
+    }
+    fence_mbar_init();
+  }
+  if (warp == NCW && lane == 0) {
+    prefetch_tmap(&map64);
+    prefetch_tmap(&map8);
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // ---- 1. rows per sequence and the cost prefix (identical in every block)
   const int per = (B + 127) / 128;
@@ -178,7 +204,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
         ok = false;
       }
       sm.meta[b] = (uint32_t)L | (ok ? kMetaMergeOk : 0u);
-      sum += L + (with_merge ? p.merge_cost : 0);
+      sum += L + mcost;
     }
     sm.scan[tid] = sum;
   }
@@ -197,70 +223,47 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
     int64_t ex = incl - run;
 #pragma unroll
     for (int i = 0; i < 4; ++i) { const int64_t t = v[i]; sm.scan[lane * 4 + i] = ex; ex += t; }
+    if (lane == 31) sm.prefix[B] = ex;  // total cost
   }
   __syncthreads();
   if (tid < 128) {
     int64_t run = sm.scan[tid];
     for (int b = tid * per; b < B && b < (tid + 1) * per; ++b) {
       sm.prefix[b] = run;
-      run += (int64_t)(sm.meta[b] & (kMetaMergeOk - 1)) + (with_merge ? p.merge_cost : 0);
+      run += rows_of(sm.meta, b) + mcost;
     }
   }
-  if (tid == 0) {
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(&sm.full_bar[i], 1);
-      mbar_init(&sm.empty_bar[i], NCW);
-    }
-    fence_mbar_init();
-  }
+  const int64_t C = sm.prefix[B];
+  // share starts: block c owns cost positions [lo[c], lo[c+1])
+  for (int c = tid; c <= G; c += NT) sm.lo[c] = C > 0 ? (int64_t)c * C / G : 0;
   __syncthreads();
-  if (tid == 0) {
-    // total = prefix of the last sequence + its cost
-    const int64_t last = B > 0 ? sm.prefix[B - 1] + (int64_t)(sm.meta[B - 1] & (kMetaMergeOk - 1)) +
-                                     (with_merge ? p.merge_cost : 0)
-                               : 0;
-    sm.prefix[B] = last;
+  // first sequence with rows in each share (B if none)
+  for (int c = tid; c < G; c += NT) {
+    const int64_t x = sm.lo[c];
+    int b = upper_bound_i64(sm.prefix, B + 1, x) - 1;
+    if (b < 0) b = 0;
+    if (b < B && x - sm.prefix[b] >= rows_of(sm.meta, b)) ++b;
+    sm.fs[c] = (x < sm.lo[c + 1]) ? b : B;
   }
   __syncthreads();
 
-  Part part;
-  part.prefix = sm.prefix;
-  part.meta = sm.meta;
-  part.B = B;
-  part.G = G;
-  part.C = sm.prefix[B];
-  const int64_t my_lo = part.C > 0 ? part.lo(cta) : 0;
-  const int64_t my_hi = part.C > 0 ? part.lo(cta + 1) : 0;
-  const int b_first = part.C > 0 ? part.first_seq(cta) : B;
-
+  const int64_t my_lo = sm.lo[cta], my_hi = sm.lo[cta + 1];
+  const int b_first = sm.fs[cta];
   const __nv_bfloat16* cache = reinterpret_cast<const __nv_bfloat16*>(p.a.cache);
 
   // ======================= producer warp =======================
   if (warp == NCW) {
     if (lane == 0 && my_lo < my_hi) {
-      prefetch_tmap(&map64);
-      prefetch_tmap(&map8);
       uint32_t job = 0;
       bool ok = true;
       for (int b = b_first; b < B && sm.prefix[b] < my_hi && ok; ++b) {
-        const int64_t Lb = part.rows(b);
+        const int64_t Lb = rows_of(sm.meta, b);
         const int64_t r_lo = (my_lo > sm.prefix[b] ? my_lo : sm.prefix[b]) - sm.prefix[b];
         const int64_t r_end = sm.prefix[b] + Lb < my_hi ? sm.prefix[b] + Lb : my_hi;
         const int64_t r_hi = r_end - sm.prefix[b];
         if (r_lo >= r_hi) continue;
-        const bool merge_here = (sm.meta[b] & kMetaMergeOk) && r_hi == Lb;
         const int64_t row0 = p.a.seq_offset[b];
         for (int64_t u = r_lo; u < r_hi && ok; u += UNIT) {
-          const bool is_tail = merge_here && u + UNIT >= r_hi;
-          if (is_tail) {
-            for (int w = 0; w < N_WC && ok; ++w, ++job) {
-              const int st = job % NS;
-              if (job >= NS && !mbar_wait(&sm.empty_bar[st], ((job / NS) & 1) ^ 1)) { ok = false; break; }
-              mbar_arrive_expect_tx(&sm.full_bar[st], STAGE);
-              bulk_load(sm.stages + st * STAGE, p.m.W_c + (size_t)w * WC_ROWS * D, STAGE, &sm.full_bar[st]);
-            }
-            if (!ok) break;
-          }
           const int st = job % NS;
           if (job >= NS && !mbar_wait(&sm.empty_bar[st], ((job / NS) & 1) ^ 1)) { ok = false; break; }
           const int64_t nrows = r_hi - u < UNIT ? r_hi - u : UNIT;
@@ -289,11 +292,65 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
   const int cw = warp, ctid = tid;  // 0..127
   const int g = lane >> 2, q = lane & 3;
   const float sl2 = p.scale_log2;
+  // per-lane ldmatrix rows: scores (A = rows, K-major) and values (A = C_hat^T, trans)
+  const int w_lo = 16 * cw;
+  const int arow = w_lo + (lane & 7) + ((lane >> 3) & 1) * 8;
+  const int ach = lane >> 4;
+  const int vrow = w_lo + (lane & 7) + (lane >> 4) * 8;
+  const int vch = (lane >> 3) & 1;
   uint32_t job = 0;
   bool ok = true;
 
+  // ---- merge gates: this block's slice of Linear(c_t) = c_t W_c + b_c,
+  // channel-major (index k * B + b), while its first tiles are in flight
+  if (with_merge) {
+    const int N = B * D;
+    const int i_lo = (int)((int64_t)cta * N / G), i_hi = (int)((int64_t)(cta + 1) * N / G);
+    float* wcol = sm.c_sm;  // one column of W_c
+    const uint4* cnew = reinterpret_cast<const uint4*>(p.m.c_new);
+    for (int k = i_lo / B; i_lo < i_hi && k <= (i_hi - 1) / B; ++k) {
+      const int b_lo = i_lo - k * B > 0 ? i_lo - k * B : 0;
+      const int b_hi = i_hi - k * B < B ? i_hi - k * B : B;
+      for (int i = ctid; i < R; i += 128) wcol[i] = __ldg(p.m.W_c + (size_t)i * D + k);
+      named_bar(1, 128);
+      float wv[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) wv[e] = wcol[8 * lane + e];
+      const float bias = __ldg(p.m.b_c + k);
+      // warp cw takes sequences b_lo + cw, + NCW, ...; four at a time so that
+      // their loads overlap; lane covers inputs 8 lane .. 8 lane + 7
+      for (int b0 = b_lo + cw; b0 < b_hi; b0 += 4 * NCW) {
+        uint4 cv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int bb = b0 + u * NCW;
+          cv[u] = bb < b_hi ? __ldg(cnew + (size_t)bb * (R / 8) + lane) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&cv[u]);
+          float acc = 0.f;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(h2[e]);
+            acc = fmaf(f.x, wv[2 * e], acc);
+            acc = fmaf(f.y, wv[2 * e + 1], acc);
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+          const int bb = b0 + u * NCW;
+          if (lane == 0 && bb < b_hi) p.gates[(size_t)bb * D + k] = acc + bias;
+        }
+      }
+      named_bar(1, 128);  // the column buffer is reused for the next channel
+    }
+    __threadfence();
+    named_bar(1, 128);
+    if (ctid == 0) atomicAdd(p.gate_done, 1);
+  }
+
   for (int b = b_first; b < B && sm.prefix[b] < my_hi; ++b) {
-    const int64_t Lb = part.rows(b);
+    const int64_t Lb = rows_of(sm.meta, b);
     const int64_t r_lo = (my_lo > sm.prefix[b] ? my_lo : sm.prefix[b]) - sm.prefix[b];
     const int64_t r_end = sm.prefix[b] + Lb < my_hi ? sm.prefix[b] + Lb : my_hi;
     const int64_t r_hi = r_end - sm.prefix[b];
@@ -301,70 +358,60 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
     const bool merge_here = (sm.meta[b] & kMetaMergeOk) && r_hi == Lb;
     const bool full = (r_lo == 0 && r_hi == Lb);
 
-    // B operand of the score MMA: [q_abs ; q_rope] of head g, k = 16kk + 2q (+1, +8, +9)
-    uint32_t bq[18][2];
+    // [q_abs ; q_rope] of the 8 heads into shared memory (rows padded to
+    // QSTR words so the B-fragment loads below are free of bank conflicts);
+    // the buffer shares space with the combine buffer, which is only used
+    // after the segment's last tile
     {
       const uint32_t* qa = reinterpret_cast<const uint32_t*>(
-          reinterpret_cast<const __nv_bfloat16*>(p.o.q_abs) + ((size_t)b * H + g) * R);
+          reinterpret_cast<const __nv_bfloat16*>(p.o.q_abs) + (size_t)b * H * R);
       const uint32_t* qr = reinterpret_cast<const uint32_t*>(
-          reinterpret_cast<const __nv_bfloat16*>(p.o.q_rope) + ((size_t)b * H + g) * DR);
-#pragma unroll
-      for (int kk = 0; kk < 16; ++kk) {
-        bq[kk][0] = __ldg(qa + kk * 8 + q);
-        bq[kk][1] = __ldg(qa + kk * 8 + q + 4);
+          reinterpret_cast<const __nv_bfloat16*>(p.o.q_rope) + (size_t)b * H * DR);
+      uint32_t* qs = reinterpret_cast<uint32_t*>(sm.comb_o);
+      for (int i = ctid; i < H * (D / 2); i += 128) {
+        const int h = i / (D / 2), w = i % (D / 2);
+        qs[h * QSTR + w] = w < R / 2 ? __ldg(qa + h * (R / 2) + w) : __ldg(qr + h * (DR / 2) + (w - R / 2));
       }
-#pragma unroll
-      for (int kk = 0; kk < 2; ++kk) {
-        bq[16 + kk][0] = __ldg(qr + kk * 8 + q);
-        bq[16 + kk][1] = __ldg(qr + kk * 8 + q + 4);
-      }
+      named_bar(1, 128);
     }
+    // B operand of the score MMA for head g: words 8kk + q and 8kk + q + 4 of its row
+    const uint32_t qrow = smem_u32(sm.comb_o) + (uint32_t)(g * QSTR + q) * 4u;
     float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
     float O[16][4];
 #pragma unroll
     for (int mb = 0; mb < 16; ++mb) O[mb][0] = O[mb][1] = O[mb][2] = O[mb][3] = 0.f;
 
-    float gacc[3] = {0.f, 0.f, 0.f};
-    if (merge_here) {
-      const __nv_bfloat16* c = reinterpret_cast<const __nv_bfloat16*>(p.m.c_new) + (size_t)b * R;
-      for (int i = ctid; i < R; i += 128) sm.c_sm[i] = __bfloat162float(c[i]);
-      named_bar(1, 128);
-    }
 
     for (int64_t u = r_lo; u < r_hi; u += UNIT) {
       const bool is_tail = merge_here && u + UNIT >= r_hi;
       if (is_tail) {
-        for (int w = 0; w < N_WC; ++w, ++job) {
-          const int st = job % NS;
-          if (ok && !mbar_wait(&sm.full_bar[st], (job / NS) & 1)) ok = false;
-          const float* Wsm = reinterpret_cast<const float*>(sm.stages + st * STAGE);
-#pragma unroll
-          for (int ci = 0; ci < 3; ++ci) {
-            const int k = ctid + 128 * ci;
-            if (k < D) {
-              float a = gacc[ci];
-#pragma unroll 8
-              for (int i = 0; i < WC_ROWS; ++i) a = fmaf(sm.c_sm[w * WC_ROWS + i], Wsm[i * D + k], a);
-              gacc[ci] = a;
+        // every block's slice of the gates must be written (bounded wait)
+        if (ctid == 0) {
+          uint32_t it = 0;
+          while (ld_acquire_gpu(p.gate_done) < G) {
+            if (++it > kSpinLimit) {
+              set_err(p.a.dev_err, MTLA_DEVERR_TIMEOUT);
+              break;
             }
+            __nanosleep(64);
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.empty_bar[st]);
         }
+        named_bar(1, 128);
         // gate, gated entry and the updated tail row (fp32 math, bf16 storage)
         const int64_t t = (int64_t)p.a.t_processed[b] + 1;
         const int64_t j = group_of(t, s);
         const bool opens = opens_row(t, s);
         __nv_bfloat16* row = const_cast<__nv_bfloat16*>(cache) + (p.a.seq_offset[b] + j - 1) * p.a.row_stride;
+        const __nv_bfloat16* cn = reinterpret_cast<const __nv_bfloat16*>(p.m.c_new) + (size_t)b * R;
         const __nv_bfloat16* kR = reinterpret_cast<const __nv_bfloat16*>(p.m.kR_new) + (size_t)b * DR;
         const float* Pj = p.m.P + (j - 1) * D;
 #pragma unroll
         for (int ci = 0; ci < 3; ++ci) {
           const int k = ctid + 128 * ci;
           if (k < D) {
-            const float gv = __fadd_rn(gacc[ci], p.m.b_c[k]);
+            const float gv = __ldcg(p.gates + (size_t)b * D + k);
             const float w = sigmoidf_(__fmul_rn(gv, Pj[k]));
-            const float x = k < R ? sm.c_sm[k] : __bfloat162float(kR[k - R]);
+            const float x = __bfloat162float(k < R ? cn[k] : kR[k - R]);
             const float e = __fmul_rn(w, x);
             const float v = opens ? e : __fadd_rn(__bfloat162float(row[k]), e);
             const __nv_bfloat16 vb = __float2bfloat16_rn(v);
@@ -377,16 +424,17 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
 
       const int st = job % NS;
       if (ok && !mbar_wait(&sm.full_bar[st], (job / NS) & 1)) ok = false;
-      const uint32_t tile = smem_u32(sm.stages + st * STAGE);
+      uint8_t* tile_ptr = sm.stages + st * STAGE;
+      const uint32_t tile = smem_u32(tile_ptr);
       const int rows = (int)(r_hi - u < UNIT ? r_hi - u : UNIT);
-      const int w_lo = 16 * cw;
       if (w_lo < rows) {
         bool wrote = false;
         if (w_lo + 16 > rows) {
           // rows past the segment's end: zero them (they may hold anything)
           for (int i = lane; i < (w_lo + 16 - rows) * 36; i += 32) {
             const int rr = rows + i / 36, ch = i % 36;
-            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(swz(tile, rr, ch)), "r"(0u) : "memory");
+            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(tile + swz_off(rr, ch)), "r"(0u)
+                         : "memory");
           }
           wrote = true;
         }
@@ -396,8 +444,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
             const uint4* src = reinterpret_cast<const uint4*>(sm.tail_sm);
             for (int ch = lane; ch < 36; ch += 32) {
               const uint4 v = src[ch];
-              asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(swz(tile, lr, ch)), "r"(v.x), "r"(v.y),
-                           "r"(v.z), "r"(v.w) : "memory");
+              asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(tile + swz_off(lr, ch)), "r"(v.x),
+                           "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
             }
             wrote = true;
           }
@@ -405,22 +453,24 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
         if (wrote) fence_proxy_async_smem();
         __syncwarp();
 
-        // scores S^T (16 rows x 8 heads) = rows . [q_abs ; q_rope]^T
-        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
-        const int arow = w_lo + (lane & 7) + ((lane >> 3) & 1) * 8;
+        // scores S^T (16 rows x 8 heads) = rows . [q_abs ; q_rope]^T, two
+        // independent accumulator chains
+        float sacc[2][4];
 #pragma unroll
-        for (int kk = 0; kk < 18; kk += 2) {
-          uint32_t a0, a1, a2, a3, c0, c1, c2, c3;
-          ldsm_x4(swz(tile, arow, 2 * kk + (lane >> 4)), a0, a1, a2, a3);
-          ldsm_x4(swz(tile, arow, 2 * kk + 2 + (lane >> 4)), c0, c1, c2, c3);
-          mma_bf16(sa, a0, a1, a2, a3, bq[kk][0], bq[kk][1]);
-          mma_bf16(sb, c0, c1, c2, c3, bq[kk + 1][0], bq[kk + 1][1]);
+        for (int i = 0; i < 2; ++i) sacc[i][0] = sacc[i][1] = sacc[i][2] = sacc[i][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 18; ++kk) {
+          uint32_t a0, a1, a2, a3, b0, b1;
+          ldsm_x4(tile + swz_off(arow, 2 * kk + ach), a0, a1, a2, a3);
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(b0) : "r"(qrow + kk * 32u));
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(b1) : "r"(qrow + kk * 32u + 16u));
+          mma_bf16(sacc[kk & 1], a0, a1, a2, a3, b0, b1);
         }
         const bool v0 = (w_lo + g) < rows, v1 = (w_lo + g + 8) < rows;
-        const float xA0 = v0 ? (sa[0] + sb[0]) * sl2 : -INFINITY;
-        const float xB0 = v0 ? (sa[1] + sb[1]) * sl2 : -INFINITY;
-        const float xA1 = v1 ? (sa[2] + sb[2]) * sl2 : -INFINITY;
-        const float xB1 = v1 ? (sa[3] + sb[3]) * sl2 : -INFINITY;
+        const float xA0 = v0 ? (sacc[0][0] + sacc[1][0]) * sl2 : -INFINITY;
+        const float xB0 = v0 ? (sacc[0][1] + sacc[1][1]) * sl2 : -INFINITY;
+        const float xA1 = v1 ? (sacc[0][2] + sacc[1][2]) * sl2 : -INFINITY;
+        const float xB1 = v1 ? (sacc[0][3] + sacc[1][3]) * sl2 : -INFINITY;
         float mxA = fmaxf(xA0, xA1), mxB = fmaxf(xB0, xB1);
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
@@ -446,12 +496,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
         const uint32_t pb0 = movmatrix_t(pack_bf16x2(pA0, pB0));
         const uint32_t pb1 = movmatrix_t(pack_bf16x2(pA1, pB1));
         // values O^T (256 channels x 8 heads) += C_hat^T . P^T
-        const int vrow = w_lo + (lane & 7) + (lane >> 4) * 8;
-        const int vch = (lane >> 3) & 1;
 #pragma unroll
         for (int mb = 0; mb < 16; ++mb) {
           uint32_t a0, a1, a2, a3;
-          ldsm_x4_t(swz(tile, vrow, 2 * mb + vch), a0, a1, a2, a3);
+          ldsm_x4_t(tile + swz_off(vrow, 2 * mb + vch), a0, a1, a2, a3);
           mma_bf16(O[mb], a0, a1, a2, a3, pb0, pb1);
         }
       }
@@ -461,6 +509,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
     }
 
     // ---- segment end: combine the four warps, then write out or a partial
+    named_bar(1, 128);  // every warp is done with the query buffer
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
       lA += __shfl_xor_sync(0xffffffffu, lA, o);
@@ -472,87 +521,138 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
       sm.comb_ml[(cw * H + 2 * q + 1) * 2 + 0] = mB;
       sm.comb_ml[(cw * H + 2 * q + 1) * 2 + 1] = lB;
     }
-#pragma unroll
-    for (int mb = 0; mb < 16; ++mb) {
-      float* oA = sm.comb_o + (cw * H + 2 * q) * OSTR + 16 * mb + g;
-      float* oB = sm.comb_o + (cw * H + 2 * q + 1) * OSTR + 16 * mb + g;
-      oA[0] = O[mb][0];
-      oB[0] = O[mb][1];
-      oA[8] = O[mb][2];
-      oB[8] = O[mb][3];
-    }
-    named_bar(1, 128);
-
     const int nslot = full ? -1 : 2 * cta + (b == b_first ? 0 : 1);
 #pragma unroll 1
-    for (int h = 0; h < H; ++h) {
-      float M = -INFINITY;
+    for (int pass = 0; pass < 2; ++pass) {
+      // heads 4 pass .. 4 pass + 3 belong to the lanes with q >> 1 == pass
+      if ((q >> 1) == pass) {
+        const int hl = 2 * q - kCombHeads * pass;  // local head of O[.][0]
 #pragma unroll
-      for (int w = 0; w < NCW; ++w) M = fmaxf(M, sm.comb_ml[(w * H + h) * 2]);
-      float Ls = 0.f, o0 = 0.f, o1 = 0.f;
-#pragma unroll
-      for (int w = 0; w < NCW; ++w) {
-        const float mw = sm.comb_ml[(w * H + h) * 2];
-        const float sc = mw == -INFINITY ? 0.f : exp2f(mw - M);
-        Ls += sc * sm.comb_ml[(w * H + h) * 2 + 1];
-        const float2 ov = *reinterpret_cast<const float2*>(sm.comb_o + (w * H + h) * OSTR + 2 * ctid);
-        o0 += sc * ov.x;
-        o1 += sc * ov.y;
-      }
-      if (full) {
-        const float inv = 1.f / Ls;
-        *reinterpret_cast<float2*>(p.o.out + ((size_t)b * H + h) * R + 2 * ctid) = make_float2(o0 * inv, o1 * inv);
-        if (p.o.lse && ctid == 0) p.o.lse[(size_t)b * H + h] = (M + log2f(Ls)) * 0.69314718055994531f;
-      } else {
-        *reinterpret_cast<float2*>(p.ws_o + ((size_t)nslot * H + h) * R + 2 * ctid) = make_float2(o0, o1);
-        if (ctid == 0) {
-          p.ws_ml[((size_t)nslot * H + h) * 2 + 0] = M;
-          p.ws_ml[((size_t)nslot * H + h) * 2 + 1] = Ls;
+        for (int mb = 0; mb < 16; ++mb) {
+          float* oA = sm.comb_o + (cw * kCombHeads + hl) * OSTR + 16 * mb + g;
+          float* oB = oA + OSTR;
+          oA[0] = O[mb][0];
+          oB[0] = O[mb][1];
+          oA[8] = O[mb][2];
+          oB[8] = O[mb][3];
         }
       }
+      named_bar(1, 128);
+#pragma unroll 1
+      for (int hl = 0; hl < kCombHeads; ++hl) {
+        const int h = kCombHeads * pass + hl;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NCW; ++w) M = fmaxf(M, sm.comb_ml[(w * H + h) * 2]);
+        float Ls = 0.f, o0 = 0.f, o1 = 0.f;
+#pragma unroll
+        for (int w = 0; w < NCW; ++w) {
+          const float mw = sm.comb_ml[(w * H + h) * 2];
+          const float sc = mw == -INFINITY ? 0.f : exp2f(mw - M);
+          Ls += sc * sm.comb_ml[(w * H + h) * 2 + 1];
+          const float2 ov = *reinterpret_cast<const float2*>(sm.comb_o + (w * kCombHeads + hl) * OSTR + 2 * ctid);
+          o0 += sc * ov.x;
+          o1 += sc * ov.y;
+        }
+        if (full) {
+          const float inv = 1.f / Ls;
+          *reinterpret_cast<float2*>(p.o.out + ((size_t)b * H + h) * R + 2 * ctid) =
+              make_float2(o0 * inv, o1 * inv);
+          if (p.o.lse && ctid == 0) p.o.lse[(size_t)b * H + h] = (M + log2f(Ls)) * 0.69314718055994531f;
+        } else {
+          *reinterpret_cast<float2*>(p.ws_o + ((size_t)nslot * H + h) * R + 2 * ctid) = make_float2(o0, o1);
+          if (ctid == 0) {
+            p.ws_ml[((size_t)nslot * H + h) * 2 + 0] = M;
+            p.ws_ml[((size_t)nslot * H + h) * 2 + 1] = Ls;
+          }
+        }
+      }
+      named_bar(1, 128);  // the buffer is rewritten by the next pass / segment
     }
     if (!full) {
       __threadfence();
       named_bar(1, 128);
-      const int c_first = part.owner(sm.prefix[b]);
-      const int c_last = part.owner(sm.prefix[b] + Lb - 1);
       if (ctid == 0) {
+        // the blocks holding part of sequence b and their workspace slots
+        const int64_t first_pos = sm.prefix[b], last_pos = sm.prefix[b] + Lb - 1;
+        const int c_first = upper_bound_i64(sm.lo, G + 1, first_pos) - 1;
+        const int c_last = upper_bound_i64(sm.lo, G + 1, last_pos) - 1;
         int nparts = 0;
-        for (int c = c_first; c <= c_last; ++c) nparts += part.lo(c) < part.lo(c + 1) ? 1 : 0;
+        for (int c = c_first; c <= c_last; ++c)
+          if (sm.lo[c] < sm.lo[c + 1]) sm.slots[nparts++] = 2 * c + (sm.fs[c] == b ? 0 : 1);
         const int old = atomicAdd(&p.tickets[b], 1);
-        sm.flags[0] = (old == nparts - 1) ? 1 : 0;
+        sm.flags[0] = (old == nparts - 1) ? nparts : 0;
         __threadfence();
       }
       named_bar(1, 128);
-      if (sm.flags[0]) {
-        // last block of this sequence: combine every block's partial
-#pragma unroll 1
-        for (int h = 0; h < H; ++h) {
-          float M = -INFINITY;
-          for (int c = c_first; c <= c_last; ++c) {
-            if (part.lo(c) >= part.lo(c + 1)) continue;
-            const int slot = 2 * c + (part.first_seq(c) == b ? 0 : 1);
-            M = fmaxf(M, __ldcg(p.ws_ml + ((size_t)slot * H + h) * 2));
+      const int nparts = sm.flags[0];
+      if (nparts) {
+        // last block of this sequence: combine every block's partial.  All
+        // loads of a phase are independent, so each phase costs about one L2
+        // round trip whatever the number of parts.
+        // phase 1: per head, running (max, sum) over the parts, 16 groups of 8 threads
+        float* red = sm.comb_o;  // [16][H][2], free at this point
+        {
+          const int h = ctid & 7, grp = ctid >> 3;
+          float M = -INFINITY, Ls = 0.f;
+          for (int i = grp; i < nparts; i += 16) {
+            const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.ws_ml) + (size_t)sm.slots[i] * H + h);
+            if (ml.x == -INFINITY) continue;
+            const float nM = fmaxf(M, ml.x);
+            Ls = Ls * exp2f(M - nM) + ml.y * exp2f(ml.x - nM);
+            M = nM;
           }
-          float Ls = 0.f, o0 = 0.f, o1 = 0.f;
-          for (int c = c_first; c <= c_last; ++c) {
-            if (part.lo(c) >= part.lo(c + 1)) continue;
-            const int slot = 2 * c + (part.first_seq(c) == b ? 0 : 1);
+          red[(grp * H + h) * 2 + 0] = M;
+          red[(grp * H + h) * 2 + 1] = Ls;
+        }
+        named_bar(1, 128);
+        if (ctid < H) {
+          float M = -INFINITY, Ls = 0.f;
+          for (int grp = 0; grp < 16; ++grp) {
+            const float m = red[(grp * H + ctid) * 2], l = red[(grp * H + ctid) * 2 + 1];
+            if (m == -INFINITY) continue;
+            const float nM = fmaxf(M, m);
+            Ls = Ls * exp2f(M - nM) + l * exp2f(m - nM);
+            M = nM;
+          }
+          red[(16 * H + ctid) * 2 + 0] = M;
+          red[(16 * H + ctid) * 2 + 1] = Ls;
+          if (p.o.lse) p.o.lse[(size_t)b * H + ctid] = (M + log2f(Ls)) * 0.69314718055994531f;
+        }
+        named_bar(1, 128);
+        // phase 2: thread -> head ctid >> 4, 16 channels; parts weighted by exp2(m_i - M) / L
+        {
+          const int h = ctid >> 4, c0 = (ctid & 15) * 16;
+          const float M = red[(16 * H + h) * 2], inv = 1.f / red[(16 * H + h) * 2 + 1];
+          float4 acc[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+          for (int i = 0; i < nparts; ++i) {
+            const int slot = sm.slots[i];
             const float mc = __ldcg(p.ws_ml + ((size_t)slot * H + h) * 2);
+            const float4* src = reinterpret_cast<const float4*>(p.ws_o + ((size_t)slot * H + h) * R + c0);
+            float4 v[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) v[k] = __ldcg(src + k);
             const float sc = mc == -INFINITY ? 0.f : exp2f(mc - M);
-            Ls += sc * __ldcg(p.ws_ml + ((size_t)slot * H + h) * 2 + 1);
-            const float2 ov = __ldcg(reinterpret_cast<const float2*>(p.ws_o + ((size_t)slot * H + h) * R + 2 * ctid));
-            o0 += sc * ov.x;
-            o1 += sc * ov.y;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              acc[k].x += sc * v[k].x;
+              acc[k].y += sc * v[k].y;
+              acc[k].z += sc * v[k].z;
+              acc[k].w += sc * v[k].w;
+            }
           }
-          const float inv = 1.f / Ls;
-          *reinterpret_cast<float2*>(p.o.out + ((size_t)b * H + h) * R + 2 * ctid) = make_float2(o0 * inv, o1 * inv);
-          if (p.o.lse && ctid == 0) p.o.lse[(size_t)b * H + h] = (M + log2f(Ls)) * 0.69314718055994531f;
+          float4* dst = reinterpret_cast<float4*>(p.o.out + ((size_t)b * H + h) * R + c0);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            dst[k] = make_float4(acc[k].x * inv, acc[k].y * inv, acc[k].z * inv, acc[k].w * inv);
         }
         if (ctid == 0) p.tickets[b] = 0;
       }
+      named_bar(1, 128);  // slots / flags are reused by the next segment
     }
-    named_bar(1, 128);  // combine buffers are reused by the next segment
   }
   if (!ok && ctid == 0) set_err(p.a.dev_err, MTLA_DEVERR_TIMEOUT);
 
@@ -567,7 +667,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
   named_bar(1, 128);
   if (sm.flags[1]) {
     for (int b = ctid; b < B; b += 128) {
-      const int64_t Lb = part.rows(b);
+      const int64_t Lb = rows_of(sm.meta, b);
       if (with_merge && (sm.meta[b] & kMetaMergeOk)) p.a.t_processed[b] = p.a.t_processed[b] + 1;
       if (p.a.cache_len) p.a.cache_len[b] = (int32_t)Lb;
       if (Lb == 0) {
@@ -577,8 +677,29 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
           for (int h = 0; h < H; ++h) p.o.lse[(size_t)b * H + h] = -INFINITY;
       }
     }
-    if (ctid == 0) *p.done = 0;
+    if (ctid == 0) {
+      *p.done = 0;
+      *p.gate_done = 0;
+    }
   }
+}
+
+int grid_size() {
+  int dev = 0, sms = 0, occ = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes()) !=
+      cudaSuccess)
+    return 0;
+  // two blocks of ~110 KB need the largest shared-memory configuration
+  if (cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+    return 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_tc_kernel, NT, smem_bytes()) != cudaSuccess)
+    return 0;
+  if (occ < 1) return 0;
+  const int g = sms * (occ < 2 ? occ : 2);
+  return g < MAXG ? g : MAXG;
 }
 
 }  // namespace dtc
@@ -594,10 +715,22 @@ cudaError_t launch_decode_tc(const dtc::Params& p, const CUtensorMap& map64, con
   if (dev >= 64 || !(done_mask & (1ull << dev))) {
     e = cudaFuncSetAttribute(dtc::decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(dtc::decode_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
     if (dev < 64) done_mask |= 1ull << dev;
   }
-  dtc::decode_tc_kernel<<<grid, dtc::NT, smem, st>>>(map64, map8, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(dtc::NT);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, dtc::decode_tc_kernel, map64, map8, p);
 }
 
 }  // namespace mtla

@@ -63,14 +63,13 @@ constexpr int UNIT = 64;                 // rows per full TMA box
 constexpr int SUB = 8;                   // rows per box of a ragged last unit
 constexpr int ROWB = D * 2;              // bytes per cache row (576)
 constexpr int STAGE = UNIT * ROWB;       // 36864 bytes per pipeline stage
-constexpr int NS = 4;                    // pipeline depth
+constexpr int NS = 2;                    // pipeline depth per block (two blocks per SM)
 constexpr int NCW = 4;                   // consumer warps
 constexpr int NT = 32 * (NCW + 1);       // + 1 producer warp
-constexpr int WC_ROWS = STAGE / (D * 4); // W_c rows per stage (32)
-constexpr int N_WC = R / WC_ROWS;        // W_c stages per merge (8)
-constexpr int MAXB = 2048;
+constexpr int MAXB = 1024;               // sequences per call
+constexpr int MAXG = 320;                // blocks per launch
 constexpr int OSTR = 260;                // head stride of the combine buffer (floats)
-constexpr int MERGE_COST = 128;          // partition weight of one merge, in rows
+constexpr int MERGE_COST = 32;           // partition weight of one merge, in rows
 
 struct Params {
   SeqArgs a;
@@ -81,13 +80,16 @@ struct Params {
   int merge_cost;
   float scale_log2;     // log2(e) / sqrt(d_h)
   int32_t* tickets;     // [B]
-  int32_t* done;        // [1]
+  int32_t* done;        // [1] blocks finished
+  int32_t* gate_done;   // [1] blocks whose share of the merge gates is written
+  float* gates;         // [B][D] Linear(c_t) of every new token
   float* ws_ml;         // [2 * grid][H][2]
   float* ws_o;          // [2 * grid][H][R]
 };
 
 size_t smem_bytes();
 size_t workspace_bytes(int B, int grid);
+int grid_size();  // blocks of the persistent grid on the current device (0 on error)
 }  // namespace dtc
 
 cudaError_t launch_merge_append(const SeqArgs& a, const MergeArgsDev& m, int B, int dtype, cudaStream_t st);

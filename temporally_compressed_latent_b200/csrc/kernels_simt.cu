@@ -219,8 +219,9 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(SeqArgs a, Me
 // Block = 256 threads as 16 x 16; a chunk of TC = 16*TPT tokens times 16*CPT
 // channels is computed per pass with W_c streamed through shared memory in
 // slabs of 32 input rows.  The scan then runs over the chunk's tokens in
-// order, carrying the running merge (rounded to the storage type after every
-// token, exactly as the decode's in-place update does).
+// order, carrying each group's running merge in fp32 and rounding only the
+// values it stores (a decode step, whose tail row lives in the cache, rounds
+// the stored row after every token instead).
 template <typename T, int TPT, int CPT>
 __global__ void __launch_bounds__(256) partial_merge_kernel(PrefillArgs p) {
   constexpr int TC = 16 * TPT;
@@ -309,7 +310,7 @@ __global__ void __launch_bounds__(256) partial_merge_kernel(PrefillArgs p) {
       for (int tt = 0; tt < tc; ++tt) {
         const int64_t n1 = n0 + tt + 1;
         const float e = e_sm[tt * D + ch];
-        v = opens_row(n1, s) ? round_to<T>(e) : round_to<T>(__fadd_rn(v, e));
+        v = opens_row(n1, s) ? e : __fadd_rn(v, e);
         st_elem(cp + (n1 - 1) * D + ch, v);
         if (cache && (n1 % s == 0 || n1 == Tn)) {
           const int64_t g = group_of(n1, s);

@@ -117,7 +117,7 @@ def test_decode_workspace_reused_many_calls():
     for _ in range(19):
         again, _ = run.step(case.q_abs, case.q_rope)
         np.testing.assert_array_equal(again, first)
-    ws = run.ws[:4 * (case.B + 1)].view(torch.int32)
+    ws = run.ws[:4 * (case.B + 2)].view(torch.int32)
     assert int(ws.abs().sum().item()) == 0
 
 

@@ -159,8 +159,9 @@ def test_prefill_equals_gpu_decode_steps():
     torch.cuda.synchronize()
     assert int(drun.err.item()) == 0
     assert drun.t.cpu().tolist() == [T] and drun.cache_len.cpu().tolist() == [T // 2]
-    # identical merge arithmetic: the decode cache equals the prefill cache bit for bit
-    np.testing.assert_array_equal(drun.cache.rows(0, T // 2), host(run.cache[0]))
+    # same gates; decode rounds the stored tail row after each token, the
+    # prefill only once per stored state: equal within the bf16 tolerance
+    assert_close(drun.cache.rows(0, T // 2), host(run.cache[0]), "bf16", "decode-built vs prefill cache")
     assert_close(host(run.out[0]), host(outs), "bf16", "parallel vs incremental (GPU)")
 
 
