@@ -60,13 +60,16 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D view of a bf16 cache: {32 elements, 9 chunks of 32, cache_rows rows}.
-bool encode_cache_map(CUtensorMap* map, void* cache, int64_t cache_rows, int64_t row_stride, uint32_t box_rows) {
+// 3-D view of a bf16 cache: {32 elements, cache_rows rows, 9 segments of 32};
+// with the segment as the outermost dimension a box lands in shared memory as
+// one [rows x 64 B] plane per segment.
+bool encode_cache_map(CUtensorMap* map, void* cache, int64_t cache_rows, int64_t row_stride, uint32_t box_rows,
+                      uint32_t box_planes) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
-  const cuuint64_t dims[3] = {32, (cuuint64_t)(dtc::D / 32), (cuuint64_t)cache_rows};
-  const cuuint64_t strides[2] = {64, (cuuint64_t)row_stride * 2};
-  const cuuint32_t box[3] = {32, (cuuint32_t)(dtc::D / 32), box_rows};
+  const cuuint64_t dims[3] = {32, (cuuint64_t)cache_rows, (cuuint64_t)(dtc::D / 32)};
+  const cuuint64_t strides[2] = {(cuuint64_t)row_stride * 2, 64};
+  const cuuint32_t box[3] = {32, box_rows, box_planes};
   const cuuint32_t estr[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, cache, dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -210,8 +213,8 @@ mtla_status mtla_decode_attn(const mtla_dims* dims, int32_t B, const void* q_abs
 
   thread_local CacheMaps maps;
   if (maps.ptr != cache || maps.rows != cache_rows || maps.stride != row_stride) {
-    if (!encode_cache_map(&maps.m64, cache, cache_rows, row_stride, dtc::UNIT) ||
-        !encode_cache_map(&maps.m8, cache, cache_rows, row_stride, dtc::SUB)) {
+    if (!encode_cache_map(&maps.m64, cache, cache_rows, row_stride, dtc::UNIT, dtc::D / 32) ||
+        !encode_cache_map(&maps.m8, cache, cache_rows, row_stride, dtc::SUB, 1)) {
       maps.ptr = nullptr;
       return MTLA_ERR_CUDA;
     }
@@ -229,10 +232,11 @@ mtla_status mtla_decode_attn(const mtla_dims* dims, int32_t B, const void* q_abs
   p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->d_h));
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   size_t off = 0;
-  p.tickets = reinterpret_cast<int32_t*>(ws + off);
-  p.done = p.tickets + B;
-  p.gate_done = p.tickets + B + 1;
-  off += ((size_t)B + 2) * 4;
+  p.seq_info = reinterpret_cast<int4*>(ws + off);
+  off += (size_t)B * 16;
+  off = (off + 255) & ~(size_t)255;
+  p.fs = reinterpret_cast<int32_t*>(ws + off);
+  off += (size_t)grid * 4;
   off = (off + 255) & ~(size_t)255;
   p.gates = reinterpret_cast<float*>(ws + off);
   off += (size_t)B * dtc::D * 4;

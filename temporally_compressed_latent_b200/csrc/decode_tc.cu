@@ -13,8 +13,12 @@
 //    into equal shares for a persistent grid of two blocks per SM (split-L,
 //    balanced to the row; a merge counts as MERGE_COST rows).
 //  * One producer warp streams 64-row tiles HBM -> shared memory with 3-D TMA
-//    boxes {32 elements, 9 chunks, 64 rows} and 64-byte swizzle (a ragged last
-//    tile uses 8-row boxes), NS stages deep, completion on mbarriers.
+//    boxes {32 elements, 64 rows, 9 planes}: the tensor map orders the row's
+//    nine 32-element segments as the outer dimension, so a tile lands as nine
+//    [64 rows x 64 B] planes with the 64-byte swizzle, whose XOR phase then
+//    depends on the row only (every ldmatrix address is a per-lane base plus a
+//    constant; this is also the canonical K-major SW64 operand layout).  A
+//    ragged last tile uses {32, 8, 1} boxes.  NS stages, mbarrier completion.
 //  * Four consumer warps each own 16 rows of a tile.  Scores S^T = rows . Q^T
 //    (M = rows, N = the 8 heads, K = 288) and values O^T += C_hat^T . P^T
 //    (M = 256 latent channels, N = 8 heads, K = rows) run on the tensor cores
@@ -22,22 +26,25 @@
 //    value-MMA operand with one in-register 8x8 transpose (movmatrix).  Each
 //    warp keeps its own online-softmax state, so no block barrier is needed
 //    per tile.
-//  * The merge of the new tokens is spread over the whole grid: the gate
-//    pre-activations Linear(c_t) = c_t W_c + b_c of all B tokens are cut into
-//    channel-major slices, one per block, computed while the block's first
-//    tiles are in flight (each block reads about one column of W_c).  The
-//    block owning a sequence's tail row waits (bounded) for all slices, then
-//    forms the gate, the gated entry and the updated row in fp32, writes it to
-//    the cache in bf16 and patches it into the tile before the tile is used.
+//  * The gate pre-activations Linear(c_t) = c_t W_c + b_c of all B new tokens
+//    come from a small kernel launched just before (32 channels x 8 tokens per
+//    block, W_c read as coalesced row segments).  It releases the decode grid
+//    at once (programmatic dependent launch), so the decode blocks run their
+//    set-up and stream their tiles meanwhile; only the block owning a
+//    sequence's tail row waits for it, then forms the gate, the gated entry
+//    and the updated row in fp32, writes the row to the cache in bf16 and
+//    patches it into the tile before the tile is used.
 //  * Launched with programmatic dependent launch: the next call's blocks are
 //    scheduled while this call's last blocks finish and wait for it before
 //    touching memory.
-//  * Partial results of sequences split between blocks go to the workspace;
-//    the last block to finish a sequence (atomic ticket) combines them.  No
-//    block ever waits for another.  The last block of the grid advances
-//    t_processed and resets the counters.  Every block's share and first
-//    sequence are tabulated once in shared memory, so the bookkeeping in the
-//    loops needs no integer division.
+//  * A block that holds only part of a sequence writes its partial (max, sum,
+//    unnormalised output) to the workspace and moves on: no fence, no atomic,
+//    no block ever waits for another at a segment boundary.  A second, small
+//    kernel chained with programmatic dependent launch (its blocks are resident
+//    and waiting before the first kernel ends) combines the split sequences,
+//    advances t_processed / cache_len and resets the gate counter.  Every
+//    block's share and first sequence are tabulated once in shared memory, so
+//    the bookkeeping in the loops needs no integer division.
 #include "kernels.cuh"
 
 namespace mtla {
@@ -53,13 +60,12 @@ static_assert(17 * H * 2 <= NCW * kCombHeads * OSTR, "combine scratch must fit t
 static_assert((size_t)H * QSTR * 4 <= (size_t)NCW * kCombHeads * OSTR * 4, "query buffer must fit the combine buffer");
 constexpr size_t kOffComb = rup((size_t)NS * STAGE);
 constexpr size_t kOffCombMl = kOffComb + rup((size_t)NCW * kCombHeads * OSTR * 4);
-constexpr size_t kOffPrefix = kOffCombMl + rup((size_t)NCW * H * 2 * 4);
+constexpr size_t kOffPrefix = kOffCombMl + rup((size_t)NCW * H * 2 * 4 + (size_t)(NCW + 2) * H * 4);
 constexpr size_t kOffMeta = kOffPrefix + rup((size_t)(MAXB + 1) * 8);
 constexpr size_t kOffScan = kOffMeta + rup((size_t)MAXB * 4);
 constexpr size_t kOffLo = kOffScan + rup(128 * 8);
 constexpr size_t kOffFs = kOffLo + rup((size_t)(MAXG + 1) * 8);
-constexpr size_t kOffSlots = kOffFs + rup((size_t)MAXG * 4);
-constexpr size_t kOffC = kOffSlots + rup((size_t)MAXG * 4);
+constexpr size_t kOffC = kOffFs + rup((size_t)MAXG * 4);
 constexpr size_t kOffTail = kOffC + rup((size_t)R * 4);
 constexpr size_t kOffBar = kOffTail + rup((size_t)D * 2);
 constexpr size_t kOffFlags = kOffBar + rup(2 * NS * 8);
@@ -70,7 +76,9 @@ size_t smem_bytes() { return kSmemUsed + 1024; }  // + slack to align the base t
 
 size_t workspace_bytes(int B, int grid) {
   size_t b = 0;
-  b += ((size_t)B + 2) * 4;
+  b += (size_t)B * 16;  // seq_info
+  b = (b + 255) & ~(size_t)255;
+  b += (size_t)grid * 4;  // fs
   b = (b + 255) & ~(size_t)255;
   b += (size_t)B * D * 4;
   b = (b + 255) & ~(size_t)255;
@@ -80,11 +88,11 @@ size_t workspace_bytes(int B, int grid) {
   return b;
 }
 
-// byte offset, inside a swizzled tile, of row `row`, 16-byte chunk `ch` (0..35):
-// TMA's 64-byte swizzle XORs chunk bits [4:5] with address bits [7:8]
+// byte offset, inside a tile, of row `row`, 16-byte chunk `ch` (0..35): plane
+// ch / 4 holds the row's 64-byte segment, TMA's 64-byte swizzle XORs chunk
+// bits [4:5] with address bits [7:8], i.e. with (row / 2) mod 4
 __host__ __device__ __forceinline__ uint32_t swz_off(int row, int ch) {
-  const uint32_t seg = (uint32_t)row * ROWB + (uint32_t)(ch >> 2) * 64u;
-  return seg + ((((uint32_t)ch & 3u) ^ ((seg >> 7) & 3u)) << 4);
+  return (uint32_t)(ch >> 2) * SEGB + (uint32_t)row * 64u + ((((uint32_t)ch & 3u) ^ (((uint32_t)row >> 1) & 3u)) << 4);
 }
 
 constexpr uint32_t kMetaMergeOk = 1u << 30;
@@ -98,7 +106,6 @@ struct Smem {
   int64_t* scan;
   int64_t* lo;        // [G + 1] first cost position of each block's share
   int32_t* fs;        // [G] first sequence with rows in each block's share
-  int32_t* slots;     // [G] workspace slots of the sequence being combined
   float* c_sm;
   __nv_bfloat16* tail_sm;
   uint64_t* full_bar;
@@ -117,7 +124,6 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   s.scan = reinterpret_cast<int64_t*>(p + kOffScan);
   s.lo = reinterpret_cast<int64_t*>(p + kOffLo);
   s.fs = reinterpret_cast<int32_t*>(p + kOffFs);
-  s.slots = reinterpret_cast<int32_t*>(p + kOffSlots);
   s.c_sm = reinterpret_cast<float*>(p + kOffC);
   s.tail_sm = reinterpret_cast<__nv_bfloat16*>(p + kOffTail);
   s.full_bar = reinterpret_cast<uint64_t*>(p + kOffBar);
@@ -136,14 +142,7 @@ __device__ __forceinline__ int upper_bound_i64(const int64_t* a, int n, int64_t 
   return lo;
 }
 
-constexpr uint32_t kSpinLimit = 1u << 22;  // x 64 ns sleeps: gives up after ~0.3 s
-
-__device__ __forceinline__ int ld_acquire_gpu(const int32_t* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
+constexpr int PRO_T = 32 * (NCW + 1);  // threads of the consumer and producer warps
 __device__ __forceinline__ int64_t rows_of(const uint32_t* meta, int b) {
   return (int64_t)(meta[b] & (kMetaMergeOk - 1));
 }
@@ -158,8 +157,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
   const bool with_merge = p.with_merge != 0;
   const int64_t mcost = with_merge ? p.merge_cost : 0;
 
-  // let the next launch on the stream be scheduled as soon as blocks retire;
-  // then wait for the previous launch before reading anything it may write
+  // let the next launch on the stream be scheduled as soon as blocks retire.
+  // Without a merge, wait for the previous launch before reading anything it
+  // may write; with a merge the gate kernel just before has already waited
+  // for it, and only the gates themselves (read at a tail row) need the gate
+  // kernel to be complete.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (tid == 0) {
     for (int i = 0; i < NS; ++i) {
@@ -168,11 +170,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
     }
     fence_mbar_init();
   }
-  if (warp == NCW && lane == 0) {
+  if (warp == PRODUCER_WARP && lane == 0) {
     prefetch_tmap(&map64);
     prefetch_tmap(&map8);
   }
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (!with_merge) asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // ---- 1. rows per sequence and the cost prefix (identical in every block)
   const int per = (B + 127) / 128;
@@ -208,7 +210,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
     }
     sm.scan[tid] = sum;
   }
-  __syncthreads();
+  named_bar(2, PRO_T);
   if (warp == 0) {
     // exclusive scan of the 128 partial sums (4 per lane)
     int64_t v[4], run = 0;
@@ -225,7 +227,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
     for (int i = 0; i < 4; ++i) { const int64_t t = v[i]; sm.scan[lane * 4 + i] = ex; ex += t; }
     if (lane == 31) sm.prefix[B] = ex;  // total cost
   }
-  __syncthreads();
+  named_bar(2, PRO_T);
   if (tid < 128) {
     int64_t run = sm.scan[tid];
     for (int b = tid * per; b < B && b < (tid + 1) * per; ++b) {
@@ -235,24 +237,37 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
   }
   const int64_t C = sm.prefix[B];
   // share starts: block c owns cost positions [lo[c], lo[c+1])
-  for (int c = tid; c <= G; c += NT) sm.lo[c] = C > 0 ? (int64_t)c * C / G : 0;
-  __syncthreads();
+  for (int c = tid; c <= G; c += PRO_T) sm.lo[c] = C > 0 ? (int64_t)c * C / G : 0;
+  named_bar(2, PRO_T);
   // first sequence with rows in each share (B if none)
-  for (int c = tid; c < G; c += NT) {
+  for (int c = tid; c < G; c += PRO_T) {
     const int64_t x = sm.lo[c];
     int b = upper_bound_i64(sm.prefix, B + 1, x) - 1;
     if (b < 0) b = 0;
     if (b < B && x - sm.prefix[b] >= rows_of(sm.meta, b)) ++b;
     sm.fs[c] = (x < sm.lo[c + 1]) ? b : B;
   }
-  __syncthreads();
+  named_bar(2, PRO_T);
 
+  if (cta == 0) {
+    // the partition, for the combine kernel (read after this grid completes)
+    for (int c = tid; c < G; c += PRO_T) p.fs[c] = sm.fs[c];
+    for (int b = tid; b < B; b += PRO_T) {
+      const int64_t Lb = rows_of(sm.meta, b);
+      int cf = -1, cl = -1;
+      if (Lb > 0) {
+        cf = upper_bound_i64(sm.lo, G + 1, sm.prefix[b]) - 1;
+        cl = upper_bound_i64(sm.lo, G + 1, sm.prefix[b] + Lb - 1) - 1;
+      }
+      p.seq_info[b] = make_int4((int)Lb, (sm.meta[b] & kMetaMergeOk) ? 1 : 0, cf, cl);
+    }
+  }
   const int64_t my_lo = sm.lo[cta], my_hi = sm.lo[cta + 1];
   const int b_first = sm.fs[cta];
   const __nv_bfloat16* cache = reinterpret_cast<const __nv_bfloat16*>(p.a.cache);
 
   // ======================= producer warp =======================
-  if (warp == NCW) {
+  if (warp == PRODUCER_WARP) {
     if (lane == 0 && my_lo < my_hi) {
       uint32_t job = 0;
       bool ok = true;
@@ -270,12 +285,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
           uint8_t* dst = sm.stages + st * STAGE;
           if (nrows == UNIT) {
             mbar_arrive_expect_tx(&sm.full_bar[st], STAGE);
-            tma_load_3d(dst, &map64, 0, 0, (int32_t)(row0 + u), &sm.full_bar[st]);
+            tma_load_3d(dst, &map64, 0, (int32_t)(row0 + u), 0, &sm.full_bar[st]);
           } else {
+            // 8-row boxes of one plane each, into the same plane layout
             const int nsub = (int)((nrows + SUB - 1) / SUB);
             mbar_arrive_expect_tx(&sm.full_bar[st], (uint32_t)(nsub * SUB * ROWB));
             for (int i = 0; i < nsub; ++i)
-              tma_load_3d(dst + i * SUB * ROWB, &map8, 0, 0, (int32_t)(row0 + u + i * SUB), &sm.full_bar[st]);
+              for (int c = 0; c < D / 32; ++c)
+                tma_load_3d(dst + c * SEGB + i * SUB * 64, &map8, 0, (int32_t)(row0 + u + i * SUB), c,
+                            &sm.full_bar[st]);
           }
           ++job;
         }
@@ -298,56 +316,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
   const int ach = lane >> 4;
   const int vrow = w_lo + (lane & 7) + (lane >> 4) * 8;
   const int vch = (lane >> 3) & 1;
+  // ldmatrix offsets inside a tile: chunk 2 kk + ach of row arow sits in plane
+  // kk / 2 at swz_off(arow, ach) (kk even) or swz_off(arow, 2 + ach) (kk odd)
+  const uint32_t offA0 = swz_off(arow, ach), offA1 = swz_off(arow, 2 + ach);
+  const uint32_t offV0 = swz_off(vrow, vch), offV1 = swz_off(vrow, 2 + vch);
   uint32_t job = 0;
   bool ok = true;
-
-  // ---- merge gates: this block's slice of Linear(c_t) = c_t W_c + b_c,
-  // channel-major (index k * B + b), while its first tiles are in flight
-  if (with_merge) {
-    const int N = B * D;
-    const int i_lo = (int)((int64_t)cta * N / G), i_hi = (int)((int64_t)(cta + 1) * N / G);
-    float* wcol = sm.c_sm;  // one column of W_c
-    const uint4* cnew = reinterpret_cast<const uint4*>(p.m.c_new);
-    for (int k = i_lo / B; i_lo < i_hi && k <= (i_hi - 1) / B; ++k) {
-      const int b_lo = i_lo - k * B > 0 ? i_lo - k * B : 0;
-      const int b_hi = i_hi - k * B < B ? i_hi - k * B : B;
-      for (int i = ctid; i < R; i += 128) wcol[i] = __ldg(p.m.W_c + (size_t)i * D + k);
-      named_bar(1, 128);
-      float wv[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) wv[e] = wcol[8 * lane + e];
-      const float bias = __ldg(p.m.b_c + k);
-      // warp cw takes sequences b_lo + cw, + NCW, ...; four at a time so that
-      // their loads overlap; lane covers inputs 8 lane .. 8 lane + 7
-      for (int b0 = b_lo + cw; b0 < b_hi; b0 += 4 * NCW) {
-        uint4 cv[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int bb = b0 + u * NCW;
-          cv[u] = bb < b_hi ? __ldg(cnew + (size_t)bb * (R / 8) + lane) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&cv[u]);
-          float acc = 0.f;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(h2[e]);
-            acc = fmaf(f.x, wv[2 * e], acc);
-            acc = fmaf(f.y, wv[2 * e + 1], acc);
-          }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-          const int bb = b0 + u * NCW;
-          if (lane == 0 && bb < b_hi) p.gates[(size_t)bb * D + k] = acc + bias;
-        }
-      }
-      named_bar(1, 128);  // the column buffer is reused for the next channel
-    }
-    __threadfence();
-    named_bar(1, 128);
-    if (ctid == 0) atomicAdd(p.gate_done, 1);
-  }
 
   for (int b = b_first; b < B && sm.prefix[b] < my_hi; ++b) {
     const int64_t Lb = rows_of(sm.meta, b);
@@ -385,18 +359,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
     for (int64_t u = r_lo; u < r_hi; u += UNIT) {
       const bool is_tail = merge_here && u + UNIT >= r_hi;
       if (is_tail) {
-        // every block's slice of the gates must be written (bounded wait)
-        if (ctid == 0) {
-          uint32_t it = 0;
-          while (ld_acquire_gpu(p.gate_done) < G) {
-            if (++it > kSpinLimit) {
-              set_err(p.a.dev_err, MTLA_DEVERR_TIMEOUT);
-              break;
-            }
-            __nanosleep(64);
-          }
-        }
-        named_bar(1, 128);
+        // the gate kernel must be complete (hardware-tracked, no polling)
+        asm volatile("griddepcontrol.wait;" ::: "memory");
         // gate, gated entry and the updated tail row (fp32 math, bf16 storage)
         const int64_t t = (int64_t)p.a.t_processed[b] + 1;
         const int64_t j = group_of(t, s);
@@ -461,7 +425,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
 #pragma unroll
         for (int kk = 0; kk < 18; ++kk) {
           uint32_t a0, a1, a2, a3, b0, b1;
-          ldsm_x4(tile + swz_off(arow, 2 * kk + ach), a0, a1, a2, a3);
+          ldsm_x4(tile + (kk >> 1) * SEGB + ((kk & 1) ? offA1 : offA0), a0, a1, a2, a3);
           asm volatile("ld.shared.u32 %0, [%1];" : "=r"(b0) : "r"(qrow + kk * 32u));
           asm volatile("ld.shared.u32 %0, [%1];" : "=r"(b1) : "r"(qrow + kk * 32u + 16u));
           mma_bf16(sacc[kk & 1], a0, a1, a2, a3, b0, b1);
@@ -485,12 +449,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
         lB = lB * aB + pB0 + pB1;
         mA = nA;
         mB = nB;
+        if (__any_sync(0xffffffffu, aA != 1.f || aB != 1.f)) {  // some head's max moved
 #pragma unroll
-        for (int mb = 0; mb < 16; ++mb) {
-          O[mb][0] *= aA;
-          O[mb][1] *= aB;
-          O[mb][2] *= aA;
-          O[mb][3] *= aB;
+          for (int mb = 0; mb < 16; ++mb) {
+            O[mb][0] *= aA;
+            O[mb][1] *= aB;
+            O[mb][2] *= aA;
+            O[mb][3] *= aB;
+          }
         }
         // P^T fragments (k = rows, n = heads) by an 8x8 transpose of the score fragment
         const uint32_t pb0 = movmatrix_t(pack_bf16x2(pA0, pB0));
@@ -499,7 +465,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
 #pragma unroll
         for (int mb = 0; mb < 16; ++mb) {
           uint32_t a0, a1, a2, a3;
-          ldsm_x4_t(tile + swz_off(vrow, 2 * mb + vch), a0, a1, a2, a3);
+          ldsm_x4_t(tile + (mb >> 1) * SEGB + ((mb & 1) ? offV1 : offV0), a0, a1, a2, a3);
           mma_bf16(O[mb], a0, a1, a2, a3, pb0, pb1);
         }
       }
@@ -522,6 +488,23 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
       sm.comb_ml[(cw * H + 2 * q + 1) * 2 + 1] = lB;
     }
     const int nslot = full ? -1 : 2 * cta + (b == b_first ? 0 : 1);
+    named_bar(1, 128);  // comb_ml complete
+    float* wsc = sm.comb_ml + NCW * H * 2;  // [NCW][H] weights exp2(m_w - M), then [H] M and [H] 1/L
+    if (ctid < H) {
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < NCW; ++w) M = fmaxf(M, sm.comb_ml[(w * H + ctid) * 2]);
+      float Ls = 0.f;
+#pragma unroll
+      for (int w = 0; w < NCW; ++w) {
+        const float mw = sm.comb_ml[(w * H + ctid) * 2];
+        const float sc = mw == -INFINITY ? 0.f : exp2f(mw - M);
+        wsc[w * H + ctid] = sc;
+        Ls += sc * sm.comb_ml[(w * H + ctid) * 2 + 1];
+      }
+      wsc[NCW * H + ctid] = M;
+      wsc[NCW * H + H + ctid] = Ls;
+    }
 #pragma unroll 1
     for (int pass = 0; pass < 2; ++pass) {
       // heads 4 pass .. 4 pass + 3 belong to the lanes with q >> 1 == pass
@@ -538,18 +521,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
         }
       }
       named_bar(1, 128);
-#pragma unroll 1
+#pragma unroll
       for (int hl = 0; hl < kCombHeads; ++hl) {
         const int h = kCombHeads * pass + hl;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < NCW; ++w) M = fmaxf(M, sm.comb_ml[(w * H + h) * 2]);
-        float Ls = 0.f, o0 = 0.f, o1 = 0.f;
+        const float M = wsc[NCW * H + h], Ls = wsc[NCW * H + H + h];
+        float o0 = 0.f, o1 = 0.f;
 #pragma unroll
         for (int w = 0; w < NCW; ++w) {
-          const float mw = sm.comb_ml[(w * H + h) * 2];
-          const float sc = mw == -INFINITY ? 0.f : exp2f(mw - M);
-          Ls += sc * sm.comb_ml[(w * H + h) * 2 + 1];
+          const float sc = wsc[w * H + h];
           const float2 ov = *reinterpret_cast<const float2*>(sm.comb_o + (w * kCombHeads + hl) * OSTR + 2 * ctid);
           o0 += sc * ov.x;
           o1 += sc * ov.y;
@@ -569,119 +548,153 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
       }
       named_bar(1, 128);  // the buffer is rewritten by the next pass / segment
     }
-    if (!full) {
-      __threadfence();
-      named_bar(1, 128);
-      if (ctid == 0) {
-        // the blocks holding part of sequence b and their workspace slots
-        const int64_t first_pos = sm.prefix[b], last_pos = sm.prefix[b] + Lb - 1;
-        const int c_first = upper_bound_i64(sm.lo, G + 1, first_pos) - 1;
-        const int c_last = upper_bound_i64(sm.lo, G + 1, last_pos) - 1;
-        int nparts = 0;
-        for (int c = c_first; c <= c_last; ++c)
-          if (sm.lo[c] < sm.lo[c + 1]) sm.slots[nparts++] = 2 * c + (sm.fs[c] == b ? 0 : 1);
-        const int old = atomicAdd(&p.tickets[b], 1);
-        sm.flags[0] = (old == nparts - 1) ? nparts : 0;
-        __threadfence();
-      }
-      named_bar(1, 128);
-      const int nparts = sm.flags[0];
-      if (nparts) {
-        // last block of this sequence: combine every block's partial.  All
-        // loads of a phase are independent, so each phase costs about one L2
-        // round trip whatever the number of parts.
-        // phase 1: per head, running (max, sum) over the parts, 16 groups of 8 threads
-        float* red = sm.comb_o;  // [16][H][2], free at this point
-        {
-          const int h = ctid & 7, grp = ctid >> 3;
-          float M = -INFINITY, Ls = 0.f;
-          for (int i = grp; i < nparts; i += 16) {
-            const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.ws_ml) + (size_t)sm.slots[i] * H + h);
-            if (ml.x == -INFINITY) continue;
-            const float nM = fmaxf(M, ml.x);
-            Ls = Ls * exp2f(M - nM) + ml.y * exp2f(ml.x - nM);
-            M = nM;
-          }
-          red[(grp * H + h) * 2 + 0] = M;
-          red[(grp * H + h) * 2 + 1] = Ls;
-        }
-        named_bar(1, 128);
-        if (ctid < H) {
-          float M = -INFINITY, Ls = 0.f;
-          for (int grp = 0; grp < 16; ++grp) {
-            const float m = red[(grp * H + ctid) * 2], l = red[(grp * H + ctid) * 2 + 1];
-            if (m == -INFINITY) continue;
-            const float nM = fmaxf(M, m);
-            Ls = Ls * exp2f(M - nM) + l * exp2f(m - nM);
-            M = nM;
-          }
-          red[(16 * H + ctid) * 2 + 0] = M;
-          red[(16 * H + ctid) * 2 + 1] = Ls;
-          if (p.o.lse) p.o.lse[(size_t)b * H + ctid] = (M + log2f(Ls)) * 0.69314718055994531f;
-        }
-        named_bar(1, 128);
-        // phase 2: thread -> head ctid >> 4, 16 channels; parts weighted by exp2(m_i - M) / L
-        {
-          const int h = ctid >> 4, c0 = (ctid & 15) * 16;
-          const float M = red[(16 * H + h) * 2], inv = 1.f / red[(16 * H + h) * 2 + 1];
-          float4 acc[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 2
-          for (int i = 0; i < nparts; ++i) {
-            const int slot = sm.slots[i];
-            const float mc = __ldcg(p.ws_ml + ((size_t)slot * H + h) * 2);
-            const float4* src = reinterpret_cast<const float4*>(p.ws_o + ((size_t)slot * H + h) * R + c0);
-            float4 v[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) v[k] = __ldcg(src + k);
-            const float sc = mc == -INFINITY ? 0.f : exp2f(mc - M);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              acc[k].x += sc * v[k].x;
-              acc[k].y += sc * v[k].y;
-              acc[k].z += sc * v[k].z;
-              acc[k].w += sc * v[k].w;
-            }
-          }
-          float4* dst = reinterpret_cast<float4*>(p.o.out + ((size_t)b * H + h) * R + c0);
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            dst[k] = make_float4(acc[k].x * inv, acc[k].y * inv, acc[k].z * inv, acc[k].w * inv);
-        }
-        if (ctid == 0) p.tickets[b] = 0;
-      }
-      named_bar(1, 128);  // slots / flags are reused by the next segment
-    }
   }
   if (!ok && ctid == 0) set_err(p.a.dev_err, MTLA_DEVERR_TIMEOUT);
 
-  // ---- grid epilogue: the last block advances the per-sequence state
-  named_bar(1, 128);
-  if (ctid == 0) {
-    __threadfence();
-    const int old = atomicAdd(p.done, 1);
-    sm.flags[1] = (old == G - 1) ? 1 : 0;
-    __threadfence();
+}
+
+// Combine of the sequences split between blocks; one block of 128 threads per
+// sequence.  Launched right after the decode kernel with programmatic
+// dependent launch: its blocks are scheduled early and wait for the decode
+// grid to complete before reading anything.
+__global__ void __launch_bounds__(256) decode_combine_kernel(const Params p) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  __shared__ int slots[MAXG];
+  __shared__ float scale[MAXG * H];  // exp2(m_i - M_h) / L_h for every part and head
+  __shared__ float red[32 * H * 2];
+  __shared__ int wsum[8];
+  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int4 info = p.seq_info[b];  // rows, merge ok, first block, last block
+  if (tid == 0) {
+    if (p.with_merge && info.y) p.a.t_processed[b] = p.a.t_processed[b] + 1;
+    if (p.a.cache_len) p.a.cache_len[b] = info.x;
   }
-  named_bar(1, 128);
-  if (sm.flags[1]) {
-    for (int b = ctid; b < B; b += 128) {
-      const int64_t Lb = rows_of(sm.meta, b);
-      if (with_merge && (sm.meta[b] & kMetaMergeOk)) p.a.t_processed[b] = p.a.t_processed[b] + 1;
-      if (p.a.cache_len) p.a.cache_len[b] = (int32_t)Lb;
-      if (Lb == 0) {
-        set_err(p.a.dev_err, MTLA_DEVERR_EMPTY);
-        for (int i = 0; i < H * R; ++i) p.o.out[(size_t)b * H * R + i] = 0.f;
-        if (p.o.lse)
-          for (int h = 0; h < H; ++h) p.o.lse[(size_t)b * H + h] = -INFINITY;
+  if (info.x == 0) {
+    if (tid == 0) set_err(p.a.dev_err, MTLA_DEVERR_EMPTY);
+    for (int i = tid; i < H * R; i += 256) p.o.out[(size_t)b * H * R + i] = 0.f;
+    if (p.o.lse && tid < H) p.o.lse[(size_t)b * H + tid] = -INFINITY;
+    return;
+  }
+  // the workspace slots of the blocks that hold part of sequence b, in block
+  // order: every candidate block is looked up at once and compacted by ballots
+  const int ncand = info.w - info.z + 1;
+  if (ncand <= 1) return;  // one block held the whole sequence and wrote it
+  int nparts = 0;
+  for (int base = 0; base < ncand; base += 256) {
+    const int t = base + tid;
+    int slot = -1;
+    if (t < ncand) {
+      const int c = info.z + t;
+      const int f = p.fs[c];
+      if (f != p.B) slot = 2 * c + (f == b ? 0 : 1);
+    }
+    const unsigned bal = __ballot_sync(0xffffffffu, slot >= 0);
+    if (lane == 0) wsum[wid] = __popc(bal);
+    __syncthreads();
+    int off = nparts;
+    for (int w = 0; w < wid; ++w) off += wsum[w];
+    if (slot >= 0) slots[off + __popc(bal & ((1u << lane) - 1u))] = slot;
+    for (int w = 0; w < 8; ++w) nparts += wsum[w];
+    __syncthreads();
+  }
+  if (nparts <= 1) return;
+  // phase 1: per head, running (max, sum) over the parts: 32 groups x 8 heads
+  {
+    const int h = tid & 7, grp = tid >> 3;
+    float M = -INFINITY, Ls = 0.f;
+    for (int i = grp; i < nparts; i += 32) {
+      const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.ws_ml) + (size_t)slots[i] * H + h);
+      if (ml.x == -INFINITY) continue;
+      const float nM = fmaxf(M, ml.x);
+      Ls = Ls * exp2f(M - nM) + ml.y * exp2f(ml.x - nM);
+      M = nM;
+    }
+    red[(grp * H + h) * 2 + 0] = M;
+    red[(grp * H + h) * 2 + 1] = Ls;
+  }
+  __syncthreads();
+  if (tid < H) {
+    float M = -INFINITY, Ls = 0.f;
+    for (int grp = 0; grp < 32; ++grp) {
+      const float m = red[(grp * H + tid) * 2], l = red[(grp * H + tid) * 2 + 1];
+      if (m == -INFINITY) continue;
+      const float nM = fmaxf(M, m);
+      Ls = Ls * exp2f(M - nM) + l * exp2f(m - nM);
+      M = nM;
+    }
+    red[tid * 2 + 0] = M;  // group 0's entries are no longer needed
+    red[tid * 2 + 1] = Ls;
+    if (p.o.lse) p.o.lse[(size_t)b * H + tid] = (M + log2f(Ls)) * 0.69314718055994531f;
+  }
+  __syncthreads();
+  for (int i = tid; i < nparts * H; i += 256) {
+    const int part = i / H, h = i % H;
+    const float mc = __ldcg(p.ws_ml + ((size_t)slots[part] * H + h) * 2);
+    scale[i] = mc == -INFINITY ? 0.f : exp2f(mc - red[h * 2]) / red[h * 2 + 1];
+  }
+  __syncthreads();
+  // phase 2: thread -> head tid >> 5, 8 channels; eight parts' loads in flight at a time
+  const int h = tid >> 5, c0 = (tid & 31) * 8;
+  float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+  for (int i0 = 0; i0 < nparts; i0 += 8) {
+    float4 v0[8], v1[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (i0 + u < nparts) {
+        const float4* src = reinterpret_cast<const float4*>(p.ws_o + ((size_t)slots[i0 + u] * H + h) * R + c0);
+        v0[u] = __ldcg(src);
+        v1[u] = __ldcg(src + 1);
       }
     }
-    if (ctid == 0) {
-      *p.done = 0;
-      *p.gate_done = 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (i0 + u < nparts) {
+        const float sc = scale[(i0 + u) * H + h];
+        acc0.x += sc * v0[u].x; acc0.y += sc * v0[u].y; acc0.z += sc * v0[u].z; acc0.w += sc * v0[u].w;
+        acc1.x += sc * v1[u].x; acc1.y += sc * v1[u].y; acc1.z += sc * v1[u].z; acc1.w += sc * v1[u].w;
+      }
     }
   }
+  float4* dst = reinterpret_cast<float4*>(p.o.out + ((size_t)b * H + h) * R + c0);
+  dst[0] = acc0;
+  dst[1] = acc1;
+}
+
+// Gate pre-activations g[b][k] = sum_i c_b[i] W_c[i][k] + b_c[k] of the new
+// tokens (Linear(c_t) of the merge).  Block = 32 channels x 8 tokens; warp w
+// takes input rows 32w .. 32w+31 (one coalesced 128-byte segment of W_c per
+// row, all in flight at once), lanes are channels; the eight warps' partial
+// sums are added in a fixed order, so the result is deterministic.
+__global__ void __launch_bounds__(256) decode_gate_kernel(const Params p) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __shared__ float part[8][8][32];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kt = blockIdx.x % (D / 32), bt = blockIdx.x / (D / 32);
+  const int k = kt * 32 + lane, b0 = bt * 8, i0 = w * 32;
+  float wv[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) wv[i] = __ldg(p.m.W_c + (size_t)(i0 + i) * D + k);
+  const __nv_bfloat16* cn = reinterpret_cast<const __nv_bfloat16*>(p.m.c_new);
+  float cv[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) cv[u] = b0 + u < p.B ? __bfloat162float(cn[(size_t)(b0 + u) * R + i0 + lane]) : 0.f;
+  float acc[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) acc[u] = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc[u] = fmaf(__shfl_sync(0xffffffffu, cv[u], i), wv[i], acc[u]);
+#pragma unroll
+  for (int u = 0; u < 8; ++u) part[w][u][lane] = acc[u];
+  __syncthreads();
+  const int u = w;  // thread -> token b0 + u, channel k
+  float g = 0.f;
+#pragma unroll
+  for (int ww = 0; ww < 8; ++ww) g += part[ww][u][lane];
+  if (b0 + u < p.B) p.gates[(size_t)(b0 + u) * D + k] = g + __ldg(p.m.b_c + k);
 }
 
 int grid_size() {
@@ -720,17 +733,36 @@ cudaError_t launch_decode_tc(const dtc::Params& p, const CUtensorMap& map64, con
     if (e != cudaSuccess) return e;
     if (dev < 64) done_mask |= 1ull << dev;
   }
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
   cfg.blockDim = dim3(dtc::NT);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, dtc::decode_tc_kernel, map64, map8, p);
+  if (p.with_merge) {
+    cudaLaunchConfig_t cfg0 = {};
+    cfg0.gridDim = dim3((unsigned)((dtc::D / 32) * ((p.B + 7) / 8)));
+    cfg0.blockDim = dim3(256);
+    cfg0.stream = st;
+    cfg0.attrs = attr;
+    cfg0.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg0, dtc::decode_gate_kernel, p);
+    if (e != cudaSuccess) return e;
+  }
+  e = cudaLaunchKernelEx(&cfg, dtc::decode_tc_kernel, map64, map8, p);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg2 = {};
+  cfg2.gridDim = dim3((unsigned)p.B);
+  cfg2.blockDim = dim3(256);
+  cfg2.dynamicSmemBytes = 0;
+  cfg2.stream = st;
+  cfg2.attrs = attr;
+  cfg2.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg2, dtc::decode_combine_kernel, p);
 }
 
 }  // namespace mtla

@@ -65,7 +65,9 @@ constexpr int ROWB = D * 2;              // bytes per cache row (576)
 constexpr int STAGE = UNIT * ROWB;       // 36864 bytes per pipeline stage
 constexpr int NS = 2;                    // pipeline depth per block (two blocks per SM)
 constexpr int NCW = 4;                   // consumer warps
-constexpr int NT = 32 * (NCW + 1);       // + 1 producer warp
+constexpr int PRODUCER_WARP = NCW;       // streams the tiles
+constexpr int NT = 32 * (NCW + 1);
+constexpr int SEGB = UNIT * 64;          // bytes of one 32-element plane of a tile (4096)
 constexpr int MAXB = 1024;               // sequences per call
 constexpr int MAXG = 320;                // blocks per launch
 constexpr int OSTR = 260;                // head stride of the combine buffer (floats)
@@ -79,10 +81,9 @@ struct Params {
   int B;
   int merge_cost;
   float scale_log2;     // log2(e) / sqrt(d_h)
-  int32_t* tickets;     // [B]
-  int32_t* done;        // [1] blocks finished
-  int32_t* gate_done;   // [1] blocks whose share of the merge gates is written
-  float* gates;         // [B][D] Linear(c_t) of every new token
+  int4* seq_info;       // [B] {rows, merge ok, first block, last block} for the combine
+  int32_t* fs;          // [grid] first sequence with rows in each block's share (B: none)
+  float* gates;         // [B][D] Linear(c_t) of every new token (gate kernel)
   float* ws_ml;         // [2 * grid][H][2]
   float* ws_o;          // [2 * grid][H][R]
 };
