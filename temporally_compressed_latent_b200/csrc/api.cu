@@ -76,6 +76,22 @@ bool encode_cache_map(CUtensorMap* map, void* cache, int64_t cache_rows, int64_t
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Generic tiled map of a bf16 tensor with the 64-byte swizzle (dims innermost first).
+bool encode_bf16_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+                     const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool tc_prefill_dims(const mtla_dims* d, int B, int T) {
+  return d->dtype == MTLA_BF16 && d->H == 8 && d->r == 256 && d->d_R == 32 && T % 16 == 0 && T >= 16 &&
+         (int64_t)B * T * 8 < (int64_t(1) << 31);
+}
+
 struct CacheMaps {
   void* ptr = nullptr;
   int64_t rows = -1, stride = -1;
@@ -289,7 +305,48 @@ mtla_status mtla_prefill_masked_attn(const mtla_dims* dims, int32_t B, int32_t T
   cudaError_t e = launch_partial_merge(p, B, dims->dtype, cs);
   if (e != cudaSuccess) return MTLA_ERR_CUDA;
   if (!out) return MTLA_OK;
-  return from_cuda(launch_prefill_simt(p, B, dims->dtype, cs));
+  if (!tc_prefill_dims(dims, B, T)) return from_cuda(launch_prefill_simt(p, B, dims->dtype, cs));
+
+  // tensor-core path: queries as 9 planes of 32, own rows, and the completed
+  // groups C_hat'_{g s} read through a map whose row stride is s rows
+  const int s = dims->s;
+  const cuuint64_t rows_q = (cuuint64_t)B * T * 8, rows_c = (cuuint64_t)B * T;
+  CUtensorMap qmap, rmap, smap, kmap;
+  {
+    const cuuint64_t dims3[3] = {32, rows_q, 8}, str[2] = {512, 64};
+    const cuuint32_t box[3] = {32, 128, 8};
+    if (!encode_bf16_map(&qmap, q_abs, 3, dims3, str, box)) return MTLA_ERR_CUDA;
+  }
+  {
+    const cuuint64_t dims2[2] = {32, rows_q}, str[1] = {64};
+    const cuuint32_t box[2] = {32, 128};
+    if (!encode_bf16_map(&rmap, q_rope, 2, dims2, str, box)) return MTLA_ERR_CUDA;
+  }
+  {
+    const cuuint64_t dims3[3] = {32, rows_c, 9}, str[2] = {576, 64};
+    const cuuint32_t box[3] = {32, 16, 9};
+    if (!encode_bf16_map(&smap, c_partial, 3, dims3, str, box)) return MTLA_ERR_CUDA;
+  }
+  {
+    const int64_t groups = T / s;
+    const cuuint64_t dims4[4] = {32, (cuuint64_t)(groups > 0 ? groups : 1), 9, (cuuint64_t)B};
+    const cuuint64_t str[3] = {(cuuint64_t)s * 576, 64, (cuuint64_t)T * 576};
+    const cuuint32_t box[4] = {32, 64, 9, 1};
+    const __nv_bfloat16* base = reinterpret_cast<const __nv_bfloat16*>(c_partial) + (s - 1) * 288;
+    if (!encode_bf16_map(&kmap, base, 4, dims4, str, box)) return MTLA_ERR_CUDA;
+  }
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return MTLA_ERR_CUDA;
+  PrefillTcLaunch a;
+  a.B = B;
+  a.T = T;
+  a.s = s;
+  a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->d_h));
+  a.out = out;
+  a.dev_err = dev_err;
+  const int tiles = B * (T / 16);
+  return from_cuda(launch_prefill_tc_args(a, qmap, rmap, smap, kmap, tiles < sms ? tiles : sms, cs));
 }
 
 }  // extern "C"

@@ -99,6 +99,20 @@ cudaError_t launch_decode_simt(const SeqArgs& a, const MergeArgsDev& m, bool wit
 cudaError_t launch_decode_tc(const dtc::Params& p, const CUtensorMap& map64, const CUtensorMap& map8, int grid,
                              cudaStream_t st);
 cudaError_t launch_partial_merge(const PrefillArgs& p, int B, int dtype, cudaStream_t st);
+
+// Masked prefill on tcgen05 (bf16, H = 8, r = 256, d_R = 32, T % 16 == 0).
+namespace ptc {
+struct Params;
+size_t smem_bytes();
+}
+struct PrefillTcLaunch {
+  int B, T, s;
+  float scale_log2;
+  void* out;
+  int32_t* dev_err;
+};
+cudaError_t launch_prefill_tc_args(const PrefillTcLaunch& a, const CUtensorMap& qmap, const CUtensorMap& rmap,
+                                   const CUtensorMap& smap, const CUtensorMap& kmap, int grid, cudaStream_t st);
 cudaError_t launch_prefill_simt(const PrefillArgs& p, int B, int dtype, cudaStream_t st);
 
 }  // namespace mtla

@@ -1,0 +1,442 @@
+// Stride-aware masked parallel forward on the 5th-generation tensor cores
+// (tcgen05 + TMEM), bf16 with H = 8, r = 256, d_R = 32.
+//
+// What it computes (MTLA paper notes, "Key designs: stride-aware causal mask"
+// and "decoupled RoPE with temporal compression"; Figure 2(c) of the abstract
+// page): query m (1-based) of sequence b, head h, attends the columns n of the
+// running merge C_hat' with n == m, or n < m and n mod s == 0.  The columns
+// n = g s (g < ceil(m/s)) are the completed groups, i.e. the compressed cache
+// rows C_hat_g; the only other column is the query's own partial row C_hat'_m.
+// So: out[m, h] = softmax over {C_hat_1 .. C_hat_{ceil(m/s)-1}, C_hat'_m} of
+// (q_abs . c_hat + q_rope . k_hat^R) / sqrt(d_h), weighting the latent parts.
+//
+// Design (B200):
+//  * An M tile is 16 consecutive queries x 8 heads = 128 rows (the heads share
+//    every key, so each key tile is loaded once for all of them); a key tile is
+//    64 completed groups, read straight out of C_hat' through a 4-D tensor map
+//    whose row stride is s rows.  Queries, keys and the 16 own rows land as
+//    nine [rows x 64 B] planes with the 64-byte swizzle: the canonical K-major
+//    operand layout for the score MMA and, for the latent planes, the
+//    MN-major operand layout for the value MMA (the key tile is also V).
+//  * Scores S = Q K^T (M 128, N 64, K 288) and values O += P V (M 128, N 256,
+//    K 64) are tcgen05.mma ops with fp32 accumulators in TMEM (S double-
+//    buffered, O 256 columns), issued by one thread.  Only complete groups up
+//    to the staircase are visited, so no tile is empty.
+//  * Four softmax warps own one (query, head) row each (a TMEM lane): mask,
+//    online softmax with lazy rescaling (O is rescaled in TMEM only when the
+//    running max grows by more than 2^8), bf16 P written 128-byte swizzled for
+//    the value MMA.  The epilogue adds the own-row term and writes bf16 out.
+//  * One TMA warp, one MMA warp, mbarrier pipelines; a persistent grid visits
+//    the M tiles heaviest first.
+#include "kernels.cuh"
+
+namespace mtla {
+namespace ptc {
+
+constexpr int H = 8, R = 256, DR = 32, D = R + DR;
+constexpr int QM = 16;                 // query positions per M tile
+constexpr int BM = QM * H;             // 128 rows
+constexpr int BN = 64;                 // groups per key tile
+constexpr int NPL = D / 32;            // 9 planes of 32 elements
+constexpr int QPL = BM * 64;           // bytes of one query plane (8192)
+constexpr int KPL = BN * 64;           // bytes of one key plane (4096)
+constexpr int SPL = QM * 64;           // bytes of one own-row plane (1024)
+constexpr int QBYTES = NPL * QPL;      // 73728
+constexpr int KBYTES = NPL * KPL;      // 36864
+constexpr int SBYTES = NPL * SPL;      // 9216
+constexpr int PBYTES = BM * BN * 2;    // 16384
+constexpr int KS = 2;                  // key-tile stages
+constexpr int NT = 192;                // 4 softmax warps, TMA warp, MMA warp
+constexpr int TMA_WARP = 4, MMA_WARP = 5;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t S_COL0 = 0, S_COL1 = 64, O_COL = 256;
+constexpr uint32_t IDESC_S = umma_idesc_bf16(BM, BN, false, false);
+constexpr uint32_t IDESC_O = umma_idesc_bf16(BM, R, false, true);
+
+constexpr size_t OFF_Q = 0;
+constexpr size_t OFF_SELF = OFF_Q + QBYTES;            // 2 buffers
+constexpr size_t OFF_K = OFF_SELF + 2 * SBYTES;        // KS stages
+constexpr size_t OFF_P = OFF_K + (size_t)KS * KBYTES;  // 2 buffers
+constexpr size_t OFF_BAR = OFF_P + 2 * PBYTES;
+constexpr int NBAR = 21;
+constexpr size_t OFF_TMEM = OFF_BAR + NBAR * 8;
+constexpr size_t SMEM_USED = OFF_TMEM + 16;
+static_assert(OFF_K % 1024 == 0 && OFF_P % 1024 == 0 && OFF_SELF % 1024 == 0, "tile bases must be 1024-aligned");
+
+size_t smem_bytes() { return SMEM_USED + 1024; }
+
+struct Params {
+  int B, T, s;
+  int n_mtiles;            // B * T / QM
+  int n_groups;            // complete groups per sequence, floor(T / s)
+  float scale_log2;        // log2(e) / sqrt(d_h)
+  __nv_bfloat16* out;      // [B, T, H, R]
+  int32_t* dev_err;
+};
+
+
+// 16-byte chunk ch (0..35) of row `row` inside a plane-layout tile whose planes
+// hold `rows` rows: plane ch / 4, 64-byte swizzle phase (row / 2) mod 4
+__device__ __forceinline__ uint32_t plane_off(int rows, int row, int ch) {
+  return (uint32_t)(ch >> 2) * (uint32_t)(rows * 64) + (uint32_t)row * 64u +
+         ((((uint32_t)ch & 3u) ^ (((uint32_t)row >> 1) & 3u)) << 4);
+}
+
+// work of an M tile, heaviest first: index o -> (b, first query m0 1-based, key tiles)
+struct Tile {
+  int b, m0, nkt;
+};
+// mbarrier wait taken by every lane of a warp, with a warp-uniform result:
+// the tcgen05.ld / st that follow are warp-collective, so no lane may leave
+// the common path on its own
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+}
+
+__device__ __forceinline__ Tile tile_of(const Params& p, int o) {
+  const int per_seq = p.T / QM;
+  Tile t;
+  t.b = o % p.B;
+  const int mb = per_seq - 1 - o / p.B;
+  t.m0 = mb * QM + 1;
+  const int vis_max = (int)group_of(t.m0 + QM - 1, p.s) - 1;  // groups seen by the last query
+  t.nkt = (vis_max + BN - 1) / BN;
+  return t;
+}
+
+__global__ void __launch_bounds__(NT, 1)
+prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap rmap,
+                  const __grid_constant__ CUtensorMap smap, const __grid_constant__ CUtensorMap kmap,
+                  const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+  uint64_t* const q_full = bar + 0;
+  uint64_t* const q_empty = bar + 1;
+  uint64_t* const self_full = bar + 2;   // [2]
+  uint64_t* const self_empty = bar + 4;  // [2]
+  uint64_t* const k_full = bar + 6;      // [2]
+  uint64_t* const k_empty = bar + 8;     // [2]
+  uint64_t* const s_full = bar + 10;     // [2]
+  uint64_t* const s_empty = bar + 12;    // [2]
+  uint64_t* const p_full = bar + 14;     // [2]
+  uint64_t* const p_empty = bar + 16;    // [2]
+  uint64_t* const o_full = bar + 18;
+  uint64_t* const o_empty = bar + 19;
+  uint64_t* const mma_done = bar + 20;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (tid == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&self_full[i], 1);
+      mbar_init(&self_empty[i], 4);
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], 4);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&p_empty[i], 1);
+    }
+    mbar_init(o_full, 1);
+    mbar_init(o_empty, 4);
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_holder, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == TMA_WARP && lane == 0) {
+    prefetch_tmap(&qmap);
+    prefetch_tmap(&rmap);
+    prefetch_tmap(&smap);
+    prefetch_tmap(&kmap);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const uint32_t sQ = smem_u32(sm + OFF_Q);
+  const uint32_t sSelf = smem_u32(sm + OFF_SELF);
+  const uint32_t sK = smem_u32(sm + OFF_K);
+  const uint32_t sP = smem_u32(sm + OFF_P);
+  const int G = gridDim.x;
+  bool ok = true;
+
+  if (warp == TMA_WARP) {
+    // ======================= TMA producer =======================
+    if (lane == 0) {
+      uint32_t tc = 0, kc = 0, q_issued = 0, self_issued = 0;
+      for (int o = blockIdx.x; o < p.n_mtiles && ok; o += G, ++tc) {
+        const Tile t = tile_of(p, o);
+        const int qrow0 = ((t.b * p.T) + (t.m0 - 1)) * H;  // first row of [B*T*H, .]
+        const int crow0 = t.b * p.T + (t.m0 - 1);         // first own row of [B*T, .]
+        if (tc > 0 && !mbar_wait(q_empty, (tc - 1) & 1)) { ok = false; break; }
+        mbar_arrive_expect_tx(q_full, QBYTES);
+        tma_load_3d(sm + OFF_Q, &qmap, 0, qrow0, 0, q_full);
+        tma_load_2d(sm + OFF_Q + 8 * QPL, &rmap, 0, qrow0, q_full);
+        q_issued = tc + 1;
+        const int sb = tc & 1;
+        if (tc >= 2 && !mbar_wait(&self_empty[sb], ((tc >> 1) & 1) ^ 1)) { ok = false; break; }
+        mbar_arrive_expect_tx(&self_full[sb], SBYTES);
+        tma_load_3d(sm + OFF_SELF + sb * SBYTES, &smap, 0, crow0, 0, &self_full[sb]);
+        self_issued = tc + 1;
+        for (int kt = 0; kt < t.nkt; ++kt, ++kc) {
+          const int st = kc % KS;
+          if (kc >= KS && !mbar_wait(&k_empty[st], ((kc / KS) & 1) ^ 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(&k_full[st], KBYTES);
+          tma_load_4d(sm + OFF_K + st * KBYTES, &kmap, 0, kt * BN, 0, t.b, &k_full[st]);
+        }
+      }
+      if (!ok) set_err(p.dev_err, MTLA_DEVERR_TIMEOUT);
+      // drain: no copy may still be writing shared memory when the block exits
+      if (q_issued) mbar_wait(q_full, (q_issued - 1) & 1);
+      for (uint32_t u = self_issued > 2 ? self_issued - 2 : 0; u < self_issued; ++u)
+        mbar_wait(&self_full[u & 1], (u >> 1) & 1);
+      for (uint32_t j = kc > (uint32_t)KS ? kc - KS : 0; j < kc; ++j) mbar_wait(&k_full[j % KS], (j / KS) & 1);
+    }
+  } else if (warp == MMA_WARP) {
+    // ======================= MMA issuer =======================
+    if (lane == 0) {
+      uint32_t tc = 0, kc = 0;
+      for (int o = blockIdx.x; o < p.n_mtiles && ok; o += G, ++tc) {
+        const Tile t = tile_of(p, o);
+        if (!mbar_wait(q_full, tc & 1)) { ok = false; break; }
+        tc_fence_after();
+        auto issue_pv = [&](uint32_t j, int kt) {
+          const int pb = j & 1, st = j % KS;
+          if (!mbar_wait(&p_full[pb], (j >> 1) & 1)) ok = false;
+          if (kt == 0 && tc > 0 && !mbar_wait(o_empty, (tc - 1) & 1)) ok = false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            const uint64_t ad = umma_desc(sP + pb * PBYTES + kk * 32, 16, 1024, 2);
+            const uint64_t bd = umma_desc(sK + st * KBYTES + kk * 16 * 64, KPL, 512, 4);
+            umma_bf16(tmem + O_COL, ad, bd, IDESC_O, (kt > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&k_empty[st]);
+          umma_commit(&p_empty[pb]);
+        };
+        for (int kt = 0; kt < t.nkt && ok; ++kt) {
+          const uint32_t j = kc + kt;
+          const int st = j % KS, sb = j & 1;
+          if (!mbar_wait(&k_full[st], (j / KS) & 1)) { ok = false; break; }
+          if (j >= 2 && !mbar_wait(&s_empty[sb], ((j >> 1) & 1) ^ 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t scol = sb ? S_COL1 : S_COL0;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ad = umma_desc(sQ + (kk >> 1) * QPL + (kk & 1) * 32, 16, 512, 4);
+            const uint64_t bd = umma_desc(sK + st * KBYTES + (kk >> 1) * KPL + (kk & 1) * 32, 16, 512, 4);
+            umma_bf16(tmem + scol, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&s_full[sb]);
+          if (kt >= 1) issue_pv(j - 1, kt - 1);
+        }
+        if (t.nkt >= 1 && ok) issue_pv(kc + t.nkt - 1, t.nkt - 1);
+        umma_commit(o_full);
+        kc += t.nkt;
+      }
+      if (!ok) set_err(p.dev_err, MTLA_DEVERR_TIMEOUT);
+      // every MMA of this thread has completed before TMEM is released
+      umma_commit(mma_done);
+      mbar_wait(mma_done, 0);
+    }
+  } else {
+    // ======================= softmax / epilogue warps =======================
+    const int i = tid;                         // row of the M tile = TMEM lane
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const float sl2 = p.scale_log2;
+    uint32_t tc = 0, kc = 0;
+    for (int o = blockIdx.x; o < p.n_mtiles && ok; o += G, ++tc) {
+      const Tile t = tile_of(p, o);
+      const int m = t.m0 + i / H;              // this row's query (1-based)
+      const int h = i % H;
+      const int vis = (int)group_of(m, p.s) - 1;  // completed groups it sees
+      float m_run = -INFINITY, l = 0.f;
+      for (int kt = 0; kt < t.nkt && ok; ++kt) {
+        const uint32_t j = kc + kt;
+        const int sb = j & 1;
+        if (!warp_wait(&s_full[sb], (j >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t sr[2][32];
+        tmem_ld32(lane_base + (sb ? S_COL1 : S_COL0), sr[0]);
+        tmem_ld32(lane_base + (sb ? S_COL1 : S_COL0) + 32, sr[1]);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[sb]);
+        // mask (group kt*BN + c + 1 visible iff <= vis) and scale
+        const int nvis = vis - kt * BN;        // visible columns of this tile
+        float x[64];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          x[c] = c < nvis ? __uint_as_float(sr[c >> 5][c & 31]) * sl2 : -INFINITY;
+          mx = fmaxf(mx, x[c]);
+        }
+        // the running max moves by more than 2^8: rescale l and, once the
+        // previous value MMA has landed, this row of O in TMEM.  The TMEM
+        // accesses are warp-collective, so the whole warp takes the branch
+        // when any of its rows needs it (factor 1 for the others).
+        const bool grow = mx > m_run + 8.f;
+        const bool resc = grow && m_run != -INFINITY;
+        if (kt > 0 && __any_sync(0xffffffffu, resc)) {
+          const uint32_t jp = j - 1;
+          if (!warp_wait(&p_empty[jp & 1], (jp >> 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+          const float a = resc ? exp2f(m_run - mx) : 1.f;
+#pragma unroll 1
+          for (int ch = 0; ch < R / 32; ++ch) {
+            uint32_t ov[32];
+            tmem_ld32(lane_base + O_COL + ch * 32, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * a);
+            tmem_st32(lane_base + O_COL + ch * 32, ov);
+          }
+          tmem_wait_st();
+          l *= a;
+        }
+        if (grow) m_run = mx;
+        // probabilities (relative to the possibly stale max, at most 2^8)
+        uint32_t pk[32];
+        float ls = 0.f;
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const float p0 = x[c] == -INFINITY ? 0.f : exp2f(x[c] - m_run);
+          const float p1 = x[c + 1] == -INFINITY ? 0.f : exp2f(x[c + 1] - m_run);
+          ls += p0 + p1;
+          pk[c >> 1] = pack_bf16x2(p0, p1);
+        }
+        l += ls;
+        // P row i of buffer sb (the previous value MMA on this buffer must be done)
+        if (j >= 2 && !warp_wait(&p_empty[sb], ((j >> 1) & 1) ^ 1)) { ok = false; break; }
+        const uint32_t prow = sP + sb * PBYTES + i * 128;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint32_t a = prow + ((uint32_t)(ch ^ (i & 7)) << 4);
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[4 * ch]), "r"(pk[4 * ch + 1]),
+                       "r"(pk[4 * ch + 2]), "r"(pk[4 * ch + 3]) : "memory");
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[sb]);
+      }
+      if (!ok) break;
+      // ---- epilogue: own partial row C_hat'_m, then out = normalised (O + own term)
+      const int sbuf = tc & 1;
+      if (!warp_wait(&self_full[sbuf], (tc >> 1) & 1)) { ok = false; break; }
+      const uint32_t selfb = sSelf + sbuf * SBYTES;
+      const int srow = i / H;
+      float dot = 0.f;
+#pragma unroll 4
+      for (int ch = 0; ch < D / 8; ++ch) {
+        uint32_t qv[4], cv[4];
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(qv[0]), "=r"(qv[1]), "=r"(qv[2]), "=r"(qv[3])
+                     : "r"(sQ + plane_off(BM, i, ch)));
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(cv[0]), "=r"(cv[1]), "=r"(cv[2]), "=r"(cv[3])
+                     : "r"(selfb + plane_off(QM, srow, ch)));
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qv[e]));
+          const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cv[e]));
+          dot = fmaf(a.x, c.x, dot);
+          dot = fmaf(a.y, c.y, dot);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_empty);  // the query tile is no longer read
+      const float xs = dot * sl2;
+      const float mf = fmaxf(m_run, xs);
+      const float alpha = m_run == -INFINITY ? 0.f : exp2f(m_run - mf);
+      const float pself = exp2f(xs - mf);
+      const float inv = 1.f / (l * alpha + pself);
+      if (!warp_wait(o_full, tc & 1)) { ok = false; break; }
+      tc_fence_after();
+      __nv_bfloat16* orow = p.out + ((size_t)(t.b * p.T + (m - 1)) * H + h) * R;
+#pragma unroll 1
+      for (int ch = 0; ch < R / 32; ++ch) {
+        uint32_t ov[32];
+        if (t.nkt > 0) {
+          tmem_ld32(lane_base + O_COL + ch * 32, ov);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = 0u;
+        }
+        uint32_t res[16];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t cv[4];
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(cv[0]), "=r"(cv[1]), "=r"(cv[2]), "=r"(cv[3])
+                       : "r"(selfb + plane_off(QM, srow, ch * 4 + q4)));
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cv[e]));
+            const int k = q4 * 8 + e * 2;
+            const float v0 = (__uint_as_float(ov[k]) * alpha + pself * c.x) * inv;
+            const float v1 = (__uint_as_float(ov[k + 1]) * alpha + pself * c.y) * inv;
+            res[q4 * 4 + e] = pack_bf16x2(v0, v1);
+          }
+        }
+        uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) dst[q4] = make_uint4(res[4 * q4], res[4 * q4 + 1], res[4 * q4 + 2], res[4 * q4 + 3]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(o_empty);
+        mbar_arrive(&self_empty[sbuf]);
+      }
+      kc += t.nkt;
+    }
+    if (!ok && lane == 0) set_err(p.dev_err, MTLA_DEVERR_TIMEOUT);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace ptc
+
+cudaError_t launch_prefill_tc(const ptc::Params& p, const CUtensorMap& qmap, const CUtensorMap& rmap,
+                              const CUtensorMap& smap, const CUtensorMap& kmap, int grid, cudaStream_t st) {
+  const size_t smem = ptc::smem_bytes();
+  static uint64_t done_mask = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64 || !(done_mask & (1ull << dev))) {
+    e = cudaFuncSetAttribute(ptc::prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) done_mask |= 1ull << dev;
+  }
+  ptc::prefill_tc_kernel<<<grid, ptc::NT, smem, st>>>(qmap, rmap, smap, kmap, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_tc_args(const PrefillTcLaunch& a, const CUtensorMap& qmap, const CUtensorMap& rmap,
+                                   const CUtensorMap& smap, const CUtensorMap& kmap, int grid, cudaStream_t st) {
+  ptc::Params p;
+  p.B = a.B;
+  p.T = a.T;
+  p.s = a.s;
+  p.n_mtiles = a.B * (a.T / ptc::QM);
+  p.n_groups = a.T / a.s;
+  p.scale_log2 = a.scale_log2;
+  p.out = reinterpret_cast<__nv_bfloat16*>(a.out);
+  p.dev_err = a.dev_err;
+  return launch_prefill_tc(p, qmap, rmap, smap, kmap, grid, st);
+}
+
+}  // namespace mtla

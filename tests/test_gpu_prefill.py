@@ -178,3 +178,48 @@ def test_stride_mask_matches_oracle_bit_exact():
     for s in (1, 2, 3, 4, 7, 8):
         for T in (1, 9, 64):
             np.testing.assert_array_equal(mtla.mtla_debug_stride_mask(s, T).astype(bool), oracle.stride_mask(T, s))
+
+
+@pytest.mark.parametrize("s,T", [(1, 256), (2, 96), (3, 400), (4, 128), (5, 80), (8, 1024), (70, 112)])
+def test_prefill_tensor_core_path(s, T):
+    """bf16 (H, r, d_R) = (8, 256, 32) with T a multiple of 16 runs the tcgen05
+    kernel: several key tiles, ragged staircases, queries with no completed group."""
+    dims = synth.Dims(H=8, d_h=64, r=256, d_R=32, s=s)
+    case = synth.token_case(dims, B=3, T=T, seed=400 + s, dtype="bf16")
+    run = PrefillRun(dims, "bf16", case.q_abs, case.q_rope, case.c, case.kR, case.lin).run()
+    for b in range(3):
+        Cp, o = _oracle_seq(case.lin, case.c[b], case.kR[b], case.q_abs[b], case.q_rope[b], dims)
+        assert_close(host(run.out[b]), o, "bf16", f"out s={s} T={T} b={b}")
+
+
+def test_prefill_tensor_core_repeatable():
+    """Two calls give bit-identical outputs (no race between the warp roles)."""
+    dims = synth.Dims(H=8, d_h=64, r=256, d_R=32, s=2)
+    case = synth.token_case(dims, B=4, T=512, seed=77, dtype="bf16")
+    run = PrefillRun(dims, "bf16", case.q_abs, case.q_rope, case.c, case.kR, case.lin).run()
+    first = run.out.clone()
+    run.run()
+    assert torch.equal(first, run.out)
+
+
+@pytest.mark.parametrize("s,T", [(1, 512), (4, 1024)])
+def test_prefill_tensor_core_rising_scores(s, T):
+    """Key magnitudes that ramp up along the sequence and larger queries on odd
+    heads: the running max jumps at later key tiles for some rows of a warp and
+    not others, so the rescale of O in TMEM runs, and runs for part of a warp."""
+    dims = synth.Dims(H=8, d_h=64, r=256, d_R=32, s=s)
+    case = synth.token_case(dims, B=2, T=T, seed=500 + s, dtype="bf16")
+    ramp = (1.0 + 5.0 * np.arange(T) / T)[None, :, None]
+    c = synth.cast(case.c * ramp, "bf16")
+    kR = synth.cast(case.kR * ramp, "bf16")
+    head = np.where(np.arange(8) % 2 == 1, 3.0, 1.0)[None, None, :, None]
+    qa = synth.cast(case.q_abs * head, "bf16")
+    qr = synth.cast(case.q_rope * head, "bf16")
+    run = PrefillRun(dims, "bf16", qa, qr, c, kR, case.lin).run()
+    for b in range(2):
+        Cp, _ = _oracle_seq(case.lin, c[b], kR[b], qa[b], qr[b], dims, with_out=False)
+        # scores reach ~50 here, so the bf16 storage of C_hat' alone moves the
+        # fp64 answer by ~4e-2 of its range; the oracle therefore attends over
+        # its own C_hat' rounded to the cache's storage type
+        o = oracle.masked_forward(qa[b], qr[b], synth.round_to_bf16(Cp), s, dims.d_h)[0]
+        assert_close(host(run.out[b]), o, "bf16", f"out s={s} T={T} b={b}")
