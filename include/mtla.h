@@ -136,6 +136,42 @@ mtla_status mtla_decode_attn(const mtla_dims *dims, int32_t B,
                              int32_t *dev_err, void *stream);
 
 /*
+ * mtla_decode_attn_static — mtla_decode_attn with its scratch in a static
+ * device array of this library instead of a caller-provided workspace.  The
+ * MTLA paper has no counterpart: this is a library convenience, and it
+ * computes exactly what mtla_decode_attn computes, through the same kernels.
+ *
+ * For callers that cannot allocate device memory around a decode step: for
+ * example an engine that has given all free memory to its cache pages, or
+ * plain C host code with no device allocator.  Nothing in the call
+ * allocates.  The scratch is MTLA_DECODE_STATIC_SCRATCH_BYTES per device,
+ * reserved by the driver when the library's device code is loaded.
+ *
+ * Arguments, layouts and device-side errors are those of mtla_decode_attn
+ * without workspace / workspace_bytes.
+ * Set-up: the first call on a device (with that device current) looks up the
+ *   array's address and clears it on `stream`; make it before any stream
+ *   capture.
+ * Limit: a call whose workspace (mtla_workspace_bytes) would exceed
+ *   MTLA_DECODE_STATIC_SCRATCH_BYTES returns MTLA_ERR_WORKSPACE and runs
+ *   nothing.  8 MiB covers every B <= 1024 on a 148-SM B200 (about 6.1 MB at
+ *   B = 1024).
+ * Sharing: all calls on a device use the one scratch, so calls that overlap
+ *   (other streams, unordered threads) race; issue them one after another on
+ *   one stream.
+ */
+#define MTLA_DECODE_STATIC_SCRATCH_BYTES (8u << 20)
+
+mtla_status mtla_decode_attn_static(const mtla_dims *dims, int32_t B,
+                                    const void *q_abs, const void *q_rope,
+                                    const mtla_merge_args *merge,
+                                    void *cache, int64_t cache_rows, int64_t row_stride,
+                                    const int64_t *seq_offset, const int64_t *seq_capacity,
+                                    int32_t *t_processed, int32_t *cache_len,
+                                    float *out, float *lse,
+                                    int32_t *dev_err, void *stream);
+
+/*
  * mtla_prefill_masked_attn — the parallel (training / prefill) forward of B
  * sequences of T tokens, t = 1..T ([mask], [fig2](c)).
  *   1. c_partial[b, n] = C_hat'_n = sum_{i=(j(n)-1)s+1}^{n} w_i ⊙ [c_i ; k^R_i],

@@ -8,6 +8,7 @@ in the CUDA library ``libmtla.so``; this package only marshals arguments
 statuses into exceptions.  Importing it fails if the library is not built.
 """
 from ._abi import (  # noqa: F401
+    DECODE_STATIC_SCRATCH_BYTES,
     DEVERR_CAPACITY,
     DEVERR_EMPTY,
     DEVERR_PE_RANGE,
@@ -23,6 +24,7 @@ from ._abi import (  # noqa: F401
     mtla_cache_length,
     mtla_debug_stride_mask,
     mtla_decode_attn,
+    mtla_decode_attn_static,
     mtla_merge_append,
     mtla_prefill_masked_attn,
     mtla_status_string,

@@ -23,6 +23,7 @@ lib = ctypes.CDLL(LIB_PATH)
 
 MTLA_F32, MTLA_BF16 = 0, 1
 WS_DECODE = 0
+DECODE_STATIC_SCRATCH_BYTES = 8 << 20  # MTLA_DECODE_STATIC_SCRATCH_BYTES
 DEVERR_PE_RANGE, DEVERR_CAPACITY, DEVERR_EMPTY, DEVERR_TIMEOUT = 1, 2, 4, 8
 _c = ctypes
 
@@ -46,6 +47,9 @@ lib.mtla_merge_append.argtypes = [_DIMS_P, _I32, _MERGE_P, _P, _I64, _I64, _P, _
 lib.mtla_decode_attn.restype = _c.c_int
 lib.mtla_decode_attn.argtypes = [_DIMS_P, _I32, _P, _P, _MERGE_P, _P, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ,
                                  _P, _P]
+lib.mtla_decode_attn_static.restype = _c.c_int
+lib.mtla_decode_attn_static.argtypes = [_DIMS_P, _I32, _P, _P, _MERGE_P, _P, _I64, _I64, _P, _P, _P, _P, _P, _P, _P,
+                                        _P]
 lib.mtla_prefill_masked_attn.restype = _c.c_int
 lib.mtla_prefill_masked_attn.argtypes = [_DIMS_P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _P, _P, _P]
 lib.mtla_workspace_bytes.restype = _SZ
@@ -114,6 +118,14 @@ def mtla_decode_attn(d, B, q_abs, q_rope, merge, cache, cache_rows, row_stride, 
                                 row_stride, _ptr(seq_offset), _ptr(seq_capacity), _ptr(t_processed),
                                 _ptr(cache_len), _ptr(out), _ptr(lse), _ptr(workspace), workspace_bytes,
                                 _ptr(dev_err), _stream(stream)), "mtla_decode_attn")
+
+
+def mtla_decode_attn_static(d, B, q_abs, q_rope, merge, cache, cache_rows, row_stride, seq_offset, seq_capacity,
+                            t_processed, cache_len, out, lse, dev_err, stream=None):
+    _check(lib.mtla_decode_attn_static(_c.byref(d), B, _ptr(q_abs), _ptr(q_rope), _merge(merge), _ptr(cache),
+                                       cache_rows, row_stride, _ptr(seq_offset), _ptr(seq_capacity),
+                                       _ptr(t_processed), _ptr(cache_len), _ptr(out), _ptr(lse), _ptr(dev_err),
+                                       _stream(stream)), "mtla_decode_attn_static")
 
 
 def mtla_prefill_masked_attn(d, B, T, q_abs, q_rope, c, kR, W_c, b_c, P, J_max, c_partial, cache_out, out,
