@@ -85,6 +85,22 @@ def profiled_traffic():
         return None
 
 
+def max_over_ranks(value: float, dist, device) -> float:
+    """The largest of all ranks' values (every rank calls this, in the same
+    order); the value itself on a single process."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, units_per_rank_step: int, steps: int, ms_max: float) -> float:
+    """Whole-job units per second: every rank's units over the slowest rank's time."""
+    return world * units_per_rank_step * steps / (ms_max / 1e3)
+
+
 # ---------------------------------------------------------------------------
 # clocks during the timed region (NVML, read only)
 # ---------------------------------------------------------------------------
@@ -259,13 +275,9 @@ def run_ours(args, rank, world, local_rank):
     dev_err = int(err.item())
     if dev_err:
         raise RuntimeError(f"device error bits {dev_err} during the timed steps")
-    ms_max = ms
-    if dist:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_max = float(tt.item())
+    ms_max = max_over_ranks(ms, dist, dev)
     ms_step = ms_max / K
-    value = world * B * K / (ms_max / 1e3)
+    value = job_throughput(world, B, K, ms_max)
 
     hbm_peak, _, _, peak_kind = measured_peaks()
     achieved_gbs = (sum(timed_bytes) / K) / (ms / K / 1e3) / 1e9
