@@ -7,6 +7,11 @@
 
 #include "kernels.cuh"
 
+namespace mtla {
+// tensor-core running merge (merge_tc.cu)
+cudaError_t launch_merge_tc(const PrefillArgs& a, int B, const CUtensorMap& cmap, int sms, cudaStream_t st);
+}  // namespace mtla
+
 namespace {
 
 using namespace mtla;
@@ -78,13 +83,19 @@ bool encode_cache_map(CUtensorMap* map, void* cache, int64_t cache_rows, int64_t
 
 // Generic tiled map of a bf16 tensor with the 64-byte swizzle (dims innermost first).
 bool encode_bf16_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
-                     const cuuint32_t* box) {
+                     const cuuint32_t* box, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_64B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// the running merge on the tensor cores: bf16, r = 256, d_R = 32, s <= 32
+bool tc_merge_dims(const mtla_dims* d, int B, int T) {
+  return d->dtype == MTLA_BF16 && d->r == 256 && d->d_R == 32 && d->s <= 32 &&
+         (int64_t)B * T + 256 < (int64_t(1) << 31);
 }
 
 bool tc_prefill_dims(const mtla_dims* d, int B, int T) {
@@ -302,7 +313,20 @@ mtla_status mtla_prefill_masked_attn(const mtla_dims* dims, int32_t B, int32_t T
   p.s = dims->s;
   p.scale = (float)(1.0 / sqrt((double)dims->d_h));
   p.J_max = J_max;
-  cudaError_t e = launch_partial_merge(p, B, dims->dtype, cs);
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return MTLA_ERR_CUDA;
+  cudaError_t e;
+  if (tc_merge_dims(dims, B, T)) {
+    // latents as [B*T rows, 256], boxes of 64 latents x 32 rows, 128-byte swizzle
+    CUtensorMap cmap;
+    const cuuint64_t dims2[2] = {256, (cuuint64_t)B * T}, str[1] = {512};
+    const cuuint32_t box[2] = {64, 32};
+    if (!encode_bf16_map(&cmap, c, 2, dims2, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MTLA_ERR_CUDA;
+    e = launch_merge_tc(p, B, cmap, sms, cs);
+  } else {
+    e = launch_partial_merge(p, B, dims->dtype, cs);
+  }
   if (e != cudaSuccess) return MTLA_ERR_CUDA;
   if (!out) return MTLA_OK;
   if (!tc_prefill_dims(dims, B, T)) return from_cuda(launch_prefill_simt(p, B, dims->dtype, cs));
@@ -335,9 +359,6 @@ mtla_status mtla_prefill_masked_attn(const mtla_dims* dims, int32_t B, int32_t T
     const __nv_bfloat16* base = reinterpret_cast<const __nv_bfloat16*>(c_partial) + (s - 1) * 288;
     if (!encode_bf16_map(&kmap, base, 4, dims4, str, box)) return MTLA_ERR_CUDA;
   }
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return MTLA_ERR_CUDA;
   PrefillTcLaunch a;
   a.B = B;
   a.T = T;

@@ -223,3 +223,18 @@ def test_prefill_tensor_core_rising_scores(s, T):
         # its own C_hat' rounded to the cache's storage type
         o = oracle.masked_forward(qa[b], qr[b], synth.round_to_bf16(Cp), s, dims.d_h)[0]
         assert_close(host(run.out[b]), o, "bf16", f"out s={s} T={T} b={b}")
+
+
+@pytest.mark.parametrize("s,T", [(1, 300), (2, 1000), (3, 97), (4, 4096), (7, 333), (16, 160), (31, 100), (32, 97),
+                                 (33, 70)])
+def test_running_merge_strides(s, T):
+    """The running merge and the compressed cache alone (cache-only call) for
+    strides up to 32 (tensor-core kernel: warp blocks of floor(32/s)*s tokens)
+    and 33 (generic kernel), ragged prompt ends included."""
+    dims = synth.Dims(H=8, d_h=64, r=256, d_R=32, s=s)
+    case = synth.token_case(dims, B=3, T=T, seed=600 + s, dtype="bf16", with_queries=False)
+    run = PrefillRun(dims, "bf16", None, None, case.c, case.kR, case.lin, with_out=False).run()
+    for b in range(3):
+        Cp, _ = _oracle_seq(case.lin, case.c[b], case.kR[b], None, None, dims, with_out=False)
+        assert_close(host(run.cp[b]), Cp, "bf16", f"C_hat' s={s} T={T} b={b}")
+        assert_close(host(run.cache[b]), oracle.compressed_cache(Cp, s), "bf16", f"cache s={s} T={T} b={b}")
