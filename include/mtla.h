@@ -154,13 +154,13 @@ mtla_status mtla_decode_attn(const mtla_dims *dims, int32_t B,
  *   capture.
  * Limit: a call whose workspace (mtla_workspace_bytes) would exceed
  *   MTLA_DECODE_STATIC_SCRATCH_BYTES returns MTLA_ERR_WORKSPACE and runs
- *   nothing.  8 MiB covers every B <= 1024 on a 148-SM B200 (about 6.1 MB at
- *   B = 1024).
+ *   nothing.  24 MiB covers every B <= 1024 on a 148-SM B200 (about 20.2 MB
+ *   at B = 1024).
  * Sharing: all calls on a device use the one scratch, so calls that overlap
  *   (other streams, unordered threads) race; issue them one after another on
  *   one stream.
  */
-#define MTLA_DECODE_STATIC_SCRATCH_BYTES (8u << 20)
+#define MTLA_DECODE_STATIC_SCRATCH_BYTES (24u << 20)
 
 mtla_status mtla_decode_attn_static(const mtla_dims *dims, int32_t B,
                                     const void *q_abs, const void *q_rope,

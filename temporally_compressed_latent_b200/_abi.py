@@ -23,7 +23,7 @@ lib = ctypes.CDLL(LIB_PATH)
 
 MTLA_F32, MTLA_BF16 = 0, 1
 WS_DECODE = 0
-DECODE_STATIC_SCRATCH_BYTES = 8 << 20  # MTLA_DECODE_STATIC_SCRATCH_BYTES
+DECODE_STATIC_SCRATCH_BYTES = 24 << 20  # MTLA_DECODE_STATIC_SCRATCH_BYTES
 DEVERR_PE_RANGE, DEVERR_CAPACITY, DEVERR_EMPTY, DEVERR_TIMEOUT = 1, 2, 4, 8
 _c = ctypes
 

@@ -262,14 +262,11 @@ mtla_status mtla_decode_attn(const mtla_dims* dims, int32_t B, const void* q_abs
   p.seq_info = reinterpret_cast<int4*>(ws + off);
   off += (size_t)B * 16;
   off = (off + 255) & ~(size_t)255;
-  p.fs = reinterpret_cast<int32_t*>(ws + off);
-  off += (size_t)grid * 4;
-  off = (off + 255) & ~(size_t)255;
-  p.gates = reinterpret_cast<float*>(ws + off);
-  off += (size_t)B * dtc::D * 4;
+  p.tails = reinterpret_cast<__nv_bfloat16*>(ws + off);
+  off += (size_t)B * dtc::D * 2;
   off = (off + 255) & ~(size_t)255;
   p.ws_ml = reinterpret_cast<float*>(ws + off);
-  off += (size_t)2 * grid * dtc::H * 2 * 4;
+  off += (size_t)2 * grid * dtc::NCW * dtc::H * 2 * 4;
   off = (off + 255) & ~(size_t)255;
   p.ws_o = reinterpret_cast<float*>(ws + off);
   return from_cuda(launch_decode_tc(p, maps.m64, maps.m8, grid, cs));

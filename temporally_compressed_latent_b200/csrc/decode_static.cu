@@ -26,8 +26,8 @@
 namespace mtla {
 namespace {
 
-// file-scope scratch; 8 MiB covers the split-L kernel's workspace for every B
-// it accepts (B <= 1024) on a 148-SM B200 (about 6.1 MB at B = 1024)
+// file-scope scratch; 24 MiB covers the split-L kernel's workspace for every
+// B it accepts (B <= 1024) on a 148-SM B200 (about 20.2 MB at B = 1024)
 __device__ __align__(256) unsigned char g_decode_scratch[MTLA_DECODE_STATIC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;

@@ -26,25 +26,23 @@
 //    value-MMA operand with one in-register 8x8 transpose (movmatrix).  Each
 //    warp keeps its own online-softmax state, so no block barrier is needed
 //    per tile.
-//  * The gate pre-activations Linear(c_t) = c_t W_c + b_c of all B new tokens
-//    come from a small kernel launched just before (32 channels x 8 tokens per
-//    block, W_c read as coalesced row segments).  It releases the decode grid
-//    at once (programmatic dependent launch), so the decode blocks run their
-//    set-up and stream their tiles meanwhile; only the block owning a
-//    sequence's tail row waits for it, then forms the gate, the gated entry
-//    and the updated row in fp32, writes the row to the cache in bf16 and
-//    patches it into the tile before the tile is used.
-//  * Launched with programmatic dependent launch: the next call's blocks are
-//    scheduled while this call's last blocks finish and wait for it before
-//    touching memory.
+//  * The merge of the B new tokens runs in a small kernel launched just before
+//    (gate contraction with W_c read as coalesced row segments, gate, gated
+//    entry, append / in-place update of the tail row, written to the cache and
+//    to a workspace copy).  It releases the decode grid at once (programmatic
+//    dependent launch), so the decode blocks set up and stream meanwhile.
+//    Every block visits its share's sequences last to first, so a tail row is
+//    the last tile of its block; the warp holding it waits for the merge
+//    kernel (hardware-tracked) and patches the finished row into the tile.
 //  * A block that holds only part of a sequence writes its partial (max, sum,
 //    unnormalised output) to the workspace and moves on: no fence, no atomic,
-//    no block ever waits for another at a segment boundary.  A second, small
-//    kernel chained with programmatic dependent launch (its blocks are resident
-//    and waiting before the first kernel ends) combines the split sequences,
-//    advances t_processed / cache_len and resets the gate counter.  Every
-//    block's share and first sequence are tabulated once in shared memory, so
-//    the bookkeeping in the loops needs no integer division.
+//    no block ever waits for another.  A second, small kernel chained with
+//    programmatic dependent launch (its blocks are resident and waiting
+//    before the first kernel ends) combines the split sequences from a
+//    per-sequence partition summary that block 0 publishes (one dependent
+//    load, then every part's loads at once) and advances t_processed /
+//    cache_len.  Every block's share and first sequence are tabulated once in
+//    shared memory, so the bookkeeping in the loops needs no division.
 #include "kernels.cuh"
 
 namespace mtla {
@@ -56,7 +54,6 @@ constexpr size_t kAlign = 128;
 __host__ __device__ constexpr size_t rup(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 constexpr int kCombHeads = 4;  // heads per pass of the block combine
 constexpr int QSTR = D / 2 + 4;  // words per query row in shared memory (148: conflict-free)
-static_assert(17 * H * 2 <= NCW * kCombHeads * OSTR, "combine scratch must fit the combine buffer");
 static_assert((size_t)H * QSTR * 4 <= (size_t)NCW * kCombHeads * OSTR * 4, "query buffer must fit the combine buffer");
 constexpr size_t kOffComb = rup((size_t)NS * STAGE);
 constexpr size_t kOffCombMl = kOffComb + rup((size_t)NCW * kCombHeads * OSTR * 4);
@@ -65,26 +62,23 @@ constexpr size_t kOffMeta = kOffPrefix + rup((size_t)(MAXB + 1) * 8);
 constexpr size_t kOffScan = kOffMeta + rup((size_t)MAXB * 4);
 constexpr size_t kOffLo = kOffScan + rup(128 * 8);
 constexpr size_t kOffFs = kOffLo + rup((size_t)(MAXG + 1) * 8);
-constexpr size_t kOffC = kOffFs + rup((size_t)MAXG * 4);
-constexpr size_t kOffTail = kOffC + rup((size_t)R * 4);
-constexpr size_t kOffBar = kOffTail + rup((size_t)D * 2);
+constexpr size_t kOffQx = kOffFs + rup((size_t)MAXG * 4);
+constexpr size_t kOffBar = kOffQx + rup((size_t)H * QSTR * 4);
 constexpr size_t kOffFlags = kOffBar + rup(2 * NS * 8);
 constexpr size_t kSmemUsed = kOffFlags + rup(16);
-static_assert(kOffTail % 16 == 0 && kOffBar % 8 == 0, "shared-memory regions must stay aligned");
+static_assert(kOffQx % 16 == 0 && kOffBar % 8 == 0, "shared-memory regions must stay aligned");
 
 size_t smem_bytes() { return kSmemUsed + 1024; }  // + slack to align the base to 1024
 
 size_t workspace_bytes(int B, int grid) {
   size_t b = 0;
-  b += (size_t)B * 16;  // seq_info
+  b += (size_t)B * 16;  // per-sequence partition summary
   b = (b + 255) & ~(size_t)255;
-  b += (size_t)grid * 4;  // fs
+  b += (size_t)B * D * 2;  // tail rows
   b = (b + 255) & ~(size_t)255;
-  b += (size_t)B * D * 4;
+  b += (size_t)2 * grid * NCW * H * 2 * 4;  // parts: (max, sum) per head
   b = (b + 255) & ~(size_t)255;
-  b += (size_t)2 * grid * H * 2 * 4;
-  b = (b + 255) & ~(size_t)255;
-  b += (size_t)2 * grid * H * R * 4;
+  b += (size_t)2 * grid * NCW * H * R * 4;  // parts: unnormalised outputs
   return b;
 }
 
@@ -106,8 +100,7 @@ struct Smem {
   int64_t* scan;
   int64_t* lo;        // [G + 1] first cost position of each block's share
   int32_t* fs;        // [G] first sequence with rows in each block's share
-  float* c_sm;
-  __nv_bfloat16* tail_sm;
+  uint32_t* qx;       // [H][QSTR] queries of the share's second sequence (prefetched)
   uint64_t* full_bar;
   uint64_t* empty_bar;
   int32_t* flags;
@@ -124,8 +117,7 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   s.scan = reinterpret_cast<int64_t*>(p + kOffScan);
   s.lo = reinterpret_cast<int64_t*>(p + kOffLo);
   s.fs = reinterpret_cast<int32_t*>(p + kOffFs);
-  s.c_sm = reinterpret_cast<float*>(p + kOffC);
-  s.tail_sm = reinterpret_cast<__nv_bfloat16*>(p + kOffTail);
+  s.qx = reinterpret_cast<uint32_t*>(p + kOffQx);
   s.full_bar = reinterpret_cast<uint64_t*>(p + kOffBar);
   s.empty_bar = s.full_bar + NS;
   s.flags = reinterpret_cast<int32_t*>(p + kOffFlags);
@@ -143,8 +135,54 @@ __device__ __forceinline__ int upper_bound_i64(const int64_t* a, int n, int64_t 
 }
 
 constexpr int PRO_T = 32 * (NCW + 1);  // threads of the consumer and producer warps
+
+// 16-byte asynchronous global -> shared copies (completion per thread)
+__device__ __forceinline__ void cp_async16(uint32_t saddr, const void* g) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr), "l"(g) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ int64_t rows_of(const uint32_t* meta, int b) {
   return (int64_t)(meta[b] & (kMetaMergeOk - 1));
+}
+
+// Sequence b after this call: its rows, whether its new token is merged, and
+// the device-error bits the checks raise.  The merge kernel (which writes the
+// tail row) and the decode kernel (which partitions the rows) decide alike.
+struct SeqState {
+  int64_t t;        // processed tokens after the call
+  int64_t L;        // cache rows after the call
+  bool merge_ok;
+  int err;
+};
+__device__ __forceinline__ SeqState seq_state(const Params& p, int b, bool with_merge) {
+  const int s = p.a.s;
+  const int64_t t0 = p.a.t_processed[b];
+  const int64_t off = p.a.seq_offset[b], cap = p.a.seq_capacity[b];
+  SeqState st;
+  st.t = t0 + (with_merge ? 1 : 0);
+  st.L = st.t > 0 ? group_of(st.t, s) : 0;
+  st.merge_ok = with_merge;
+  st.err = 0;
+  if (t0 < 0 || off < 0 || cap < 0 || off > p.a.cache_rows || cap > p.a.cache_rows - off) {
+    st.err |= MTLA_DEVERR_CAPACITY;
+    st.L = 0;
+    st.merge_ok = false;
+  } else if (st.L > cap) {
+    st.err |= MTLA_DEVERR_CAPACITY;
+    st.L = cap;
+    st.merge_ok = false;
+  }
+  if (st.L >= (int64_t)kMetaMergeOk) {  // beyond what one call can address
+    st.err |= MTLA_DEVERR_CAPACITY;
+    st.L = 0;
+    st.merge_ok = false;
+  }
+  if (st.merge_ok && group_of(st.t, s) > p.m.J_max) {
+    st.err |= MTLA_DEVERR_PE_RANGE;
+    st.merge_ok = false;
+  }
+  return st;
 }
 
 __global__ void __launch_bounds__(NT, 2)
@@ -159,9 +197,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
 
   // let the next launch on the stream be scheduled as soon as blocks retire.
   // Without a merge, wait for the previous launch before reading anything it
-  // may write; with a merge the gate kernel just before has already waited
-  // for it, and only the gates themselves (read at a tail row) need the gate
-  // kernel to be complete.
+  // may write; with a merge the merge kernel just before has already waited
+  // for it, and only the tail rows it writes need it to be complete.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (tid == 0) {
     for (int i = 0; i < NS; ++i) {
@@ -181,32 +218,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
   if (tid < 128) {
     int64_t sum = 0;
     for (int b = tid * per; b < B && b < (tid + 1) * per; ++b) {
-      const int64_t t0 = p.a.t_processed[b];
-      const int64_t t = t0 + (with_merge ? 1 : 0);
-      const int64_t off = p.a.seq_offset[b], cap = p.a.seq_capacity[b];
-      int64_t L = t > 0 ? group_of(t, s) : 0;
-      bool ok = with_merge;
-      const bool report = (cta == 0);
-      if (t0 < 0 || off < 0 || cap < 0 || off > p.a.cache_rows || cap > p.a.cache_rows - off) {
-        if (report) set_err(p.a.dev_err, MTLA_DEVERR_CAPACITY);
-        L = 0;
-        ok = false;
-      } else if (L > cap) {
-        if (report) set_err(p.a.dev_err, MTLA_DEVERR_CAPACITY);
-        L = cap;
-        ok = false;
-      }
-      if (L >= (int64_t)kMetaMergeOk) {  // beyond what one call can address
-        if (report) set_err(p.a.dev_err, MTLA_DEVERR_CAPACITY);
-        L = 0;
-        ok = false;
-      }
-      if (ok && group_of(t, s) > p.m.J_max) {
-        if (report) set_err(p.a.dev_err, MTLA_DEVERR_PE_RANGE);
-        ok = false;
-      }
-      sm.meta[b] = (uint32_t)L | (ok ? kMetaMergeOk : 0u);
-      sum += L + mcost;
+      const SeqState st = seq_state(p, b, with_merge);
+      if (st.err && cta == 0) set_err(p.a.dev_err, st.err);
+      sm.meta[b] = (uint32_t)st.L | (st.merge_ok ? kMetaMergeOk : 0u);
+      sum += st.L + mcost;
     }
     sm.scan[tid] = sum;
   }
@@ -249,21 +264,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
   }
   named_bar(2, PRO_T);
 
-  if (cta == 0) {
-    // the partition, for the combine kernel (read after this grid completes)
-    for (int c = tid; c < G; c += PRO_T) p.fs[c] = sm.fs[c];
-    for (int b = tid; b < B; b += PRO_T) {
-      const int64_t Lb = rows_of(sm.meta, b);
-      int cf = -1, cl = -1;
-      if (Lb > 0) {
-        cf = upper_bound_i64(sm.lo, G + 1, sm.prefix[b]) - 1;
-        cl = upper_bound_i64(sm.lo, G + 1, sm.prefix[b] + Lb - 1) - 1;
-      }
-      p.seq_info[b] = make_int4((int)Lb, (sm.meta[b] & kMetaMergeOk) ? 1 : 0, cf, cl);
-    }
-  }
   const int64_t my_lo = sm.lo[cta], my_hi = sm.lo[cta + 1];
+  // the share's sequences, visited last to first so that a sequence's tail
+  // row (whose merge the merge kernel finishes meanwhile) is the block's last
+  // tile; b_first == B when the share holds no rows
   const int b_first = sm.fs[cta];
+  const int b_last = my_lo < my_hi ? upper_bound_i64(sm.prefix, B + 1, my_hi - 1) - 1 : -1;
   const __nv_bfloat16* cache = reinterpret_cast<const __nv_bfloat16*>(p.a.cache);
 
   // ======================= producer warp =======================
@@ -271,7 +277,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
     if (lane == 0 && my_lo < my_hi) {
       uint32_t job = 0;
       bool ok = true;
-      for (int b = b_first; b < B && sm.prefix[b] < my_hi && ok; ++b) {
+      for (int b = b_last; b >= b_first && ok; --b) {
         const int64_t Lb = rows_of(sm.meta, b);
         const int64_t r_lo = (my_lo > sm.prefix[b] ? my_lo : sm.prefix[b]) - sm.prefix[b];
         const int64_t r_end = sm.prefix[b] + Lb < my_hi ? sm.prefix[b] + Lb : my_hi;
@@ -323,20 +329,67 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
   uint32_t job = 0;
   bool ok = true;
 
-  for (int b = b_first; b < B && sm.prefix[b] < my_hi; ++b) {
+  // the share's second sequence (in visiting order): its queries are fetched
+  // now, so that they do not queue behind the tile stream later
+  int b_second = -1;
+  {
+    int found = 0;
+    for (int b = b_last; b >= b_first && found < 2; --b) {
+      const int64_t lo_b = my_lo > sm.prefix[b] ? my_lo : sm.prefix[b];
+      const int64_t hi_b = sm.prefix[b] + rows_of(sm.meta, b) < my_hi ? sm.prefix[b] + rows_of(sm.meta, b) : my_hi;
+      if (lo_b >= hi_b) continue;
+      if (++found == 2) b_second = b;
+    }
+  }
+  if (b_second >= 0) {
+    const __nv_bfloat16* qa = reinterpret_cast<const __nv_bfloat16*>(p.o.q_abs) + (size_t)b_second * H * R;
+    const __nv_bfloat16* qr = reinterpret_cast<const __nv_bfloat16*>(p.o.q_rope) + (size_t)b_second * H * DR;
+    for (int i = ctid; i < H * (D / 8); i += 128) {
+      const int h = i / (D / 8), c = i % (D / 8);  // 16-byte chunk c of head h's row
+      const __nv_bfloat16* src = c < R / 8 ? qa + h * R + c * 8 : qr + h * DR + (c - R / 8) * 8;
+      cp_async16(smem_u32(sm.qx) + (uint32_t)(h * QSTR + c * 4) * 4u, src);
+    }
+    cp_async_commit();
+  }
+  int seg = 0;
+
+  // the partition as the combine kernel needs it, published by block 0 while
+  // its first tile is in flight: rows, merge flag, the first part's slot and
+  // the number of parts (blocks cf..cl; block c > cf stored its part in slot
+  // 2c, block cf in 2cf or 2cf + 1)
+  if (cta == 0) {
+    for (int bb = ctid; bb < B; bb += 128) {
+      const int64_t Lb = rows_of(sm.meta, bb);
+      const int ok_m = (sm.meta[bb] & kMetaMergeOk) ? 1 : 0;
+      int first = 0, n = 0;
+      if (Lb > 0) {
+        const int cf = upper_bound_i64(sm.lo, G + 1, sm.prefix[bb]) - 1;
+        const int cl = upper_bound_i64(sm.lo, G + 1, sm.prefix[bb] + Lb - 1) - 1;
+        first = 2 * cf + (sm.fs[cf] == bb ? 0 : 1);
+        n = cl - cf + 1;
+      }
+      p.seq_info[bb] = make_int4((int)Lb, ok_m, first, n);
+    }
+  }
+
+  for (int b = b_last; b >= b_first; --b) {
     const int64_t Lb = rows_of(sm.meta, b);
     const int64_t r_lo = (my_lo > sm.prefix[b] ? my_lo : sm.prefix[b]) - sm.prefix[b];
     const int64_t r_end = sm.prefix[b] + Lb < my_hi ? sm.prefix[b] + Lb : my_hi;
     const int64_t r_hi = r_end - sm.prefix[b];
     if (r_lo >= r_hi) continue;
     const bool merge_here = (sm.meta[b] & kMetaMergeOk) && r_hi == Lb;
-    const bool full = (r_lo == 0 && r_hi == Lb);
 
     // [q_abs ; q_rope] of the 8 heads into shared memory (rows padded to
-    // QSTR words so the B-fragment loads below are free of bank conflicts);
-    // the buffer shares space with the combine buffer, which is only used
-    // after the segment's last tile
-    {
+    // QSTR words so the B-fragment loads below are free of bank conflicts):
+    // the prefetched buffer for the second sequence, else loaded now into the
+    // combine buffer, which is only used after the segment's last tile
+    const bool pre = (seg == 1 && b == b_second);
+    if (pre) {
+      cp_async_wait_all();
+      named_bar(1, 128);
+    } else {
+      if (seg > 0) named_bar(1, 128);  // every warp is done with the previous queries
       const uint32_t* qa = reinterpret_cast<const uint32_t*>(
           reinterpret_cast<const __nv_bfloat16*>(p.o.q_abs) + (size_t)b * H * R);
       const uint32_t* qr = reinterpret_cast<const uint32_t*>(
@@ -349,7 +402,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
       named_bar(1, 128);
     }
     // B operand of the score MMA for head g: words 8kk + q and 8kk + q + 4 of its row
-    const uint32_t qrow = smem_u32(sm.comb_o) + (uint32_t)(g * QSTR + q) * 4u;
+    const uint32_t qrow = smem_u32(pre ? reinterpret_cast<float*>(sm.qx) : sm.comb_o) + (uint32_t)(g * QSTR + q) * 4u;
     float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
     float O[16][4];
 #pragma unroll
@@ -358,33 +411,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
 
     for (int64_t u = r_lo; u < r_hi; u += UNIT) {
       const bool is_tail = merge_here && u + UNIT >= r_hi;
-      if (is_tail) {
-        // the gate kernel must be complete (hardware-tracked, no polling)
-        asm volatile("griddepcontrol.wait;" ::: "memory");
-        // gate, gated entry and the updated tail row (fp32 math, bf16 storage)
-        const int64_t t = (int64_t)p.a.t_processed[b] + 1;
-        const int64_t j = group_of(t, s);
-        const bool opens = opens_row(t, s);
-        __nv_bfloat16* row = const_cast<__nv_bfloat16*>(cache) + (p.a.seq_offset[b] + j - 1) * p.a.row_stride;
-        const __nv_bfloat16* cn = reinterpret_cast<const __nv_bfloat16*>(p.m.c_new) + (size_t)b * R;
-        const __nv_bfloat16* kR = reinterpret_cast<const __nv_bfloat16*>(p.m.kR_new) + (size_t)b * DR;
-        const float* Pj = p.m.P + (j - 1) * D;
-#pragma unroll
-        for (int ci = 0; ci < 3; ++ci) {
-          const int k = ctid + 128 * ci;
-          if (k < D) {
-            const float gv = __ldcg(p.gates + (size_t)b * D + k);
-            const float w = sigmoidf_(__fmul_rn(gv, Pj[k]));
-            const float x = __bfloat162float(k < R ? cn[k] : kR[k - R]);
-            const float e = __fmul_rn(w, x);
-            const float v = opens ? e : __fadd_rn(__bfloat162float(row[k]), e);
-            const __nv_bfloat16 vb = __float2bfloat16_rn(v);
-            row[k] = vb;
-            sm.tail_sm[k] = vb;
-          }
-        }
-        named_bar(1, 128);
-      }
 
       const int st = job % NS;
       if (ok && !mbar_wait(&sm.full_bar[st], (job / NS) & 1)) ok = false;
@@ -405,9 +431,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
         if (is_tail) {
           const int lr = (int)(Lb - 1 - u);
           if (lr >= w_lo && lr < w_lo + 16) {
-            const uint4* src = reinterpret_cast<const uint4*>(sm.tail_sm);
+            // the merge kernel wrote the updated row (the copy the tile holds
+            // may predate it); hardware-tracked wait for that kernel, no polling
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            const uint4* src = reinterpret_cast<const uint4*>(p.tails + (size_t)b * D);
             for (int ch = lane; ch < 36; ch += 32) {
-              const uint4 v = src[ch];
+              const uint4 v = __ldcg(src + ch);
               asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(tile + swz_off(lr, ch)), "r"(v.x),
                            "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
             }
@@ -474,227 +503,255 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
       ++job;
     }
 
-    // ---- segment end: combine the four warps, then write out or a partial
-    named_bar(1, 128);  // every warp is done with the query buffer
+    // ---- segment end
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
       lA += __shfl_xor_sync(0xffffffffu, lA, o);
       lB += __shfl_xor_sync(0xffffffffu, lB, o);
     }
-    if (g == 0) {
-      sm.comb_ml[(cw * H + 2 * q) * 2 + 0] = mA;
-      sm.comb_ml[(cw * H + 2 * q) * 2 + 1] = lA;
-      sm.comb_ml[(cw * H + 2 * q + 1) * 2 + 0] = mB;
-      sm.comb_ml[(cw * H + 2 * q + 1) * 2 + 1] = lB;
-    }
-    const int nslot = full ? -1 : 2 * cta + (b == b_first ? 0 : 1);
-    named_bar(1, 128);  // comb_ml complete
-    float* wsc = sm.comb_ml + NCW * H * 2;  // [NCW][H] weights exp2(m_w - M), then [H] M and [H] 1/L
-    if (ctid < H) {
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < NCW; ++w) M = fmaxf(M, sm.comb_ml[(w * H + ctid) * 2]);
-      float Ls = 0.f;
-#pragma unroll
-      for (int w = 0; w < NCW; ++w) {
-        const float mw = sm.comb_ml[(w * H + ctid) * 2];
-        const float sc = mw == -INFINITY ? 0.f : exp2f(mw - M);
-        wsc[w * H + ctid] = sc;
-        Ls += sc * sm.comb_ml[(w * H + ctid) * 2 + 1];
+    if (r_lo == 0 && r_hi == Lb) {
+      // a sequence held by this block alone: the four warps combine through
+      // shared memory and write out
+      named_bar(1, 128);  // every warp is done with the query buffer
+      if (g == 0) {
+        sm.comb_ml[(cw * H + 2 * q) * 2 + 0] = mA;
+        sm.comb_ml[(cw * H + 2 * q) * 2 + 1] = lA;
+        sm.comb_ml[(cw * H + 2 * q + 1) * 2 + 0] = mB;
+        sm.comb_ml[(cw * H + 2 * q + 1) * 2 + 1] = lB;
       }
-      wsc[NCW * H + ctid] = M;
-      wsc[NCW * H + H + ctid] = Ls;
-    }
-#pragma unroll 1
-    for (int pass = 0; pass < 2; ++pass) {
-      // heads 4 pass .. 4 pass + 3 belong to the lanes with q >> 1 == pass
-      if ((q >> 1) == pass) {
-        const int hl = 2 * q - kCombHeads * pass;  // local head of O[.][0]
+      named_bar(1, 128);  // comb_ml complete
+      float* wsc = sm.comb_ml + NCW * H * 2;  // [NCW][H] weights exp2(m_w - M), then [H] M and [H] L
+      if (ctid < H) {
+        float M = -INFINITY;
 #pragma unroll
-        for (int mb = 0; mb < 16; ++mb) {
-          float* oA = sm.comb_o + (cw * kCombHeads + hl) * OSTR + 16 * mb + g;
-          float* oB = oA + OSTR;
-          oA[0] = O[mb][0];
-          oB[0] = O[mb][1];
-          oA[8] = O[mb][2];
-          oB[8] = O[mb][3];
-        }
-      }
-      named_bar(1, 128);
-#pragma unroll
-      for (int hl = 0; hl < kCombHeads; ++hl) {
-        const int h = kCombHeads * pass + hl;
-        const float M = wsc[NCW * H + h], Ls = wsc[NCW * H + H + h];
-        float o0 = 0.f, o1 = 0.f;
+        for (int w = 0; w < NCW; ++w) M = fmaxf(M, sm.comb_ml[(w * H + ctid) * 2]);
+        float Ls = 0.f;
 #pragma unroll
         for (int w = 0; w < NCW; ++w) {
-          const float sc = wsc[w * H + h];
-          const float2 ov = *reinterpret_cast<const float2*>(sm.comb_o + (w * kCombHeads + hl) * OSTR + 2 * ctid);
-          o0 += sc * ov.x;
-          o1 += sc * ov.y;
+          const float mw = sm.comb_ml[(w * H + ctid) * 2];
+          const float sc = mw == -INFINITY ? 0.f : exp2f(mw - M);
+          wsc[w * H + ctid] = sc;
+          Ls += sc * sm.comb_ml[(w * H + ctid) * 2 + 1];
         }
-        if (full) {
-          const float inv = 1.f / Ls;
-          *reinterpret_cast<float2*>(p.o.out + ((size_t)b * H + h) * R + 2 * ctid) =
-              make_float2(o0 * inv, o1 * inv);
-          if (p.o.lse && ctid == 0) p.o.lse[(size_t)b * H + h] = (M + log2f(Ls)) * 0.69314718055994531f;
-        } else {
-          *reinterpret_cast<float2*>(p.ws_o + ((size_t)nslot * H + h) * R + 2 * ctid) = make_float2(o0, o1);
-          if (ctid == 0) {
-            p.ws_ml[((size_t)nslot * H + h) * 2 + 0] = M;
-            p.ws_ml[((size_t)nslot * H + h) * 2 + 1] = Ls;
+        wsc[NCW * H + ctid] = M;
+        wsc[NCW * H + H + ctid] = Ls;
+      }
+#pragma unroll 1
+      for (int pass = 0; pass < 2; ++pass) {
+        // heads 4 pass .. 4 pass + 3 belong to the lanes with q >> 1 == pass
+        if ((q >> 1) == pass) {
+          const int hl = 2 * q - kCombHeads * pass;  // local head of O[.][0]
+#pragma unroll
+          for (int mb = 0; mb < 16; ++mb) {
+            float* oA = sm.comb_o + (cw * kCombHeads + hl) * OSTR + 16 * mb + g;
+            float* oB = oA + OSTR;
+            oA[0] = O[mb][0];
+            oB[0] = O[mb][1];
+            oA[8] = O[mb][2];
+            oB[8] = O[mb][3];
           }
         }
+        named_bar(1, 128);
+#pragma unroll
+        for (int hl = 0; hl < kCombHeads; ++hl) {
+          const int h = kCombHeads * pass + hl;
+          const float M = wsc[NCW * H + h], Ls = wsc[NCW * H + H + h];
+          float o0 = 0.f, o1 = 0.f;
+#pragma unroll
+          for (int w = 0; w < NCW; ++w) {
+            const float sc = wsc[w * H + h];
+            const float2 ov = *reinterpret_cast<const float2*>(sm.comb_o + (w * kCombHeads + hl) * OSTR + 2 * ctid);
+            o0 += sc * ov.x;
+            o1 += sc * ov.y;
+          }
+          const float inv = 1.f / Ls;
+          *reinterpret_cast<float2*>(p.o.out + ((size_t)b * H + h) * R + 2 * ctid) = make_float2(o0 * inv, o1 * inv);
+          if (p.o.lse && ctid == 0) p.o.lse[(size_t)b * H + h] = (M + log2f(Ls)) * 0.69314718055994531f;
+        }
+        named_bar(1, 128);  // the buffer is rewritten by the next pass / segment
       }
-      named_bar(1, 128);  // the buffer is rewritten by the next pass / segment
+    } else {
+      // part of a split sequence: every warp writes its own part (its rows'
+      // max, sum and unnormalised output per head); no block barrier
+      const int part = NCW * (2 * cta + (b == b_first ? 0 : 1)) + cw;
+      if (g == 0) {
+        float2* pml = reinterpret_cast<float2*>(p.ws_ml) + (size_t)part * H;
+        pml[2 * q] = make_float2(mA, lA);
+        pml[2 * q + 1] = make_float2(mB, lB);
+      }
+      float* po = p.ws_o + (size_t)part * H * R + g;
+#pragma unroll
+      for (int mb = 0; mb < 16; ++mb) {
+        po[(2 * q) * R + 16 * mb] = O[mb][0];
+        po[(2 * q + 1) * R + 16 * mb] = O[mb][1];
+        po[(2 * q) * R + 16 * mb + 8] = O[mb][2];
+        po[(2 * q + 1) * R + 16 * mb + 8] = O[mb][3];
+      }
     }
+    ++seg;
   }
+  // a block with an empty share holds no parts; its slot says so to the combine
+  if (my_lo >= my_hi && ctid < NCW * H)
+    reinterpret_cast<float2*>(p.ws_ml)[(size_t)NCW * 2 * cta * H + ctid] = make_float2(-INFINITY, 0.f);
   if (!ok && ctid == 0) set_err(p.a.dev_err, MTLA_DEVERR_TIMEOUT);
-
 }
 
-// Combine of the sequences split between blocks; one block of 128 threads per
-// sequence.  Launched right after the decode kernel with programmatic
-// dependent launch: its blocks are scheduled early and wait for the decode
-// grid to complete before reading anything.
+// Combine of every sequence's parts and the length bookkeeping.  One block
+// of 256 threads per (sequence, head), thread = latent channel; launched right
+// after the decode kernel with programmatic dependent launch (its blocks wait
+// for the decode grid to complete).  The parts of sequence b are the NCW
+// warps' parts of blocks cf..cl (slot 2c, or 2cf + 1 for block cf when b is
+// not its first sequence).  Per group of up to kGroup parts: their (max, sum)
+// pairs go to shared memory while the first kChunk outputs are already in
+// flight; warp 0 turns the pairs into weights e^{m_i - M}; every thread then
+// sums its channel.  Groups merge online:
+// out = sum_i e^{m_i - M} o_i / sum_i e^{m_i - M} l_i, lse = M + ln(sum).
+constexpr int kGroup = 256, kChunk = 40;
 __global__ void __launch_bounds__(256) decode_combine_kernel(const Params p) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  __shared__ int slots[MAXG];
-  __shared__ float scale[MAXG * H];  // exp2(m_i - M_h) / L_h for every part and head
-  __shared__ float red[32 * H * 2];
-  __shared__ int wsum[8];
-  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  const int4 info = p.seq_info[b];  // rows, merge ok, first block, last block
-  if (tid == 0) {
+  __shared__ float wts[kGroup];  // maxima, then weights
+  __shared__ float lsum[kGroup];
+  __shared__ float red[2];
+  const int b = blockIdx.x / H, h = blockIdx.x % H, c = threadIdx.x;
+  const int4 info = __ldcg(p.seq_info + b);  // rows, merge ok, first block's slot, blocks
+  if (h == 0 && c == 0) {
     if (p.with_merge && info.y) p.a.t_processed[b] = p.a.t_processed[b] + 1;
     if (p.a.cache_len) p.a.cache_len[b] = info.x;
   }
+  float* out = p.o.out + ((size_t)b * H + h) * R;
   if (info.x == 0) {
-    if (tid == 0) set_err(p.a.dev_err, MTLA_DEVERR_EMPTY);
-    for (int i = tid; i < H * R; i += 256) p.o.out[(size_t)b * H * R + i] = 0.f;
-    if (p.o.lse && tid < H) p.o.lse[(size_t)b * H + tid] = -INFINITY;
+    if (h == 0 && c == 0) set_err(p.a.dev_err, MTLA_DEVERR_EMPTY);
+    out[c] = 0.f;
+    if (p.o.lse && c == 0) p.o.lse[(size_t)b * H + h] = -INFINITY;
     return;
   }
-  // the workspace slots of the blocks that hold part of sequence b, in block
-  // order: every candidate block is looked up at once and compacted by ballots
-  const int ncand = info.w - info.z + 1;
-  if (ncand <= 1) return;  // one block held the whole sequence and wrote it
-  int nparts = 0;
-  for (int base = 0; base < ncand; base += 256) {
-    const int t = base + tid;
-    int slot = -1;
-    if (t < ncand) {
-      const int c = info.z + t;
-      const int f = p.fs[c];
-      if (f != p.B) slot = 2 * c + (f == b ? 0 : 1);
-    }
-    const unsigned bal = __ballot_sync(0xffffffffu, slot >= 0);
-    if (lane == 0) wsum[wid] = __popc(bal);
-    __syncthreads();
-    int off = nparts;
-    for (int w = 0; w < wid; ++w) off += wsum[w];
-    if (slot >= 0) slots[off + __popc(bal & ((1u << lane) - 1u))] = slot;
-    for (int w = 0; w < 8; ++w) nparts += wsum[w];
-    __syncthreads();
-  }
-  if (nparts <= 1) return;
-  // phase 1: per head, running (max, sum) over the parts: 32 groups x 8 heads
-  {
-    const int h = tid & 7, grp = tid >> 3;
-    float M = -INFINITY, Ls = 0.f;
-    for (int i = grp; i < nparts; i += 32) {
-      const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.ws_ml) + (size_t)slots[i] * H + h);
-      if (ml.x == -INFINITY) continue;
-      const float nM = fmaxf(M, ml.x);
-      Ls = Ls * exp2f(M - nM) + ml.y * exp2f(ml.x - nM);
-      M = nM;
-    }
-    red[(grp * H + h) * 2 + 0] = M;
-    red[(grp * H + h) * 2 + 1] = Ls;
-  }
-  __syncthreads();
-  if (tid < H) {
-    float M = -INFINITY, Ls = 0.f;
-    for (int grp = 0; grp < 32; ++grp) {
-      const float m = red[(grp * H + tid) * 2], l = red[(grp * H + tid) * 2 + 1];
-      if (m == -INFINITY) continue;
-      const float nM = fmaxf(M, m);
-      Ls = Ls * exp2f(M - nM) + l * exp2f(m - nM);
-      M = nM;
-    }
-    red[tid * 2 + 0] = M;  // group 0's entries are no longer needed
-    red[tid * 2 + 1] = Ls;
-    if (p.o.lse) p.o.lse[(size_t)b * H + tid] = (M + log2f(Ls)) * 0.69314718055994531f;
-  }
-  __syncthreads();
-  for (int i = tid; i < nparts * H; i += 256) {
-    const int part = i / H, h = i % H;
-    const float mc = __ldcg(p.ws_ml + ((size_t)slots[part] * H + h) * 2);
-    scale[i] = mc == -INFINITY ? 0.f : exp2f(mc - red[h * 2]) / red[h * 2 + 1];
-  }
-  __syncthreads();
-  // phase 2: thread -> head tid >> 5, 8 channels; eight parts' loads in flight at a time
-  const int h = tid >> 5, c0 = (tid & 31) * 8;
-  float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
-  for (int i0 = 0; i0 < nparts; i0 += 8) {
-    float4 v0[8], v1[8];
+  if (info.w <= 1) return;  // one block held the whole sequence and wrote it
+  const int nparts = NCW * info.w;
+  const int cf = info.z >> 1;
+  auto part_of = [&](int i) {
+    const int blk = i / NCW;
+    return NCW * (blk == 0 ? info.z : 2 * (cf + blk)) + i % NCW;
+  };
+  float M = -INFINITY, S = 0.f, acc = 0.f;
+  for (int g0 = 0; g0 < nparts; g0 += kGroup) {
+    const int ng = nparts - g0 < kGroup ? nparts - g0 : kGroup;
+    float v[kChunk];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (i0 + u < nparts) {
-        const float4* src = reinterpret_cast<const float4*>(p.ws_o + ((size_t)slots[i0 + u] * H + h) * R + c0);
-        v0[u] = __ldcg(src);
-        v1[u] = __ldcg(src + 1);
+    for (int u = 0; u < kChunk; ++u)
+      v[u] = u < ng ? __ldcg(p.ws_o + ((size_t)part_of(g0 + u) * H + h) * R + c) : 0.f;
+    for (int i = c; i < ng; i += 256) {
+      const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.ws_ml) + (size_t)part_of(g0 + i) * H + h);
+      wts[i] = ml.x;
+      lsum[i] = ml.y;
+    }
+    __syncthreads();
+    if (c < 32) {
+      float Mg = -INFINITY;
+      for (int i = c; i < ng; i += 32) Mg = fmaxf(Mg, wts[i]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) Mg = fmaxf(Mg, __shfl_xor_sync(0xffffffffu, Mg, o));
+      float Sg = 0.f;
+      for (int i = c; i < ng; i += 32) {
+        const float w = wts[i] == -INFINITY ? 0.f : exp2f(wts[i] - Mg);  // a warp without rows weighs 0
+        wts[i] = w;
+        Sg += w * lsum[i];
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) Sg += __shfl_xor_sync(0xffffffffu, Sg, o);
+      if (c == 0) {
+        red[0] = Mg;
+        red[1] = Sg;
       }
     }
+    __syncthreads();
+    float accg = 0.f;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (i0 + u < nparts) {
-        const float sc = scale[(i0 + u) * H + h];
-        acc0.x += sc * v0[u].x; acc0.y += sc * v0[u].y; acc0.z += sc * v0[u].z; acc0.w += sc * v0[u].w;
-        acc1.x += sc * v1[u].x; acc1.y += sc * v1[u].y; acc1.z += sc * v1[u].z; acc1.w += sc * v1[u].w;
-      }
+    for (int u = 0; u < kChunk; ++u)
+      if (u < ng) accg += wts[u] * v[u];
+    for (int i0 = kChunk; i0 < ng; i0 += kChunk) {
+#pragma unroll
+      for (int u = 0; u < kChunk; ++u)
+        v[u] = i0 + u < ng ? __ldcg(p.ws_o + ((size_t)part_of(g0 + i0 + u) * H + h) * R + c) : 0.f;
+#pragma unroll
+      for (int u = 0; u < kChunk; ++u)
+        if (i0 + u < ng) accg += wts[i0 + u] * v[u];
     }
+    // merge this group into the running result
+    const float Mg = red[0], Sg = red[1];
+    const float nM = fmaxf(M, Mg);
+    const float a = exp2f(M - nM), bg = exp2f(Mg - nM);  // a = 0 while M is -inf
+    S = S * a + Sg * bg;
+    acc = acc * a + accg * bg;
+    M = nM;
+    __syncthreads();  // wts / red are rewritten by the next group
   }
-  float4* dst = reinterpret_cast<float4*>(p.o.out + ((size_t)b * H + h) * R + c0);
-  dst[0] = acc0;
-  dst[1] = acc1;
+  out[c] = acc / S;
+  if (p.o.lse && c == 0) p.o.lse[(size_t)b * H + h] = (M + log2f(S)) * 0.69314718055994531f;
 }
 
-// Gate pre-activations g[b][k] = sum_i c_b[i] W_c[i][k] + b_c[k] of the new
-// tokens (Linear(c_t) of the merge).  Block = 32 channels x 8 tokens; warp w
-// takes input rows 32w .. 32w+31 (one coalesced 128-byte segment of W_c per
-// row, all in flight at once), lanes are channels; the eight warps' partial
-// sums are added in a fixed order, so the result is deterministic.
-__global__ void __launch_bounds__(256) decode_gate_kernel(const Params p) {
+// The merge of every sequence's new token (Linear(c_t) of the merge, the gate,
+// the gated entry and the append / in-place update of the tail row), before
+// the decode kernel reads the cache.  Block = 32 channels x 2 tokens, 128
+// threads: warp w takes input rows 64w .. 64w+63 of the gate contraction (its
+// W_c column segments all in flight at once), lanes are channels; the four
+// warps' partial sums are added in a fixed order, so the result is
+// deterministic.  Small on purpose (1 KB of shared memory, few registers): its
+// blocks share SMs with two decode blocks, which start while it runs.  The
+// updated row goes to the cache and to the workspace copy that the decode
+// kernel patches into its tile.
+constexpr int kMergeTok = 2;
+__global__ void __launch_bounds__(128) decode_merge_kernel(const Params p) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  __shared__ float part[8][8][32];
+  __shared__ float part[4][kMergeTok][32];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kt = blockIdx.x % (D / 32), bt = blockIdx.x / (D / 32);
-  const int k = kt * 32 + lane, b0 = bt * 8, i0 = w * 32;
-  float wv[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) wv[i] = __ldg(p.m.W_c + (size_t)(i0 + i) * D + k);
+  const int k = kt * 32 + lane, b0 = bt * kMergeTok, i0 = w * 64;
   const __nv_bfloat16* cn = reinterpret_cast<const __nv_bfloat16*>(p.m.c_new);
-  float cv[8];
+  float acc[kMergeTok];
 #pragma unroll
-  for (int u = 0; u < 8; ++u) cv[u] = b0 + u < p.B ? __bfloat162float(cn[(size_t)(b0 + u) * R + i0 + lane]) : 0.f;
-  float acc[8];
+  for (int u = 0; u < kMergeTok; ++u) acc[u] = 0.f;
 #pragma unroll
-  for (int u = 0; u < 8; ++u) acc[u] = 0.f;
+  for (int half = 0; half < 2; ++half) {
+    const int ib = i0 + 32 * half;
+    float wv[32];
 #pragma unroll
-  for (int i = 0; i < 32; ++i)
+    for (int i = 0; i < 32; ++i) wv[i] = __ldg(p.m.W_c + (size_t)(ib + i) * D + k);
+    float cv[kMergeTok];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) acc[u] = fmaf(__shfl_sync(0xffffffffu, cv[u], i), wv[i], acc[u]);
+    for (int u = 0; u < kMergeTok; ++u)
+      cv[u] = b0 + u < p.B ? __bfloat162float(cn[(size_t)(b0 + u) * R + ib + lane]) : 0.f;
 #pragma unroll
-  for (int u = 0; u < 8; ++u) part[w][u][lane] = acc[u];
+    for (int i = 0; i < 32; ++i)
+#pragma unroll
+      for (int u = 0; u < kMergeTok; ++u) acc[u] = fmaf(__shfl_sync(0xffffffffu, cv[u], i), wv[i], acc[u]);
+  }
+#pragma unroll
+  for (int u = 0; u < kMergeTok; ++u) part[w][u][lane] = acc[u];
   __syncthreads();
+  if (w >= kMergeTok) return;
   const int u = w;  // thread -> token b0 + u, channel k
   float g = 0.f;
 #pragma unroll
-  for (int ww = 0; ww < 8; ++ww) g += part[ww][u][lane];
-  if (b0 + u < p.B) p.gates[(size_t)(b0 + u) * D + k] = g + __ldg(p.m.b_c + k);
+  for (int ww = 0; ww < 4; ++ww) g += part[ww][u][lane];
+  const int b = b0 + u;
+  if (b >= p.B) return;
+  const SeqState st = seq_state(p, b, true);
+  if (!st.merge_ok) return;  // the decode kernel reports why
+  const int s = p.a.s;
+  const int64_t j = group_of(st.t, s);
+  const bool opens = opens_row(st.t, s);
+  __nv_bfloat16* row = reinterpret_cast<__nv_bfloat16*>(p.a.cache) + (p.a.seq_offset[b] + j - 1) * p.a.row_stride;
+  const float gv = g + __ldg(p.m.b_c + k);
+  const float wt = sigmoidf_(__fmul_rn(gv, __ldg(p.m.P + (j - 1) * D + k)));
+  const __nv_bfloat16* xin = k < R ? reinterpret_cast<const __nv_bfloat16*>(p.m.c_new) + (size_t)b * R + k
+                                   : reinterpret_cast<const __nv_bfloat16*>(p.m.kR_new) + (size_t)b * DR + (k - R);
+  const float e = __fmul_rn(wt, __bfloat162float(*xin));
+  const float v = opens ? e : __fadd_rn(__bfloat162float(row[k]), e);
+  const __nv_bfloat16 vb = __float2bfloat16_rn(v);
+  row[k] = vb;
+  p.tails[(size_t)b * D + k] = vb;
 }
 
 int grid_size() {
@@ -745,20 +802,19 @@ cudaError_t launch_decode_tc(const dtc::Params& p, const CUtensorMap& map64, con
   cfg.numAttrs = 1;
   if (p.with_merge) {
     cudaLaunchConfig_t cfg0 = {};
-    cfg0.gridDim = dim3((unsigned)((dtc::D / 32) * ((p.B + 7) / 8)));
-    cfg0.blockDim = dim3(256);
+    cfg0.gridDim = dim3((unsigned)((dtc::D / 32) * ((p.B + dtc::kMergeTok - 1) / dtc::kMergeTok)));
+    cfg0.blockDim = dim3(128);
     cfg0.stream = st;
     cfg0.attrs = attr;
     cfg0.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg0, dtc::decode_gate_kernel, p);
+    e = cudaLaunchKernelEx(&cfg0, dtc::decode_merge_kernel, p);
     if (e != cudaSuccess) return e;
   }
   e = cudaLaunchKernelEx(&cfg, dtc::decode_tc_kernel, map64, map8, p);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg2 = {};
-  cfg2.gridDim = dim3((unsigned)p.B);
+  cfg2.gridDim = dim3((unsigned)(p.B * dtc::H));
   cfg2.blockDim = dim3(256);
-  cfg2.dynamicSmemBytes = 0;
   cfg2.stream = st;
   cfg2.attrs = attr;
   cfg2.numAttrs = 1;

@@ -81,9 +81,8 @@ struct Params {
   int B;
   int merge_cost;
   float scale_log2;     // log2(e) / sqrt(d_h)
-  int4* seq_info;       // [B] {rows, merge ok, first block, last block} for the combine
-  int32_t* fs;          // [grid] first sequence with rows in each block's share (B: none)
-  float* gates;         // [B][D] Linear(c_t) of every new token (gate kernel)
+  int4* seq_info;       // [B] {rows, merge ok, first part slot, part count} for the combine
+  __nv_bfloat16* tails; // [B][D] updated tail row of every merged sequence (merge kernel)
   float* ws_ml;         // [2 * grid][H][2]
   float* ws_o;          // [2 * grid][H][R]
 };
