@@ -59,14 +59,16 @@ constexpr size_t kOffComb = rup((size_t)NS * STAGE);
 constexpr size_t kOffCombMl = kOffComb + rup((size_t)NCW * kCombHeads * OSTR * 4);
 constexpr size_t kOffPrefix = kOffCombMl + rup((size_t)NCW * H * 2 * 4 + (size_t)(NCW + 2) * H * 4);
 constexpr size_t kOffMeta = kOffPrefix + rup((size_t)(MAXB + 1) * 8);
-constexpr size_t kOffScan = kOffMeta + rup((size_t)MAXB * 4);
-constexpr size_t kOffLo = kOffScan + rup(128 * 8);
+constexpr size_t kOffLo = kOffMeta + rup((size_t)MAXB * 4);
 constexpr size_t kOffFs = kOffLo + rup((size_t)(MAXG + 1) * 8);
 constexpr size_t kOffQx = kOffFs + rup((size_t)MAXG * 4);
 constexpr size_t kOffBar = kOffQx + rup((size_t)H * QSTR * 4);
 constexpr size_t kOffFlags = kOffBar + rup(2 * NS * 8);
 constexpr size_t kSmemUsed = kOffFlags + rup(16);
 static_assert(kOffQx % 16 == 0 && kOffBar % 8 == 0, "shared-memory regions must stay aligned");
+static_assert(128 * 8 <= (size_t)NCW * kCombHeads * OSTR * 4, "scan scratch must fit the combine buffer");
+// two decode blocks plus two merge-kernel blocks (1 KB each) fit one SM's 228 KB
+static_assert(2 * (kSmemUsed + 1024 + 1024) + 2 * (1024 + 1024) <= 233472, "shared memory per SM");
 
 size_t smem_bytes() { return kSmemUsed + 1024; }  // + slack to align the base to 1024
 
@@ -114,7 +116,8 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   s.comb_ml = reinterpret_cast<float*>(p + kOffCombMl);
   s.prefix = reinterpret_cast<int64_t*>(p + kOffPrefix);
   s.meta = reinterpret_cast<uint32_t*>(p + kOffMeta);
-  s.scan = reinterpret_cast<int64_t*>(p + kOffScan);
+  // the prologue's scan scratch shares the combine buffer, first used after it
+  s.scan = reinterpret_cast<int64_t*>(p + kOffComb);
   s.lo = reinterpret_cast<int64_t*>(p + kOffLo);
   s.fs = reinterpret_cast<int32_t*>(p + kOffFs);
   s.qx = reinterpret_cast<uint32_t*>(p + kOffQx);
@@ -788,6 +791,15 @@ cudaError_t launch_decode_tc(const dtc::Params& p, const CUtensorMap& map64, con
     e = cudaFuncSetAttribute(dtc::decode_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
+    // the same shared-memory configuration for the kernels around it, so that
+    // an SM running one of their blocks can take decode blocks at once
+    // (changing the configuration waits for the SM to drain)
+    e = cudaFuncSetAttribute(dtc::decode_merge_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(dtc::decode_combine_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
     if (dev < 64) done_mask |= 1ull << dev;
   }
   cudaLaunchAttribute attr[1];
@@ -805,8 +817,10 @@ cudaError_t launch_decode_tc(const dtc::Params& p, const CUtensorMap& map64, con
     cfg0.gridDim = dim3((unsigned)((dtc::D / 32) * ((p.B + dtc::kMergeTok - 1) / dtc::kMergeTok)));
     cfg0.blockDim = dim3(128);
     cfg0.stream = st;
-    cfg0.attrs = attr;
-    cfg0.numAttrs = 1;
+    // plain stream order (no early launch): launched early, its blocks would
+    // pile onto the SMs the previous step's kernels leave free first and keep
+    // decode blocks off them; after the previous step they spread one per SM
+    cfg0.numAttrs = 0;
     e = cudaLaunchKernelEx(&cfg0, dtc::decode_merge_kernel, p);
     if (e != cudaSuccess) return e;
   }
