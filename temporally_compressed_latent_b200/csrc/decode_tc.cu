@@ -149,6 +149,17 @@ __device__ __forceinline__ int64_t rows_of(const uint32_t* meta, int b) {
   return (int64_t)(meta[b] & (kMetaMergeOk - 1));
 }
 
+// Block c's share of the C cost positions starts at c C / G.
+__device__ __forceinline__ int64_t share_start(int c, int64_t C, int G) { return C > 0 ? (int64_t)c * C / G : 0; }
+// The first sequence with rows in the share [lo, hi), B if the share is empty.
+__device__ __forceinline__ int first_seq(const int64_t* prefix, const uint32_t* meta, int B, int64_t lo, int64_t hi) {
+  if (lo >= hi) return B;
+  int b = upper_bound_i64(prefix, B + 1, lo) - 1;
+  if (b < 0) b = 0;
+  if (b < B && lo - prefix[b] >= rows_of(meta, b)) ++b;
+  return b;
+}
+
 // Sequence b after this call: its rows, whether its new token is merged, and
 // the device-error bits the checks raise.  The merge kernel (which writes the
 // tail row) and the decode kernel (which partitions the rows) decide alike.
@@ -253,25 +264,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
       run += rows_of(sm.meta, b) + mcost;
     }
   }
+  named_bar(2, PRO_T);
   const int64_t C = sm.prefix[B];
-  // share starts: block c owns cost positions [lo[c], lo[c+1])
-  for (int c = tid; c <= G; c += PRO_T) sm.lo[c] = C > 0 ? (int64_t)c * C / G : 0;
-  named_bar(2, PRO_T);
-  // first sequence with rows in each share (B if none)
-  for (int c = tid; c < G; c += PRO_T) {
-    const int64_t x = sm.lo[c];
-    int b = upper_bound_i64(sm.prefix, B + 1, x) - 1;
-    if (b < 0) b = 0;
-    if (b < B && x - sm.prefix[b] >= rows_of(sm.meta, b)) ++b;
-    sm.fs[c] = (x < sm.lo[c + 1]) ? b : B;
-  }
-  named_bar(2, PRO_T);
-
-  const int64_t my_lo = sm.lo[cta], my_hi = sm.lo[cta + 1];
-  // the share's sequences, visited last to first so that a sequence's tail
+  // this block's share: cost positions [my_lo, my_hi); its first sequence
+  // with rows (B if none) by the rule block 0 tabulates for every block below
+  const int64_t my_lo = share_start(cta, C, G), my_hi = share_start(cta + 1, C, G);
+  const int b_first = first_seq(sm.prefix, sm.meta, B, my_lo, my_hi);
+  // the share's sequences are visited last to first so that a sequence's tail
   // row (whose merge the merge kernel finishes meanwhile) is the block's last
-  // tile; b_first == B when the share holds no rows
-  const int b_first = sm.fs[cta];
+  // tile
   const int b_last = my_lo < my_hi ? upper_bound_i64(sm.prefix, B + 1, my_hi - 1) - 1 : -1;
   const __nv_bfloat16* cache = reinterpret_cast<const __nv_bfloat16*>(p.a.cache);
 
@@ -361,6 +362,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
   // the number of parts (blocks cf..cl; block c > cf stored its part in slot
   // 2c, block cf in 2cf or 2cf + 1)
   if (cta == 0) {
+    for (int c = ctid; c <= G; c += 128) sm.lo[c] = share_start(c, C, G);
+    named_bar(1, 128);
+    for (int c = ctid; c < G; c += 128) sm.fs[c] = first_seq(sm.prefix, sm.meta, B, sm.lo[c], sm.lo[c + 1]);
+    named_bar(1, 128);
     for (int bb = ctid; bb < B; bb += 128) {
       const int64_t Lb = rows_of(sm.meta, bb);
       const int ok_m = (sm.meta[bb] & kMetaMergeOk) ? 1 : 0;
