@@ -22,10 +22,15 @@
 //    K 64) are tcgen05.mma ops with fp32 accumulators in TMEM (S double-
 //    buffered, O 256 columns), issued by one thread.  Only complete groups up
 //    to the staircase are visited, so no tile is empty.
-//  * Four softmax warps own one (query, head) row each (a TMEM lane): mask,
-//    online softmax with lazy rescaling (O is rescaled in TMEM only when the
-//    running max grows by more than 2^8), bf16 P written 128-byte swizzled for
-//    the value MMA.  The epilogue adds the own-row term and writes bf16 out.
+//  * Eight softmax warps, two per TMEM lane quarter: warps w and w + 4 own
+//    the same 32 (query, head) rows (TMEM lanes) and split the key tile's 64
+//    columns and O's 256 columns between them, so each SMSP runs two of them.
+//    Per tile the pair exchanges row maxima through shared memory (a 64-thread
+//    named barrier) and makes the same lazy-rescale decision (O is rescaled in
+//    TMEM only when the running max grows by more than 2^8); the row sums stay
+//    per half until the epilogue.  Masking, online softmax and bf16 P written
+//    128-byte swizzled for the value MMA.  The epilogue adds the own-row term
+//    and writes bf16 out.
 //  * One TMA warp, one MMA warp, mbarrier pipelines; a persistent grid visits
 //    the M tiles heaviest first.
 #include "kernels.cuh"
@@ -45,25 +50,28 @@ constexpr int QBYTES = NPL * QPL;      // 73728
 constexpr int KBYTES = NPL * KPL;      // 36864
 constexpr int SBYTES = NPL * SPL;      // 9216
 constexpr int PBYTES = BM * BN * 2;    // 16384
-constexpr int KS = 2;                  // key-tile stages
-constexpr int NT = 192;                // 4 softmax warps, TMA warp, MMA warp
-constexpr int TMA_WARP = 4, MMA_WARP = 5;
+constexpr int KS = 3;                  // key-tile stages
+constexpr int SMW = 8;                 // softmax warps: two per TMEM lane quarter
+constexpr int NT = 32 * (SMW + 2);     // + TMA warp, MMA warp
+constexpr int TMA_WARP = SMW, MMA_WARP = SMW + 1;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t S_COL0 = 0, S_COL1 = 64, O_COL = 256;
 constexpr uint32_t IDESC_S = umma_idesc_bf16(BM, BN, false, false);
 constexpr uint32_t IDESC_O = umma_idesc_bf16(BM, R, false, true);
 
 constexpr size_t OFF_Q = 0;
-constexpr size_t OFF_SELF = OFF_Q + QBYTES;            // 2 buffers
-constexpr size_t OFF_K = OFF_SELF + 2 * SBYTES;        // KS stages
+constexpr size_t OFF_SELF = OFF_Q + QBYTES;            // one buffer (read in the epilogue only)
+constexpr size_t OFF_K = OFF_SELF + SBYTES;            // KS stages
 constexpr size_t OFF_P = OFF_K + (size_t)KS * KBYTES;  // 2 buffers
-constexpr size_t OFF_BAR = OFF_P + 2 * PBYTES;
+constexpr size_t OFF_XCH = OFF_P + 2 * PBYTES;        // pair exchange: row maxima, row sums
+constexpr size_t OFF_BAR = OFF_XCH + 2 * 2 * BM * 4 + 2 * 2 * BM * 4;
 constexpr int NBAR = 21;
 constexpr size_t OFF_TMEM = OFF_BAR + NBAR * 8;
 constexpr size_t SMEM_USED = OFF_TMEM + 16;
 static_assert(OFF_K % 1024 == 0 && OFF_P % 1024 == 0 && OFF_SELF % 1024 == 0, "tile bases must be 1024-aligned");
 
 size_t smem_bytes() { return SMEM_USED + 1024; }
+static_assert(SMEM_USED + 1024 <= 232448, "one block's shared memory (227 KB)");
 
 struct Params {
   int B, T, s;
@@ -86,6 +94,14 @@ __device__ __forceinline__ uint32_t plane_off(int rows, int row, int ch) {
 struct Tile {
   int b, m0, nkt;
 };
+// 2^x with the hardware approximation (relative error about 2^-22; results
+// below 2^-126 flush to zero, 2^-inf = 0): the probabilities' exponentials
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // mbarrier wait taken by every lane of a warp, with a warp-uniform result:
 // the tcgen05.ld / st that follow are warp-collective, so no lane may leave
 // the common path on its own
@@ -113,35 +129,37 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
   uint64_t* const q_full = bar + 0;
   uint64_t* const q_empty = bar + 1;
-  uint64_t* const self_full = bar + 2;   // [2]
-  uint64_t* const self_empty = bar + 4;  // [2]
-  uint64_t* const k_full = bar + 6;      // [2]
-  uint64_t* const k_empty = bar + 8;     // [2]
-  uint64_t* const s_full = bar + 10;     // [2]
-  uint64_t* const s_empty = bar + 12;    // [2]
-  uint64_t* const p_full = bar + 14;     // [2]
-  uint64_t* const p_empty = bar + 16;    // [2]
-  uint64_t* const o_full = bar + 18;
-  uint64_t* const o_empty = bar + 19;
-  uint64_t* const mma_done = bar + 20;
+  uint64_t* const self_full = bar + 2;
+  uint64_t* const self_empty = bar + 3;
+  uint64_t* const k_full = bar + 4;             // [KS]
+  uint64_t* const k_empty = bar + 4 + KS;       // [KS]
+  uint64_t* const s_full = bar + 4 + 2 * KS;    // [2]
+  uint64_t* const s_empty = s_full + 2;         // [2]
+  uint64_t* const p_full = s_full + 4;          // [2]
+  uint64_t* const p_empty = s_full + 6;         // [2]
+  uint64_t* const o_full = s_full + 8;
+  uint64_t* const o_empty = s_full + 9;
+  uint64_t* const mma_done = s_full + 10;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
     mbar_init(q_full, 1);
-    mbar_init(q_empty, 4);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&self_full[i], 1);
-      mbar_init(&self_empty[i], 4);
+    mbar_init(q_empty, SMW);
+    mbar_init(self_full, 1);
+    mbar_init(self_empty, SMW);
+    for (int i = 0; i < KS; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 4);
-      mbar_init(&p_full[i], 4);
+      mbar_init(&s_empty[i], SMW);
+      mbar_init(&p_full[i], SMW);
       mbar_init(&p_empty[i], 1);
     }
     mbar_init(o_full, 1);
-    mbar_init(o_empty, 4);
+    mbar_init(o_empty, SMW);
     mbar_init(mma_done, 1);
     fence_mbar_init();
   }
@@ -179,10 +197,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         tma_load_3d(sm + OFF_Q, &qmap, 0, qrow0, 0, q_full);
         tma_load_2d(sm + OFF_Q + 8 * QPL, &rmap, 0, qrow0, q_full);
         q_issued = tc + 1;
-        const int sb = tc & 1;
-        if (tc >= 2 && !mbar_wait(&self_empty[sb], ((tc >> 1) & 1) ^ 1)) { ok = false; break; }
-        mbar_arrive_expect_tx(&self_full[sb], SBYTES);
-        tma_load_3d(sm + OFF_SELF + sb * SBYTES, &smap, 0, crow0, 0, &self_full[sb]);
+        if (tc > 0 && !mbar_wait(self_empty, (tc - 1) & 1)) { ok = false; break; }
+        mbar_arrive_expect_tx(self_full, SBYTES);
+        tma_load_3d(sm + OFF_SELF, &smap, 0, crow0, 0, self_full);
         self_issued = tc + 1;
         for (int kt = 0; kt < t.nkt; ++kt, ++kc) {
           const int st = kc % KS;
@@ -194,8 +211,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       if (!ok) set_err(p.dev_err, MTLA_DEVERR_TIMEOUT);
       // drain: no copy may still be writing shared memory when the block exits
       if (q_issued) mbar_wait(q_full, (q_issued - 1) & 1);
-      for (uint32_t u = self_issued > 2 ? self_issued - 2 : 0; u < self_issued; ++u)
-        mbar_wait(&self_full[u & 1], (u >> 1) & 1);
+      if (self_issued) mbar_wait(self_full, (self_issued - 1) & 1);
       for (uint32_t j = kc > (uint32_t)KS ? kc - KS : 0; j < kc; ++j) mbar_wait(&k_full[j % KS], (j / KS) & 1);
     }
   } else if (warp == MMA_WARP) {
@@ -247,93 +263,106 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     }
   } else {
     // ======================= softmax / epilogue warps =======================
-    const int i = tid;                         // row of the M tile = TMEM lane
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    // warp w: TMEM lane quarter w % 4 (rows 32 (w % 4) .. +31) and half w / 4
+    // of the key tile's 64 columns and of O's 256 columns.  Warps w and w + 4
+    // own the same rows and agree on the running max every tile (64-thread
+    // named barrier per pair; the exchange buffers alternate with the tile, so
+    // neither can overwrite a value its partner has not read).  A wait that
+    // times out only stops further waiting: every warp still takes every pair
+    // barrier, so a pair never waits for a warp that left.
+    const int qw = warp & 3, hf = warp >> 2;
+    const int i = qw * 32 + lane;              // row of the M tile = TMEM lane
+    const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
+    float* xmax = reinterpret_cast<float*>(sm + OFF_XCH);             // [2 parity][2 halves][BM]
+    float* xl = reinterpret_cast<float*>(sm + OFF_XCH + 4 * BM * 4);   // [2 parity][2 halves][BM]
     const float sl2 = p.scale_log2;
     uint32_t tc = 0, kc = 0;
-    for (int o = blockIdx.x; o < p.n_mtiles && ok; o += G, ++tc) {
+    for (int o = blockIdx.x; o < p.n_mtiles; o += G, ++tc) {
       const Tile t = tile_of(p, o);
       const int m = t.m0 + i / H;              // this row's query (1-based)
       const int h = i % H;
       const int vis = (int)group_of(m, p.s) - 1;  // completed groups it sees
-      float m_run = -INFINITY, l = 0.f;
-      for (int kt = 0; kt < t.nkt && ok; ++kt) {
+      float m_run = -INFINITY, l = 0.f;        // l: this half's sum
+      for (int kt = 0; kt < t.nkt; ++kt) {
         const uint32_t j = kc + kt;
         const int sb = j & 1;
-        if (!warp_wait(&s_full[sb], (j >> 1) & 1)) { ok = false; break; }
+        if (ok && !warp_wait(&s_full[sb], (j >> 1) & 1)) ok = false;
         tc_fence_after();
-        uint32_t sr[2][32];
-        tmem_ld32(lane_base + (sb ? S_COL1 : S_COL0), sr[0]);
-        tmem_ld32(lane_base + (sb ? S_COL1 : S_COL0) + 32, sr[1]);
+        uint32_t sr[32];
+        tmem_ld32(lane_base + (sb ? S_COL1 : S_COL0) + 32 * hf, sr);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_empty[sb]);
-        // mask (group kt*BN + c + 1 visible iff <= vis) and scale
-        const int nvis = vis - kt * BN;        // visible columns of this tile
-        float x[64];
-        float mx = -INFINITY;
+        // mask (group kt*BN + 32 hf + c + 1 visible iff <= vis) and scale
+        const int nvis = vis - kt * BN - 32 * hf;
+        float x[32];
+        float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // four independent chains
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          x[c] = c < nvis ? __uint_as_float(sr[c >> 5][c & 31]) * sl2 : -INFINITY;
-          mx = fmaxf(mx, x[c]);
+        for (int c = 0; c < 32; ++c) {
+          x[c] = c < nvis ? __uint_as_float(sr[c]) * sl2 : -INFINITY;
+          mq[c & 3] = fmaxf(mq[c & 3], x[c]);
         }
+        const float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+        xmax[(sb * 2 + hf) * BM + i] = mx;
+        named_bar(1 + qw, 64);
+        const float rmx = fmaxf(mx, xmax[(sb * 2 + (hf ^ 1)) * BM + i]);
         // the running max moves by more than 2^8: rescale l and, once the
-        // previous value MMA has landed, this row of O in TMEM.  The TMEM
-        // accesses are warp-collective, so the whole warp takes the branch
-        // when any of its rows needs it (factor 1 for the others).
-        const bool grow = mx > m_run + 8.f;
+        // previous value MMA has landed, this half of the row of O in TMEM
+        // (warp-collective: the whole warp rescales when any row needs it)
+        const bool grow = rmx > m_run + 8.f;
         const bool resc = grow && m_run != -INFINITY;
         if (kt > 0 && __any_sync(0xffffffffu, resc)) {
           const uint32_t jp = j - 1;
-          if (!warp_wait(&p_empty[jp & 1], (jp >> 1) & 1)) { ok = false; break; }
+          if (ok && !warp_wait(&p_empty[jp & 1], (jp >> 1) & 1)) ok = false;
           tc_fence_after();
-          const float a = resc ? exp2f(m_run - mx) : 1.f;
+          const float a = resc ? exp2f(m_run - rmx) : 1.f;
 #pragma unroll 1
-          for (int ch = 0; ch < R / 32; ++ch) {
+          for (int ch = 0; ch < R / 64; ++ch) {
             uint32_t ov[32];
-            tmem_ld32(lane_base + O_COL + ch * 32, ov);
+            const uint32_t col = O_COL + 128 * hf + 32 * ch;
+            tmem_ld32(lane_base + col, ov);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * a);
-            tmem_st32(lane_base + O_COL + ch * 32, ov);
+            tmem_st32(lane_base + col, ov);
           }
           tmem_wait_st();
           l *= a;
         }
-        if (grow) m_run = mx;
+        if (grow) m_run = rmx;
         // probabilities (relative to the possibly stale max, at most 2^8)
-        uint32_t pk[32];
-        float ls = 0.f;
+        // (a row with nothing visible yet keeps m_run = -inf; its x are all -inf)
+        const float mref = m_run == -INFINITY ? 0.f : m_run;
+        uint32_t pk[16];
+        float lq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float p0 = x[c] == -INFINITY ? 0.f : exp2f(x[c] - m_run);
-          const float p1 = x[c + 1] == -INFINITY ? 0.f : exp2f(x[c + 1] - m_run);
-          ls += p0 + p1;
+        for (int c = 0; c < 32; c += 2) {
+          const float p0 = ex2_approx(x[c] - mref);
+          const float p1 = ex2_approx(x[c + 1] - mref);
+          lq[(c >> 1) & 3] += p0 + p1;
           pk[c >> 1] = pack_bf16x2(p0, p1);
         }
-        l += ls;
-        // P row i of buffer sb (the previous value MMA on this buffer must be done)
-        if (j >= 2 && !warp_wait(&p_empty[sb], ((j >> 1) & 1) ^ 1)) { ok = false; break; }
+        l += (lq[0] + lq[1]) + (lq[2] + lq[3]);
+        // this half of P row i (the previous value MMA on this buffer must be done)
+        if (j >= 2 && ok && !warp_wait(&p_empty[sb], ((j >> 1) & 1) ^ 1)) ok = false;
         const uint32_t prow = sP + sb * PBYTES + i * 128;
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const uint32_t a = prow + ((uint32_t)(ch ^ (i & 7)) << 4);
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[4 * ch]), "r"(pk[4 * ch + 1]),
-                       "r"(pk[4 * ch + 2]), "r"(pk[4 * ch + 3]) : "memory");
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint32_t a = prow + ((uint32_t)((4 * hf + q4) ^ (i & 7)) << 4);
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[4 * q4]), "r"(pk[4 * q4 + 1]),
+                       "r"(pk[4 * q4 + 2]), "r"(pk[4 * q4 + 3]) : "memory");
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[sb]);
       }
-      if (!ok) break;
       // ---- epilogue: own partial row C_hat'_m, then out = normalised (O + own term)
-      const int sbuf = tc & 1;
-      if (!warp_wait(&self_full[sbuf], (tc >> 1) & 1)) { ok = false; break; }
-      const uint32_t selfb = sSelf + sbuf * SBYTES;
+      if (ok && !warp_wait(self_full, tc & 1)) ok = false;
+      const uint32_t selfb = sSelf;
       const int srow = i / H;
-      float dot = 0.f;
+      float dot = 0.f;                         // all 288 dimensions, in both warps of the pair
 #pragma unroll 4
       for (int ch = 0; ch < D / 8; ++ch) {
         uint32_t qv[4], cv[4];
@@ -349,18 +378,22 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           dot = fmaf(a.y, c.y, dot);
         }
       }
+      xl[((tc & 1) * 2 + hf) * BM + i] = l;
       __syncwarp();
-      if (lane == 0) mbar_arrive(q_empty);  // the query tile is no longer read
+      if (lane == 0) mbar_arrive(q_empty);  // this warp no longer reads the query tile
+      named_bar(1 + qw, 64);
       const float xs = dot * sl2;
+      const float lt = xl[((tc & 1) * 2 + 0) * BM + i] + xl[((tc & 1) * 2 + 1) * BM + i];
       const float mf = fmaxf(m_run, xs);
       const float alpha = m_run == -INFINITY ? 0.f : exp2f(m_run - mf);
       const float pself = exp2f(xs - mf);
-      const float inv = 1.f / (l * alpha + pself);
-      if (!warp_wait(o_full, tc & 1)) { ok = false; break; }
+      const float inv = 1.f / (lt * alpha + pself);
+      if (ok && !warp_wait(o_full, tc & 1)) ok = false;
       tc_fence_after();
       __nv_bfloat16* orow = p.out + ((size_t)(t.b * p.T + (m - 1)) * H + h) * R;
 #pragma unroll 1
-      for (int ch = 0; ch < R / 32; ++ch) {
+      for (int cc = 0; cc < R / 64; ++cc) {
+        const int ch = 4 * hf + cc;            // 32-channel chunk of this half
         uint32_t ov[32];
         if (t.nkt > 0) {
           tmem_ld32(lane_base + O_COL + ch * 32, ov);
@@ -392,7 +425,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(o_empty);
-        mbar_arrive(&self_empty[sbuf]);
+        mbar_arrive(self_empty);
       }
       kc += t.nkt;
     }
