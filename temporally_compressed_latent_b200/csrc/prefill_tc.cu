@@ -19,18 +19,20 @@
 //    operand layout for the score MMA and, for the latent planes, the
 //    MN-major operand layout for the value MMA (the key tile is also V).
 //  * Scores S = Q K^T (M 128, N 64, K 288) and values O += P V (M 128, N 256,
-//    K 64) are tcgen05.mma ops with fp32 accumulators in TMEM (S double-
-//    buffered, O 256 columns), issued by one thread.  Only complete groups up
-//    to the staircase are visited, so no tile is empty.
+//    K 64) are tcgen05.mma ops with fp32 accumulators in TMEM (three 64-column
+//    S / P buffers, O 256 columns), issued by one thread, the scores of tile
+//    j + 1 ahead of the values of tile j.  Only complete groups up to the
+//    staircase are visited, so no tile is empty.
 //  * Eight softmax warps, two per TMEM lane quarter: warps w and w + 4 own
 //    the same 32 (query, head) rows (TMEM lanes) and split the key tile's 64
 //    columns and O's 256 columns between them, so each SMSP runs two of them.
 //    Per tile the pair exchanges row maxima through shared memory (a 64-thread
 //    named barrier) and makes the same lazy-rescale decision (O is rescaled in
 //    TMEM only when the running max grows by more than 2^8); the row sums stay
-//    per half until the epilogue.  Masking, online softmax and bf16 P written
-//    128-byte swizzled for the value MMA.  The epilogue adds the own-row term
-//    and writes bf16 out.
+//    per half until the epilogue.  Masking, online softmax, and bf16 P written
+//    back into the tile's S columns of TMEM (tcgen05.st), from where the value
+//    MMA reads it as its A operand: no shared-memory round trip and no proxy
+//    fence.  The epilogue adds the own-row term and writes bf16 out.
 //  * One TMA warp, one MMA warp, mbarrier pipelines; a persistent grid visits
 //    the M tiles heaviest first.
 #include "kernels.cuh"
@@ -49,26 +51,27 @@ constexpr int SPL = QM * 64;           // bytes of one own-row plane (1024)
 constexpr int QBYTES = NPL * QPL;      // 73728
 constexpr int KBYTES = NPL * KPL;      // 36864
 constexpr int SBYTES = NPL * SPL;      // 9216
-constexpr int PBYTES = BM * BN * 2;    // 16384
 constexpr int KS = 3;                  // key-tile stages
 constexpr int SMW = 8;                 // softmax warps: two per TMEM lane quarter
 constexpr int NT = 32 * (SMW + 2);     // + TMA warp, MMA warp
 constexpr int TMA_WARP = SMW, MMA_WARP = SMW + 1;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t S_COL0 = 0, S_COL1 = 64, O_COL = 256;
+constexpr int NSB = 3;                 // S / P buffers in TMEM (64 columns each)
+constexpr uint32_t O_COL = 256;
+__host__ __device__ constexpr uint32_t s_col(int b) { return 64u * (uint32_t)b; }
+static_assert(NSB * 64 <= (int)O_COL, "S buffers below O");
 constexpr uint32_t IDESC_S = umma_idesc_bf16(BM, BN, false, false);
 constexpr uint32_t IDESC_O = umma_idesc_bf16(BM, R, false, true);
 
 constexpr size_t OFF_Q = 0;
 constexpr size_t OFF_SELF = OFF_Q + QBYTES;            // one buffer (read in the epilogue only)
 constexpr size_t OFF_K = OFF_SELF + SBYTES;            // KS stages
-constexpr size_t OFF_P = OFF_K + (size_t)KS * KBYTES;  // 2 buffers
-constexpr size_t OFF_XCH = OFF_P + 2 * PBYTES;        // pair exchange: row maxima, row sums
+constexpr size_t OFF_XCH = OFF_K + (size_t)KS * KBYTES;  // pair exchange: row maxima, row sums
 constexpr size_t OFF_BAR = OFF_XCH + 2 * 2 * BM * 4 + 2 * 2 * BM * 4;
-constexpr int NBAR = 21;
+constexpr int NBAR = 4 + 2 * KS + 4 * NSB + 3;
 constexpr size_t OFF_TMEM = OFF_BAR + NBAR * 8;
 constexpr size_t SMEM_USED = OFF_TMEM + 16;
-static_assert(OFF_K % 1024 == 0 && OFF_P % 1024 == 0 && OFF_SELF % 1024 == 0, "tile bases must be 1024-aligned");
+static_assert(OFF_K % 1024 == 0 && OFF_SELF % 1024 == 0, "tile bases must be 1024-aligned");
 
 size_t smem_bytes() { return SMEM_USED + 1024; }
 static_assert(SMEM_USED + 1024 <= 232448, "one block's shared memory (227 KB)");
@@ -102,6 +105,24 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// 16 consecutive 32-bit TMEM columns of this thread's lane
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+      "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+// D (TMEM) (+)= A (TMEM: lane = row, two bf16 of K per 32-bit column) x B (shared memory)
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.u32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
 // mbarrier wait taken by every lane of a warp, with a warp-uniform result:
 // the tcgen05.ld / st that follow are warp-collective, so no lane may leave
 // the common path on its own
@@ -133,13 +154,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   uint64_t* const self_empty = bar + 3;
   uint64_t* const k_full = bar + 4;             // [KS]
   uint64_t* const k_empty = bar + 4 + KS;       // [KS]
-  uint64_t* const s_full = bar + 4 + 2 * KS;    // [2]
-  uint64_t* const s_empty = s_full + 2;         // [2]
-  uint64_t* const p_full = s_full + 4;          // [2]
-  uint64_t* const p_empty = s_full + 6;         // [2]
-  uint64_t* const o_full = s_full + 8;
-  uint64_t* const o_empty = s_full + 9;
-  uint64_t* const mma_done = s_full + 10;
+  uint64_t* const s_full = bar + 4 + 2 * KS;    // [NSB]
+  uint64_t* const s_empty = s_full + NSB;       // [NSB]
+  uint64_t* const p_full = s_full + 2 * NSB;    // [NSB]
+  uint64_t* const p_empty = s_full + 3 * NSB;   // [NSB]
+  uint64_t* const o_full = s_full + 4 * NSB;
+  uint64_t* const o_empty = o_full + 1;
+  uint64_t* const mma_done = o_full + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -152,7 +173,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NSB; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_empty[i], SMW);
       mbar_init(&p_full[i], SMW);
@@ -180,7 +201,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   const uint32_t sQ = smem_u32(sm + OFF_Q);
   const uint32_t sSelf = smem_u32(sm + OFF_SELF);
   const uint32_t sK = smem_u32(sm + OFF_K);
-  const uint32_t sP = smem_u32(sm + OFF_P);
   const int G = gridDim.x;
   bool ok = true;
 
@@ -217,37 +237,45 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   } else if (warp == MMA_WARP) {
     // ======================= MMA issuer =======================
     if (lane == 0) {
+      // operand descriptors are built once; a K step or a stage moves only the
+      // 14-bit start-address field (shared addresses are below 2^18, no carry)
+      const uint64_t dq0 = umma_desc(sQ, 16, 512, 4);
+      const uint64_t dk0 = umma_desc(sK, 16, 512, 4);
+      const uint64_t dv0 = umma_desc(sK, KPL, 512, 4);
       uint32_t tc = 0, kc = 0;
       for (int o = blockIdx.x; o < p.n_mtiles && ok; o += G, ++tc) {
         const Tile t = tile_of(p, o);
         if (!mbar_wait(q_full, tc & 1)) { ok = false; break; }
         tc_fence_after();
+        // value MMA of key tile j (the kt-th of this M tile): O += P V, P from
+        // TMEM over the tile's S columns, V = the latent planes of its key tile
         auto issue_pv = [&](uint32_t j, int kt) {
-          const int pb = j & 1, st = j % KS;
-          if (!mbar_wait(&p_full[pb], (j >> 1) & 1)) ok = false;
+          const int pb = j % NSB, st = j % KS;
+          if (!mbar_wait(&p_full[pb], (j / NSB) & 1)) ok = false;
           if (kt == 0 && tc > 0 && !mbar_wait(o_empty, (tc - 1) & 1)) ok = false;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint64_t ad = umma_desc(sP + pb * PBYTES + kk * 32, 16, 1024, 2);
-            const uint64_t bd = umma_desc(sK + st * KBYTES + kk * 16 * 64, KPL, 512, 4);
-            umma_bf16(tmem + O_COL, ad, bd, IDESC_O, (kt > 0 || kk > 0) ? 1u : 0u);
+            const uint32_t pa = tmem + s_col(pb) + 8 * kk;  // two bf16 per column: 8 columns per K step
+            const uint64_t bd = dv0 + (uint64_t)((st * KBYTES + kk * 16 * 64) >> 4);
+            umma_bf16_ts(tmem + O_COL, pa, bd, IDESC_O, (kt > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&k_empty[st]);
           umma_commit(&p_empty[pb]);
         };
+        // scores of key tile j are issued one tile ahead of its value MMA, so
+        // the tensor core has the next scores while the softmax works
         for (int kt = 0; kt < t.nkt && ok; ++kt) {
           const uint32_t j = kc + kt;
-          const int st = j % KS, sb = j & 1;
+          const int st = j % KS, sb = j % NSB;
           if (!mbar_wait(&k_full[st], (j / KS) & 1)) { ok = false; break; }
-          if (j >= 2 && !mbar_wait(&s_empty[sb], ((j >> 1) & 1) ^ 1)) { ok = false; break; }
+          if (j >= NSB && !mbar_wait(&s_empty[sb], ((j / NSB) & 1) ^ 1)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t scol = sb ? S_COL1 : S_COL0;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t ad = umma_desc(sQ + (kk >> 1) * QPL + (kk & 1) * 32, 16, 512, 4);
-            const uint64_t bd = umma_desc(sK + st * KBYTES + (kk >> 1) * KPL + (kk & 1) * 32, 16, 512, 4);
-            umma_bf16(tmem + scol, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+            const uint64_t ad = dq0 + (uint64_t)(((kk >> 1) * QPL + (kk & 1) * 32) >> 4);
+            const uint64_t bd = dk0 + (uint64_t)((st * KBYTES + (kk >> 1) * KPL + (kk & 1) * 32) >> 4);
+            umma_bf16(tmem + s_col(sb), ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
           }
           umma_commit(&s_full[sb]);
           if (kt >= 1) issue_pv(j - 1, kt - 1);
@@ -285,11 +313,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       float m_run = -INFINITY, l = 0.f;        // l: this half's sum
       for (int kt = 0; kt < t.nkt; ++kt) {
         const uint32_t j = kc + kt;
-        const int sb = j & 1;
-        if (ok && !warp_wait(&s_full[sb], (j >> 1) & 1)) ok = false;
+        const int sb = j % NSB, xb = j & 1;    // TMEM buffer; exchange-buffer parity
+        if (ok && !warp_wait(&s_full[sb], (j / NSB) & 1)) ok = false;
         tc_fence_after();
         uint32_t sr[32];
-        tmem_ld32(lane_base + (sb ? S_COL1 : S_COL0) + 32 * hf, sr);
+        tmem_ld32(lane_base + s_col(sb) + 32 * hf, sr);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
@@ -304,9 +332,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           mq[c & 3] = fmaxf(mq[c & 3], x[c]);
         }
         const float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
-        xmax[(sb * 2 + hf) * BM + i] = mx;
+        xmax[(xb * 2 + hf) * BM + i] = mx;
+        tc_fence_before();
         named_bar(1 + qw, 64);
-        const float rmx = fmaxf(mx, xmax[(sb * 2 + (hf ^ 1)) * BM + i]);
+        tc_fence_after();
+        const float rmx = fmaxf(mx, xmax[(xb * 2 + (hf ^ 1)) * BM + i]);
         // the running max moves by more than 2^8: rescale l and, once the
         // previous value MMA has landed, this half of the row of O in TMEM
         // (warp-collective: the whole warp rescales when any row needs it)
@@ -314,7 +344,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         const bool resc = grow && m_run != -INFINITY;
         if (kt > 0 && __any_sync(0xffffffffu, resc)) {
           const uint32_t jp = j - 1;
-          if (ok && !warp_wait(&p_empty[jp & 1], (jp >> 1) & 1)) ok = false;
+          if (ok && !warp_wait(&p_empty[jp % NSB], (jp / NSB) & 1)) ok = false;
           tc_fence_after();
           const float a = resc ? exp2f(m_run - rmx) : 1.f;
 #pragma unroll 1
@@ -344,16 +374,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           pk[c >> 1] = pack_bf16x2(p0, p1);
         }
         l += (lq[0] + lq[1]) + (lq[2] + lq[3]);
-        // this half of P row i (the previous value MMA on this buffer must be done)
-        if (j >= 2 && ok && !warp_wait(&p_empty[sb], ((j >> 1) & 1) ^ 1)) ok = false;
-        const uint32_t prow = sP + sb * PBYTES + i * 128;
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const uint32_t a = prow + ((uint32_t)((4 * hf + q4) ^ (i & 7)) << 4);
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[4 * q4]), "r"(pk[4 * q4 + 1]),
-                       "r"(pk[4 * q4 + 2]), "r"(pk[4 * q4 + 3]) : "memory");
-        }
-        fence_proxy_async_smem();
+        // this half of P row i into TMEM over the tile's S columns (both halves'
+        // S are loaded: the pair barrier above), bf16 pairs, for the value MMA
+        tmem_st16(lane_base + s_col(sb) + 16 * hf, pk);
+        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[sb]);
