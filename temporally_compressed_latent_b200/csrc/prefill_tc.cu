@@ -34,7 +34,7 @@
 //    MMA reads it as its A operand: no shared-memory round trip and no proxy
 //    fence.  The epilogue adds the own-row term and writes bf16 out.
 //  * One TMA warp, one MMA warp, mbarrier pipelines; a persistent grid visits
-//    the M tiles heaviest first.
+//    the M tiles heaviest first, in rounds of alternating direction.
 #include "kernels.cuh"
 
 namespace mtla {
@@ -130,6 +130,12 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity));
 }
 
+// M tile that block x takes in its round r: tiles are numbered heaviest
+// first and the rounds alternate direction (x, then G - 1 - x), so each block
+// gets a heavy and a light tile in turn and all blocks end close together;
+// increasing in r for every block
+__device__ __forceinline__ int tile_index(int r, int x, int G) { return r * G + ((r & 1) ? G - 1 - x : x); }
+
 __device__ __forceinline__ Tile tile_of(const Params& p, int o) {
   const int per_seq = p.T / QM;
   Tile t;
@@ -208,7 +214,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     // ======================= TMA producer =======================
     if (lane == 0) {
       uint32_t tc = 0, kc = 0, q_issued = 0, self_issued = 0;
-      for (int o = blockIdx.x; o < p.n_mtiles && ok; o += G, ++tc) {
+      for (int o; (o = tile_index(tc, blockIdx.x, G)) < p.n_mtiles && ok; ++tc) {
         const Tile t = tile_of(p, o);
         const int qrow0 = ((t.b * p.T) + (t.m0 - 1)) * H;  // first row of [B*T*H, .]
         const int crow0 = t.b * p.T + (t.m0 - 1);         // first own row of [B*T, .]
@@ -243,7 +249,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       const uint64_t dk0 = umma_desc(sK, 16, 512, 4);
       const uint64_t dv0 = umma_desc(sK, KPL, 512, 4);
       uint32_t tc = 0, kc = 0;
-      for (int o = blockIdx.x; o < p.n_mtiles && ok; o += G, ++tc) {
+      for (int o; (o = tile_index(tc, blockIdx.x, G)) < p.n_mtiles && ok; ++tc) {
         const Tile t = tile_of(p, o);
         if (!mbar_wait(q_full, tc & 1)) { ok = false; break; }
         tc_fence_after();
@@ -305,7 +311,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     float* xl = reinterpret_cast<float*>(sm + OFF_XCH + 4 * BM * 4);   // [2 parity][2 halves][BM]
     const float sl2 = p.scale_log2;
     uint32_t tc = 0, kc = 0;
-    for (int o = blockIdx.x; o < p.n_mtiles; o += G, ++tc) {
+    for (int o; (o = tile_index(tc, blockIdx.x, G)) < p.n_mtiles; ++tc) {
       const Tile t = tile_of(p, o);
       const int m = t.m0 + i / H;              // this row's query (1-based)
       const int h = i % H;
