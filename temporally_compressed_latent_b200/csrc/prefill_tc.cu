@@ -18,6 +18,8 @@
 //    nine [rows x 64 B] planes with the 64-byte swizzle: the canonical K-major
 //    operand layout for the score MMA and, for the latent planes, the
 //    MN-major operand layout for the value MMA (the key tile is also V).
+//    The own rows are read from global memory (L1 / L2): four key stages fill
+//    the shared memory that a copy of them would take.
 //  * Scores S = Q K^T (M 128, N 64, K 288) and values O += P V (M 128, N 256,
 //    K 64) are tcgen05.mma ops with fp32 accumulators in TMEM (three 64-column
 //    S / P buffers, O 256 columns), issued by one thread, the scores of tile
@@ -29,7 +31,9 @@
 //    Per tile the pair exchanges row maxima through shared memory (a 64-thread
 //    named barrier) and makes the same lazy-rescale decision (O is rescaled in
 //    TMEM only when the running max grows by more than 2^8); the row sums stay
-//    per half until the epilogue.  Masking, online softmax, and bf16 P written
+//    per half until the epilogue.  The own-row score is taken when the M tile
+//    starts, so the query tile is free for the next M tile as soon as its last
+//    score MMA completes.  Masking, online softmax, and bf16 P written
 //    back into the tile's S columns of TMEM (tcgen05.st), from where the value
 //    MMA reads it as its A operand: no shared-memory round trip and no proxy
 //    fence.  The epilogue adds the own-row term and writes bf16 out.
@@ -47,11 +51,9 @@ constexpr int BN = 64;                 // groups per key tile
 constexpr int NPL = D / 32;            // 9 planes of 32 elements
 constexpr int QPL = BM * 64;           // bytes of one query plane (8192)
 constexpr int KPL = BN * 64;           // bytes of one key plane (4096)
-constexpr int SPL = QM * 64;           // bytes of one own-row plane (1024)
 constexpr int QBYTES = NPL * QPL;      // 73728
 constexpr int KBYTES = NPL * KPL;      // 36864
-constexpr int SBYTES = NPL * SPL;      // 9216
-constexpr int KS = 3;                  // key-tile stages
+constexpr int KS = 4;                  // key-tile stages
 constexpr int SMW = 8;                 // softmax warps: two per TMEM lane quarter
 constexpr int NT = 32 * (SMW + 2);     // + TMA warp, MMA warp
 constexpr int TMA_WARP = SMW, MMA_WARP = SMW + 1;
@@ -64,14 +66,13 @@ constexpr uint32_t IDESC_S = umma_idesc_bf16(BM, BN, false, false);
 constexpr uint32_t IDESC_O = umma_idesc_bf16(BM, R, false, true);
 
 constexpr size_t OFF_Q = 0;
-constexpr size_t OFF_SELF = OFF_Q + QBYTES;            // one buffer (read in the epilogue only)
-constexpr size_t OFF_K = OFF_SELF + SBYTES;            // KS stages
+constexpr size_t OFF_K = OFF_Q + QBYTES;               // KS stages
 constexpr size_t OFF_XCH = OFF_K + (size_t)KS * KBYTES;  // pair exchange: row maxima, row sums
-constexpr size_t OFF_BAR = OFF_XCH + 2 * 2 * BM * 4 + 2 * 2 * BM * 4;
-constexpr int NBAR = 4 + 2 * KS + 4 * NSB + 3;
+constexpr size_t OFF_BAR = OFF_XCH + 2 * 2 * BM * 4 + 2 * 2 * BM * 8;
+constexpr int NBAR = 2 + 2 * KS + 4 * NSB + 3;
 constexpr size_t OFF_TMEM = OFF_BAR + NBAR * 8;
 constexpr size_t SMEM_USED = OFF_TMEM + 16;
-static_assert(OFF_K % 1024 == 0 && OFF_SELF % 1024 == 0, "tile bases must be 1024-aligned");
+static_assert(OFF_K % 1024 == 0, "tile bases must be 1024-aligned");
 
 size_t smem_bytes() { return SMEM_USED + 1024; }
 static_assert(SMEM_USED + 1024 <= 232448, "one block's shared memory (227 KB)");
@@ -81,6 +82,7 @@ struct Params {
   int n_mtiles;            // B * T / QM
   int n_groups;            // complete groups per sequence, floor(T / s)
   float scale_log2;        // log2(e) / sqrt(d_h)
+  const __nv_bfloat16* c_partial;  // [B, T, D]: the own rows C_hat'_m
   __nv_bfloat16* out;      // [B, T, H, R]
   int32_t* dev_err;
 };
@@ -149,18 +151,15 @@ __device__ __forceinline__ Tile tile_of(const Params& p, int o) {
 
 __global__ void __launch_bounds__(NT, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap rmap,
-                  const __grid_constant__ CUtensorMap smap, const __grid_constant__ CUtensorMap kmap,
-                  const Params p) {
+                  const __grid_constant__ CUtensorMap kmap, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
   uint64_t* const q_full = bar + 0;
-  uint64_t* const q_empty = bar + 1;
-  uint64_t* const self_full = bar + 2;
-  uint64_t* const self_empty = bar + 3;
-  uint64_t* const k_full = bar + 4;             // [KS]
-  uint64_t* const k_empty = bar + 4 + KS;       // [KS]
-  uint64_t* const s_full = bar + 4 + 2 * KS;    // [NSB]
+  uint64_t* const q_empty = bar + 1;            // the last score MMA + every softmax warp's own-row score
+  uint64_t* const k_full = bar + 2;             // [KS]
+  uint64_t* const k_empty = bar + 2 + KS;       // [KS]
+  uint64_t* const s_full = bar + 2 + 2 * KS;    // [NSB]
   uint64_t* const s_empty = s_full + NSB;       // [NSB]
   uint64_t* const p_full = s_full + 2 * NSB;    // [NSB]
   uint64_t* const p_empty = s_full + 3 * NSB;   // [NSB]
@@ -172,9 +171,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 
   if (tid == 0) {
     mbar_init(q_full, 1);
-    mbar_init(q_empty, SMW);
-    mbar_init(self_full, 1);
-    mbar_init(self_empty, SMW);
+    mbar_init(q_empty, SMW + 1);
     for (int i = 0; i < KS; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
@@ -197,7 +194,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   if (warp == TMA_WARP && lane == 0) {
     prefetch_tmap(&qmap);
     prefetch_tmap(&rmap);
-    prefetch_tmap(&smap);
     prefetch_tmap(&kmap);
   }
   tc_fence_before();
@@ -205,7 +201,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const uint32_t sQ = smem_u32(sm + OFF_Q);
-  const uint32_t sSelf = smem_u32(sm + OFF_SELF);
   const uint32_t sK = smem_u32(sm + OFF_K);
   const int G = gridDim.x;
   bool ok = true;
@@ -213,20 +208,15 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   if (warp == TMA_WARP) {
     // ======================= TMA producer =======================
     if (lane == 0) {
-      uint32_t tc = 0, kc = 0, q_issued = 0, self_issued = 0;
+      uint32_t tc = 0, kc = 0, q_issued = 0;
       for (int o; (o = tile_index(tc, blockIdx.x, G)) < p.n_mtiles && ok; ++tc) {
         const Tile t = tile_of(p, o);
         const int qrow0 = ((t.b * p.T) + (t.m0 - 1)) * H;  // first row of [B*T*H, .]
-        const int crow0 = t.b * p.T + (t.m0 - 1);         // first own row of [B*T, .]
         if (tc > 0 && !mbar_wait(q_empty, (tc - 1) & 1)) { ok = false; break; }
         mbar_arrive_expect_tx(q_full, QBYTES);
         tma_load_3d(sm + OFF_Q, &qmap, 0, qrow0, 0, q_full);
         tma_load_2d(sm + OFF_Q + 8 * QPL, &rmap, 0, qrow0, q_full);
         q_issued = tc + 1;
-        if (tc > 0 && !mbar_wait(self_empty, (tc - 1) & 1)) { ok = false; break; }
-        mbar_arrive_expect_tx(self_full, SBYTES);
-        tma_load_3d(sm + OFF_SELF, &smap, 0, crow0, 0, self_full);
-        self_issued = tc + 1;
         for (int kt = 0; kt < t.nkt; ++kt, ++kc) {
           const int st = kc % KS;
           if (kc >= KS && !mbar_wait(&k_empty[st], ((kc / KS) & 1) ^ 1)) { ok = false; break; }
@@ -237,29 +227,30 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       if (!ok) set_err(p.dev_err, MTLA_DEVERR_TIMEOUT);
       // drain: no copy may still be writing shared memory when the block exits
       if (q_issued) mbar_wait(q_full, (q_issued - 1) & 1);
-      if (self_issued) mbar_wait(self_full, (self_issued - 1) & 1);
       for (uint32_t j = kc > (uint32_t)KS ? kc - KS : 0; j < kc; ++j) mbar_wait(&k_full[j % KS], (j / KS) & 1);
     }
   } else if (warp == MMA_WARP) {
     // ======================= MMA issuer =======================
-    if (lane == 0) {
-      // operand descriptors are built once; a K step or a stage moves only the
-      // 14-bit start-address field (shared addresses are below 2^18, no carry)
-      const uint64_t dq0 = umma_desc(sQ, 16, 512, 4);
-      const uint64_t dk0 = umma_desc(sK, 16, 512, 4);
-      const uint64_t dv0 = umma_desc(sK, KPL, 512, 4);
-      uint32_t tc = 0, kc = 0;
-      for (int o; (o = tile_index(tc, blockIdx.x, G)) < p.n_mtiles && ok; ++tc) {
-        const Tile t = tile_of(p, o);
-        if (!mbar_wait(q_full, tc & 1)) { ok = false; break; }
+    // The whole warp runs the loop, so every operand is warp-uniform; one
+    // elected lane issues each group of MMAs and the commits that track it.
+    // Operand descriptors are built once; a K step or a stage moves only the
+    // 14-bit start-address field (shared addresses are below 2^18, no carry).
+    const uint64_t dq0 = umma_desc(sQ, 16, 512, 4);
+    const uint64_t dk0 = umma_desc(sK, 16, 512, 4);
+    const uint64_t dv0 = umma_desc(sK, KPL, 512, 4);
+    uint32_t tc = 0, kc = 0;
+    for (int o; (o = tile_index(tc, blockIdx.x, G)) < p.n_mtiles && ok; ++tc) {
+      const Tile t = tile_of(p, o);
+      if (!warp_wait(q_full, tc & 1)) { ok = false; break; }
+      tc_fence_after();
+      // value MMA of key tile j (the kt-th of this M tile): O += P V, P from
+      // TMEM over the tile's S columns, V = the latent planes of its key tile
+      auto issue_pv = [&](uint32_t j, int kt) {
+        const int pb = j % NSB, st = j % KS;
+        if (!warp_wait(&p_full[pb], (j / NSB) & 1)) ok = false;
+        if (kt == 0 && tc > 0 && !warp_wait(o_empty, (tc - 1) & 1)) ok = false;
         tc_fence_after();
-        // value MMA of key tile j (the kt-th of this M tile): O += P V, P from
-        // TMEM over the tile's S columns, V = the latent planes of its key tile
-        auto issue_pv = [&](uint32_t j, int kt) {
-          const int pb = j % NSB, st = j % KS;
-          if (!mbar_wait(&p_full[pb], (j / NSB) & 1)) ok = false;
-          if (kt == 0 && tc > 0 && !mbar_wait(o_empty, (tc - 1) & 1)) ok = false;
-          tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {
             const uint32_t pa = tmem + s_col(pb) + 8 * kk;  // two bf16 per column: 8 columns per K step
@@ -268,15 +259,18 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           }
           umma_commit(&k_empty[st]);
           umma_commit(&p_empty[pb]);
-        };
-        // scores of key tile j are issued one tile ahead of its value MMA, so
-        // the tensor core has the next scores while the softmax works
-        for (int kt = 0; kt < t.nkt && ok; ++kt) {
-          const uint32_t j = kc + kt;
-          const int st = j % KS, sb = j % NSB;
-          if (!mbar_wait(&k_full[st], (j / KS) & 1)) { ok = false; break; }
-          if (j >= NSB && !mbar_wait(&s_empty[sb], ((j / NSB) & 1) ^ 1)) { ok = false; break; }
-          tc_fence_after();
+        }
+        __syncwarp();
+      };
+      // scores of key tile j + 1 are issued ahead of the values of tile j, so
+      // the tensor core has the next scores while the softmax works
+      for (int kt = 0; kt < t.nkt && ok; ++kt) {
+        const uint32_t j = kc + kt;
+        const int st = j % KS, sb = j % NSB;
+        if (!warp_wait(&k_full[st], (j / KS) & 1)) { ok = false; break; }
+        if (j >= NSB && !warp_wait(&s_empty[sb], ((j / NSB) & 1) ^ 1)) { ok = false; break; }
+        tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t ad = dq0 + (uint64_t)(((kk >> 1) * QPL + (kk & 1) * 32) >> 4);
@@ -284,17 +278,25 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             umma_bf16(tmem + s_col(sb), ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
           }
           umma_commit(&s_full[sb]);
-          if (kt >= 1) issue_pv(j - 1, kt - 1);
+          if (kt + 1 == t.nkt) umma_commit(q_empty);  // the tile's scores no longer read Q
         }
-        if (t.nkt >= 1 && ok) issue_pv(kc + t.nkt - 1, t.nkt - 1);
-        umma_commit(o_full);
-        kc += t.nkt;
+        __syncwarp();
+        if (kt >= 1) issue_pv(j - 1, kt - 1);
       }
-      if (!ok) set_err(p.dev_err, MTLA_DEVERR_TIMEOUT);
-      // every MMA of this thread has completed before TMEM is released
-      umma_commit(mma_done);
-      mbar_wait(mma_done, 0);
+      if (t.nkt == 0) {
+        if (elect_one()) umma_commit(q_empty);
+        __syncwarp();
+      }
+      if (t.nkt >= 1 && ok) issue_pv(kc + t.nkt - 1, t.nkt - 1);
+      if (elect_one()) umma_commit(o_full);
+      __syncwarp();
+      kc += t.nkt;
     }
+    if (!ok && lane == 0) set_err(p.dev_err, MTLA_DEVERR_TIMEOUT);
+    // every MMA of this warp has completed before TMEM is released
+    if (elect_one()) umma_commit(mma_done);
+    __syncwarp();
+    warp_wait(mma_done, 0);
   } else {
     // ======================= softmax / epilogue warps =======================
     // warp w: TMEM lane quarter w % 4 (rows 32 (w % 4) .. +31) and half w / 4
@@ -307,8 +309,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     const int qw = warp & 3, hf = warp >> 2;
     const int i = qw * 32 + lane;              // row of the M tile = TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
-    float* xmax = reinterpret_cast<float*>(sm + OFF_XCH);             // [2 parity][2 halves][BM]
-    float* xl = reinterpret_cast<float*>(sm + OFF_XCH + 4 * BM * 4);   // [2 parity][2 halves][BM]
+    float* xmax = reinterpret_cast<float*>(sm + OFF_XCH);              // [2 parity][2 halves][BM]
+    float2* xl = reinterpret_cast<float2*>(sm + OFF_XCH + 4 * BM * 4);  // [2 parity][2 halves][BM]: row sum, own-row dot
     const float sl2 = p.scale_log2;
     uint32_t tc = 0, kc = 0;
     for (int o; (o = tile_index(tc, blockIdx.x, G)) < p.n_mtiles; ++tc) {
@@ -317,6 +319,34 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       const int h = i % H;
       const int vis = (int)group_of(m, p.s) - 1;  // completed groups it sees
       float m_run = -INFINITY, l = 0.f;        // l: this half's sum
+      // own row C_hat'_m from global memory; this warp's half of its score
+      // (16-byte chunks 18 hf .. 18 hf + 17 of the 288 dimensions), taken
+      // while the first scores are computed; then the warp is done with Q
+      const uint4* self_row = reinterpret_cast<const uint4*>(p.c_partial + (size_t)(t.b * p.T + (m - 1)) * D);
+      float dot = 0.f;
+      {
+        constexpr int NCH = D / 16;            // 18 chunks per half
+        uint4 cs[NCH];
+#pragma unroll
+        for (int k = 0; k < NCH; ++k) cs[k] = __ldg(self_row + NCH * hf + k);
+        if (ok && !warp_wait(q_full, tc & 1)) ok = false;
+#pragma unroll
+        for (int k = 0; k < NCH; ++k) {
+          uint32_t qv[4];
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(qv[0]), "=r"(qv[1]), "=r"(qv[2]), "=r"(qv[3])
+                       : "r"(sQ + plane_off(BM, i, NCH * hf + k)));
+          const uint32_t cv[4] = {cs[k].x, cs[k].y, cs[k].z, cs[k].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qv[e]));
+            const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cv[e]));
+            dot = fmaf(a.x, c.x, dot);
+            dot = fmaf(a.y, c.y, dot);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(q_empty);
+      }
       for (int kt = 0; kt < t.nkt; ++kt) {
         const uint32_t j = kc + kt;
         const int sb = j % NSB, xb = j & 1;    // TMEM buffer; exchange-buffer parity
@@ -388,32 +418,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[sb]);
       }
-      // ---- epilogue: own partial row C_hat'_m, then out = normalised (O + own term)
-      if (ok && !warp_wait(self_full, tc & 1)) ok = false;
-      const uint32_t selfb = sSelf;
-      const int srow = i / H;
-      float dot = 0.f;                         // all 288 dimensions, in both warps of the pair
-#pragma unroll 4
-      for (int ch = 0; ch < D / 8; ++ch) {
-        uint32_t qv[4], cv[4];
-        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(qv[0]), "=r"(qv[1]), "=r"(qv[2]), "=r"(qv[3])
-                     : "r"(sQ + plane_off(BM, i, ch)));
-        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(cv[0]), "=r"(cv[1]), "=r"(cv[2]), "=r"(cv[3])
-                     : "r"(selfb + plane_off(QM, srow, ch)));
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qv[e]));
-          const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cv[e]));
-          dot = fmaf(a.x, c.x, dot);
-          dot = fmaf(a.y, c.y, dot);
-        }
-      }
-      xl[((tc & 1) * 2 + hf) * BM + i] = l;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(q_empty);  // this warp no longer reads the query tile
+      // ---- epilogue: the own row's term, then out = normalised (O + own term)
+      xl[((tc & 1) * 2 + hf) * BM + i] = make_float2(l, dot);
       named_bar(1 + qw, 64);
-      const float xs = dot * sl2;
-      const float lt = xl[((tc & 1) * 2 + 0) * BM + i] + xl[((tc & 1) * 2 + 1) * BM + i];
+      const float2 e0 = xl[((tc & 1) * 2 + 0) * BM + i], e1 = xl[((tc & 1) * 2 + 1) * BM + i];
+      const float xs = (e0.y + e1.y) * sl2;
+      const float lt = e0.x + e1.x;
       const float mf = fmaxf(m_run, xs);
       const float alpha = m_run == -INFINITY ? 0.f : exp2f(m_run - mf);
       const float pself = exp2f(xs - mf);
@@ -435,9 +445,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         uint32_t res[16];
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t cv[4];
-          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(cv[0]), "=r"(cv[1]), "=r"(cv[2]), "=r"(cv[3])
-                       : "r"(selfb + plane_off(QM, srow, ch * 4 + q4)));
+          const uint4 c4 = __ldg(self_row + ch * 4 + q4);   // latent dims 32 ch + 8 q4 ..
+          const uint32_t cv[4] = {c4.x, c4.y, c4.z, c4.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cv[e]));
@@ -453,10 +462,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(o_empty);
-        mbar_arrive(self_empty);
-      }
+      if (lane == 0) mbar_arrive(o_empty);
       kc += t.nkt;
     }
     if (!ok && lane == 0) set_err(p.dev_err, MTLA_DEVERR_TIMEOUT);
@@ -473,7 +479,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 }  // namespace ptc
 
 cudaError_t launch_prefill_tc(const ptc::Params& p, const CUtensorMap& qmap, const CUtensorMap& rmap,
-                              const CUtensorMap& smap, const CUtensorMap& kmap, int grid, cudaStream_t st) {
+                              const CUtensorMap& kmap, int grid, cudaStream_t st) {
   const size_t smem = ptc::smem_bytes();
   static uint64_t done_mask = 0;
   int dev = 0;
@@ -484,12 +490,12 @@ cudaError_t launch_prefill_tc(const ptc::Params& p, const CUtensorMap& qmap, con
     if (e != cudaSuccess) return e;
     if (dev < 64) done_mask |= 1ull << dev;
   }
-  ptc::prefill_tc_kernel<<<grid, ptc::NT, smem, st>>>(qmap, rmap, smap, kmap, p);
+  ptc::prefill_tc_kernel<<<grid, ptc::NT, smem, st>>>(qmap, rmap, kmap, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_prefill_tc_args(const PrefillTcLaunch& a, const CUtensorMap& qmap, const CUtensorMap& rmap,
-                                   const CUtensorMap& smap, const CUtensorMap& kmap, int grid, cudaStream_t st) {
+                                   const CUtensorMap& kmap, int grid, cudaStream_t st) {
   ptc::Params p;
   p.B = a.B;
   p.T = a.T;
@@ -497,9 +503,10 @@ cudaError_t launch_prefill_tc_args(const PrefillTcLaunch& a, const CUtensorMap& 
   p.n_mtiles = a.B * (a.T / ptc::QM);
   p.n_groups = a.T / a.s;
   p.scale_log2 = a.scale_log2;
+  p.c_partial = reinterpret_cast<const __nv_bfloat16*>(a.c_partial);
   p.out = reinterpret_cast<__nv_bfloat16*>(a.out);
   p.dev_err = a.dev_err;
-  return launch_prefill_tc(p, qmap, rmap, smap, kmap, grid, st);
+  return launch_prefill_tc(p, qmap, rmap, kmap, grid, st);
 }
 
 }  // namespace mtla
