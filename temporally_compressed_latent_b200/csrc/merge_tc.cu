@@ -190,18 +190,20 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
     }
   } else if (warp == MMA_WARP) {
     // ======================= MMA issuer =======================
-    if (lane == 0) {
-      const uint32_t sA = smem_u32(sm + OFF_A), sHi = smem_u32(sm + OFF_WHI), sLo = smem_u32(sm + OFF_WLO);
-      uint32_t kc = 0, tc = 0;
-      for (int it = first; it < p.n_tiles && ok; it += G2, ++tc) {
-        const int ab = tc & 1;
-        if (tc >= 2 && !mbar_wait(&acc_empty[ab], ((tc >> 1) & 1) ^ 1)) { ok = false; break; }
+    // The whole warp runs the loop (warp-uniform operands); one elected lane
+    // issues the MMAs and the commits that track them.
+    const uint32_t sA = smem_u32(sm + OFF_A), sHi = smem_u32(sm + OFF_WHI), sLo = smem_u32(sm + OFF_WLO);
+    uint32_t kc = 0, tc = 0;
+    for (int it = first; it < p.n_tiles && ok; it += G2, ++tc) {
+      const int ab = tc & 1;
+      if (tc >= 2 && !warp_wait(&acc_empty[ab], ((tc >> 1) & 1) ^ 1)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t dcol = tmem + ab * ACC_STRIDE;
+      for (int kb = 0; kb < KB; ++kb, ++kc) {
+        const int st = kc % KS;
+        if (!warp_wait(&k_full[st], (kc / KS) & 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t dcol = tmem + ab * ACC_STRIDE;
-        for (int kb = 0; kb < KB; ++kb, ++kc) {
-          const int st = kc % KS;
-          if (!mbar_wait(&k_full[st], (kc / KS) & 1)) { ok = false; break; }
-          tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t ad = umma_desc(sA + st * ABLK + kk * 32, 16, 1024, 2);
@@ -212,14 +214,17 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
           }
           umma_commit(&k_empty[st]);
         }
-        if (!ok) break;
-        umma_commit(&acc_full[ab]);
+        __syncwarp();
       }
-      if (!ok) set_err(p.dev_err, MTLA_DEVERR_TIMEOUT);
-      // every MMA of this thread has completed before TMEM is released
-      umma_commit(mma_done);
-      mbar_wait(mma_done, 0);
+      if (!ok) break;
+      if (elect_one()) umma_commit(&acc_full[ab]);
+      __syncwarp();
     }
+    if (!ok && lane == 0) set_err(p.dev_err, MTLA_DEVERR_TIMEOUT);
+    // every MMA of this warp has completed before TMEM is released
+    if (elect_one()) umma_commit(mma_done);
+    __syncwarp();
+    warp_wait(mma_done, 0);
   } else {
     // ======================= epilogue: gate, gated entry, group scan =======================
     const int q = warp & 3;                            // TMEM lane quarter = warp block

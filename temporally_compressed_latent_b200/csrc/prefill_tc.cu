@@ -21,10 +21,11 @@
 //    The own rows are read from global memory (L1 / L2): four key stages fill
 //    the shared memory that a copy of them would take.
 //  * Scores S = Q K^T (M 128, N 64, K 288) and values O += P V (M 128, N 256,
-//    K 64) are tcgen05.mma ops with fp32 accumulators in TMEM (three 64-column
-//    S / P buffers, O 256 columns), issued by one thread, the scores of tile
-//    j + 1 ahead of the values of tile j.  Only complete groups up to the
-//    staircase are visited, so no tile is empty.
+//    K 64) are tcgen05.mma ops with fp32 accumulators in TMEM (four 64-column
+//    S / P buffers, O 256 columns: all 512 columns).  A score warp and a value
+//    warp issue them, each as soon as its inputs are ready, so the tensor pipe
+//    holds the next group before the current one ends.  Only complete groups
+//    up to the staircase are visited, so no tile is empty.
 //  * Eight softmax warps, two per TMEM lane quarter: warps w and w + 4 own
 //    the same 32 (query, head) rows (TMEM lanes) and split the key tile's 64
 //    columns and O's 256 columns between them, so each SMSP runs two of them.
@@ -37,7 +38,7 @@
 //    back into the tile's S columns of TMEM (tcgen05.st), from where the value
 //    MMA reads it as its A operand: no shared-memory round trip and no proxy
 //    fence.  The epilogue adds the own-row term and writes bf16 out.
-//  * One TMA warp, one MMA warp, mbarrier pipelines; a persistent grid visits
+//  * One TMA warp, two MMA warps, mbarrier pipelines; a persistent grid visits
 //    the M tiles heaviest first, in rounds of alternating direction.
 #include "kernels.cuh"
 
@@ -55,10 +56,10 @@ constexpr int QBYTES = NPL * QPL;      // 73728
 constexpr int KBYTES = NPL * KPL;      // 36864
 constexpr int KS = 4;                  // key-tile stages
 constexpr int SMW = 8;                 // softmax warps: two per TMEM lane quarter
-constexpr int NT = 32 * (SMW + 2);     // + TMA warp, MMA warp
-constexpr int TMA_WARP = SMW, MMA_WARP = SMW + 1;
+constexpr int NT = 32 * (SMW + 3);     // + TMA warp, score-MMA warp, value-MMA warp
+constexpr int TMA_WARP = SMW, SMMA_WARP = SMW + 1, PMMA_WARP = SMW + 2;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr int NSB = 3;                 // S / P buffers in TMEM (64 columns each)
+constexpr int NSB = 4;                 // S / P buffers in TMEM (64 columns each)
 constexpr uint32_t O_COL = 256;
 __host__ __device__ constexpr uint32_t s_col(int b) { return 64u * (uint32_t)b; }
 static_assert(NSB * 64 <= (int)O_COL, "S buffers below O");
@@ -69,7 +70,7 @@ constexpr size_t OFF_Q = 0;
 constexpr size_t OFF_K = OFF_Q + QBYTES;               // KS stages
 constexpr size_t OFF_XCH = OFF_K + (size_t)KS * KBYTES;  // pair exchange: row maxima, row sums
 constexpr size_t OFF_BAR = OFF_XCH + 2 * 2 * BM * 4 + 2 * 2 * BM * 8;
-constexpr int NBAR = 2 + 2 * KS + 4 * NSB + 3;
+constexpr int NBAR = 2 + 2 * KS + 3 * NSB + 3;
 constexpr size_t OFF_TMEM = OFF_BAR + NBAR * 8;
 constexpr size_t SMEM_USED = OFF_TMEM + 16;
 static_assert(OFF_K % 1024 == 0, "tile bases must be 1024-aligned");
@@ -160,10 +161,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   uint64_t* const k_full = bar + 2;             // [KS]
   uint64_t* const k_empty = bar + 2 + KS;       // [KS]
   uint64_t* const s_full = bar + 2 + 2 * KS;    // [NSB]
-  uint64_t* const s_empty = s_full + NSB;       // [NSB]
-  uint64_t* const p_full = s_full + 2 * NSB;    // [NSB]
-  uint64_t* const p_empty = s_full + 3 * NSB;   // [NSB]
-  uint64_t* const o_full = s_full + 4 * NSB;
+  uint64_t* const p_full = s_full + NSB;        // [NSB]
+  uint64_t* const p_empty = s_full + 2 * NSB;   // [NSB]: the value MMA has read P (and so the buffer is free)
+  uint64_t* const o_full = s_full + 3 * NSB;
   uint64_t* const o_empty = o_full + 1;
   uint64_t* const mma_done = o_full + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
@@ -178,13 +178,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     }
     for (int i = 0; i < NSB; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], SMW);
       mbar_init(&p_full[i], SMW);
       mbar_init(&p_empty[i], 1);
     }
     mbar_init(o_full, 1);
     mbar_init(o_empty, SMW);
-    mbar_init(mma_done, 1);
+    mbar_init(mma_done, 2);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -229,71 +228,80 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       if (q_issued) mbar_wait(q_full, (q_issued - 1) & 1);
       for (uint32_t j = kc > (uint32_t)KS ? kc - KS : 0; j < kc; ++j) mbar_wait(&k_full[j % KS], (j / KS) & 1);
     }
-  } else if (warp == MMA_WARP) {
-    // ======================= MMA issuer =======================
-    // The whole warp runs the loop, so every operand is warp-uniform; one
-    // elected lane issues each group of MMAs and the commits that track it.
-    // Operand descriptors are built once; a K step or a stage moves only the
-    // 14-bit start-address field (shared addresses are below 2^18, no carry).
+  } else if (warp == SMMA_WARP || warp == PMMA_WARP) {
+    // ======================= MMA issuers =======================
+    // Two warps feed the one tensor pipe: the score warp issues S(j) as soon
+    // as its key tile has landed and its TMEM buffer is free, the value warp
+    // issues O += P(j) V(j) as soon as the softmax has written P(j), so the
+    // pipe holds the next group before the current one ends.  Each warp runs
+    // its loop with all 32 lanes (warp-uniform operands); one elected lane
+    // issues the MMAs and the commits that track them.  Operand descriptors
+    // are built once; a K step or a stage moves only the 14-bit start-address
+    // field (shared addresses are below 2^18, no carry).
+    const bool scores = warp == SMMA_WARP;
     const uint64_t dq0 = umma_desc(sQ, 16, 512, 4);
     const uint64_t dk0 = umma_desc(sK, 16, 512, 4);
     const uint64_t dv0 = umma_desc(sK, KPL, 512, 4);
     uint32_t tc = 0, kc = 0;
     for (int o; (o = tile_index(tc, blockIdx.x, G)) < p.n_mtiles && ok; ++tc) {
       const Tile t = tile_of(p, o);
-      if (!warp_wait(q_full, tc & 1)) { ok = false; break; }
-      tc_fence_after();
-      // value MMA of key tile j (the kt-th of this M tile): O += P V, P from
-      // TMEM over the tile's S columns, V = the latent planes of its key tile
-      auto issue_pv = [&](uint32_t j, int kt) {
-        const int pb = j % NSB, st = j % KS;
-        if (!warp_wait(&p_full[pb], (j / NSB) & 1)) ok = false;
-        if (kt == 0 && tc > 0 && !warp_wait(o_empty, (tc - 1) & 1)) ok = false;
-        tc_fence_after();
-        if (elect_one()) {
+      if (scores) {
+        // S(j) = Q K(j)^T into buffer j mod NSB, once the value MMA of tile
+        // j - NSB has read that buffer (which also means its scores were read)
+        if (!warp_wait(q_full, tc & 1)) { ok = false; break; }
+        for (int kt = 0; kt < t.nkt && ok; ++kt) {
+          const uint32_t j = kc + kt;
+          const int st = j % KS, sb = j % NSB;
+          if (!warp_wait(&k_full[st], (j / KS) & 1)) { ok = false; break; }
+          if (j >= NSB && !warp_wait(&p_empty[sb], ((j / NSB) & 1) ^ 1)) { ok = false; break; }
+          tc_fence_after();
+          if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint32_t pa = tmem + s_col(pb) + 8 * kk;  // two bf16 per column: 8 columns per K step
-            const uint64_t bd = dv0 + (uint64_t)((st * KBYTES + kk * 16 * 64) >> 4);
-            umma_bf16_ts(tmem + O_COL, pa, bd, IDESC_O, (kt > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t ad = dq0 + (uint64_t)(((kk >> 1) * QPL + (kk & 1) * 32) >> 4);
+              const uint64_t bd = dk0 + (uint64_t)((st * KBYTES + (kk >> 1) * KPL + (kk & 1) * 32) >> 4);
+              umma_bf16(tmem + s_col(sb), ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&s_full[sb]);
+            if (kt + 1 == t.nkt) umma_commit(q_empty);  // the tile's scores no longer read Q
           }
-          umma_commit(&k_empty[st]);
-          umma_commit(&p_empty[pb]);
+          __syncwarp();
         }
-        __syncwarp();
-      };
-      // scores of key tile j + 1 are issued ahead of the values of tile j, so
-      // the tensor core has the next scores while the softmax works
-      for (int kt = 0; kt < t.nkt && ok; ++kt) {
-        const uint32_t j = kc + kt;
-        const int st = j % KS, sb = j % NSB;
-        if (!warp_wait(&k_full[st], (j / KS) & 1)) { ok = false; break; }
-        if (j >= NSB && !warp_wait(&s_empty[sb], ((j / NSB) & 1) ^ 1)) { ok = false; break; }
-        tc_fence_after();
-        if (elect_one()) {
+        if (t.nkt == 0) {
+          if (elect_one()) umma_commit(q_empty);
+          __syncwarp();
+        }
+      } else {
+        // O += P(j) V(j): P from TMEM over the tile's S columns, V = the
+        // latent planes of its key tile.  Its completion frees the key stage
+        // (the scores of tile j completed before the softmax wrote P(j)).
+        for (int kt = 0; kt < t.nkt && ok; ++kt) {
+          const uint32_t j = kc + kt;
+          const int pb = j % NSB, st = j % KS;
+          if (!warp_wait(&p_full[pb], (j / NSB) & 1)) { ok = false; break; }
+          if (kt == 0 && tc > 0 && !warp_wait(o_empty, (tc - 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+          if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t ad = dq0 + (uint64_t)(((kk >> 1) * QPL + (kk & 1) * 32) >> 4);
-            const uint64_t bd = dk0 + (uint64_t)((st * KBYTES + (kk >> 1) * KPL + (kk & 1) * 32) >> 4);
-            umma_bf16(tmem + s_col(sb), ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < BN / 16; ++kk) {
+              const uint32_t pa = tmem + s_col(pb) + 8 * kk;  // two bf16 per column: 8 columns per K step
+              const uint64_t bd = dv0 + (uint64_t)((st * KBYTES + kk * 16 * 64) >> 4);
+              umma_bf16_ts(tmem + O_COL, pa, bd, IDESC_O, (kt > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(&k_empty[st]);
+            umma_commit(&p_empty[pb]);
           }
-          umma_commit(&s_full[sb]);
-          if (kt + 1 == t.nkt) umma_commit(q_empty);  // the tile's scores no longer read Q
+          __syncwarp();
         }
-        __syncwarp();
-        if (kt >= 1) issue_pv(j - 1, kt - 1);
+        if (ok) {
+          if (elect_one()) umma_commit(o_full);
+          __syncwarp();
+        }
       }
-      if (t.nkt == 0) {
-        if (elect_one()) umma_commit(q_empty);
-        __syncwarp();
-      }
-      if (t.nkt >= 1 && ok) issue_pv(kc + t.nkt - 1, t.nkt - 1);
-      if (elect_one()) umma_commit(o_full);
-      __syncwarp();
       kc += t.nkt;
     }
     if (!ok && lane == 0) set_err(p.dev_err, MTLA_DEVERR_TIMEOUT);
-    // every MMA of this warp has completed before TMEM is released
+    // every MMA of both warps has completed before TMEM is released
     if (elect_one()) umma_commit(mma_done);
     __syncwarp();
     warp_wait(mma_done, 0);
@@ -355,9 +363,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         uint32_t sr[32];
         tmem_ld32(lane_base + s_col(sb) + 32 * hf, sr);
         tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_empty[sb]);
         // mask (group kt*BN + 32 hf + c + 1 visible iff <= vis) and scale
         const int nvis = vis - kt * BN - 32 * hf;
         float x[32];
