@@ -107,12 +107,12 @@ size_t smem_bytes();
 struct PrefillTcLaunch {
   int B, T, s;
   float scale_log2;
-  const void* c_partial;
   void* out;
   int32_t* dev_err;
 };
 cudaError_t launch_prefill_tc_args(const PrefillTcLaunch& a, const CUtensorMap& qmap, const CUtensorMap& rmap,
-                                   const CUtensorMap& kmap, int grid, cudaStream_t st);
+                                   const CUtensorMap& smap, const CUtensorMap& kmap, const CUtensorMap& omap,
+                                   int grid, cudaStream_t st);
 cudaError_t launch_prefill_simt(const PrefillArgs& p, int B, int dtype, cudaStream_t st);
 
 }  // namespace mtla

@@ -52,12 +52,14 @@ constexpr int BN = 64;                 // groups per key tile
 constexpr int NPL = D / 32;            // 9 planes of 32 elements
 constexpr int QPL = BM * 64;           // bytes of one query plane (8192)
 constexpr int KPL = BN * 64;           // bytes of one key plane (4096)
+constexpr int SPL = QM * 64;           // bytes of one own-row plane (1024)
 constexpr int QBYTES = NPL * QPL;      // 73728
 constexpr int KBYTES = NPL * KPL;      // 36864
-constexpr int KS = 4;                  // key-tile stages
+constexpr int SBYTES = NPL * SPL;      // 9216
+constexpr int KS = 3;                  // key-tile stages
 constexpr int SMW = 8;                 // softmax warps: two per TMEM lane quarter
-constexpr int NT = 32 * (SMW + 3);     // + TMA warp, score-MMA warp, value-MMA warp
-constexpr int TMA_WARP = SMW, SMMA_WARP = SMW + 1, PMMA_WARP = SMW + 2;
+constexpr int NT = 32 * (SMW + 4);     // + TMA warp, score-MMA warp, value-MMA warp, own-row warp
+constexpr int TMA_WARP = SMW, SMMA_WARP = SMW + 1, PMMA_WARP = SMW + 2, DOT_WARP = SMW + 3;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int NSB = 4;                 // S / P buffers in TMEM (64 columns each)
 constexpr uint32_t O_COL = 256;
@@ -66,14 +68,18 @@ static_assert(NSB * 64 <= (int)O_COL, "S buffers below O");
 constexpr uint32_t IDESC_S = umma_idesc_bf16(BM, BN, false, false);
 constexpr uint32_t IDESC_O = umma_idesc_bf16(BM, R, false, true);
 
+constexpr int OST_BYTES = 32 * 64;     // output staging of one warp: 32 rows x 32 channels bf16
+
 constexpr size_t OFF_Q = 0;
-constexpr size_t OFF_K = OFF_Q + QBYTES;               // KS stages
-constexpr size_t OFF_XCH = OFF_K + (size_t)KS * KBYTES;  // pair exchange: row maxima, row sums
-constexpr size_t OFF_BAR = OFF_XCH + 2 * 2 * BM * 4 + 2 * 2 * BM * 8;
-constexpr int NBAR = 2 + 2 * KS + 3 * NSB + 3;
+constexpr size_t OFF_SELF = OFF_Q + QBYTES;              // two own-row buffers (M tile parity)
+constexpr size_t OFF_K = OFF_SELF + 2 * SBYTES;          // KS stages
+constexpr size_t OFF_OST = OFF_K + (size_t)KS * KBYTES;  // SMW output staging buffers
+constexpr size_t OFF_XCH = OFF_OST + (size_t)SMW * OST_BYTES;  // row maxima, row sums, own-row scores
+constexpr size_t OFF_BAR = OFF_XCH + 2 * 2 * BM * 4 + 2 * 2 * BM * 4 + 2 * BM * 4;
+constexpr int NBAR = 2 + 8 + 2 * KS + 3 * NSB + 3;
 constexpr size_t OFF_TMEM = OFF_BAR + NBAR * 8;
 constexpr size_t SMEM_USED = OFF_TMEM + 16;
-static_assert(OFF_K % 1024 == 0, "tile bases must be 1024-aligned");
+static_assert(OFF_K % 1024 == 0 && OFF_SELF % 1024 == 0 && OFF_OST % 1024 == 0, "tile bases must be 1024-aligned");
 
 size_t smem_bytes() { return SMEM_USED + 1024; }
 static_assert(SMEM_USED + 1024 <= 232448, "one block's shared memory (227 KB)");
@@ -83,7 +89,6 @@ struct Params {
   int n_mtiles;            // B * T / QM
   int n_groups;            // complete groups per sequence, floor(T / s)
   float scale_log2;        // log2(e) / sqrt(d_h)
-  const __nv_bfloat16* c_partial;  // [B, T, D]: the own rows C_hat'_m
   __nv_bfloat16* out;      // [B, T, H, R]
   int32_t* dev_err;
 };
@@ -152,26 +157,40 @@ __device__ __forceinline__ Tile tile_of(const Params& p, int o) {
 
 __global__ void __launch_bounds__(NT, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap rmap,
-                  const __grid_constant__ CUtensorMap kmap, const Params p) {
+                  const __grid_constant__ CUtensorMap smap, const __grid_constant__ CUtensorMap kmap,
+                  const __grid_constant__ CUtensorMap omap, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
   uint64_t* const q_full = bar + 0;
-  uint64_t* const q_empty = bar + 1;            // the last score MMA + every softmax warp's own-row score
-  uint64_t* const k_full = bar + 2;             // [KS]
-  uint64_t* const k_empty = bar + 2 + KS;       // [KS]
-  uint64_t* const s_full = bar + 2 + 2 * KS;    // [NSB]
+  uint64_t* const q_empty = bar + 1;            // the tile's last score MMA + the own-row warp
+  uint64_t* const self_full = bar + 2;          // [2] own rows of M tile parity b landed
+  uint64_t* const self_empty = bar + 4;         // [2] the epilogue is done with them
+  uint64_t* const dot_full = bar + 6;           // [2] own-row scores written
+  uint64_t* const dot_empty = bar + 8;          // [2] the epilogue has read them
+  uint64_t* const k_full = bar + 10;            // [KS]
+  uint64_t* const k_empty = bar + 10 + KS;      // [KS]
+  uint64_t* const s_full = bar + 10 + 2 * KS;   // [NSB]
   uint64_t* const p_full = s_full + NSB;        // [NSB]
   uint64_t* const p_empty = s_full + 2 * NSB;   // [NSB]: the value MMA has read P (and so the buffer is free)
   uint64_t* const o_full = s_full + 3 * NSB;
   uint64_t* const o_empty = o_full + 1;
   uint64_t* const mma_done = o_full + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
+  float* xmax = reinterpret_cast<float*>(sm + OFF_XCH);                 // [2 parity][2 halves][BM]
+  float* xl = reinterpret_cast<float*>(sm + OFF_XCH + 4 * BM * 4);      // [2 parity][2 halves][BM]
+  float* xdot = reinterpret_cast<float*>(sm + OFF_XCH + 8 * BM * 4);    // [2 parity][BM]: own-row scores
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
     mbar_init(q_full, 1);
-    mbar_init(q_empty, SMW + 1);
+    mbar_init(q_empty, 2);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&self_full[b], 1);
+      mbar_init(&self_empty[b], SMW);
+      mbar_init(&dot_full[b], 1);
+      mbar_init(&dot_empty[b], SMW);
+    }
     for (int i = 0; i < KS; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
@@ -193,13 +212,16 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   if (warp == TMA_WARP && lane == 0) {
     prefetch_tmap(&qmap);
     prefetch_tmap(&rmap);
+    prefetch_tmap(&smap);
     prefetch_tmap(&kmap);
+    prefetch_tmap(&omap);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const uint32_t sQ = smem_u32(sm + OFF_Q);
+  const uint32_t sSelf = smem_u32(sm + OFF_SELF);
   const uint32_t sK = smem_u32(sm + OFF_K);
   const int G = gridDim.x;
   bool ok = true;
@@ -211,11 +233,18 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       for (int o; (o = tile_index(tc, blockIdx.x, G)) < p.n_mtiles && ok; ++tc) {
         const Tile t = tile_of(p, o);
         const int qrow0 = ((t.b * p.T) + (t.m0 - 1)) * H;  // first row of [B*T*H, .]
+        const int crow0 = t.b * p.T + (t.m0 - 1);         // first own row of [B*T, .]
+        const int sb2 = tc & 1;
         if (tc > 0 && !mbar_wait(q_empty, (tc - 1) & 1)) { ok = false; break; }
         mbar_arrive_expect_tx(q_full, QBYTES);
         tma_load_3d(sm + OFF_Q, &qmap, 0, qrow0, 0, q_full);
         tma_load_2d(sm + OFF_Q + 8 * QPL, &rmap, 0, qrow0, q_full);
         q_issued = tc + 1;
+        // own rows into the buffer of this tile's parity, once the epilogue of
+        // tile tc - 2 is done with it
+        if (tc >= 2 && !mbar_wait(&self_empty[sb2], ((tc >> 1) & 1) ^ 1)) { ok = false; break; }
+        mbar_arrive_expect_tx(&self_full[sb2], SBYTES);
+        tma_load_3d(sm + OFF_SELF + sb2 * SBYTES, &smap, 0, crow0, 0, &self_full[sb2]);
         for (int kt = 0; kt < t.nkt; ++kt, ++kc) {
           const int st = kc % KS;
           if (kc >= KS && !mbar_wait(&k_empty[st], ((kc / KS) & 1) ^ 1)) { ok = false; break; }
@@ -226,8 +255,50 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       if (!ok) set_err(p.dev_err, MTLA_DEVERR_TIMEOUT);
       // drain: no copy may still be writing shared memory when the block exits
       if (q_issued) mbar_wait(q_full, (q_issued - 1) & 1);
+      for (uint32_t u = q_issued > 2 ? q_issued - 2 : 0; u < q_issued; ++u) mbar_wait(&self_full[u & 1], (u >> 1) & 1);
       for (uint32_t j = kc > (uint32_t)KS ? kc - KS : 0; j < kc; ++j) mbar_wait(&k_full[j % KS], (j / KS) & 1);
     }
+  } else if (warp == DOT_WARP) {
+    // ======================= own-row scores =======================
+    // x_self = q_abs . c_hat'_m + q^R . k_hat^R'_m for the 128 rows of the M
+    // tile (lane: rows lane + 32 r), from the query tile and the own rows in
+    // shared memory, while the key tiles run.  Then this warp is done with Q.
+    for (uint32_t tc = 0; tile_index(tc, blockIdx.x, G) < p.n_mtiles; ++tc) {
+      const int sb2 = tc & 1;
+      if (ok && !warp_wait(q_full, tc & 1)) ok = false;
+      if (ok && !warp_wait(&self_full[sb2], (tc >> 1) & 1)) ok = false;
+      // the epilogue of tile tc - 2 has read this parity's scores
+      if (ok && tc >= 2 && !warp_wait(&dot_empty[sb2], ((tc >> 1) & 1) ^ 1)) ok = false;
+      const uint32_t selfb = sSelf + sb2 * SBYTES;
+#pragma unroll 1
+      for (int r = 0; r < BM / 32; ++r) {
+        const int i = r * 32 + lane;
+        const int srow = i / H;
+        float dot = 0.f;
+#pragma unroll 4
+        for (int ch = 0; ch < D / 8; ++ch) {
+          uint32_t qv[4], cv[4];
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(qv[0]), "=r"(qv[1]), "=r"(qv[2]), "=r"(qv[3])
+                       : "r"(sQ + plane_off(BM, i, ch)));
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(cv[0]), "=r"(cv[1]), "=r"(cv[2]), "=r"(cv[3])
+                       : "r"(selfb + plane_off(QM, srow, ch)));
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qv[e]));
+            const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cv[e]));
+            dot = fmaf(a.x, c.x, dot);
+            dot = fmaf(a.y, c.y, dot);
+          }
+        }
+        xdot[sb2 * BM + i] = dot;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(q_empty);
+        mbar_arrive(&dot_full[sb2]);
+      }
+    }
+    if (!ok && lane == 0) set_err(p.dev_err, MTLA_DEVERR_TIMEOUT);
   } else if (warp == SMMA_WARP || warp == PMMA_WARP) {
     // ======================= MMA issuers =======================
     // Two warps feed the one tensor pipe: the score warp issues S(j) as soon
@@ -317,44 +388,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     const int qw = warp & 3, hf = warp >> 2;
     const int i = qw * 32 + lane;              // row of the M tile = TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
-    float* xmax = reinterpret_cast<float*>(sm + OFF_XCH);              // [2 parity][2 halves][BM]
-    float2* xl = reinterpret_cast<float2*>(sm + OFF_XCH + 4 * BM * 4);  // [2 parity][2 halves][BM]: row sum, own-row dot
+    uint8_t* const ost = sm + OFF_OST + warp * OST_BYTES;  // this warp's output staging
     const float sl2 = p.scale_log2;
     uint32_t tc = 0, kc = 0;
     for (int o; (o = tile_index(tc, blockIdx.x, G)) < p.n_mtiles; ++tc) {
       const Tile t = tile_of(p, o);
       const int m = t.m0 + i / H;              // this row's query (1-based)
-      const int h = i % H;
       const int vis = (int)group_of(m, p.s) - 1;  // completed groups it sees
       float m_run = -INFINITY, l = 0.f;        // l: this half's sum
-      // own row C_hat'_m from global memory; this warp's half of its score
-      // (16-byte chunks 18 hf .. 18 hf + 17 of the 288 dimensions), taken
-      // while the first scores are computed; then the warp is done with Q
-      const uint4* self_row = reinterpret_cast<const uint4*>(p.c_partial + (size_t)(t.b * p.T + (m - 1)) * D);
-      float dot = 0.f;
-      {
-        constexpr int NCH = D / 16;            // 18 chunks per half
-        uint4 cs[NCH];
-#pragma unroll
-        for (int k = 0; k < NCH; ++k) cs[k] = __ldg(self_row + NCH * hf + k);
-        if (ok && !warp_wait(q_full, tc & 1)) ok = false;
-#pragma unroll
-        for (int k = 0; k < NCH; ++k) {
-          uint32_t qv[4];
-          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(qv[0]), "=r"(qv[1]), "=r"(qv[2]), "=r"(qv[3])
-                       : "r"(sQ + plane_off(BM, i, NCH * hf + k)));
-          const uint32_t cv[4] = {cs[k].x, cs[k].y, cs[k].z, cs[k].w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qv[e]));
-            const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cv[e]));
-            dot = fmaf(a.x, c.x, dot);
-            dot = fmaf(a.y, c.y, dot);
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(q_empty);
-      }
       for (int kt = 0; kt < t.nkt; ++kt) {
         const uint32_t j = kc + kt;
         const int sb = j % NSB, xb = j & 1;    // TMEM buffer; exchange-buffer parity
@@ -424,18 +465,24 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         if (lane == 0) mbar_arrive(&p_full[sb]);
       }
       // ---- epilogue: the own row's term, then out = normalised (O + own term)
-      xl[((tc & 1) * 2 + hf) * BM + i] = make_float2(l, dot);
+      const int sb2 = tc & 1;
+      xl[(sb2 * 2 + hf) * BM + i] = l;
       named_bar(1 + qw, 64);
-      const float2 e0 = xl[((tc & 1) * 2 + 0) * BM + i], e1 = xl[((tc & 1) * 2 + 1) * BM + i];
-      const float xs = (e0.y + e1.y) * sl2;
-      const float lt = e0.x + e1.x;
+      const float lt = xl[(sb2 * 2 + 0) * BM + i] + xl[(sb2 * 2 + 1) * BM + i];
+      if (ok && !warp_wait(&dot_full[sb2], (tc >> 1) & 1)) ok = false;
+      if (ok && !warp_wait(&self_full[sb2], (tc >> 1) & 1)) ok = false;
+      const float xs = xdot[sb2 * BM + i] * sl2;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&dot_empty[sb2]);
       const float mf = fmaxf(m_run, xs);
       const float alpha = m_run == -INFINITY ? 0.f : exp2f(m_run - mf);
       const float pself = exp2f(xs - mf);
       const float inv = 1.f / (lt * alpha + pself);
       if (ok && !warp_wait(o_full, tc & 1)) ok = false;
       tc_fence_after();
-      __nv_bfloat16* orow = p.out + ((size_t)(t.b * p.T + (m - 1)) * H + h) * R;
+      const uint32_t selfb = sSelf + sb2 * SBYTES;
+      const int srow = i / H;
+      const int orow0 = ((t.b * p.T) + (t.m0 - 1)) * H + 32 * qw;  // first output row of this warp
 #pragma unroll 1
       for (int cc = 0; cc < R / 64; ++cc) {
         const int ch = 4 * hf + cc;            // 32-channel chunk of this half
@@ -447,11 +494,18 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 #pragma unroll
           for (int e = 0; e < 32; ++e) ov[e] = 0u;
         }
+        if (cc == R / 64 - 1) {
+          // the last read of O in TMEM: the next M tile's value MMAs may start
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(o_empty);
+        }
         uint32_t res[16];
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-          const uint4 c4 = __ldg(self_row + ch * 4 + q4);   // latent dims 32 ch + 8 q4 ..
-          const uint32_t cv[4] = {c4.x, c4.y, c4.z, c4.w};
+          uint32_t cv[4];
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(cv[0]), "=r"(cv[1]), "=r"(cv[2]), "=r"(cv[3])
+                       : "r"(selfb + plane_off(QM, srow, ch * 4 + q4)));
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cv[e]));
@@ -461,16 +515,30 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
             res[q4 * 4 + e] = pack_bf16x2(v0, v1);
           }
         }
-        uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+        // stage row `lane` of the warp's 32 x 32 output block (64-byte swizzle,
+        // the tensor map's layout) once the previous block's store has read it,
+        // then one TMA store writes the block to rows orow0.., channels 32 ch..
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) dst[q4] = make_uint4(res[4 * q4], res[4 * q4 + 1], res[4 * q4 + 2], res[4 * q4 + 3]);
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint32_t off = (uint32_t)lane * 64u + ((((uint32_t)q4) ^ (((uint32_t)lane >> 1) & 3u)) << 4);
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(ost) + off), "r"(res[4 * q4]),
+                       "r"(res[4 * q4 + 1]), "r"(res[4 * q4 + 2]), "r"(res[4 * q4 + 3]) : "memory");
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&omap, ost, ch * 32, orow0);
+          bulk_commit();
+        }
       }
-      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(o_empty);
+      if (lane == 0) mbar_arrive(&self_empty[sb2]);
       kc += t.nkt;
     }
     if (!ok && lane == 0) set_err(p.dev_err, MTLA_DEVERR_TIMEOUT);
+    if (lane == 0) bulk_wait_all();  // the output stores have completed
   }
 
   tc_fence_before();
@@ -484,7 +552,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 }  // namespace ptc
 
 cudaError_t launch_prefill_tc(const ptc::Params& p, const CUtensorMap& qmap, const CUtensorMap& rmap,
-                              const CUtensorMap& kmap, int grid, cudaStream_t st) {
+                              const CUtensorMap& smap, const CUtensorMap& kmap, const CUtensorMap& omap, int grid,
+                              cudaStream_t st) {
   const size_t smem = ptc::smem_bytes();
   static uint64_t done_mask = 0;
   int dev = 0;
@@ -495,12 +564,13 @@ cudaError_t launch_prefill_tc(const ptc::Params& p, const CUtensorMap& qmap, con
     if (e != cudaSuccess) return e;
     if (dev < 64) done_mask |= 1ull << dev;
   }
-  ptc::prefill_tc_kernel<<<grid, ptc::NT, smem, st>>>(qmap, rmap, kmap, p);
+  ptc::prefill_tc_kernel<<<grid, ptc::NT, smem, st>>>(qmap, rmap, smap, kmap, omap, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_prefill_tc_args(const PrefillTcLaunch& a, const CUtensorMap& qmap, const CUtensorMap& rmap,
-                                   const CUtensorMap& kmap, int grid, cudaStream_t st) {
+                                   const CUtensorMap& smap, const CUtensorMap& kmap, const CUtensorMap& omap,
+                                   int grid, cudaStream_t st) {
   ptc::Params p;
   p.B = a.B;
   p.T = a.T;
@@ -508,10 +578,9 @@ cudaError_t launch_prefill_tc_args(const PrefillTcLaunch& a, const CUtensorMap& 
   p.n_mtiles = a.B * (a.T / ptc::QM);
   p.n_groups = a.T / a.s;
   p.scale_log2 = a.scale_log2;
-  p.c_partial = reinterpret_cast<const __nv_bfloat16*>(a.c_partial);
   p.out = reinterpret_cast<__nv_bfloat16*>(a.out);
   p.dev_err = a.dev_err;
-  return launch_prefill_tc(p, qmap, rmap, kmap, grid, st);
+  return launch_prefill_tc(p, qmap, rmap, smap, kmap, omap, grid, st);
 }
 
 }  // namespace mtla
