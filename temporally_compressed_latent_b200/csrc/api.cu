@@ -328,12 +328,11 @@ mtla_status mtla_prefill_masked_attn(const mtla_dims* dims, int32_t B, int32_t T
   if (!out) return MTLA_OK;
   if (!tc_prefill_dims(dims, B, T)) return from_cuda(launch_prefill_simt(p, B, dims->dtype, cs));
 
-  // tensor-core path: queries as 9 planes of 32, own rows, the completed
-  // groups C_hat'_{g s} read through a map whose row stride is s rows, and
-  // the output as 32 x 32 blocks
+  // tensor-core path: queries as 9 planes of 32, own rows, and the completed
+  // groups C_hat'_{g s} read through a map whose row stride is s rows
   const int s = dims->s;
   const cuuint64_t rows_q = (cuuint64_t)B * T * 8, rows_c = (cuuint64_t)B * T;
-  CUtensorMap qmap, rmap, smap, kmap, omap;
+  CUtensorMap qmap, rmap, smap, kmap;
   {
     const cuuint64_t dims3[3] = {32, rows_q, 8}, str[2] = {512, 64};
     const cuuint32_t box[3] = {32, 128, 8};
@@ -348,11 +347,6 @@ mtla_status mtla_prefill_masked_attn(const mtla_dims* dims, int32_t B, int32_t T
     const cuuint64_t dims3[3] = {32, rows_c, 9}, str[2] = {576, 64};
     const cuuint32_t box[3] = {32, 16, 9};
     if (!encode_bf16_map(&smap, c_partial, 3, dims3, str, box)) return MTLA_ERR_CUDA;
-  }
-  {
-    const cuuint64_t dims2[2] = {256, rows_q}, str[1] = {512};
-    const cuuint32_t box[2] = {32, 32};
-    if (!encode_bf16_map(&omap, out, 2, dims2, str, box)) return MTLA_ERR_CUDA;
   }
   {
     const int64_t groups = T / s;
@@ -370,7 +364,7 @@ mtla_status mtla_prefill_masked_attn(const mtla_dims* dims, int32_t B, int32_t T
   a.out = out;
   a.dev_err = dev_err;
   const int tiles = B * (T / 16);
-  return from_cuda(launch_prefill_tc_args(a, qmap, rmap, smap, kmap, omap, tiles < sms ? tiles : sms, cs));
+  return from_cuda(launch_prefill_tc_args(a, qmap, rmap, smap, kmap, tiles < sms ? tiles : sms, cs));
 }
 
 }  // extern "C"

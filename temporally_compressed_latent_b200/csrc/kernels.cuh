@@ -111,8 +111,7 @@ struct PrefillTcLaunch {
   int32_t* dev_err;
 };
 cudaError_t launch_prefill_tc_args(const PrefillTcLaunch& a, const CUtensorMap& qmap, const CUtensorMap& rmap,
-                                   const CUtensorMap& smap, const CUtensorMap& kmap, const CUtensorMap& omap,
-                                   int grid, cudaStream_t st);
+                                   const CUtensorMap& smap, const CUtensorMap& kmap, int grid, cudaStream_t st);
 cudaError_t launch_prefill_simt(const PrefillArgs& p, int B, int dtype, cudaStream_t st);
 
 }  // namespace mtla

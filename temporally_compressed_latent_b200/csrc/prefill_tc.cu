@@ -58,8 +58,10 @@ constexpr int KBYTES = NPL * KPL;      // 36864
 constexpr int SBYTES = NPL * SPL;      // 9216
 constexpr int KS = 3;                  // key-tile stages
 constexpr int SMW = 8;                 // softmax warps: two per TMEM lane quarter
-constexpr int NT = 32 * (SMW + 4);     // + TMA warp, score-MMA warp, value-MMA warp, own-row warp
-constexpr int TMA_WARP = SMW, SMMA_WARP = SMW + 1, PMMA_WARP = SMW + 2, DOT_WARP = SMW + 3;
+constexpr int EPW = 4;                 // epilogue warps: one per TMEM lane quarter
+constexpr int NT = 32 * (SMW + 4 + EPW);  // + TMA warp, score-MMA warp, value-MMA warp, own-row warp, epilogue
+constexpr int TMA_WARP = SMW, SMMA_WARP = SMW + 1, PMMA_WARP = SMW + 2, DOT_WARP = SMW + 3, EPI_WARP0 = SMW + 4;
+static_assert(EPI_WARP0 % 4 == 0, "epilogue warp e reads TMEM lane quarter e");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int NSB = 4;                 // S / P buffers in TMEM (64 columns each)
 constexpr uint32_t O_COL = 256;
@@ -68,15 +70,15 @@ static_assert(NSB * 64 <= (int)O_COL, "S buffers below O");
 constexpr uint32_t IDESC_S = umma_idesc_bf16(BM, BN, false, false);
 constexpr uint32_t IDESC_O = umma_idesc_bf16(BM, R, false, true);
 
-constexpr int OST_BYTES = 32 * 64;     // output staging of one warp: 32 rows x 32 channels bf16
+constexpr int OST_BYTES = 32 * 64;     // output staging of one epilogue warp: 32 rows x 32 channels bf16
 
 constexpr size_t OFF_Q = 0;
 constexpr size_t OFF_SELF = OFF_Q + QBYTES;              // two own-row buffers (M tile parity)
 constexpr size_t OFF_K = OFF_SELF + 2 * SBYTES;          // KS stages
-constexpr size_t OFF_OST = OFF_K + (size_t)KS * KBYTES;  // SMW output staging buffers
-constexpr size_t OFF_XCH = OFF_OST + (size_t)SMW * OST_BYTES;  // row maxima, row sums, own-row scores
-constexpr size_t OFF_BAR = OFF_XCH + 2 * 2 * BM * 4 + 2 * 2 * BM * 4 + 2 * BM * 4;
-constexpr int NBAR = 2 + 8 + 2 * KS + 3 * NSB + 3;
+constexpr size_t OFF_OST = OFF_K + (size_t)KS * KBYTES;  // EPW output staging blocks
+constexpr size_t OFF_XCH = OFF_OST + (size_t)EPW * OST_BYTES;  // row maxima, sums, final maxima, own-row scores
+constexpr size_t OFF_BAR = OFF_XCH + 2 * 2 * BM * 4 + 2 * 2 * BM * 4 + 2 * BM * 4 + 2 * BM * 4;
+constexpr int NBAR = 2 + 12 + 2 * KS + 3 * NSB + 3;
 constexpr size_t OFF_TMEM = OFF_BAR + NBAR * 8;
 constexpr size_t SMEM_USED = OFF_TMEM + 16;
 static_assert(OFF_K % 1024 == 0 && OFF_SELF % 1024 == 0 && OFF_OST % 1024 == 0, "tile bases must be 1024-aligned");
@@ -158,7 +160,7 @@ __device__ __forceinline__ Tile tile_of(const Params& p, int o) {
 __global__ void __launch_bounds__(NT, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap rmap,
                   const __grid_constant__ CUtensorMap smap, const __grid_constant__ CUtensorMap kmap,
-                  const __grid_constant__ CUtensorMap omap, const Params p) {
+                  const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
@@ -168,9 +170,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   uint64_t* const self_empty = bar + 4;         // [2] the epilogue is done with them
   uint64_t* const dot_full = bar + 6;           // [2] own-row scores written
   uint64_t* const dot_empty = bar + 8;          // [2] the epilogue has read them
-  uint64_t* const k_full = bar + 10;            // [KS]
-  uint64_t* const k_empty = bar + 10 + KS;      // [KS]
-  uint64_t* const s_full = bar + 10 + 2 * KS;   // [NSB]
+  uint64_t* const stat_full = bar + 10;         // [2] the softmax has written a tile's row maxima and sums
+  uint64_t* const stat_empty = bar + 12;        // [2] the epilogue has read them
+  uint64_t* const k_full = bar + 14;            // [KS]
+  uint64_t* const k_empty = bar + 14 + KS;      // [KS]
+  uint64_t* const s_full = bar + 14 + 2 * KS;   // [NSB]
   uint64_t* const p_full = s_full + NSB;        // [NSB]
   uint64_t* const p_empty = s_full + 2 * NSB;   // [NSB]: the value MMA has read P (and so the buffer is free)
   uint64_t* const o_full = s_full + 3 * NSB;
@@ -178,8 +182,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   uint64_t* const mma_done = o_full + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
   float* xmax = reinterpret_cast<float*>(sm + OFF_XCH);                 // [2 parity][2 halves][BM]
-  float* xl = reinterpret_cast<float*>(sm + OFF_XCH + 4 * BM * 4);      // [2 parity][2 halves][BM]
+  float* xl = reinterpret_cast<float*>(sm + OFF_XCH + 4 * BM * 4);      // [2 parity][2 halves][BM]: row sums
   float* xdot = reinterpret_cast<float*>(sm + OFF_XCH + 8 * BM * 4);    // [2 parity][BM]: own-row scores
+  float* xm = reinterpret_cast<float*>(sm + OFF_XCH + 10 * BM * 4);     // [2 parity][BM]: final row maxima
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
@@ -187,9 +192,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     mbar_init(q_empty, 2);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&self_full[b], 1);
-      mbar_init(&self_empty[b], SMW);
+      mbar_init(&self_empty[b], EPW);
       mbar_init(&dot_full[b], 1);
-      mbar_init(&dot_empty[b], SMW);
+      mbar_init(&dot_empty[b], EPW);
+      mbar_init(&stat_full[b], SMW);
+      mbar_init(&stat_empty[b], EPW);
     }
     for (int i = 0; i < KS; ++i) {
       mbar_init(&k_full[i], 1);
@@ -201,7 +208,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       mbar_init(&p_empty[i], 1);
     }
     mbar_init(o_full, 1);
-    mbar_init(o_empty, SMW);
+    mbar_init(o_empty, EPW);
     mbar_init(mma_done, 2);
     fence_mbar_init();
   }
@@ -214,7 +221,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     prefetch_tmap(&rmap);
     prefetch_tmap(&smap);
     prefetch_tmap(&kmap);
-    prefetch_tmap(&omap);
   }
   tc_fence_before();
   __syncthreads();
@@ -376,8 +382,108 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     if (elect_one()) umma_commit(mma_done);
     __syncwarp();
     warp_wait(mma_done, 0);
+  } else if (warp >= EPI_WARP0) {
+    // ======================= epilogue warps =======================
+    // warp EPI_WARP0 + e owns rows 32 e .. 32 e + 31 (TMEM lane quarter e) and
+    // all 256 channels: out = (alpha O + p_self c_hat'_m) / (alpha l + p_self)
+    // with the own row as one more key, in bf16.  It runs while the softmax
+    // warps start the next M tile; that tile's value MMAs wait until O has
+    // been read.  O is read 64 channels at a time; each 32 x 32 block goes
+    // through a staging block in shared memory (64-byte swizzle, no bank
+    // conflicts either way) so that every store writes 64 contiguous bytes
+    // of 8 rows.
+    const int qe = warp - EPI_WARP0;
+    const int i = qe * 32 + lane;
+    const int srow = i / H;
+    const uint32_t lane_base = tmem + ((uint32_t)(qe * 32) << 16);
+    const uint32_t ost = smem_u32(sm + OFF_OST + (size_t)qe * OST_BYTES);
+    const float sl2 = p.scale_log2;
+    uint32_t tc = 0;
+    for (int o; (o = tile_index(tc, blockIdx.x, G)) < p.n_mtiles; ++tc) {
+      const Tile t = tile_of(p, o);
+      const int sb2 = tc & 1;
+      if (ok && !warp_wait(&stat_full[sb2], (tc >> 1) & 1)) ok = false;
+      if (ok && !warp_wait(&dot_full[sb2], (tc >> 1) & 1)) ok = false;
+      if (ok && !warp_wait(&self_full[sb2], (tc >> 1) & 1)) ok = false;
+      const float m_run = xm[sb2 * BM + i];
+      const float lt = xl[(sb2 * 2 + 0) * BM + i] + xl[(sb2 * 2 + 1) * BM + i];
+      const float xs = xdot[sb2 * BM + i] * sl2;
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&stat_empty[sb2]);
+        mbar_arrive(&dot_empty[sb2]);
+      }
+      const float mf = fmaxf(m_run, xs);
+      const float alpha = m_run == -INFINITY ? 0.f : exp2f(m_run - mf);
+      const float pself = exp2f(xs - mf);
+      const float inv = 1.f / (lt * alpha + pself);
+      if (ok && !warp_wait(o_full, tc & 1)) ok = false;
+      tc_fence_after();
+      const uint32_t selfb = sSelf + sb2 * SBYTES;
+      // this warp's 32 output rows, and the row / 16-byte piece each lane
+      // stores in the transposed pass
+      __nv_bfloat16* const obase = p.out + ((size_t)((t.b * p.T) + (t.m0 - 1)) * H + 32 * qe) * R;
+      const int tr = lane >> 2, tq = lane & 3;
+#pragma unroll 1
+      for (int c2 = 0; c2 < R / 64; ++c2) {
+        uint32_t ov[64];
+        if (t.nkt > 0) {
+          tmem_ld32(lane_base + O_COL + c2 * 64, *reinterpret_cast<uint32_t(*)[32]>(&ov[0]));
+          tmem_ld32(lane_base + O_COL + c2 * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[32]));
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 64; ++e) ov[e] = 0u;
+        }
+        if (c2 == R / 64 - 1) {
+          // the last read of O in TMEM: the next M tile's value MMAs may start
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(o_empty);
+        }
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int ch = 2 * c2 + hh;          // 32-channel block
+          uint32_t res[16];
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t cv[4];
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(cv[0]), "=r"(cv[1]), "=r"(cv[2]), "=r"(cv[3])
+                         : "r"(selfb + plane_off(QM, srow, ch * 4 + q4)));
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cv[e]));
+              const int k = hh * 32 + q4 * 8 + e * 2;
+              const float v0 = (__uint_as_float(ov[k]) * alpha + pself * c.x) * inv;
+              const float v1 = (__uint_as_float(ov[k + 1]) * alpha + pself * c.y) * inv;
+              res[q4 * 4 + e] = pack_bf16x2(v0, v1);
+            }
+          }
+          __syncwarp();                        // the previous block's transposed reads are done
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const uint32_t off = (uint32_t)lane * 64u + ((((uint32_t)q4) ^ (((uint32_t)lane >> 1) & 3u)) << 4);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(ost + off), "r"(res[4 * q4]),
+                         "r"(res[4 * q4 + 1]), "r"(res[4 * q4 + 2]), "r"(res[4 * q4 + 3]) : "memory");
+          }
+          __syncwarp();
+#pragma unroll
+          for (int k8 = 0; k8 < 4; ++k8) {
+            const int r = 8 * k8 + tr;         // row of the block this lane stores
+            uint32_t w[4];
+            const uint32_t off = (uint32_t)r * 64u + ((((uint32_t)tq) ^ (((uint32_t)r >> 1) & 3u)) << 4);
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                         : "r"(ost + off));
+            *reinterpret_cast<uint4*>(obase + (size_t)r * R + ch * 32 + tq * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&self_empty[sb2]);
+    }
+    if (!ok && lane == 0) set_err(p.dev_err, MTLA_DEVERR_TIMEOUT);
   } else {
-    // ======================= softmax / epilogue warps =======================
+    // ======================= softmax warps =======================
     // warp w: TMEM lane quarter w % 4 (rows 32 (w % 4) .. +31) and half w / 4
     // of the key tile's 64 columns and of O's 256 columns.  Warps w and w + 4
     // own the same rows and agree on the running max every tile (64-thread
@@ -388,7 +494,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     const int qw = warp & 3, hf = warp >> 2;
     const int i = qw * 32 + lane;              // row of the M tile = TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
-    uint8_t* const ost = sm + OFF_OST + warp * OST_BYTES;  // this warp's output staging
     const float sl2 = p.scale_log2;
     uint32_t tc = 0, kc = 0;
     for (int o; (o = tile_index(tc, blockIdx.x, G)) < p.n_mtiles; ++tc) {
@@ -464,81 +569,18 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[sb]);
       }
-      // ---- epilogue: the own row's term, then out = normalised (O + own term)
+      // ---- hand the tile to the epilogue warps: this half's row sum and the
+      // running max (both halves hold the same), once the epilogue of tile
+      // tc - 2 has read this parity's slots
       const int sb2 = tc & 1;
+      if (ok && tc >= 2 && !warp_wait(&stat_empty[sb2], ((tc >> 1) & 1) ^ 1)) ok = false;
       xl[(sb2 * 2 + hf) * BM + i] = l;
-      named_bar(1 + qw, 64);
-      const float lt = xl[(sb2 * 2 + 0) * BM + i] + xl[(sb2 * 2 + 1) * BM + i];
-      if (ok && !warp_wait(&dot_full[sb2], (tc >> 1) & 1)) ok = false;
-      if (ok && !warp_wait(&self_full[sb2], (tc >> 1) & 1)) ok = false;
-      const float xs = xdot[sb2 * BM + i] * sl2;
+      if (hf == 0) xm[sb2 * BM + i] = m_run;
       __syncwarp();
-      if (lane == 0) mbar_arrive(&dot_empty[sb2]);
-      const float mf = fmaxf(m_run, xs);
-      const float alpha = m_run == -INFINITY ? 0.f : exp2f(m_run - mf);
-      const float pself = exp2f(xs - mf);
-      const float inv = 1.f / (lt * alpha + pself);
-      if (ok && !warp_wait(o_full, tc & 1)) ok = false;
-      tc_fence_after();
-      const uint32_t selfb = sSelf + sb2 * SBYTES;
-      const int srow = i / H;
-      const int orow0 = ((t.b * p.T) + (t.m0 - 1)) * H + 32 * qw;  // first output row of this warp
-#pragma unroll 1
-      for (int cc = 0; cc < R / 64; ++cc) {
-        const int ch = 4 * hf + cc;            // 32-channel chunk of this half
-        uint32_t ov[32];
-        if (t.nkt > 0) {
-          tmem_ld32(lane_base + O_COL + ch * 32, ov);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] = 0u;
-        }
-        if (cc == R / 64 - 1) {
-          // the last read of O in TMEM: the next M tile's value MMAs may start
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(o_empty);
-        }
-        uint32_t res[16];
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t cv[4];
-          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(cv[0]), "=r"(cv[1]), "=r"(cv[2]), "=r"(cv[3])
-                       : "r"(selfb + plane_off(QM, srow, ch * 4 + q4)));
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cv[e]));
-            const int k = q4 * 8 + e * 2;
-            const float v0 = (__uint_as_float(ov[k]) * alpha + pself * c.x) * inv;
-            const float v1 = (__uint_as_float(ov[k + 1]) * alpha + pself * c.y) * inv;
-            res[q4 * 4 + e] = pack_bf16x2(v0, v1);
-          }
-        }
-        // stage row `lane` of the warp's 32 x 32 output block (64-byte swizzle,
-        // the tensor map's layout) once the previous block's store has read it,
-        // then one TMA store writes the block to rows orow0.., channels 32 ch..
-        if (lane == 0) bulk_wait_read_all();
-        __syncwarp();
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const uint32_t off = (uint32_t)lane * 64u + ((((uint32_t)q4) ^ (((uint32_t)lane >> 1) & 3u)) << 4);
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(ost) + off), "r"(res[4 * q4]),
-                       "r"(res[4 * q4 + 1]), "r"(res[4 * q4 + 2]), "r"(res[4 * q4 + 3]) : "memory");
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&omap, ost, ch * 32, orow0);
-          bulk_commit();
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&self_empty[sb2]);
+      if (lane == 0) mbar_arrive(&stat_full[sb2]);
       kc += t.nkt;
     }
     if (!ok && lane == 0) set_err(p.dev_err, MTLA_DEVERR_TIMEOUT);
-    if (lane == 0) bulk_wait_all();  // the output stores have completed
   }
 
   tc_fence_before();
@@ -552,8 +594,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 }  // namespace ptc
 
 cudaError_t launch_prefill_tc(const ptc::Params& p, const CUtensorMap& qmap, const CUtensorMap& rmap,
-                              const CUtensorMap& smap, const CUtensorMap& kmap, const CUtensorMap& omap, int grid,
-                              cudaStream_t st) {
+                              const CUtensorMap& smap, const CUtensorMap& kmap, int grid, cudaStream_t st) {
   const size_t smem = ptc::smem_bytes();
   static uint64_t done_mask = 0;
   int dev = 0;
@@ -564,13 +605,12 @@ cudaError_t launch_prefill_tc(const ptc::Params& p, const CUtensorMap& qmap, con
     if (e != cudaSuccess) return e;
     if (dev < 64) done_mask |= 1ull << dev;
   }
-  ptc::prefill_tc_kernel<<<grid, ptc::NT, smem, st>>>(qmap, rmap, smap, kmap, omap, p);
+  ptc::prefill_tc_kernel<<<grid, ptc::NT, smem, st>>>(qmap, rmap, smap, kmap, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_prefill_tc_args(const PrefillTcLaunch& a, const CUtensorMap& qmap, const CUtensorMap& rmap,
-                                   const CUtensorMap& smap, const CUtensorMap& kmap, const CUtensorMap& omap,
-                                   int grid, cudaStream_t st) {
+                                   const CUtensorMap& smap, const CUtensorMap& kmap, int grid, cudaStream_t st) {
   ptc::Params p;
   p.B = a.B;
   p.T = a.T;
@@ -580,7 +620,7 @@ cudaError_t launch_prefill_tc_args(const PrefillTcLaunch& a, const CUtensorMap& 
   p.scale_log2 = a.scale_log2;
   p.out = reinterpret_cast<__nv_bfloat16*>(a.out);
   p.dev_err = a.dev_err;
-  return launch_prefill_tc(p, qmap, rmap, smap, kmap, omap, grid, st);
+  return launch_prefill_tc(p, qmap, rmap, smap, kmap, grid, st);
 }
 
 }  // namespace mtla
