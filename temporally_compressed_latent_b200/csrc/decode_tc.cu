@@ -150,7 +150,13 @@ __device__ __forceinline__ int64_t rows_of(const uint32_t* meta, int b) {
 }
 
 // Block c's share of the C cost positions starts at c C / G.
-__device__ __forceinline__ int64_t share_start(int c, int64_t C, int G) { return C > 0 ? (int64_t)c * C / G : 0; }
+// floor(c C / G) in double precision: c C < 2^53 is exact, and a quotient
+// that is not an integer lies at least 1/G from one, far beyond the rounding
+// error (below 2^-3 ulp of 2^40), so truncation gives the integer quotient
+// without a 64-bit integer division
+__device__ __forceinline__ int64_t share_start(int c, int64_t C, int G) {
+  return C > 0 ? (int64_t)(((double)c * (double)C) / (double)G) : 0;
+}
 // The first sequence with rows in the share [lo, hi), B if the share is empty.
 __device__ __forceinline__ int first_seq(const int64_t* prefix, const uint32_t* meta, int B, int64_t lo, int64_t hi) {
   if (lo >= hi) return B;
@@ -257,23 +263,31 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
     if (lane == 31) sm.prefix[B] = ex;  // total cost
   }
   named_bar(2, PRO_T);
+  const int64_t C = sm.prefix[B];
+  // this block's share: cost positions [my_lo, my_hi).  While the prefix is
+  // written, the threads that own the sequences holding its first and last
+  // positions record them: its first sequence with rows (B if none, the rule
+  // block 0 tabulates for every block below with first_seq) and the sequence
+  // of its last position
+  const int64_t my_lo = share_start(cta, C, G), my_hi = share_start(cta + 1, C, G);
   if (tid < 128) {
     int64_t run = sm.scan[tid];
     for (int b = tid * per; b < B && b < (tid + 1) * per; ++b) {
       sm.prefix[b] = run;
-      run += rows_of(sm.meta, b) + mcost;
+      const int64_t next = run + rows_of(sm.meta, b) + mcost;
+      if (my_lo < my_hi) {
+        if (run <= my_lo && my_lo < next) sm.flags[0] = my_lo - run >= rows_of(sm.meta, b) ? b + 1 : b;
+        if (run <= my_hi - 1 && my_hi - 1 < next) sm.flags[1] = b;
+      }
+      run = next;
     }
   }
   named_bar(2, PRO_T);
-  const int64_t C = sm.prefix[B];
-  // this block's share: cost positions [my_lo, my_hi); its first sequence
-  // with rows (B if none) by the rule block 0 tabulates for every block below
-  const int64_t my_lo = share_start(cta, C, G), my_hi = share_start(cta + 1, C, G);
-  const int b_first = first_seq(sm.prefix, sm.meta, B, my_lo, my_hi);
   // the share's sequences are visited last to first so that a sequence's tail
   // row (whose merge the merge kernel finishes meanwhile) is the block's last
   // tile
-  const int b_last = my_lo < my_hi ? upper_bound_i64(sm.prefix, B + 1, my_hi - 1) - 1 : -1;
+  const int b_first = my_lo < my_hi ? sm.flags[0] : B;
+  const int b_last = my_lo < my_hi ? sm.flags[1] : -1;
   const __nv_bfloat16* cache = reinterpret_cast<const __nv_bfloat16*>(p.a.cache);
 
   // ======================= producer warp =======================
