@@ -56,7 +56,8 @@ constexpr size_t OFF_A = OFF_WLO + WBYTES;
 constexpr size_t OFF_BAR = OFF_A + (size_t)KS * ABLK;
 constexpr int NBAR = 2 * KS + 2 + 2 + 1;
 constexpr size_t OFF_TMEM = OFF_BAR + NBAR * 8;
-constexpr size_t SMEM_USED = OFF_TMEM + 16;
+constexpr size_t OFF_BC = OFF_TMEM + 16;             // this CTA's half of b_c (fp32)
+constexpr size_t SMEM_USED = OFF_BC + NH * 4;
 static_assert(OFF_WLO % 1024 == 0 && OFF_A % 1024 == 0 && WKB % 1024 == 0, "swizzle atoms must be 1024-aligned");
 static_assert(NH % 16 == 0 && NH <= 256, "N of one MMA");
 
@@ -90,6 +91,11 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr) : "memory");
 }
+
+// The gate's sigmoid with the hardware exponential and divide: a few fp32 ulp
+// (relative error near 1e-6), far below the bf16 rounding of what it scales;
+// the fp32 paths of the library keep the correctly rounded form.
+__device__ __forceinline__ float gate_sigmoid(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
 
 __device__ __forceinline__ void unpack8(const uint4& u, float* f) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -157,6 +163,8 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(sm + OFF_WLO + off)), "r"(lo[0]),
                  "r"(lo[1]), "r"(lo[2]), "r"(lo[3]) : "memory");
   }
+  float* const bc_s = reinterpret_cast<float*>(sm + OFF_BC);
+  for (int n = tid; n < NH; n += NT) bc_s[n] = __ldg(p.b_c + half * NH + n);
   fence_proxy_async_smem();  // the tensor core reads what the threads wrote
   tc_fence_before();
   __syncthreads();
@@ -242,30 +250,43 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
       const int64_t tok = (int64_t)b * p.T + nn;
       const int64_t grp = nn / s;                       // 0-based group = P row = cache row
       const bool closes = valid && (pos == s - 1 || n == p.T - 1);
+      // a chunk's inputs (the token's latent or RoPE key, its group's P row)
+      // do not depend on the accumulator: the first chunk's are requested
+      // before the wait, every next chunk's while the current one is processed
+      uint4 vin_c[2], vin_n[2];
+      float4 pr_c[4], pr_n[4];
+      auto fetch = [&](int c16, uint4 (&vi)[2], float4 (&pr)[4]) {
+        if (!valid || c16 >= cend) return;
+        const int ch0 = half * NH + c16 * 16;
+        const __nv_bfloat16* vin = ch0 < R ? p.c + tok * R + ch0 : p.kR + tok * DR + (ch0 - R);
+        vi[0] = __ldg(reinterpret_cast<const uint4*>(vin));
+        vi[1] = __ldg(reinterpret_cast<const uint4*>(vin) + 1);
+        const float4* Pr = reinterpret_cast<const float4*>(p.P + grp * D + ch0);
+#pragma unroll
+        for (int e4 = 0; e4 < 4; ++e4) pr[e4] = __ldg(Pr + e4);
+      };
+      fetch(cbeg, vin_c, pr_c);
       if (!warp_wait(&acc_full[ab], (tc >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
       for (int c16 = cbeg; c16 < cend; ++c16) {
+        fetch(c16 + 1, vin_n, pr_n);
         uint32_t g[16];
         tmem_ld16(lane_base + ab * ACC_STRIDE + c16 * 16, g);
         tmem_wait_ld();
         const int ch0 = half * NH + c16 * 16;
         float x[16];
         if (valid) {
-          const __nv_bfloat16* vin = ch0 < R ? p.c + tok * R + ch0 : p.kR + tok * DR + (ch0 - R);
           float v[16];
-          unpack8(__ldg(reinterpret_cast<const uint4*>(vin)), v);
-          unpack8(__ldg(reinterpret_cast<const uint4*>(vin) + 1), v + 8);
-          const float4* Pr = reinterpret_cast<const float4*>(p.P + grp * D + ch0);
-          const float4* bc = reinterpret_cast<const float4*>(p.b_c + ch0);
+          unpack8(vin_c[0], v);
+          unpack8(vin_c[1], v + 8);
 #pragma unroll
           for (int e4 = 0; e4 < 4; ++e4) {
-            const float4 pv = __ldg(Pr + e4), bv = __ldg(bc + e4);
-            const float pe[4] = {pv.x, pv.y, pv.z, pv.w}, be[4] = {bv.x, bv.y, bv.z, bv.w};
+            const float pe[4] = {pr_c[e4].x, pr_c[e4].y, pr_c[e4].z, pr_c[e4].w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int k = 4 * e4 + e;
-              const float gate = __fadd_rn(__uint_as_float(g[k]), be[e]);
-              const float w = sigmoidf_(__fmul_rn(gate, pe[e]));
+              const float gate = __fadd_rn(__uint_as_float(g[k]), bc_s[c16 * 16 + k]);
+              const float w = gate_sigmoid(__fmul_rn(gate, pe[e]));
               x[k] = __fmul_rn(w, v[k]);
             }
           }
@@ -273,6 +294,10 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
 #pragma unroll
           for (int k = 0; k < 16; ++k) x[k] = 0.f;
         }
+        vin_c[0] = vin_n[0];
+        vin_c[1] = vin_n[1];
+#pragma unroll
+        for (int e4 = 0; e4 < 4; ++e4) pr_c[e4] = pr_n[e4];
         // running merge inside the group: groups start at lanes that are multiples of s
         for (int d = 1; d < s; d <<= 1) {
 #pragma unroll
