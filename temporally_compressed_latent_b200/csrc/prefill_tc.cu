@@ -89,7 +89,6 @@ static_assert(SMEM_USED + 1024 <= 232448, "one block's shared memory (227 KB)");
 struct Params {
   int B, T, s;
   int n_mtiles;            // B * T / QM
-  int n_groups;            // complete groups per sequence, floor(T / s)
   float scale_log2;        // log2(e) / sqrt(d_h)
   __nv_bfloat16* out;      // [B, T, H, R]
   int32_t* dev_err;
@@ -616,7 +615,6 @@ cudaError_t launch_prefill_tc_args(const PrefillTcLaunch& a, const CUtensorMap& 
   p.T = a.T;
   p.s = a.s;
   p.n_mtiles = a.B * (a.T / ptc::QM);
-  p.n_groups = a.T / a.s;
   p.scale_log2 = a.scale_log2;
   p.out = reinterpret_cast<__nv_bfloat16*>(a.out);
   p.dev_err = a.dev_err;
