@@ -71,7 +71,7 @@ constexpr int SEGB = UNIT * 64;          // bytes of one 32-element plane of a t
 constexpr int MAXB = 1024;               // sequences per call
 constexpr int MAXG = 320;                // blocks per launch
 constexpr int OSTR = 260;                // head stride of the combine buffer (floats)
-constexpr int MERGE_COST = 32;           // partition weight of one merge, in rows
+constexpr int MERGE_COST = 128;          // partition weight of one merged sequence, in rows: its tail owner's extra work (merge wait, tail patch, segment ends); 128 measured best of 32-256
 
 struct Params {
   SeqArgs a;
