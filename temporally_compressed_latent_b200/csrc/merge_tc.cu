@@ -24,8 +24,10 @@
 //    Hillis-Steele scan over lanes of ceil(log2 s) shuffle steps, with no
 //    carry between warps or tiles.  TMA loads the four 32-row boxes of a K
 //    block (64 latents, 128 B per row) into one pipeline stage.
-//  * Roles: one TMA warp, one MMA-issuing thread, eight epilogue warps (two
-//    per TMEM lane quarter, splitting the 144 channels).  The accumulator is
+//  * Roles: one TMA warp, one MMA warp (one elected lane issues), twelve
+//    epilogue warps (three per TMEM lane quarter, 48 of the 144 channels
+//    each: the epilogue is latency-bound, so more warps overlap more of it).
+//    The accumulator is
 //    double-buffered in TMEM so a tile's epilogue overlaps the next tile's
 //    MMAs.  The epilogue reads each token's P row, b_c and its own latent /
 //    RoPE key (just loaded, so L2-resident), forms the gate and the gated
@@ -44,8 +46,8 @@ constexpr int ABLK = ROWS * 128;     // one K block of the latent tile: 16384 B
 constexpr int KS = 4;                // latent-tile stages
 constexpr int WKB = NH * 128;        // one K block of a W part: 18432 B
 constexpr int WBYTES = KB * WKB;     // one W part (hi or lo): 73728 B
-constexpr int NEPI = 8;              // epilogue warps
-constexpr int TMA_WARP = 8, MMA_WARP = 9, NT = 320;
+constexpr int NEPI = 12;             // epilogue warps: three per TMEM lane quarter, three chunks each
+constexpr int TMA_WARP = NEPI, MMA_WARP = NEPI + 1, NT = 32 * (NEPI + 2);
 constexpr int NCH = NH / 16;         // 16-column chunks per half: 9
 constexpr uint32_t TMEM_COLS = 512, ACC_STRIDE = 256;
 constexpr uint32_t IDESC = umma_idesc_bf16(ROWS, NH, false, false);
@@ -236,7 +238,7 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
   } else {
     // ======================= epilogue: gate, gated entry, group scan =======================
     const int q = warp & 3;                            // TMEM lane quarter = warp block
-    const int cbeg = warp < 4 ? 0 : 5, cend = warp < 4 ? 5 : NCH;
+    const int cbeg = (warp >> 2) * (NCH / 3), cend = cbeg + NCH / 3;
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     const int s = p.s;
     const int pos = lane % s;                          // position inside the token's group
