@@ -323,28 +323,37 @@ def run_ours(args, rank, world, local_rank):
 
 
 def run_e2e(torch, mtla, md, case, reps, W_c, b_c, P, J_max, ws, ws_bytes, err, stream, dev, K, W):
+    """The decode step through the public API with host buffers: every step
+    copies its inputs (queries, RoPE queries, new latents, new RoPE keys,
+    packed in one pinned buffer) to the device in one copy, runs
+    mtla_decode_attn, reads `out` back and synchronises."""
     B = case.B
     d = case.dims
-    pin = lambda shape, dt: torch.empty(shape, dtype=dt, pin_memory=True)
-    h_qa, h_qr = pin((B, d.H, d.r), torch.bfloat16), pin((B, d.H, d.d_R), torch.bfloat16)
-    h_c, h_k = pin((B, d.r), torch.bfloat16), pin((B, d.d_R), torch.bfloat16)
-    h_out = pin((B, d.H, d.r), torch.float32)
-    h_qa.copy_(torch.from_numpy(case.q_abs).to(torch.bfloat16))
-    h_qr.copy_(torch.from_numpy(case.q_rope).to(torch.bfloat16))
-    h_c.copy_(torch.from_numpy(case.c_new).to(torch.bfloat16))
-    h_k.copy_(torch.from_numpy(case.kR_new).to(torch.bfloat16))
+    parts = [(B, d.H, d.r), (B, d.H, d.d_R), (B, d.r), (B, d.d_R)]  # bf16 each
+    sizes = [int(np.prod(sh)) * 2 for sh in parts]
+    offs = [0]
+    for n_b in sizes[:-1]:
+        offs.append(offs[-1] + (n_b + 15) // 16 * 16)
+    total = offs[-1] + sizes[-1]
+    h_in = torch.empty(total, dtype=torch.uint8, pin_memory=True)
+    d_in = torch.empty(total, dtype=torch.uint8, device=dev)
+    h_out = torch.empty((B, d.H, d.r), dtype=torch.float32, pin_memory=True)
+
+    def view(buf, k):
+        return buf[offs[k]:offs[k] + sizes[k]].view(torch.bfloat16).view(parts[k])
+
+    for k, arr in enumerate([case.q_abs, case.q_rope, case.c_new, case.kR_new]):
+        view(h_in, k).copy_(torch.from_numpy(arr).to(torch.bfloat16))
+    qa, qr, cn, kn = (view(d_in, k) for k in range(4))
     n = min(K, E2E_STEPS)
-    h2d = (h_qa.numel() + h_qr.numel() + h_c.numel() + h_k.numel()) * 2
+    h2d = sum(sizes)
     d2h = h_out.numel() * 4
 
     def one(i):
         rep = reps[i % N_REPLICAS]
-        rep.q_abs.copy_(h_qa, non_blocking=True)
-        rep.q_rope.copy_(h_qr, non_blocking=True)
-        rep.c_new.copy_(h_c, non_blocking=True)
-        rep.kR_new.copy_(h_k, non_blocking=True)
-        merge = {"c_new": rep.c_new, "kR_new": rep.kR_new, "W_c": W_c, "b_c": b_c, "P": P, "J_max": J_max}
-        mtla.mtla_decode_attn(md, B, rep.q_abs, rep.q_rope, merge, rep.cache, rep.cache_rows, d.D, rep.offset,
+        d_in.copy_(h_in, non_blocking=True)
+        merge = {"c_new": cn, "kR_new": kn, "W_c": W_c, "b_c": b_c, "P": P, "J_max": J_max}
+        mtla.mtla_decode_attn(md, B, qa, qr, merge, rep.cache, rep.cache_rows, d.D, rep.offset,
                               rep.capacity, rep.t, rep.cache_len, rep.out, rep.lse, ws, ws_bytes, err,
                               stream=torch.cuda.current_stream())
         h_out.copy_(rep.out, non_blocking=True)
