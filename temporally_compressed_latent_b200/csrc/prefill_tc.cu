@@ -369,6 +369,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           }
           __syncwarp();
         }
+        // a tile without key tiles still waits for the epilogue of tile
+        // tc - 1 before it completes o_full: otherwise o_full could complete
+        // twice before the epilogue waits on the earlier phase
+        if (ok && t.nkt == 0 && tc > 0 && !warp_wait(o_empty, (tc - 1) & 1)) ok = false;
         if (ok) {
           if (elect_one()) umma_commit(o_full);
           __syncwarp();

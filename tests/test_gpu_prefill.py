@@ -238,3 +238,27 @@ def test_running_merge_strides(s, T):
         Cp, _ = _oracle_seq(case.lin, case.c[b], case.kR[b], None, None, dims, with_out=False)
         assert_close(host(run.cp[b]), Cp, "bf16", f"C_hat' s={s} T={T} b={b}")
         assert_close(host(run.cache[b]), oracle.compressed_cache(Cp, s), "bf16", f"cache s={s} T={T} b={b}")
+
+
+@pytest.mark.parametrize("B,s,T", [(1, 1, 16), (5, 2, 16), (1, 3, 48), (2, 16, 4096), (2, 64, 4096),
+                                   (1, 128, 4096)])
+def test_prefill_tensor_core_edges(B, s, T):
+    """Shapes of the tcgen05 kernel the other cases miss: one 16-token query
+    tile per sequence, a single sequence, and long prompts at large strides
+    (most query tiles then see one or two key tiles).  Sampled queries around
+    the group and tile boundaries vs the oracle, every stored row checked."""
+    dims = synth.Dims(H=8, d_h=64, r=256, d_R=32, s=s)
+    case = synth.token_case(dims, B=B, T=T, seed=700 + 7 * s + B, dtype="bf16")
+    run = PrefillRun(dims, "bf16", case.q_abs, case.q_rope, case.c, case.kR, case.lin).run()
+    rng = np.random.default_rng(s + T)
+    edges = [1, 2, s - 1, s, s + 1, 2 * s, 2 * s + 1, 16, 17, 64, 65, 128, 129, T - s, T - 1, T]
+    ms = sorted(set(m for m in edges + rng.integers(1, T + 1, size=16).tolist() if 1 <= m <= T))
+    idx = np.array(ms) - 1
+    P = oracle.pe_table(run.J, case.lin["W_p"], case.lin["b_p"])
+    for b in range(B):
+        Cp = oracle.partial_merge_sequence(case.c[b], case.kR[b], case.lin["W_c"], case.lin["b_c"], P, s)
+        ref = np.stack([oracle.masked_forward_query(m, case.q_abs[b, m - 1], case.q_rope[b, m - 1], Cp, s,
+                                                    dims.d_h)[0] for m in ms])
+        assert_close(host(run.out[b])[idx], ref, "bf16", f"out B={B} s={s} T={T} b={b}")
+        assert_close(host(run.cp[b]), Cp, "bf16", f"C_hat' b={b}")
+        assert_close(host(run.cache[b]), oracle.compressed_cache(Cp, s), "bf16", f"cache b={b}")
