@@ -46,7 +46,7 @@ def test_decode_ragged_b128():
     _check_step(DecodeRun(synth.decode_ragged(), gap=3), what="ragged")
 
 
-@pytest.mark.parametrize("s", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("s", [1, 2, 3, 4, 8, 16, 64])
 @pytest.mark.parametrize("merge", [True, False])
 def test_decode_small_ragged(s, merge):
     dims = synth.Dims(H=8, d_h=64, r=256, d_R=32, s=s)
@@ -76,6 +76,16 @@ def test_decode_many_short_sequences():
     rng = np.random.default_rng(9)
     case = synth.decode_case(dims, rng.integers(1, 12, size=700), seed=9, dtype="bf16")
     _check_step(DecodeRun(case, extra_capacity=1), what="B=700 short")
+
+
+@pytest.mark.parametrize("B", [1024, 1025])
+def test_decode_batch_limit(B):
+    """The largest batch the tensor-core decode takes (1024 sequences) and one
+    more (the generic kernel): short ragged sequences, merge at every step."""
+    dims = synth.Dims(H=8, d_h=64, r=256, d_R=32, s=2)
+    rng = np.random.default_rng(15 + B)
+    case = synth.decode_case(dims, rng.integers(1, 40, size=B), seed=16 + B, dtype="bf16")
+    _check_step(DecodeRun(case, extra_capacity=1), what=f"B={B}")
 
 
 def test_decode_consecutive_steps():
