@@ -115,10 +115,10 @@ mtla_status mtla_merge_append(const mtla_dims *dims, int32_t B, const mtla_merge
  *   out[b,h,:] = sum_j softmax(score)_j c_hat_j,  lse[b,h] = ln sum_j e^score_j.
  *   q_abs [B, H, r], q_rope [B, H, d_R]   cache dtype
  *   out   [B, H, r] fp32;  lse [B, H] fp32 (nullable)
- *   workspace: mtla_workspace_bytes(dims, B, MTLA_WS_DECODE) bytes, zeroed
- *              by the caller ONCE before first use; every call leaves it zeroed
- *              again, so one workspace serves calls that run one after another
- *              on a stream (not calls that overlap).
+ *   workspace: mtla_workspace_bytes(dims, B, MTLA_WS_DECODE) bytes of device
+ *              memory owned by the caller; it needs no initialisation (a call
+ *              reads only what it wrote itself), and one workspace serves calls
+ *              that run one after another on a stream (not calls that overlap).
  * Kernels: bf16 with (H, r, d_R) = (8, 256, 32) and B <= 1024 runs the
  * split-L tensor-core kernel (workspace required); any other supported dims
  * run a one-block-per-sequence kernel (workspace unused, may be NULL).

@@ -258,17 +258,11 @@ mtla_status mtla_decode_attn(const mtla_dims* dims, int32_t B, const void* q_abs
   p.merge_cost = dtc::MERGE_COST;
   p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->d_h));
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  size_t off = 0;
-  p.seq_info = reinterpret_cast<int4*>(ws + off);
-  off += (size_t)B * 16;
-  off = (off + 255) & ~(size_t)255;
-  p.tails = reinterpret_cast<__nv_bfloat16*>(ws + off);
-  off += (size_t)B * dtc::D * 2;
-  off = (off + 255) & ~(size_t)255;
-  p.ws_ml = reinterpret_cast<float*>(ws + off);
-  off += (size_t)2 * grid * dtc::NCW * dtc::H * 2 * 4;
-  off = (off + 255) & ~(size_t)255;
-  p.ws_o = reinterpret_cast<float*>(ws + off);
+  const dtc::WsLayout wl = dtc::ws_layout(B, grid);
+  p.seq_info = reinterpret_cast<int4*>(ws + wl.seq_info);
+  p.tails = reinterpret_cast<__nv_bfloat16*>(ws + wl.tails);
+  p.ws_ml = reinterpret_cast<float*>(ws + wl.ml);
+  p.ws_o = reinterpret_cast<float*>(ws + wl.o);
   return from_cuda(launch_decode_tc(p, maps.m64, maps.m8, grid, cs));
 }
 

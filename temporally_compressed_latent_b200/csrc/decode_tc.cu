@@ -34,9 +34,11 @@
 //    Every block visits its share's sequences last to first, so a tail row is
 //    the last tile of its block; the warp holding it waits for the merge
 //    kernel (hardware-tracked) and patches the finished row into the tile.
-//  * A block that holds only part of a sequence writes its partial (max, sum,
-//    unnormalised output) to the workspace and moves on: no fence, no atomic,
-//    no block ever waits for another.  A second, small kernel chained with
+//  * At the end of each of its sequences a block's four warps combine their
+//    online-softmax states through shared memory.  A sequence held by one
+//    block is written out; otherwise the block writes one partial (max, sum,
+//    unnormalised output per head) to the workspace and moves on: no fence,
+//    no atomic, no block ever waits for another.  A second, small kernel chained with
 //    programmatic dependent launch (its blocks are resident and waiting
 //    before the first kernel ends) combines the split sequences from a
 //    per-sequence partition summary that block 0 publishes (one dependent
@@ -72,17 +74,18 @@ static_assert(2 * (kSmemUsed + 1024 + 1024) + 2 * (1024 + 1024) <= 233472, "shar
 
 size_t smem_bytes() { return kSmemUsed + 1024; }  // + slack to align the base to 1024
 
-size_t workspace_bytes(int B, int grid) {
-  size_t b = 0;
-  b += (size_t)B * 16;  // per-sequence partition summary
-  b = (b + 255) & ~(size_t)255;
-  b += (size_t)B * D * 2;  // tail rows
-  b = (b + 255) & ~(size_t)255;
-  b += (size_t)2 * grid * NCW * H * 2 * 4;  // parts: (max, sum) per head
-  b = (b + 255) & ~(size_t)255;
-  b += (size_t)2 * grid * NCW * H * R * 4;  // parts: unnormalised outputs
-  return b;
+WsLayout ws_layout(int B, int grid) {
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  WsLayout l;
+  l.seq_info = 0;                                     // [B] per-sequence partition summary
+  l.tails = up(l.seq_info + (size_t)B * 16);          // [B][D] tail rows
+  l.ml = up(l.tails + (size_t)B * D * 2);             // parts: (max, sum) per head, two slots per block
+  l.o = up(l.ml + (size_t)2 * grid * H * 2 * 4);      // parts: unnormalised outputs
+  l.total = l.o + (size_t)2 * grid * H * R * 4;
+  return l;
 }
+
+size_t workspace_bytes(int B, int grid) { return ws_layout(B, grid).total; }
 
 // byte offset, inside a tile, of row `row`, 16-byte chunk `ch` (0..35): plane
 // ch / 4 holds the row's 64-byte segment, TMA's 64-byte swizzle XORs chunk
@@ -531,99 +534,90 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
       lA += __shfl_xor_sync(0xffffffffu, lA, o);
       lB += __shfl_xor_sync(0xffffffffu, lB, o);
     }
-    if (r_lo == 0 && r_hi == Lb) {
-      // a sequence held by this block alone: the four warps combine through
-      // shared memory and write out
-      named_bar(1, 128);  // every warp is done with the query buffer
-      if (g == 0) {
-        sm.comb_ml[(cw * H + 2 * q) * 2 + 0] = mA;
-        sm.comb_ml[(cw * H + 2 * q) * 2 + 1] = lA;
-        sm.comb_ml[(cw * H + 2 * q + 1) * 2 + 0] = mB;
-        sm.comb_ml[(cw * H + 2 * q + 1) * 2 + 1] = lB;
-      }
-      named_bar(1, 128);  // comb_ml complete
-      float* wsc = sm.comb_ml + NCW * H * 2;  // [NCW][H] weights exp2(m_w - M), then [H] M and [H] L
-      if (ctid < H) {
-        float M = -INFINITY;
+    // the four warps combine through shared memory: a sequence held by this
+    // block alone is normalised and written out; the block's share of a split
+    // sequence becomes one part (its max, sum and unnormalised output per
+    // head) for the combine kernel
+    const bool whole = r_lo == 0 && r_hi == Lb;
+    const int part = 2 * cta + (b == b_first ? 0 : 1);
+    named_bar(1, 128);  // every warp is done with the query buffer
+    if (g == 0) {
+      sm.comb_ml[(cw * H + 2 * q) * 2 + 0] = mA;
+      sm.comb_ml[(cw * H + 2 * q) * 2 + 1] = lA;
+      sm.comb_ml[(cw * H + 2 * q + 1) * 2 + 0] = mB;
+      sm.comb_ml[(cw * H + 2 * q + 1) * 2 + 1] = lB;
+    }
+    named_bar(1, 128);  // comb_ml complete
+    float* wsc = sm.comb_ml + NCW * H * 2;  // [NCW][H] weights exp2(m_w - M), then [H] M and [H] L
+    if (ctid < H) {
+      float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < NCW; ++w) M = fmaxf(M, sm.comb_ml[(w * H + ctid) * 2]);
-        float Ls = 0.f;
+      for (int w = 0; w < NCW; ++w) M = fmaxf(M, sm.comb_ml[(w * H + ctid) * 2]);
+      float Ls = 0.f;
+#pragma unroll
+      for (int w = 0; w < NCW; ++w) {
+        const float mw = sm.comb_ml[(w * H + ctid) * 2];
+        const float sc = mw == -INFINITY ? 0.f : exp2f(mw - M);
+        wsc[w * H + ctid] = sc;
+        Ls += sc * sm.comb_ml[(w * H + ctid) * 2 + 1];
+      }
+      wsc[NCW * H + ctid] = M;
+      wsc[NCW * H + H + ctid] = Ls;
+    }
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+      // heads 4 pass .. 4 pass + 3 belong to the lanes with q >> 1 == pass
+      if ((q >> 1) == pass) {
+        const int hl = 2 * q - kCombHeads * pass;  // local head of O[.][0]
+#pragma unroll
+        for (int mb = 0; mb < 16; ++mb) {
+          float* oA = sm.comb_o + (cw * kCombHeads + hl) * OSTR + 16 * mb + g;
+          float* oB = oA + OSTR;
+          oA[0] = O[mb][0];
+          oB[0] = O[mb][1];
+          oA[8] = O[mb][2];
+          oB[8] = O[mb][3];
+        }
+      }
+      named_bar(1, 128);
+#pragma unroll
+      for (int hl = 0; hl < kCombHeads; ++hl) {
+        const int h = kCombHeads * pass + hl;
+        const float M = wsc[NCW * H + h], Ls = wsc[NCW * H + H + h];
+        float o0 = 0.f, o1 = 0.f;
 #pragma unroll
         for (int w = 0; w < NCW; ++w) {
-          const float mw = sm.comb_ml[(w * H + ctid) * 2];
-          const float sc = mw == -INFINITY ? 0.f : exp2f(mw - M);
-          wsc[w * H + ctid] = sc;
-          Ls += sc * sm.comb_ml[(w * H + ctid) * 2 + 1];
+          const float sc = wsc[w * H + h];
+          const float2 ov = *reinterpret_cast<const float2*>(sm.comb_o + (w * kCombHeads + hl) * OSTR + 2 * ctid);
+          o0 += sc * ov.x;
+          o1 += sc * ov.y;
         }
-        wsc[NCW * H + ctid] = M;
-        wsc[NCW * H + H + ctid] = Ls;
-      }
-#pragma unroll 1
-      for (int pass = 0; pass < 2; ++pass) {
-        // heads 4 pass .. 4 pass + 3 belong to the lanes with q >> 1 == pass
-        if ((q >> 1) == pass) {
-          const int hl = 2 * q - kCombHeads * pass;  // local head of O[.][0]
-#pragma unroll
-          for (int mb = 0; mb < 16; ++mb) {
-            float* oA = sm.comb_o + (cw * kCombHeads + hl) * OSTR + 16 * mb + g;
-            float* oB = oA + OSTR;
-            oA[0] = O[mb][0];
-            oB[0] = O[mb][1];
-            oA[8] = O[mb][2];
-            oB[8] = O[mb][3];
-          }
-        }
-        named_bar(1, 128);
-#pragma unroll
-        for (int hl = 0; hl < kCombHeads; ++hl) {
-          const int h = kCombHeads * pass + hl;
-          const float M = wsc[NCW * H + h], Ls = wsc[NCW * H + H + h];
-          float o0 = 0.f, o1 = 0.f;
-#pragma unroll
-          for (int w = 0; w < NCW; ++w) {
-            const float sc = wsc[w * H + h];
-            const float2 ov = *reinterpret_cast<const float2*>(sm.comb_o + (w * kCombHeads + hl) * OSTR + 2 * ctid);
-            o0 += sc * ov.x;
-            o1 += sc * ov.y;
-          }
+        if (whole) {
           const float inv = 1.f / Ls;
           *reinterpret_cast<float2*>(p.o.out + ((size_t)b * H + h) * R + 2 * ctid) = make_float2(o0 * inv, o1 * inv);
           if (p.o.lse && ctid == 0) p.o.lse[(size_t)b * H + h] = (M + log2f(Ls)) * 0.69314718055994531f;
+        } else {
+          *reinterpret_cast<float2*>(p.ws_o + ((size_t)part * H + h) * R + 2 * ctid) = make_float2(o0, o1);
+          if (ctid == 0) reinterpret_cast<float2*>(p.ws_ml)[(size_t)part * H + h] = make_float2(M, Ls);
         }
-        named_bar(1, 128);  // the buffer is rewritten by the next pass / segment
       }
-    } else {
-      // part of a split sequence: every warp writes its own part (its rows'
-      // max, sum and unnormalised output per head); no block barrier
-      const int part = NCW * (2 * cta + (b == b_first ? 0 : 1)) + cw;
-      if (g == 0) {
-        float2* pml = reinterpret_cast<float2*>(p.ws_ml) + (size_t)part * H;
-        pml[2 * q] = make_float2(mA, lA);
-        pml[2 * q + 1] = make_float2(mB, lB);
-      }
-      float* po = p.ws_o + (size_t)part * H * R + g;
-#pragma unroll
-      for (int mb = 0; mb < 16; ++mb) {
-        po[(2 * q) * R + 16 * mb] = O[mb][0];
-        po[(2 * q + 1) * R + 16 * mb] = O[mb][1];
-        po[(2 * q) * R + 16 * mb + 8] = O[mb][2];
-        po[(2 * q + 1) * R + 16 * mb + 8] = O[mb][3];
-      }
+      named_bar(1, 128);  // the buffer is rewritten by the next pass / segment
     }
     ++seg;
   }
   // a block with an empty share holds no parts; its slot says so to the combine
-  if (my_lo >= my_hi && ctid < NCW * H)
-    reinterpret_cast<float2*>(p.ws_ml)[(size_t)NCW * 2 * cta * H + ctid] = make_float2(-INFINITY, 0.f);
+  if (my_lo >= my_hi && ctid < H)
+    reinterpret_cast<float2*>(p.ws_ml)[(size_t)2 * cta * H + ctid] = make_float2(-INFINITY, 0.f);
   if (!ok && ctid == 0) set_err(p.a.dev_err, MTLA_DEVERR_TIMEOUT);
 }
 
 // Combine of every sequence's parts and the length bookkeeping.  One block
 // of 256 threads per (sequence, head), thread = latent channel; launched right
 // after the decode kernel with programmatic dependent launch (its blocks wait
-// for the decode grid to complete).  The parts of sequence b are the NCW
-// warps' parts of blocks cf..cl (slot 2c, or 2cf + 1 for block cf when b is
-// not its first sequence).  Per group of up to kGroup parts: their (max, sum)
+// for the decode grid to complete).  The parts of sequence b are those of
+// blocks cf..cl (slot 2c, or 2cf + 1 for block cf when b is not its first
+// sequence); a block whose share is empty marks its slot with a zero weight,
+// and a part of weight zero is never read.  Per group of up to kGroup parts: their (max, sum)
 // pairs go to shared memory while the first kChunk outputs are already in
 // flight; warp 0 turns the pairs into weights e^{m_i - M}; every thread then
 // sums its channel.  Groups merge online:
@@ -649,12 +643,9 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const Params p) {
     return;
   }
   if (info.w <= 1) return;  // one block held the whole sequence and wrote it
-  const int nparts = NCW * info.w;
+  const int nparts = info.w;
   const int cf = info.z >> 1;
-  auto part_of = [&](int i) {
-    const int blk = i / NCW;
-    return NCW * (blk == 0 ? info.z : 2 * (cf + blk)) + i % NCW;
-  };
+  auto part_of = [&](int i) { return i == 0 ? info.z : 2 * (cf + i); };
   float M = -INFINITY, S = 0.f, acc = 0.f;
   for (int g0 = 0; g0 < nparts; g0 += kGroup) {
     const int ng = nparts - g0 < kGroup ? nparts - g0 : kGroup;
@@ -690,14 +681,14 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const Params p) {
     float accg = 0.f;
 #pragma unroll
     for (int u = 0; u < kChunk; ++u)
-      if (u < ng) accg += wts[u] * v[u];
+      if (u < ng && wts[u] != 0.f) accg += wts[u] * v[u];  // a part without rows is never read
     for (int i0 = kChunk; i0 < ng; i0 += kChunk) {
 #pragma unroll
       for (int u = 0; u < kChunk; ++u)
         v[u] = i0 + u < ng ? __ldcg(p.ws_o + ((size_t)part_of(g0 + i0 + u) * H + h) * R + c) : 0.f;
 #pragma unroll
       for (int u = 0; u < kChunk; ++u)
-        if (i0 + u < ng) accg += wts[i0 + u] * v[u];
+        if (i0 + u < ng && wts[i0 + u] != 0.f) accg += wts[i0 + u] * v[u];
     }
     // merge this group into the running result
     const float Mg = red[0], Sg = red[1];

@@ -88,6 +88,12 @@ struct Params {
 };
 
 size_t smem_bytes();
+// Byte offsets of the workspace regions (each on a 256-byte boundary) and its
+// size: one layout for the size query and for the pointers a call carves.
+struct WsLayout {
+  size_t seq_info, tails, ml, o, total;
+};
+WsLayout ws_layout(int B, int grid);
 size_t workspace_bytes(int B, int grid);
 int grid_size();  // blocks of the persistent grid on the current device (0 on error)
 }  // namespace dtc

@@ -130,6 +130,19 @@ def test_decode_workspace_reused_many_calls():
 
 
 
+def test_decode_workspace_needs_no_zeroing():
+    """A workspace full of NaN bytes: short sequences leave some blocks of the
+    split-L grid with empty shares inside a split sequence's block range."""
+    dims = synth.Dims(H=8, d_h=64, r=256, d_R=32, s=2)
+    # fewer cost positions (rows, plus the merge weight of a merged sequence)
+    # than the grid's blocks: one merged sequence, then three without merge
+    for t_prev, merge in (([180], True), ([180, 3, 61], False)):
+        case = synth.decode_case(dims, t_prev, seed=17, dtype="bf16")
+        run = DecodeRun(case)
+        run.ws.fill_(0xFF)
+        _check_step(run, merge=merge, what=f"NaN workspace {t_prev}")
+
+
 def test_decode_device_errors():
     dims = synth.Dims(H=8, d_h=64, r=256, d_R=32, s=2)
     case = synth.decode_case(dims, [8, 9, 0], seed=14, dtype="bf16")
