@@ -12,9 +12,9 @@
 //
 // Set-up: the first call on a device, with that device current, looks up the
 // array's device address (cudaGetSymbolAddress) and clears it on the caller's
-// stream.  That is the "zeroed once before first use" that mtla_decode_attn
-// asks of a workspace; every call then leaves it valid for the next.  Make
-// the first call on each device before any stream capture.
+// stream.  The decode reads only what the same call wrote, so the clearing is
+// not needed for correctness; it only keeps the scratch's first contents
+// defined.  Make the first call on each device before any stream capture.
 //
 // Sharing: every call on a device uses the same scratch, so calls that can
 // overlap (different streams, or threads without ordering between them) race
@@ -27,7 +27,7 @@ namespace mtla {
 namespace {
 
 // file-scope scratch; 24 MiB covers the split-L kernel's workspace for every
-// B it accepts (B <= 1024) on a 148-SM B200 (about 20.2 MB at B = 1024)
+// B it accepts (B <= 1024) on a 148-SM B200 (about 5.5 MB at B = 1024)
 __device__ __align__(256) unsigned char g_decode_scratch[MTLA_DECODE_STATIC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
