@@ -96,6 +96,17 @@ def max_over_ranks(value: float, dist, device) -> float:
     return float(t.item())
 
 
+def decode_step_bytes(t_after, d) -> int:
+    """Algorithmic bytes of one decode step with the merge, for B sequences that
+    hold t_after[b] tokens after it: every cache row read once for all heads,
+    the tail row written, the queries, the new token, out and lse, W_c and b_c
+    once, one P row per sequence."""
+    B = len(t_after)
+    rows = int(sum(synth.ceil_div(int(x), d.s) for x in t_after))
+    return (rows * ROW_BYTES + B * ROW_BYTES + B * d.H * d.D * 2 + B * d.D * 2 + B * d.H * d.r * 4 +
+            B * d.H * 4 + d.r * d.D * 4 + d.D * 4 + B * d.D * 4)
+
+
 def job_throughput(world: int, units_per_rank_step: int, steps: int, ms_max: float) -> float:
     """Whole-job units per second: every rank's units over the slowest rank's time."""
     return world * units_per_rank_step * steps / (ms_max / 1e3)
@@ -204,7 +215,9 @@ def run_ours(args, rank, world, local_rank):
     d = case.dims
     B = case.B
     W, K = args.warmup, args.steps
-    visits = math.ceil((W + K + E2E_STEPS + 8) / N_REPLICAS) + 1
+    # the timed graph is replayed twice (an untimed first replay, then the
+    # timed one), so every replica needs room for W + 2K steps plus e2e
+    visits = math.ceil((W + 2 * K + E2E_STEPS + 8) / N_REPLICAS) + 1
     extra = visits // d.s + 4
     J_max = synth.ceil_div(int(case.t_prev.max()) + visits + 8, d.s) + 1
     W_c = torch.from_numpy(case.lin["W_c"]).to(dev)
@@ -229,13 +242,11 @@ def run_ours(args, rank, world, local_rank):
         rep_i = i % N_REPLICAS
         v = visit[rep_i]
         visit[rep_i] += 1
-        t = case.t_prev + v + 1
-        rows = int(sum(synth.ceil_div(int(x), d.s) for x in t))
-        return (rows * ROW_BYTES + B * ROW_BYTES + B * d.H * d.D * 2 + B * d.D * 2 + B * d.H * d.r * 4 +
-                B * d.H * 4 + d.r * d.D * 4 + d.D * 4 + B * d.D * 4)
+        return decode_step_bytes(case.t_prev + v + 1, d)
 
-    bytes_per_step = [step_bytes(i) for i in range(W + K)]
-    timed_bytes = bytes_per_step[W:]
+    # warm-up graph, the untimed first replay of the timed graph, the timed replay
+    bytes_per_step = [step_bytes(i) for i in list(range(W)) + list(range(W, W + K)) * 2]
+    timed_bytes = bytes_per_step[W + K:]
 
     # capture W warm-up steps and K timed steps as two CUDA graphs (launch cost
     # of a ~6 us kernel must not be Python's); replica i % 8 at step i
@@ -255,14 +266,22 @@ def run_ours(args, rank, world, local_rank):
             step(reps[i % N_REPLICAS], torch.cuda.current_stream())
     torch.cuda.synchronize()
 
+    # the first replay of a graph pays its upload, and the replicas the warm-up
+    # did not reach are cold: replay the timed graph once untimed, so the timed
+    # replay measures steady-state steps whatever K and W are
     with torch.cuda.stream(stream):
         g_warm.replay()
+        g_timed.replay()
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index) as clk:
+        # a short device-side sleep keeps the GPU busy while the host launches
+        # the graph, so the timed region holds steps only, not launch latency
+        with torch.cuda.stream(stream):
+            torch.cuda._sleep(200_000)
         e0.record(stream)
         with torch.cuda.stream(stream):
             g_timed.replay()
@@ -290,6 +309,9 @@ def run_ours(args, rank, world, local_rank):
     prefill = None
     if not args.no_prefill and rank == 0:
         prefill = run_prefill(torch, mtla, glue, dev)
+    configs = None
+    if not args.no_configs and rank == 0:
+        configs = run_configs(torch, mtla, glue, dev)
 
     if dist:
         dist.barrier()
@@ -304,19 +326,22 @@ def run_ours(args, rank, world, local_rank):
                    "s": d.s, "parallelism": f"independent sequences per GPU x{world}",
                    "l2": f"inputs larger than L2: {N_REPLICAS} rotating cache replicas "
                          f"(~{N_REPLICAS * 37.8:.0f} MB > 126 MB L2)",
-                   "timing": "CUDA graph of K steps (3 kernels each: gate, decode, split combine, chained by "
-                             "programmatic dependent launch), CUDA events on the launching stream"},
+                   "timing": "CUDA graph of K steps (one kernel each: merge, attention and split combine; "
+                             "consecutive steps chained by programmatic dependent launch), replayed once untimed, "
+                             "then timed with CUDA events on the launching stream"},
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved_gbs / hbm_peak, "traffic": traffic,
-                     "kernel": "mtla::dtc::decode_tc_kernel (+ its split-combine kernel)",
+                     "kernel": "mtla::dtc::decode_tc_kernel (the whole step)",
                      "peak_kind": f"{peak_kind} copy bandwidth",
                      "algorithmic_bytes_per_launch": sum(timed_bytes) / K},
-        "gpu_launches": 3 * K,  # gate, decode and split-combine kernels per step
+        "gpu_launches": K,  # one decode kernel per step
         "e2e": e2e,
         "clocks": clk.report(),
     }
     if prefill:
         res["prefill"] = prefill
+    if configs:
+        res["configs"] = configs
     if args.cpu_baseline and world == 1:
         res["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     return res
@@ -432,63 +457,296 @@ def run_prefill(torch, mtla, glue, dev):
                     "L2 flushed before each call"}
 
 
+class DecodeState:
+    """One decode workload resident on the device: a paged-contiguous cache
+    with spare rows, lengths, queries and the merge inputs."""
+
+    def __init__(self, torch, mtla, glue, dev, d, t_prev, cache_rows_dev, lin, q_abs, q_rope, c_new, kR_new,
+                 spare_tokens):
+        B = len(t_prev)
+        self.B, self.d, self.mtla = B, d, mtla
+        L = [synth.ceil_div(int(t), d.s) for t in t_prev]
+        caps = [l + spare_tokens // d.s + 2 for l in L]
+        offs = np.concatenate([[0], np.cumsum(caps)])[:-1]
+        self.cache_rows = int(sum(caps))
+        self.cache = torch.zeros(self.cache_rows, d.D, dtype=torch.bfloat16, device=dev)
+        for b in range(B):
+            self.cache[int(offs[b]):int(offs[b]) + L[b]] = cache_rows_dev(b)
+        self.offset = torch.tensor(offs, dtype=torch.int64, device=dev)
+        self.capacity = torch.tensor(caps, dtype=torch.int64, device=dev)
+        self.t_host = np.asarray(t_prev, dtype=np.int64).copy()
+        self.t = torch.tensor(t_prev, dtype=torch.int32, device=dev)
+        self.cache_len = torch.zeros(B, dtype=torch.int32, device=dev)
+        J = synth.ceil_div(int(max(t_prev)) + spare_tokens + 1, d.s) + 1
+        bf = lambda a: (a if torch.is_tensor(a) else torch.from_numpy(np.ascontiguousarray(a, np.float32))).to(
+            dev).to(torch.bfloat16).contiguous()
+        self.q_abs, self.q_rope, c, k = bf(q_abs), bf(q_rope), bf(c_new), bf(kR_new)
+        W_c, b_c = torch.from_numpy(lin["W_c"]).to(dev), torch.from_numpy(lin["b_c"]).to(dev)
+        P = glue.pe_table(J, torch.from_numpy(lin["W_p"]).to(dev), torch.from_numpy(lin["b_p"]).to(dev))
+        self.merge = {"c_new": c, "kR_new": k, "W_c": W_c, "b_c": b_c, "P": P, "J_max": J}
+        self.md = mtla.dims(d.H, d.d_h, d.r, d.d_R, d.s, "bf16")
+        self.ws_bytes = mtla.mtla_workspace_bytes(self.md, B)
+        self.ws = torch.zeros(max(self.ws_bytes, 16), dtype=torch.uint8, device=dev)
+        self.out = torch.empty(B, d.H, d.r, dtype=torch.float32, device=dev)
+        self.lse = torch.empty(B, d.H, dtype=torch.float32, device=dev)
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def call(self):
+        self.mtla.mtla_decode_attn(self.md, self.B, self.q_abs, self.q_rope, self.merge, self.cache,
+                                   self.cache_rows, self.d.D, self.offset, self.capacity, self.t, self.cache_len,
+                                   self.out, self.lse, self.ws, self.ws_bytes, self.err)
+        self.t_host += 1
+
+
+def time_decode_calls(torch, state: DecodeState, n: int, warm: int, flush):
+    """Median time of single decode calls (merge + attention + combine) with
+    L2 flushed before each: the flush also keeps the GPU busy while the call is
+    launched, so the events bracket the call's own kernels.  Each call really
+    advances the state; its algorithmic bytes come from its lengths."""
+    for _ in range(warm):
+        state.call()
+    torch.cuda.synchronize()
+    times, nbytes = [], []
+    for _ in range(n):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        state.call()
+        e1.record()
+        nbytes.append(decode_step_bytes(state.t_host, state.d))
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    if int(state.err.item()):
+        raise RuntimeError(f"device error bits {int(state.err.item())}")
+    ms = statistics.median(times)
+    by = statistics.median(nbytes)
+    hbm_peak, _, _, kind = measured_peaks()
+    gbs = by / (ms / 1e3) / 1e9
+    return {"ms_per_step": ms, "value": state.B / (ms / 1e3), "unit": UNIT, "algorithmic_bytes_per_step": by,
+            "achieved_gbs": gbs, "frac": gbs / hbm_peak, "peak_gbs": hbm_peak, "peak_kind": kind,
+            "roofline_ms": by / (hbm_peak * 1e9) * 1e3, "calls": n}
+
+
+def run_configs(torch, mtla, glue, dev):
+    """The other decode workloads, one call at a time (L2 flushed before each):
+    ragged B=128 (processed lengths uniform in [512, 8192], seed 1) and the
+    compression-ratio sweep B=64, T=16384, s in {1, 2, 3, 4, 8}, whose caches
+    are built on the device by the library's cache-only prefill from latents
+    and RoPE keys drawn on the device (torch generator seeded 4 + s; the merge
+    Linears are the shared generator's draws for that seed)."""
+    import dataclasses
+    n, warm = 20, 3
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    res = {"timing": f"median of {n} single calls after {warm}, CUDA events, L2 flushed before each call"}
+    case = synth.decode_ragged()
+    d = case.dims
+    rows_dev = lambda b: torch.from_numpy(case.rows[b]).to(dev).to(torch.bfloat16)
+    st = DecodeState(torch, mtla, glue, dev, d, case.t_prev, rows_dev, case.lin, case.q_abs, case.q_rope,
+                     case.c_new, case.kR_new, n + warm + 2)
+    r = time_decode_calls(torch, st, n, warm, flush)
+    r["workload"] = ("ragged decode bf16: B=128, H=8, d_h=64, r=256, d_R=32, s=2, processed lengths uniform in "
+                     f"[512, 8192] (seed 1), {int(sum(len(x) for x in case.rows))} cache rows before the calls")
+    res["ragged_b128"] = r
+    del st
+    sweep = {}
+    B, T = 64, 16384
+    for s in (1, 2, 3, 4, 8):
+        d = dataclasses.replace(synth.MAIN, s=s)
+        lin = synth.merge_linears(synth.rng_for(4 + s), d)
+        g = torch.Generator(device=dev)
+        g.manual_seed(4 + s)
+        c = torch.randn(B, T, d.r, generator=g, device=dev).to(torch.bfloat16)
+        kR = torch.randn(B, T, d.d_R, generator=g, device=dev).to(torch.bfloat16)
+        L = synth.ceil_div(T, s)
+        J = synth.ceil_div(T + n + warm + 4, s) + 1
+        P = glue.pe_table(J, torch.from_numpy(lin["W_p"]).to(dev), torch.from_numpy(lin["b_p"]).to(dev))
+        cp = torch.empty(B, T, d.D, dtype=torch.bfloat16, device=dev)
+        built = torch.empty(B, L, d.D, dtype=torch.bfloat16, device=dev)
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+        mtla.mtla_prefill_masked_attn(mtla.dims(d.H, d.d_h, d.r, d.d_R, s, "bf16"), B, T, None, None, c, kR,
+                                      torch.from_numpy(lin["W_c"]).to(dev), torch.from_numpy(lin["b_c"]).to(dev),
+                                      P, J, cp, built, None, err)
+        torch.cuda.synchronize()
+        if int(err.item()):
+            raise RuntimeError(f"device error bits {int(err.item())} building the s={s} cache")
+        del cp, c, kR
+        qa, qr, cn, kn = synth.sweep_step(s, B=B)
+        st = DecodeState(torch, mtla, glue, dev, d, [T] * B, lambda b: built[b], lin, qa, qr, cn, kn,
+                         n + warm + 2)
+        del built
+        r = time_decode_calls(torch, st, n, warm, flush)
+        r["rows_per_sequence_before"] = L
+        sweep[f"s={s}"] = r
+        del st
+        torch.cuda.empty_cache()
+    res["sweep_b64_t16384"] = {"workload": "compression-ratio sweep bf16: B=64, t=16384 processed tokens, H=8, "
+                                           "d_h=64, r=256, d_R=32; cache merged from N(0,1) latents with the "
+                                           "sigmoid gates", **sweep}
+    return res
+
+
 # ---------------------------------------------------------------------------
 # the oracle on the host cores (reference arm and cpu_baseline)
 # ---------------------------------------------------------------------------
-def cpu_baseline(seconds: float):
+# Worker processes are started with "spawn" (never forked from a process that
+# may hold a CUDA context) and read the B=32 workload from one shared-memory
+# block; each runs numpy with one BLAS thread, so the core count is the number
+# of worker processes.
+_WK = {}
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover - non-Linux
+        return os.cpu_count() or 1
+
+
+def _oracle_inputs():
+    """The B=32 decode workload and its P table, as the oracle sees them."""
     import oracle
-    from threadpoolctl import threadpool_limits
     case = synth.decode_uniform(B=32, seed=2)
     d = case.dims
     P = oracle.pe_table(synth.ceil_div(int(case.t_prev.max()) + 1, d.s) + 1, case.lin["W_p"], case.lin["b_p"])
-    done = 0
-    with threadpool_limits(limits=1):
-        t0 = time.perf_counter()
-        while time.perf_counter() - t0 < seconds:
-            b = done % case.B
-            oracle.decode_step(case.rows[b], int(case.t_prev[b]), d.s, case.c_new[b], case.kR_new[b],
-                               case.q_abs[b], case.q_rope[b], case.lin["W_c"], case.lin["b_c"], P, d.d_h)
-            done += 1
-        el = time.perf_counter() - t0
-    return {"value": done / el, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{done} sequence-steps of the B=32 workload (cycling over its sequences) in {el:.1f} s, "
-                      "numpy float64, one thread"}
+    arrays = {"rows": np.concatenate(case.rows).astype(np.float32), "q_abs": case.q_abs, "q_rope": case.q_rope,
+              "c_new": case.c_new, "kR_new": case.kR_new, "W_c": case.lin["W_c"], "b_c": case.lin["b_c"],
+              "P": P.astype(np.float64)}
+    lens = [len(r) for r in case.rows]
+    return case, arrays, lens
+
+
+def _worker_init(shm_name, layout, lens, t_prev, dims):
+    from multiprocessing import shared_memory
+
+    from threadpoolctl import threadpool_limits
+    threadpool_limits(limits=1)
+    # spawned children share the parent's resource tracker: attaching registers
+    # the same name again, and the parent's unlink is the one that counts
+    shm = shared_memory.SharedMemory(name=shm_name)
+    a = {k: np.ndarray(shape, dtype=np.dtype(dt), buffer=shm.buf, offset=off) for k, (off, shape, dt) in
+         layout.items()}
+    starts = np.concatenate([[0], np.cumsum(lens)])
+    _WK.update(shm=shm, a=a, rows=[a["rows"][starts[b]:starts[b + 1]] for b in range(len(lens))],
+               t_prev=t_prev, dims=dims)
+
+
+def _worker_seq(b):
+    """The oracle's decode step (merge + attention) of sequence b."""
+    import oracle
+    a, (H, d_h, r, d_R, s) = _WK["a"], _WK["dims"]
+    oracle.decode_step(_WK["rows"][b], int(_WK["t_prev"][b]), s, a["c_new"][b], a["kR_new"][b], a["q_abs"][b],
+                       a["q_rope"][b], a["W_c"], a["b_c"], a["P"], d_h)
+    return b
+
+
+def _worker_loop(k, n, seconds):
+    """Sequences k, k + n, ... (cyclically) for `seconds`: (steps done, seconds taken)."""
+    B = len(_WK["rows"])
+    done, b = 0, k % B
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < seconds:
+        _worker_seq(b)
+        done += 1
+        b = (b + n) % B
+    return done, time.perf_counter() - t0
+
+
+class OraclePool:
+    """A pool of spawned oracle workers over the shared B=32 workload."""
+
+    def __init__(self, workers: int):
+        import multiprocessing as mp
+        from multiprocessing import shared_memory
+        case, arrays, lens = _oracle_inputs()
+        self.case = case
+        layout, off = {}, 0
+        for k, v in arrays.items():
+            v = np.ascontiguousarray(v)
+            layout[k] = (off, v.shape, v.dtype.str)
+            off += (v.nbytes + 63) // 64 * 64
+        self.shm = shared_memory.SharedMemory(create=True, size=max(off, 64))
+        for k, v in arrays.items():
+            o, shape, dt = layout[k]
+            np.ndarray(shape, dtype=np.dtype(dt), buffer=self.shm.buf, offset=o)[...] = v
+        d = case.dims
+        env_keys = ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")
+        saved = {k: os.environ.get(k) for k in env_keys}
+        os.environ.update({k: "1" for k in env_keys})
+        try:
+            self.pool = mp.get_context("spawn").Pool(
+                workers, initializer=_worker_init,
+                initargs=(self.shm.name, layout, lens, case.t_prev, (d.H, d.d_h, d.r, d.d_R, d.s)))
+        finally:
+            for k, v in saved.items():
+                if v is None:
+                    os.environ.pop(k, None)
+                else:
+                    os.environ[k] = v
+        self.workers = workers
+        # every worker imported numpy and attached the block before timing starts
+        self.pool.map(_worker_seq, [b % case.B for b in range(workers)], chunksize=1)
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+        self.shm.close()
+        self.shm.unlink()
+
+
+def cpu_baseline(seconds: float):
+    """The oracle as it stands on the host: one worker (one thread) for
+    `seconds`, then every host core for `seconds`, each cycling over the
+    32 sequences of the B=32 decode step (merge + attention per sequence)."""
+    cores = host_cores()
+    one = OraclePool(1)
+    try:
+        n1, el1 = one.pool.apply(_worker_loop, (0, 1, seconds))
+    finally:
+        one.close()
+    allp = OraclePool(cores)
+    try:
+        res = allp.pool.starmap(_worker_loop, [(k, cores, seconds) for k in range(cores)], chunksize=1)
+    finally:
+        allp.close()
+    n_all = sum(r[0] for r in res)
+    el_all = max(r[1] for r in res)
+    return {"value": n_all / el_all, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n_all} sequence-steps of the B=32 decode workload (merge + attention over 2048/2049 rows "
+                      f"per sequence, cycling over the 32 sequences) by {cores} worker processes with one "
+                      f"numpy float64 thread each, {el_all:.1f} s; host cores (sched_getaffinity): {cores}",
+            "single_thread": {"value": n1 / el1, "unit": UNIT, "cores": 1,
+                              "sample": f"{n1} sequence-steps in {el1:.1f} s, one worker, one thread"}}
 
 
 def run_reference(args, rank, world):
-    """The oracle, as it stands, on the host cores: each step is a bounded
-    sample of the B=32 decode step (one sequence's merge + attention, cycling
-    over the 32 sequences); W untimed steps, then K timed ones."""
+    """The oracle, as it stands, on the host cores: a step is the whole B=32
+    decode step (every sequence's merge and attention), its 32 sequences spread
+    over min(host cores, 32) worker processes; W untimed steps, then K timed."""
     if rank != 0:
         return None
-    import oracle
-    from threadpoolctl import threadpool_limits
     W, K = args.warmup, args.steps
-    case = synth.decode_uniform(B=32, seed=2)
-    d = case.dims
-    P = oracle.pe_table(synth.ceil_div(int(case.t_prev.max()) + 1, d.s) + 1, case.lin["W_p"], case.lin["b_p"])
-
-    def one(i):
-        b = i % case.B
-        oracle.decode_step(case.rows[b], int(case.t_prev[b]), d.s, case.c_new[b], case.kR_new[b], case.q_abs[b],
-                           case.q_rope[b], case.lin["W_c"], case.lin["b_c"], P, d.d_h)
-
-    with threadpool_limits(limits=1):
-        for i in range(W):
-            one(i)
+    cores = host_cores()
+    workers = min(cores, 32)
+    pool = OraclePool(workers)
+    B = pool.case.B
+    try:
+        for _ in range(W):
+            pool.pool.map(_worker_seq, range(B), chunksize=1)
         t0 = time.perf_counter()
-        for i in range(K):
-            one(W + i)
+        for _ in range(K):
+            pool.pool.map(_worker_seq, range(B), chunksize=1)
         el = time.perf_counter() - t0
-    value = K / el
-    cb = {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-          "sample": f"{K} timed steps, each one sequence of the B=32 workload (merge + attention over "
-                    f"2048/2049 rows), numpy float64, one thread, {el:.1f} s"}
+    finally:
+        pool.close()
+    value = B * K / el
+    cb = {"value": value, "unit": UNIT, "cores": workers, "kind": "oracle",
+          "sample": f"{K} timed steps of the whole B=32 decode workload (merge + attention of all 32 sequences, "
+                    f"2048/2049 rows each) over {workers} worker processes, numpy float64, one thread each, "
+                    f"{el:.1f} s; host cores: {cores}"}
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": W, "ms_per_step": el / K * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1))",
-            "config": {"workload": WORKLOAD, "B_per_gpu": 32,
-                       "step": "one sequence of the B=32 step (bounded sample)"},
+            "config": {"workload": WORKLOAD, "B_per_gpu": B, "step": "the whole B=32 step on the host cores"},
             "cpu_baseline": cb,
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -500,9 +758,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=500)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the ragged and s-sweep decode workloads")
     ap.add_argument("--cpu-baseline", dest="cpu_baseline", action="store_true", default=True)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--cpu-seconds", type=float, default=8.0)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
