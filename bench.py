@@ -326,15 +326,15 @@ def run_ours(args, rank, world, local_rank):
                    "s": d.s, "parallelism": f"independent sequences per GPU x{world}",
                    "l2": f"inputs larger than L2: {N_REPLICAS} rotating cache replicas "
                          f"(~{N_REPLICAS * 37.8:.0f} MB > 126 MB L2)",
-                   "timing": "CUDA graph of K steps (one kernel each: merge, attention and split combine; "
-                             "consecutive steps chained by programmatic dependent launch), replayed once untimed, "
-                             "then timed with CUDA events on the launching stream"},
+                   "timing": "CUDA graph of K steps (3 kernels each: gate and tail row, attention, split combine, "
+                             "chained by programmatic dependent launch), replayed once untimed, then timed with "
+                             "CUDA events on the launching stream"},
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved_gbs / hbm_peak, "traffic": traffic,
-                     "kernel": "mtla::dtc::decode_tc_kernel (the whole step)",
+                     "kernel": "mtla::dtc::decode_tc_kernel with its merge and split-combine kernels (the whole step)",
                      "peak_kind": f"{peak_kind} copy bandwidth",
                      "algorithmic_bytes_per_launch": sum(timed_bytes) / K},
-        "gpu_launches": K,  # one decode kernel per step
+        "gpu_launches": 3 * K,  # merge, decode and split-combine kernels per step
         "e2e": e2e,
         "clocks": clk.report(),
     }

@@ -107,26 +107,25 @@ mtla_status mtla_merge_append(const mtla_dims *dims, int32_t B, const mtla_merge
 /*
  * mtla_decode_attn — one incremental decode step ([rope], [fig2](a)).
  * If merge != NULL the new token is first merged exactly as mtla_merge_append
- * does, in the same launch, and t_processed advances by one; if merge == NULL
- * the cache is read as it stands (t_processed unchanged).  Then for every
- * sequence b and head h, over the L = ceil(t/s) cached rows (the partial tail
- * included):
+ * does, before the attention reads the tail row, and t_processed advances by
+ * one; if merge == NULL the cache is read as it stands (t_processed
+ * unchanged).  Then for every sequence b and head h, over the L = ceil(t/s)
+ * cached rows (the partial tail included):
  *   score_j = (q_abs[b,h] · c_hat_j + q_rope[b,h] · k_hat^R_j) / sqrt(d_h),
  *   out[b,h,:] = sum_j softmax(score)_j c_hat_j,  lse[b,h] = ln sum_j e^score_j.
  *   q_abs [B, H, r], q_rope [B, H, d_R]   cache dtype
  *   out   [B, H, r] fp32;  lse [B, H] fp32 (nullable)
  *   workspace: mtla_workspace_bytes(dims, B, MTLA_WS_DECODE) bytes of device
- *              memory owned by the caller.  Zero it once before its first
- *              call (e.g. cudaMemsetAsync); every call that completes leaves
- *              it ready for the next, so it is not zeroed again, except after
- *              a call that set MTLA_DEVERR_TIMEOUT.  One workspace serves calls
- *              that run one after another on a stream, whatever their B (it
- *              must be at least the size the largest B needs); calls that
- *              overlap need one workspace each.
- * Kernels: bf16 with (H, r, d_R) = (8, 256, 32) and B <= 1024 runs one
- * split-L tensor-core kernel per call (merge, attention and split combine in
- * one launch; workspace required); any other supported dims run a
- * one-block-per-sequence kernel (workspace unused, may be NULL).
+ *              memory owned by the caller; it needs no initialisation (a call
+ *              reads only what it wrote itself), and one workspace serves calls
+ *              that run one after another on a stream (not calls that overlap).
+ * Kernels: bf16 with (H, r, d_R) = (8, 256, 32) and B <= 1024 runs the
+ * split-L tensor-core path as three launches on `stream`, chained by
+ * programmatic dependent launch: the merge (gate, append or in-place update of
+ * the tail row; only if merge != NULL), the attention over row shares, and the
+ * split combine with the length update (workspace required).  Any other
+ * supported dims run a one-block-per-sequence kernel (one launch, merge
+ * included; workspace unused, may be NULL).
  * Supported dims everywhere: H <= 16, r <= 512, r + d_R <= 576, r and d_R
  * multiples of 8 (bf16) or 4 (fp32); otherwise MTLA_ERR_UNSUPPORTED.
  */
@@ -156,17 +155,18 @@ mtla_status mtla_decode_attn(const mtla_dims *dims, int32_t B,
  * without workspace / workspace_bytes.
  * Set-up: the first call on a device (with that device current) looks up the
  *   array's address and clears it on `stream`; make it before any stream
- *   capture.  The address is kept for the life of the process: do not use
- *   this entry point on a device after cudaDeviceReset.
+ *   capture.  The driver reserves the array when it loads this library's
+ *   device code into the context: under lazy module loading (the CUDA
+ *   default) that is this first call.  The address is kept for the life of
+ *   the process: do not use this entry point on a device after
+ *   cudaDeviceReset.
  * Limit: a call whose workspace (mtla_workspace_bytes) would exceed
  *   MTLA_DECODE_STATIC_SCRATCH_BYTES returns MTLA_ERR_WORKSPACE and runs
- *   nothing.  24 MiB covers every B <= 1024 on a 148-SM B200 (about 6.1 MB
+ *   nothing.  24 MiB covers every B <= 1024 on a 148-SM B200 (about 5.5 MB
  *   at B = 1024).
  * Sharing: all calls on a device use the one scratch, so calls that overlap
  *   (other streams, unordered threads) race; issue them one after another on
- *   one stream.  A call that set MTLA_DEVERR_TIMEOUT leaves the scratch's
- *   counters unknown: such an error ends the use of this entry point in the
- *   process.
+ *   one stream.
  */
 #define MTLA_DECODE_STATIC_SCRATCH_BYTES (24u << 20)
 

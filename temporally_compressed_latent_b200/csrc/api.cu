@@ -99,7 +99,7 @@ bool tc_merge_dims(const mtla_dims* d, int B, int T) {
 }
 
 bool tc_prefill_dims(const mtla_dims* d, int B, int T) {
-  return d->dtype == MTLA_BF16 && d->H == 8 && d->r == 256 && d->d_R == 32 && T % 16 == 0 && T >= 16 &&
+  return d->dtype == MTLA_BF16 && d->H == 8 && d->r == 256 && d->d_R == 32 && T >= 1 &&
          (int64_t)B * T * 8 < (int64_t(1) << 31);
 }
 
@@ -256,14 +256,11 @@ mtla_status mtla_decode_attn(const mtla_dims* dims, int32_t B, const void* q_abs
   p.with_merge = merge != nullptr;
   p.B = B;
   p.merge_cost = dtc::MERGE_COST;
-  // gate units of two tokens while they fit one per block, else of eight
-  p.tok_per_unit = (int64_t)((B + 1) / 2) * dtc::GATE_CHUNKS <= (int64_t)grid ? 2 : 8;
   p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->d_h));
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const dtc::WsLayout wl = dtc::ws_layout(B, grid);
-  p.gate_cnt = reinterpret_cast<uint32_t*>(ws);
   p.seq_info = reinterpret_cast<int4*>(ws + wl.seq_info);
-  p.ws_e = reinterpret_cast<float*>(ws + wl.e);
+  p.tails = reinterpret_cast<__nv_bfloat16*>(ws + wl.tails);
   p.ws_ml = reinterpret_cast<float*>(ws + wl.ml);
   p.ws_o = reinterpret_cast<float*>(ws + wl.o);
   return from_cuda(launch_decode_tc(p, maps.m64, maps.m8, grid, cs));
@@ -360,7 +357,7 @@ mtla_status mtla_prefill_masked_attn(const mtla_dims* dims, int32_t B, int32_t T
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->d_h));
   a.out = out;
   a.dev_err = dev_err;
-  const int tiles = B * (T / 16);
+  const int tiles = B * ((T + 15) / 16);
   return from_cuda(launch_prefill_tc_args(a, qmap, rmap, smap, kmap, tiles < sms ? tiles : sms, cs));
 }
 

@@ -12,12 +12,14 @@
 //
 // Set-up: the first call on a device, with that device current, looks up the
 // array's device address (cudaGetSymbolAddress) and clears it on the caller's
-// stream.  The decode keeps a few counters in its scratch that must start at
-// zero, and every call that completes leaves them at zero; the clearing at
-// set-up is what the first call needs.  Make the first call on each device
-// before any stream capture.  The address is kept for the life of the
-// process, so the entry point must not be used on a device after
-// cudaDeviceReset (which unloads the array).
+// stream.  The decode reads only what the same call wrote, so the clearing is
+// not needed for correctness; it only keeps the scratch's first contents
+// defined.  Make the first call on each device before any stream capture.
+// The driver reserves the array when it loads this library's device code
+// into a context; under lazy module loading (the CUDA default) that happens
+// at this first call.  The address is kept for the life of the process, so
+// the entry point must not be used on a device after cudaDeviceReset (which
+// unloads the array).
 //
 // Sharing: every call on a device uses the same scratch, so calls that can
 // overlap (different streams, or threads without ordering between them) race
@@ -30,7 +32,7 @@ namespace mtla {
 namespace {
 
 // file-scope scratch; 24 MiB covers the split-L kernel's workspace for every
-// B it accepts (B <= 1024) on a 148-SM B200 (about 6.1 MB at B = 1024)
+// B it accepts (B <= 1024) on a 148-SM B200 (about 5.5 MB at B = 1024)
 __device__ __align__(256) unsigned char g_decode_scratch[MTLA_DECODE_STATIC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;

@@ -1,6 +1,4 @@
-// Split-L tensor-core decode step for bf16 caches with H = 8, r = 256, d_R = 32:
-// one kernel for the merge of the new tokens and the attention, one for the
-// split combine and the lengths.
+// Split-L tensor-core decode step for bf16 caches with H = 8, r = 256, d_R = 32.
 //
 // What it computes (MTLA paper notes, "Key designs: decoupled RoPE with
 // temporal compression"; Figure 2(a) of the abstract page): for every
@@ -13,15 +11,14 @@
 //  * The H heads share one latent cache, so every cache row (576 B) is read
 //    from HBM exactly once for all heads.  The rows of all sequences are cut
 //    into equal shares for a persistent grid of two blocks per SM (split-L,
-//    balanced to the row; a merged sequence weighs MERGE_COST extra rows).
-//    Every block reads all lengths and derives the same partition.
+//    balanced to the row; a merge counts as MERGE_COST rows).
 //  * One producer warp streams 64-row tiles HBM -> shared memory with 3-D TMA
 //    boxes {32 elements, 64 rows, 9 planes}: the tensor map orders the row's
 //    nine 32-element segments as the outer dimension, so a tile lands as nine
 //    [64 rows x 64 B] planes with the 64-byte swizzle, whose XOR phase then
 //    depends on the row only (every ldmatrix address is a per-lane base plus a
-//    constant).  A ragged last tile uses {32, 8, 1} boxes.  NS stages per
-//    block, mbarrier completion.
+//    constant; this is also the canonical K-major SW64 operand layout).  A
+//    ragged last tile uses {32, 8, 1} boxes.  NS stages, mbarrier completion.
 //  * Four consumer warps each own 16 rows of a tile.  Scores S^T = rows . Q^T
 //    (M = rows, N = the 8 heads, K = 288) and values O^T += C_hat^T . P^T
 //    (M = 256 latent channels, N = 8 heads, K = rows) run on the tensor cores
@@ -29,60 +26,61 @@
 //    value-MMA operand with one in-register 8x8 transpose (movmatrix).  Each
 //    warp keeps its own online-softmax state, so no block barrier is needed
 //    per tile.
-//  * The merge's gate contraction Linear(c_t) (r x D per token) is cut into
-//    units of a few tokens x 32 channels that the consumer warps of the
-//    blocks run while their first tiles are in flight.  A unit writes its
-//    gated entries w * [c_t ; k^R_t] (fp32) to the workspace and counts itself
-//    in its tokens' counters.  Every block visits its share's sequences last
-//    to first, so a tail row is the last tile of its sequence's segment; the
-//    warp holding it waits (bounded) until the nine units of the token are
-//    in, patches the appended or updated row into its tile and writes it to
-//    the cache.
+//  * The merge of the B new tokens runs in a small kernel launched just before
+//    (gate contraction with W_c read as coalesced row segments, gate, gated
+//    entry, append / in-place update of the tail row, written to the cache and
+//    to a workspace copy).  It releases the decode grid at once (programmatic
+//    dependent launch), so the decode blocks set up and stream meanwhile.
+//    Every block visits its share's sequences last to first, so a tail row is
+//    the last tile of its block; the warp holding it waits for the merge
+//    kernel (hardware-tracked) and patches the finished row into the tile.
 //  * At the end of each of its sequences a block's four warps combine their
 //    online-softmax states through shared memory.  A sequence held by one
-//    block is written out; otherwise the block writes one part (max, sum,
-//    unnormalised output per head).  A second kernel, launched behind it with
+//    block is written out; otherwise the block writes one partial (max, sum,
+//    unnormalised output per head) to the workspace and moves on: no fence,
+//    no atomic, no block ever waits for another.  A second, small kernel chained with
 //    programmatic dependent launch (its blocks are resident and waiting
-//    before the first ends), combines the parts of every split sequence, one
-//    block per (sequence, head), from a per-sequence summary the first kernel
-//    writes, advances t_processed / cache_len and resets the gate counters.
+//    before the first kernel ends) combines the split sequences from a
+//    per-sequence partition summary that block 0 publishes (one dependent
+//    load, then every part's loads at once) and advances t_processed /
+//    cache_len.  Every block's share and first sequence are tabulated once in
+//    shared memory, so the bookkeeping in the loops needs no division.
 #include "kernels.cuh"
 
 namespace mtla {
 namespace dtc {
 
-// every region starts on a 128-byte boundary (the queries are read with
+// every region starts on a 128-byte boundary (the tail row is read with
 // 16-byte vector loads, the mbarriers need 8)
 constexpr size_t kAlign = 128;
 __host__ __device__ constexpr size_t rup(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 constexpr int kCombHeads = 4;  // heads per pass of the block combine
 constexpr int QSTR = D / 2 + 4;  // words per query row in shared memory (148: conflict-free)
-constexpr size_t kCombBytes = (size_t)NCW * kCombHeads * OSTR * 4;
-static_assert((size_t)H * QSTR * 4 <= kCombBytes, "query buffer must fit the combine buffer");
-static_assert((size_t)4 * 8 * 32 * 4 <= kCombBytes, "gate partial sums must fit the combine buffer");
+static_assert((size_t)H * QSTR * 4 <= (size_t)NCW * kCombHeads * OSTR * 4, "query buffer must fit the combine buffer");
 constexpr size_t kOffComb = rup((size_t)NS * STAGE);
-constexpr size_t kOffCombMl = kOffComb + rup(kCombBytes);
+constexpr size_t kOffCombMl = kOffComb + rup((size_t)NCW * kCombHeads * OSTR * 4);
 constexpr size_t kOffPrefix = kOffCombMl + rup((size_t)NCW * H * 2 * 4 + (size_t)(NCW + 2) * H * 4);
 constexpr size_t kOffMeta = kOffPrefix + rup((size_t)(MAXB + 1) * 8);
-constexpr size_t kOffQx = kOffMeta + rup((size_t)MAXB * 4);
+constexpr size_t kOffLo = kOffMeta + rup((size_t)MAXB * 4);
+constexpr size_t kOffFs = kOffLo + rup((size_t)(MAXG + 1) * 8);
+constexpr size_t kOffQx = kOffFs + rup((size_t)MAXG * 4);
 constexpr size_t kOffBar = kOffQx + rup((size_t)H * QSTR * 4);
 constexpr size_t kOffFlags = kOffBar + rup(2 * NS * 8);
-constexpr size_t kSmemUsed = kOffFlags + rup(16 * 4);
+constexpr size_t kSmemUsed = kOffFlags + rup(16);
 static_assert(kOffQx % 16 == 0 && kOffBar % 8 == 0, "shared-memory regions must stay aligned");
-static_assert(128 * 8 <= kCombBytes, "scan scratch must fit the combine buffer");
-// two blocks (each with 1 KB of alignment slack and 1 KB the system reserves) fit one SM's 228 KB
-static_assert(2 * (kSmemUsed + 1024 + 1024) <= 233472, "shared memory per SM");
+static_assert(128 * 8 <= (size_t)NCW * kCombHeads * OSTR * 4, "scan scratch must fit the combine buffer");
+// two decode blocks plus two merge-kernel blocks (1 KB each) fit one SM's 228 KB
+static_assert(2 * (kSmemUsed + 1024 + 1024) + 2 * (1024 + 1024) <= 233472, "shared memory per SM");
 
 size_t smem_bytes() { return kSmemUsed + 1024; }  // + slack to align the base to 1024
 
 WsLayout ws_layout(int B, int grid) {
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
   WsLayout l;
-  l.counters = up((size_t)B * 4);                    // gate counters
-  l.seq_info = l.counters;                           // [B] partition summary
-  l.e = up(l.seq_info + (size_t)B * 16);             // [B][D] fp32 gated entries
-  l.ml = up(l.e + (size_t)B * D * 4);                // parts: (max, sum) per head, two slots per block
-  l.o = up(l.ml + (size_t)2 * grid * H * 2 * 4);     // parts: unnormalised outputs
+  l.seq_info = 0;                                     // [B] per-sequence partition summary
+  l.tails = up(l.seq_info + (size_t)B * 16);          // [B][D] tail rows
+  l.ml = up(l.tails + (size_t)B * D * 2);             // parts: (max, sum) per head, two slots per block
+  l.o = up(l.ml + (size_t)2 * grid * H * 2 * 4);      // parts: unnormalised outputs
   l.total = l.o + (size_t)2 * grid * H * R * 4;
   return l;
 }
@@ -96,10 +94,6 @@ __host__ __device__ __forceinline__ uint32_t swz_off(int row, int ch) {
   return (uint32_t)(ch >> 2) * SEGB + (uint32_t)row * 64u + ((((uint32_t)ch & 3u) ^ (((uint32_t)row >> 1) & 3u)) << 4);
 }
 
-// per-sequence summary in shared memory: rows after the call (bits 0..28),
-// whether the new token opens its row (bit 29), whether it is merged (bit 30)
-constexpr uint32_t kMetaRows = (1u << 29) - 1;
-constexpr uint32_t kMetaOpens = 1u << 29;
 constexpr uint32_t kMetaMergeOk = 1u << 30;
 
 struct Smem {
@@ -107,8 +101,10 @@ struct Smem {
   float* comb_o;
   float* comb_ml;
   int64_t* prefix;
-  uint32_t* meta;
+  uint32_t* meta;     // rows (bits 0..29) | merge ok (bit 30)
   int64_t* scan;
+  int64_t* lo;        // [G + 1] first cost position of each block's share
+  int32_t* fs;        // [G] first sequence with rows in each block's share
   uint32_t* qx;       // [H][QSTR] queries of the share's second sequence (prefetched)
   uint64_t* full_bar;
   uint64_t* empty_bar;
@@ -125,6 +121,8 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   s.meta = reinterpret_cast<uint32_t*>(p + kOffMeta);
   // the prologue's scan scratch shares the combine buffer, first used after it
   s.scan = reinterpret_cast<int64_t*>(p + kOffComb);
+  s.lo = reinterpret_cast<int64_t*>(p + kOffLo);
+  s.fs = reinterpret_cast<int32_t*>(p + kOffFs);
   s.qx = reinterpret_cast<uint32_t*>(p + kOffQx);
   s.full_bar = reinterpret_cast<uint64_t*>(p + kOffBar);
   s.empty_bar = s.full_bar + NS;
@@ -142,8 +140,7 @@ __device__ __forceinline__ int upper_bound_i64(const int64_t* a, int n, int64_t 
   return lo;
 }
 
-constexpr int PRO_T = NT;               // every warp takes part in the prologue
-constexpr int CON_T = 32 * NCW;        // threads of the consumer warps
+constexpr int PRO_T = 32 * (NCW + 1);  // threads of the consumer and producer warps
 
 // 16-byte asynchronous global -> shared copies (completion per thread)
 __device__ __forceinline__ void cp_async16(uint32_t saddr, const void* g) {
@@ -151,25 +148,17 @@ __device__ __forceinline__ void cp_async16(uint32_t saddr, const void* g) {
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ int64_t rows_of(const uint32_t* meta, int b) { return (int64_t)(meta[b] & kMetaRows); }
+__device__ __forceinline__ int64_t rows_of(const uint32_t* meta, int b) {
+  return (int64_t)(meta[b] & (kMetaMergeOk - 1));
+}
 
-// Block c of the G_eff blocks that share C cost positions starts at floor(c C / G_eff).
+// Block c's share of the C cost positions starts at c C / G.
 // floor(c C / G) in double precision: c C < 2^53 is exact, and a quotient
 // that is not an integer lies at least 1/G from one, far beyond the rounding
 // error (below 2^-3 ulp of 2^40), so truncation gives the integer quotient
 // without a 64-bit integer division
 __device__ __forceinline__ int64_t share_start(int c, int64_t C, int G) {
   return C > 0 ? (int64_t)(((double)c * (double)C) / (double)G) : 0;
-}
-// The block whose share holds cost position x (0 <= x < C): shares are not
-// empty because G_eff <= C.
-__device__ __forceinline__ int block_of(int64_t x, int64_t C, int G) {
-  int c = (int)(((double)x * (double)G) / (double)C);
-  if (c > G - 1) c = G - 1;
-  if (c < 0) c = 0;
-  while (c > 0 && share_start(c, C, G) > x) --c;
-  while (c + 1 < G && share_start(c + 1, C, G) <= x) ++c;
-  return c;
 }
 // The first sequence with rows in the share [lo, hi), B if the share is empty.
 __device__ __forceinline__ int first_seq(const int64_t* prefix, const uint32_t* meta, int B, int64_t lo, int64_t hi) {
@@ -180,13 +169,13 @@ __device__ __forceinline__ int first_seq(const int64_t* prefix, const uint32_t* 
   return b;
 }
 
-// Sequence b after this call: its rows, whether its new token is merged and
-// opens a row, and the device-error bits the checks raise.
+// Sequence b after this call: its rows, whether its new token is merged, and
+// the device-error bits the checks raise.  The merge kernel (which writes the
+// tail row) and the decode kernel (which partitions the rows) decide alike.
 struct SeqState {
   int64_t t;        // processed tokens after the call
   int64_t L;        // cache rows after the call
   bool merge_ok;
-  bool opens;
   int err;
 };
 __device__ __forceinline__ SeqState seq_state(const Params& p, int b, bool with_merge) {
@@ -197,7 +186,6 @@ __device__ __forceinline__ SeqState seq_state(const Params& p, int b, bool with_
   st.t = t0 + (with_merge ? 1 : 0);
   st.L = st.t > 0 ? group_of(st.t, s) : 0;
   st.merge_ok = with_merge;
-  st.opens = st.t > 0 && opens_row(st.t, s);
   st.err = 0;
   if (t0 < 0 || off < 0 || cap < 0 || off > p.a.cache_rows || cap > p.a.cache_rows - off) {
     st.err |= MTLA_DEVERR_CAPACITY;
@@ -208,7 +196,7 @@ __device__ __forceinline__ SeqState seq_state(const Params& p, int b, bool with_
     st.L = cap;
     st.merge_ok = false;
   }
-  if (st.L > (int64_t)kMetaRows) {  // beyond what one call can address
+  if (st.L >= (int64_t)kMetaMergeOk) {  // beyond what one call can address
     st.err |= MTLA_DEVERR_CAPACITY;
     st.L = 0;
     st.merge_ok = false;
@@ -220,138 +208,20 @@ __device__ __forceinline__ SeqState seq_state(const Params& p, int b, bool with_
   return st;
 }
 
-// Bounded wait (about one second) until *cnt reaches `target`; acquire order
-// for the reads that follow.  False on timeout.
-__device__ __forceinline__ bool wait_count(const uint32_t* cnt, uint32_t target) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
-  if (v >= target) return true;
-  const uint64_t t0 = global_ns();
-  for (;;) {
-    for (int i = 0; i < 64; ++i) {
-      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
-      if (v >= target) return true;
-    }
-    if (global_ns() - t0 > kWaitNs) return false;
-    __nanosleep(64);
-  }
-}
-
-// Release form of the counters' atomic (no full fence needed).
-__device__ __forceinline__ void red_add_release(uint32_t* p, uint32_t v) {
-  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// One gate unit: tokens b0 .. b0 + TPU - 1, channels k0 .. k0 + 31 of the
-// merge gate (MTLA paper notes, "Key designs: hyper-network temporal
-// merging"): w = sigmoid((c_t W_c + b_c) * P[j - 1]) and the gated entry
-// w * [c_t ; k^R_t], written to ws_e.  The four consumer warps run it: warp w
-// takes input rows 64 w .. 64 w + 63 of the contraction, lanes are channels,
-// and every load of the unit is issued at once (gate_issue, then the P row
-// once t_processed has arrived); a block's first unit is issued right after
-// the kernel starts, beside the length loads and before the tile stream
-// floods the memory system.  The warps' partial sums meet in shared memory
-// and are added in a fixed order (deterministic).  The unit then counts
-// itself in each of its tokens' gate counters (release: the entries are
-// visible to the reader that sees the count).
-template <int TPU>
-struct GateIn {
-  static constexpr int NF = (TPU + NCW - 1) / NCW;  // tokens warp w finishes: w, w + 4
-  float wv[64];           // W_c rows 64 w .. 64 w + 63, channel k
-  float cv[2][TPU];       // the tokens' latents of rows 64 w + lane and 64 w + 32 + lane
-  float fb[NF], fp[NF], fx[NF];  // b_c[k], P[j - 1][k] and the entry [c_t ; k^R_t][k] of a finished token
-  int32_t t0[NF];         // its t_processed before the call
-};
-
-template <int TPU>
-__device__ __forceinline__ void gate_issue(const Params& p, int k0, int b0, GateIn<TPU>& g) {
-  const int ctid = threadIdx.x, w = ctid >> 5, lane = ctid & 31;
-  const int k = k0 + lane, i0 = w * 64;
-  const __nv_bfloat16* cn = reinterpret_cast<const __nv_bfloat16*>(p.m.c_new);
-#pragma unroll
-  for (int i = 0; i < 64; ++i) g.wv[i] = __ldg(p.m.W_c + (size_t)(i0 + i) * D + k);
-#pragma unroll
-  for (int half = 0; half < 2; ++half)
-#pragma unroll
-    for (int u = 0; u < TPU; ++u)
-      g.cv[half][u] = b0 + u < p.B ? __bfloat162float(cn[(size_t)(b0 + u) * R + i0 + 32 * half + lane]) : 0.f;
-#pragma unroll
-  for (int f = 0; f < GateIn<TPU>::NF; ++f) {
-    const int b = b0 + w + NCW * f;
-    g.fb[f] = g.fp[f] = g.fx[f] = 0.f;
-    g.t0[f] = -1;
-    if (w + NCW * f < TPU && b < p.B) {
-      g.fb[f] = __ldg(p.m.b_c + k);
-      g.fx[f] = __bfloat162float(k < R ? cn[(size_t)b * R + k]
-                                       : reinterpret_cast<const __nv_bfloat16*>(p.m.kR_new)[(size_t)b * DR + (k - R)]);
-      g.t0[f] = p.a.t_processed[b];
-    }
-  }
-}
-
-// The P row of each finished token's group j = ceil((t0 + 1) / s); a group
-// outside the table is not loaded (that token is not merged: PE_RANGE).
-template <int TPU>
-__device__ __forceinline__ void gate_issue_p(const Params& p, int k0, GateIn<TPU>& g) {
-  const int k = k0 + (threadIdx.x & 31);
-#pragma unroll
-  for (int f = 0; f < GateIn<TPU>::NF; ++f) {
-    if (g.t0[f] < 0) continue;
-    const int64_t j = group_of((int64_t)g.t0[f] + 1, p.a.s);
-    if (j <= p.m.J_max) g.fp[f] = __ldg(p.m.P + (j - 1) * D + k);
-  }
-}
-
-template <int TPU>
-__device__ __forceinline__ void gate_finish(const Params& p, const Smem& sm, int k0, int b0, const GateIn<TPU>& g) {
-  const int ctid = threadIdx.x, w = ctid >> 5, lane = ctid & 31;
-  float* part = sm.comb_o;  // [4 warps][TPU][32]
-  const int k = k0 + lane;
-  float acc[TPU];
-#pragma unroll
-  for (int u = 0; u < TPU; ++u) acc[u] = 0.f;
-#pragma unroll
-  for (int i = 0; i < 64; ++i)
-#pragma unroll
-    for (int u = 0; u < TPU; ++u) acc[u] = fmaf(__shfl_sync(0xffffffffu, g.cv[i >> 5][u], i & 31), g.wv[i], acc[u]);
-#pragma unroll
-  for (int u = 0; u < TPU; ++u) part[(w * TPU + u) * 32 + lane] = acc[u];
-  named_bar(1, CON_T);
-#pragma unroll
-  for (int f = 0; f < GateIn<TPU>::NF; ++f) {
-    const int u = w + NCW * f;
-    const int b = b0 + u;
-    if (u >= TPU || b >= p.B || !(sm.meta[b] & kMetaMergeOk)) continue;
-    float gs = 0.f;
-#pragma unroll
-    for (int ww = 0; ww < NCW; ++ww) gs += part[(ww * TPU + u) * 32 + lane];
-    const float gv = gs + g.fb[f];
-    const float wt = sigmoidf_(__fmul_rn(gv, g.fp[f]));
-    p.ws_e[(size_t)b * D + k] = __fmul_rn(wt, g.fx[f]);
-  }
-  named_bar(1, CON_T);  // every entry of the unit is written (and `part` may be reused)
-  if (ctid < TPU) {
-    const int b = b0 + ctid;
-    if (b < p.B && (sm.meta[b] & kMetaMergeOk)) red_add_release(p.gate_cnt + b, 1u);
-  }
-}
-
-template <int TPU>
-__device__ __forceinline__ int gate_unit_count(int B) { return ((B + TPU - 1) / TPU) * GATE_CHUNKS; }
-
-template <int TPU>
 __global__ void __launch_bounds__(NT, 2)
 decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constant__ CUtensorMap map8,
                  const Params p) {
   extern __shared__ uint8_t smem_raw[];
   const Smem sm = carve(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int B = p.B, G = gridDim.x, cta = blockIdx.x;
+  const int B = p.B, s = p.a.s, G = gridDim.x, cta = blockIdx.x;
   const bool with_merge = p.with_merge != 0;
   const int64_t mcost = with_merge ? p.merge_cost : 0;
 
-  // the next launch on the stream may be scheduled as soon as blocks retire;
-  // it waits for this grid before reading anything (griddepcontrol.wait)
+  // let the next launch on the stream be scheduled as soon as blocks retire.
+  // Without a merge, wait for the previous launch before reading anything it
+  // may write; with a merge the merge kernel just before has already waited
+  // for it, and only the tail rows it writes need it to be complete.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (tid == 0) {
     for (int i = 0; i < NS; ++i) {
@@ -364,15 +234,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
     prefetch_tmap(&map64);
     prefetch_tmap(&map8);
   }
-  // the previous launch may write everything read below: lengths, the cache,
-  // the workspace's counters, this step's inputs
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  // this block's first gate unit: its loads go out now, beside the lengths
-  const int n_units = with_merge ? gate_unit_count<TPU>(B) : 0;
-  const bool first_unit = tid < CON_T && cta < n_units;
-  const int gk0 = (cta % GATE_CHUNKS) * GATE_CH, gb0 = (cta / GATE_CHUNKS) * TPU;
-  GateIn<TPU> gi;
-  if (first_unit) gate_issue<TPU>(p, gk0, gb0, gi);
+  if (!with_merge) asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // ---- 1. rows per sequence and the cost prefix (identical in every block)
   const int per = (B + 127) / 128;
@@ -381,12 +243,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
     for (int b = tid * per; b < B && b < (tid + 1) * per; ++b) {
       const SeqState st = seq_state(p, b, with_merge);
       if (st.err && cta == 0) set_err(p.a.dev_err, st.err);
-      sm.meta[b] = (uint32_t)st.L | (st.merge_ok ? kMetaMergeOk : 0u) | (st.opens ? kMetaOpens : 0u);
+      sm.meta[b] = (uint32_t)st.L | (st.merge_ok ? kMetaMergeOk : 0u);
       sum += st.L + mcost;
     }
     sm.scan[tid] = sum;
   }
-  if (first_unit) gate_issue_p<TPU>(p, gk0, gi);
   named_bar(2, PRO_T);
   if (warp == 0) {
     // exclusive scan of the 128 partial sums (4 per lane)
@@ -406,14 +267,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
   }
   named_bar(2, PRO_T);
   const int64_t C = sm.prefix[B];
-  // shares of the first G_eff blocks (no share is empty); the rest hold none
-  const int Ge = C < (int64_t)G ? (int)C : G;
   // this block's share: cost positions [my_lo, my_hi).  While the prefix is
   // written, the threads that own the sequences holding its first and last
-  // positions record them: its first sequence with rows (B if none) and the
-  // sequence of its last position
-  const int64_t my_lo = cta < Ge ? share_start(cta, C, Ge) : 0;
-  const int64_t my_hi = cta < Ge ? share_start(cta + 1, C, Ge) : 0;
+  // positions record them: its first sequence with rows (B if none, the rule
+  // block 0 tabulates for every block below with first_seq) and the sequence
+  // of its last position
+  const int64_t my_lo = share_start(cta, C, G), my_hi = share_start(cta + 1, C, G);
   if (tid < 128) {
     int64_t run = sm.scan[tid];
     for (int b = tid * per; b < B && b < (tid + 1) * per; ++b) {
@@ -428,10 +287,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
   }
   named_bar(2, PRO_T);
   // the share's sequences are visited last to first so that a sequence's tail
-  // row (whose gated entry other blocks compute meanwhile) is the last tile
-  // of its segment
+  // row (whose merge the merge kernel finishes meanwhile) is the block's last
+  // tile
   const int b_first = my_lo < my_hi ? sm.flags[0] : B;
   const int b_last = my_lo < my_hi ? sm.flags[1] : -1;
+  const __nv_bfloat16* cache = reinterpret_cast<const __nv_bfloat16*>(p.a.cache);
 
   // ======================= producer warp =======================
   if (warp == PRODUCER_WARP) {
@@ -477,6 +337,18 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
   const int cw = warp, ctid = tid;  // 0..127
   const int g = lane >> 2, q = lane & 3;
   const float sl2 = p.scale_log2;
+  // per-lane ldmatrix rows: scores (A = rows, K-major) and values (A = C_hat^T, trans)
+  const int w_lo = 16 * cw;
+  const int arow = w_lo + (lane & 7) + ((lane >> 3) & 1) * 8;
+  const int ach = lane >> 4;
+  const int vrow = w_lo + (lane & 7) + (lane >> 4) * 8;
+  const int vch = (lane >> 3) & 1;
+  // ldmatrix offsets inside a tile: chunk 2 kk + ach of row arow sits in plane
+  // kk / 2 at swz_off(arow, ach) (kk even) or swz_off(arow, 2 + ach) (kk odd)
+  const uint32_t offA0 = swz_off(arow, ach), offA1 = swz_off(arow, 2 + ach);
+  const uint32_t offV0 = swz_off(vrow, vch), offV1 = swz_off(vrow, 2 + vch);
+  uint32_t job = 0;
+  bool ok = true;
 
   // the share's second sequence (in visiting order): its queries are fetched
   // now, so that they do not queue behind the tile stream later
@@ -500,47 +372,30 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
     }
     cp_async_commit();
   }
-
-
-  // the partition as the combine kernel needs it (block c takes sequences
-  // c, c + G, ...): rows, merged, the first part's slot and the number of
-  // parts (blocks cf .. cl hold its rows; block cf's part is in slot 2 cf or
-  // 2 cf + 1, block c > cf's in slot 2 c)
-  for (int b = cta + G * ctid; b < B; b += G * CON_T) {
-    const uint32_t mt = sm.meta[b];
-    const int64_t Lb = (int64_t)(mt & kMetaRows);
-    int first = 0, n = 0;
-    if (Lb > 0) {
-      const int cf = block_of(sm.prefix[b], C, Ge), cl = block_of(sm.prefix[b] + Lb - 1, C, Ge);
-      const int fs = first_seq(sm.prefix, sm.meta, B, share_start(cf, C, Ge), share_start(cf + 1, C, Ge));
-      first = 2 * cf + (fs == b ? 0 : 1);
-      n = cl - cf + 1;
-    }
-    p.seq_info[b] = make_int4((int)Lb, (mt & kMetaMergeOk) ? 1 : 0, first, n);
-  }
-
-  // this block's gate units (the first one's inputs have arrived meanwhile)
-  if (first_unit) gate_finish<TPU>(p, sm, gk0, gb0, gi);
-  for (int u = cta + G; u < n_units; u += G) {
-    const int k0 = (u % GATE_CHUNKS) * GATE_CH, b0 = (u / GATE_CHUNKS) * TPU;
-    gate_issue<TPU>(p, k0, b0, gi);
-    gate_issue_p<TPU>(p, k0, gi);
-    gate_finish<TPU>(p, sm, k0, b0, gi);
-  }
-
-  // per-lane ldmatrix rows: scores (A = rows, K-major) and values (A = C_hat^T, trans)
-  const int w_lo = 16 * cw;
-  const int arow = w_lo + (lane & 7) + ((lane >> 3) & 1) * 8;
-  const int ach = lane >> 4;
-  const int vrow = w_lo + (lane & 7) + (lane >> 4) * 8;
-  const int vch = (lane >> 3) & 1;
-  // ldmatrix offsets inside a tile: chunk 2 kk + ach of row arow sits in plane
-  // kk / 2 at swz_off(arow, ach) (kk even) or swz_off(arow, 2 + ach) (kk odd)
-  const uint32_t offA0 = swz_off(arow, ach), offA1 = swz_off(arow, 2 + ach);
-  const uint32_t offV0 = swz_off(vrow, vch), offV1 = swz_off(vrow, 2 + vch);
-  uint32_t job = 0;
-  bool ok = true;
   int seg = 0;
+
+  // the partition as the combine kernel needs it, published by block 0 while
+  // its first tile is in flight: rows, merge flag, the first part's slot and
+  // the number of parts (blocks cf..cl; block c > cf stored its part in slot
+  // 2c, block cf in 2cf or 2cf + 1)
+  if (cta == 0) {
+    for (int c = ctid; c <= G; c += 128) sm.lo[c] = share_start(c, C, G);
+    named_bar(1, 128);
+    for (int c = ctid; c < G; c += 128) sm.fs[c] = first_seq(sm.prefix, sm.meta, B, sm.lo[c], sm.lo[c + 1]);
+    named_bar(1, 128);
+    for (int bb = ctid; bb < B; bb += 128) {
+      const int64_t Lb = rows_of(sm.meta, bb);
+      const int ok_m = (sm.meta[bb] & kMetaMergeOk) ? 1 : 0;
+      int first = 0, n = 0;
+      if (Lb > 0) {
+        const int cf = upper_bound_i64(sm.lo, G + 1, sm.prefix[bb]) - 1;
+        const int cl = upper_bound_i64(sm.lo, G + 1, sm.prefix[bb] + Lb - 1) - 1;
+        first = 2 * cf + (sm.fs[cf] == bb ? 0 : 1);
+        n = cl - cf + 1;
+      }
+      p.seq_info[bb] = make_int4((int)Lb, ok_m, first, n);
+    }
+  }
 
   for (int b = b_last; b >= b_first; --b) {
     const int64_t Lb = rows_of(sm.meta, b);
@@ -548,8 +403,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
     const int64_t r_end = sm.prefix[b] + Lb < my_hi ? sm.prefix[b] + Lb : my_hi;
     const int64_t r_hi = r_end - sm.prefix[b];
     if (r_lo >= r_hi) continue;
-    const uint32_t mt = sm.meta[b];
-    const bool merge_here = (mt & kMetaMergeOk) && r_hi == Lb;
+    const bool merge_here = (sm.meta[b] & kMetaMergeOk) && r_hi == Lb;
 
     // [q_abs ; q_rope] of the 8 heads into shared memory (rows padded to
     // QSTR words so the B-fragment loads below are free of bank conflicts):
@@ -558,9 +412,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
     const bool pre = (seg == 1 && b == b_second);
     if (pre) {
       cp_async_wait_all();
-      named_bar(1, CON_T);
+      named_bar(1, 128);
     } else {
-      named_bar(1, CON_T);  // every warp is done with the buffer (previous queries, gate sums)
+      if (seg > 0) named_bar(1, 128);  // every warp is done with the previous queries
       const uint32_t* qa = reinterpret_cast<const uint32_t*>(
           reinterpret_cast<const __nv_bfloat16*>(p.o.q_abs) + (size_t)b * H * R);
       const uint32_t* qr = reinterpret_cast<const uint32_t*>(
@@ -570,7 +424,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
         const int h = i / (D / 2), w = i % (D / 2);
         qs[h * QSTR + w] = w < R / 2 ? __ldg(qa + h * (R / 2) + w) : __ldg(qr + h * (DR / 2) + (w - R / 2));
       }
-      named_bar(1, CON_T);
+      named_bar(1, 128);
     }
     // B operand of the score MMA for head g: words 8kk + q and 8kk + q + 4 of its row
     const uint32_t qrow = smem_u32(pre ? reinterpret_cast<float*>(sm.qx) : sm.comb_o) + (uint32_t)(g * QSTR + q) * 4u;
@@ -578,6 +432,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
     float O[16][4];
 #pragma unroll
     for (int mb = 0; mb < 16; ++mb) O[mb][0] = O[mb][1] = O[mb][2] = O[mb][3] = 0.f;
+
 
     for (int64_t u = r_lo; u < r_hi; u += UNIT) {
       const bool is_tail = merge_here && u + UNIT >= r_hi;
@@ -601,38 +456,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
         if (is_tail) {
           const int lr = (int)(Lb - 1 - u);
           if (lr >= w_lo && lr < w_lo + 16) {
-            // the nine gate units of b's new token are in (bounded wait; they
-            // ran first thing in their blocks), then the appended or updated
-            // row: in the tile for the attention and in the cache
-            bool ready = true;
-            if (lane == 0) ready = wait_count(p.gate_cnt + b, GATE_CHUNKS);
-            ready = __shfl_sync(0xffffffffu, ready ? 1 : 0, 0) != 0;
-            __syncwarp();
-            if (!ready) {
-              ok = false;
-            } else {
-              const bool opens = (mt & kMetaOpens) != 0;
-              const float4* e4 = reinterpret_cast<const float4*>(p.ws_e + (size_t)b * D);
-              uint4* crow = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.a.cache) +
-                                                     (p.a.seq_offset[b] + Lb - 1) * p.a.row_stride);
-              for (int ch = lane; ch < 36; ch += 32) {
-                const float4 ea = __ldcg(e4 + 2 * ch), eb = __ldcg(e4 + 2 * ch + 1);
-                const float e[8] = {ea.x, ea.y, ea.z, ea.w, eb.x, eb.y, eb.z, eb.w};
-                uint32_t old[4];
-                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(old[0]), "=r"(old[1]), "=r"(old[2]),
-                             "=r"(old[3]) : "r"(tile + swz_off(lr, ch)));
-                uint32_t nv[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  const float2 o2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&old[i]));
-                  const float v0 = opens ? e[2 * i] : __fadd_rn(o2.x, e[2 * i]);
-                  const float v1 = opens ? e[2 * i + 1] : __fadd_rn(o2.y, e[2 * i + 1]);
-                  nv[i] = pack_bf16x2(v0, v1);
-                }
-                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(tile + swz_off(lr, ch)), "r"(nv[0]),
-                             "r"(nv[1]), "r"(nv[2]), "r"(nv[3]) : "memory");
-                crow[ch] = make_uint4(nv[0], nv[1], nv[2], nv[3]);
-              }
+            // the merge kernel wrote the updated row (the copy the tile holds
+            // may predate it); hardware-tracked wait for that kernel, no polling
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            const uint4* src = reinterpret_cast<const uint4*>(p.tails + (size_t)b * D);
+            for (int ch = lane; ch < 36; ch += 32) {
+              const uint4 v = __ldcg(src + ch);
+              asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(tile + swz_off(lr, ch)), "r"(v.x),
+                           "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
             }
             wrote = true;
           }
@@ -706,17 +537,17 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
     // the four warps combine through shared memory: a sequence held by this
     // block alone is normalised and written out; the block's share of a split
     // sequence becomes one part (its max, sum and unnormalised output per
-    // head)
+    // head) for the combine kernel
     const bool whole = r_lo == 0 && r_hi == Lb;
     const int part = 2 * cta + (b == b_first ? 0 : 1);
-    named_bar(1, CON_T);  // every warp is done with the query buffer
+    named_bar(1, 128);  // every warp is done with the query buffer
     if (g == 0) {
       sm.comb_ml[(cw * H + 2 * q) * 2 + 0] = mA;
       sm.comb_ml[(cw * H + 2 * q) * 2 + 1] = lA;
       sm.comb_ml[(cw * H + 2 * q + 1) * 2 + 0] = mB;
       sm.comb_ml[(cw * H + 2 * q + 1) * 2 + 1] = lB;
     }
-    named_bar(1, CON_T);  // comb_ml complete
+    named_bar(1, 128);  // comb_ml complete
     float* wsc = sm.comb_ml + NCW * H * 2;  // [NCW][H] weights exp2(m_w - M), then [H] M and [H] L
     if (ctid < H) {
       float M = -INFINITY;
@@ -748,7 +579,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
           oB[8] = O[mb][3];
         }
       }
-      named_bar(1, CON_T);
+      named_bar(1, 128);
 #pragma unroll
       for (int hl = 0; hl < kCombHeads; ++hl) {
         const int h = kCombHeads * pass + hl;
@@ -770,24 +601,27 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
           if (ctid == 0) reinterpret_cast<float2*>(p.ws_ml)[(size_t)part * H + h] = make_float2(M, Ls);
         }
       }
-      named_bar(1, CON_T);  // the buffer is rewritten by the next pass / segment
+      named_bar(1, 128);  // the buffer is rewritten by the next pass / segment
     }
     ++seg;
   }
+  // a block with an empty share holds no parts; its slot says so to the combine
+  if (my_lo >= my_hi && ctid < H)
+    reinterpret_cast<float2*>(p.ws_ml)[(size_t)2 * cta * H + ctid] = make_float2(-INFINITY, 0.f);
   if (!ok && ctid == 0) set_err(p.a.dev_err, MTLA_DEVERR_TIMEOUT);
 }
 
-// Combine of every split sequence's parts and the length bookkeeping.  One
-// block of 256 threads per (sequence, head), thread = latent channel;
-// launched right after the decode kernel with programmatic dependent launch
-// (its blocks wait for the decode grid to complete).  The parts of sequence b
-// are those of blocks cf..cl (slot 2c, or first_slot for block cf).  Per
-// group of up to kGroup parts: their (max, sum) pairs go to shared memory
-// while the first kChunk outputs are already in flight; warp 0 turns the
-// pairs into weights e^{m_i - M}; every thread then sums its channel.  Groups
-// merge online: out = sum_i e^{m_i - M} o_i / sum_i e^{m_i - M} l_i,
-// lse = M + ln(sum).  Block (b, 0) also advances t_processed and cache_len
-// and resets b's gate counter for the next call.
+// Combine of every sequence's parts and the length bookkeeping.  One block
+// of 256 threads per (sequence, head), thread = latent channel; launched right
+// after the decode kernel with programmatic dependent launch (its blocks wait
+// for the decode grid to complete).  The parts of sequence b are those of
+// blocks cf..cl (slot 2c, or 2cf + 1 for block cf when b is not its first
+// sequence); a block whose share is empty marks its slot with a zero weight,
+// and a part of weight zero is never read.  Per group of up to kGroup parts: their (max, sum)
+// pairs go to shared memory while the first kChunk outputs are already in
+// flight; warp 0 turns the pairs into weights e^{m_i - M}; every thread then
+// sums its channel.  Groups merge online:
+// out = sum_i e^{m_i - M} o_i / sum_i e^{m_i - M} l_i, lse = M + ln(sum).
 constexpr int kGroup = 256, kChunk = 40;
 __global__ void __launch_bounds__(256) decode_combine_kernel(const Params p) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -796,11 +630,10 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const Params p) {
   __shared__ float lsum[kGroup];
   __shared__ float red[2];
   const int b = blockIdx.x / H, h = blockIdx.x % H, c = threadIdx.x;
-  const int4 info = __ldcg(p.seq_info + b);  // rows, merged, first part's slot, parts
+  const int4 info = __ldcg(p.seq_info + b);  // rows, merge ok, first block's slot, blocks
   if (h == 0 && c == 0) {
-    if (info.y) p.a.t_processed[b] = p.a.t_processed[b] + 1;
+    if (p.with_merge && info.y) p.a.t_processed[b] = p.a.t_processed[b] + 1;
     if (p.a.cache_len) p.a.cache_len[b] = info.x;
-    p.gate_cnt[b] = 0u;
   }
   float* out = p.o.out + ((size_t)b * H + h) * R;
   if (info.x == 0) {
@@ -833,7 +666,7 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const Params p) {
       for (int o = 16; o > 0; o >>= 1) Mg = fmaxf(Mg, __shfl_xor_sync(0xffffffffu, Mg, o));
       float Sg = 0.f;
       for (int i = c; i < ng; i += 32) {
-        const float w = wts[i] == -INFINITY ? 0.f : exp2f(wts[i] - Mg);
+        const float w = wts[i] == -INFINITY ? 0.f : exp2f(wts[i] - Mg);  // a warp without rows weighs 0
         wts[i] = w;
         Sg += w * lsum[i];
       }
@@ -848,14 +681,14 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const Params p) {
     float accg = 0.f;
 #pragma unroll
     for (int u = 0; u < kChunk; ++u)
-      if (u < ng) accg += wts[u] * v[u];
+      if (u < ng && wts[u] != 0.f) accg += wts[u] * v[u];  // a part without rows is never read
     for (int i0 = kChunk; i0 < ng; i0 += kChunk) {
 #pragma unroll
       for (int u = 0; u < kChunk; ++u)
         v[u] = i0 + u < ng ? __ldcg(p.ws_o + ((size_t)part_of(g0 + i0 + u) * H + h) * R + c) : 0.f;
 #pragma unroll
       for (int u = 0; u < kChunk; ++u)
-        if (i0 + u < ng) accg += wts[i0 + u] * v[u];
+        if (i0 + u < ng && wts[i0 + u] != 0.f) accg += wts[i0 + u] * v[u];
     }
     // merge this group into the running result
     const float Mg = red[0], Sg = red[1];
@@ -870,21 +703,83 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const Params p) {
   if (p.o.lse && c == 0) p.o.lse[(size_t)b * H + h] = (M + log2f(S)) * 0.69314718055994531f;
 }
 
+// The merge of every sequence's new token (Linear(c_t) of the merge, the gate,
+// the gated entry and the append / in-place update of the tail row), before
+// the decode kernel reads the cache.  Block = 32 channels x 2 tokens, 128
+// threads: warp w takes input rows 64w .. 64w+63 of the gate contraction (its
+// W_c column segments all in flight at once), lanes are channels; the four
+// warps' partial sums are added in a fixed order, so the result is
+// deterministic.  Small on purpose (1 KB of shared memory, few registers): its
+// blocks share SMs with two decode blocks, which start while it runs.  The
+// updated row goes to the cache and to the workspace copy that the decode
+// kernel patches into its tile.
+constexpr int kMergeTok = 2;
+__global__ void __launch_bounds__(128) decode_merge_kernel(const Params p) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __shared__ float part[4][kMergeTok][32];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kt = blockIdx.x % (D / 32), bt = blockIdx.x / (D / 32);
+  const int k = kt * 32 + lane, b0 = bt * kMergeTok, i0 = w * 64;
+  const __nv_bfloat16* cn = reinterpret_cast<const __nv_bfloat16*>(p.m.c_new);
+  float acc[kMergeTok];
+#pragma unroll
+  for (int u = 0; u < kMergeTok; ++u) acc[u] = 0.f;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int ib = i0 + 32 * half;
+    float wv[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) wv[i] = __ldg(p.m.W_c + (size_t)(ib + i) * D + k);
+    float cv[kMergeTok];
+#pragma unroll
+    for (int u = 0; u < kMergeTok; ++u)
+      cv[u] = b0 + u < p.B ? __bfloat162float(cn[(size_t)(b0 + u) * R + ib + lane]) : 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+#pragma unroll
+      for (int u = 0; u < kMergeTok; ++u) acc[u] = fmaf(__shfl_sync(0xffffffffu, cv[u], i), wv[i], acc[u]);
+  }
+#pragma unroll
+  for (int u = 0; u < kMergeTok; ++u) part[w][u][lane] = acc[u];
+  __syncthreads();
+  if (w >= kMergeTok) return;
+  const int u = w;  // thread -> token b0 + u, channel k
+  float g = 0.f;
+#pragma unroll
+  for (int ww = 0; ww < 4; ++ww) g += part[ww][u][lane];
+  const int b = b0 + u;
+  if (b >= p.B) return;
+  const SeqState st = seq_state(p, b, true);
+  if (!st.merge_ok) return;  // the decode kernel reports why
+  const int s = p.a.s;
+  const int64_t j = group_of(st.t, s);
+  const bool opens = opens_row(st.t, s);
+  __nv_bfloat16* row = reinterpret_cast<__nv_bfloat16*>(p.a.cache) + (p.a.seq_offset[b] + j - 1) * p.a.row_stride;
+  const float gv = g + __ldg(p.m.b_c + k);
+  const float wt = sigmoidf_(__fmul_rn(gv, __ldg(p.m.P + (j - 1) * D + k)));
+  const __nv_bfloat16* xin = k < R ? reinterpret_cast<const __nv_bfloat16*>(p.m.c_new) + (size_t)b * R + k
+                                   : reinterpret_cast<const __nv_bfloat16*>(p.m.kR_new) + (size_t)b * DR + (k - R);
+  const float e = __fmul_rn(wt, __bfloat162float(*xin));
+  const float v = opens ? e : __fadd_rn(__bfloat162float(row[k]), e);
+  const __nv_bfloat16 vb = __float2bfloat16_rn(v);
+  row[k] = vb;
+  p.tails[(size_t)b * D + k] = vb;
+}
+
 int grid_size() {
   int dev = 0, sms = 0, occ = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  // two blocks of ~107 KB need the largest shared-memory configuration
-  for (const void* fn : {(const void*)decode_tc_kernel<2>, (const void*)decode_tc_kernel<8>}) {
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes()) != cudaSuccess)
-      return 0;
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared) !=
-        cudaSuccess)
-      return 0;
-    int o = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, fn, NT, smem_bytes()) != cudaSuccess) return 0;
-    occ = occ == 0 ? o : (o < occ ? o : occ);
-  }
+  if (cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes()) !=
+      cudaSuccess)
+    return 0;
+  // two blocks of ~110 KB need the largest shared-memory configuration
+  if (cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+    return 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_tc_kernel, NT, smem_bytes()) != cudaSuccess)
+    return 0;
   if (occ < 1) return 0;
   const int g = sms * (occ < 2 ? occ : 2);
   return g < MAXG ? g : MAXG;
@@ -895,28 +790,28 @@ int grid_size() {
 cudaError_t launch_decode_tc(const dtc::Params& p, const CUtensorMap& map64, const CUtensorMap& map8, int grid,
                              cudaStream_t st) {
   const size_t smem = dtc::smem_bytes();
-  // the attributes are set once per device (also keeps the call out of stream captures)
+  // the attribute is set once per device (also keeps the call out of stream captures)
   static uint64_t done_mask = 0;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 64 || !(done_mask & (1ull << dev))) {
-    for (const void* fn : {(const void*)dtc::decode_tc_kernel<2>, (const void*)dtc::decode_tc_kernel<8>}) {
-      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
-      if (e != cudaSuccess) return e;
-    }
-    // the same shared-memory configuration for the combine kernel, so that an
-    // SM running its blocks can take the next step's decode blocks at once
+    e = cudaFuncSetAttribute(dtc::decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(dtc::decode_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    // the same shared-memory configuration for the kernels around it, so that
+    // an SM running one of their blocks can take decode blocks at once
+    // (changing the configuration waits for the SM to drain)
+    e = cudaFuncSetAttribute(dtc::decode_merge_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(dtc::decode_combine_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     if (dev < 64) done_mask |= 1ull << dev;
   }
-  // programmatic dependent launch: the blocks may start (barrier set-up,
-  // tensor-map prefetch) while the previous launch on the stream finishes;
-  // griddepcontrol.wait holds them before their first read
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -927,8 +822,19 @@ cudaError_t launch_decode_tc(const dtc::Params& p, const CUtensorMap& map64, con
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = p.tok_per_unit == 2 ? cudaLaunchKernelEx(&cfg, dtc::decode_tc_kernel<2>, map64, map8, p)
-                          : cudaLaunchKernelEx(&cfg, dtc::decode_tc_kernel<8>, map64, map8, p);
+  if (p.with_merge) {
+    cudaLaunchConfig_t cfg0 = {};
+    cfg0.gridDim = dim3((unsigned)((dtc::D / 32) * ((p.B + dtc::kMergeTok - 1) / dtc::kMergeTok)));
+    cfg0.blockDim = dim3(128);
+    cfg0.stream = st;
+    // plain stream order (no early launch): launched early, its blocks would
+    // pile onto the SMs the previous step's kernels leave free first and keep
+    // decode blocks off them; after the previous step they spread one per SM
+    cfg0.numAttrs = 0;
+    e = cudaLaunchKernelEx(&cfg0, dtc::decode_merge_kernel, p);
+    if (e != cudaSuccess) return e;
+  }
+  e = cudaLaunchKernelEx(&cfg, dtc::decode_tc_kernel, map64, map8, p);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg2 = {};
   cfg2.gridDim = dim3((unsigned)(p.B * dtc::H));

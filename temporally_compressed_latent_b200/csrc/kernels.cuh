@@ -56,8 +56,7 @@ struct PrefillArgs {
   int32_t J_max;
 };
 
-// Split-L tensor-core decode (bf16, H = 8, r = 256, d_R = 32): merge,
-// attention and split combine in one kernel per step.
+// Split-L tensor-core decode (bf16, H = 8, r = 256, d_R = 32).
 namespace dtc {
 constexpr int H = 8, R = 256, DR = 32, D = R + DR;
 constexpr int UNIT = 64;                 // rows per full TMA box
@@ -72,9 +71,7 @@ constexpr int SEGB = UNIT * 64;          // bytes of one 32-element plane of a t
 constexpr int MAXB = 1024;               // sequences per call
 constexpr int MAXG = 320;                // blocks per launch
 constexpr int OSTR = 260;                // head stride of the combine buffer (floats)
-constexpr int GATE_CH = 32;              // channels of one gate unit
-constexpr int GATE_CHUNKS = D / GATE_CH; // gate units of one token (9)
-constexpr int MERGE_COST = 64;           // partition weight of one merged sequence, in rows (its tail patch)
+constexpr int MERGE_COST = 128;          // partition weight of one merged sequence, in rows: its tail owner's extra work (merge wait, tail patch, segment ends); 128 measured best of 32-256
 
 struct Params {
   SeqArgs a;
@@ -83,22 +80,18 @@ struct Params {
   int with_merge;
   int B;
   int merge_cost;
-  int tok_per_unit;     // tokens per gate unit: 2 or 8
   float scale_log2;     // log2(e) / sqrt(d_h)
-  uint32_t* gate_cnt;   // [B] gate units published per token (zero between calls)
-  int4* seq_info;       // [B] {rows, merged, first part's slot, parts} for the combine
-  float* ws_e;          // [B][D] gated entries w * [c_t ; k^R_t] of the new tokens (fp32)
-  float* ws_ml;         // [2 * grid][H][2] parts: (max, sum) per head
-  float* ws_o;          // [2 * grid][H][R] parts: unnormalised outputs
+  int4* seq_info;       // [B] {rows, merge ok, first part slot, part count} for the combine
+  __nv_bfloat16* tails; // [B][D] updated tail row of every merged sequence (merge kernel)
+  float* ws_ml;         // [2 * grid][H][2]
+  float* ws_o;          // [2 * grid][H][R]
 };
 
 size_t smem_bytes();
 // Byte offsets of the workspace regions (each on a 256-byte boundary) and its
 // size: one layout for the size query and for the pointers a call carves.
-// The counters come first: `counters` bytes from offset 0 must be zero before
-// the first call and are left zero by every call that completes.
 struct WsLayout {
-  size_t counters, seq_info, e, ml, o, total;
+  size_t seq_info, tails, ml, o, total;
 };
 WsLayout ws_layout(int B, int grid);
 size_t workspace_bytes(int B, int grid);
@@ -112,7 +105,7 @@ cudaError_t launch_decode_tc(const dtc::Params& p, const CUtensorMap& map64, con
                              cudaStream_t st);
 cudaError_t launch_partial_merge(const PrefillArgs& p, int B, int dtype, cudaStream_t st);
 
-// Masked prefill on tcgen05 (bf16, H = 8, r = 256, d_R = 32, T % 16 == 0).
+// Masked prefill on tcgen05 (bf16, H = 8, r = 256, d_R = 32, any T >= 1).
 namespace ptc {
 struct Params;
 size_t smem_bytes();

@@ -145,13 +145,17 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
 // increasing in r for every block
 __device__ __forceinline__ int tile_index(int r, int x, int G) { return r * G + ((r & 1) ? G - 1 - x : x); }
 
+// A sequence's last M tile is ragged when T is not a multiple of QM: its rows
+// past query T read finite values (the next sequence's rows, or the TMA fill
+// past the last one) and are never stored.
 __device__ __forceinline__ Tile tile_of(const Params& p, int o) {
-  const int per_seq = p.T / QM;
+  const int per_seq = (p.T + QM - 1) / QM;
   Tile t;
   t.b = o % p.B;
   const int mb = per_seq - 1 - o / p.B;
   t.m0 = mb * QM + 1;
-  const int vis_max = (int)group_of(t.m0 + QM - 1, p.s) - 1;  // groups seen by the last query
+  const int m_last = t.m0 + QM - 1 < p.T ? t.m0 + QM - 1 : p.T;
+  const int vis_max = (int)group_of(m_last, p.s) - 1;  // groups seen by the tile's last query
   t.nkt = (vis_max + BN - 1) / BN;
   return t;
 }
@@ -473,6 +477,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 #pragma unroll
           for (int k8 = 0; k8 < 4; ++k8) {
             const int r = 8 * k8 + tr;         // row of the block this lane stores
+            if (t.m0 + 4 * qe + k8 > p.T) break;  // query past the prompt (ragged last tile)
             uint32_t w[4];
             const uint32_t off = (uint32_t)r * 64u + ((((uint32_t)tq) ^ (((uint32_t)r >> 1) & 3u)) << 4);
             asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
@@ -618,7 +623,7 @@ cudaError_t launch_prefill_tc_args(const PrefillTcLaunch& a, const CUtensorMap& 
   p.B = a.B;
   p.T = a.T;
   p.s = a.s;
-  p.n_mtiles = a.B * (a.T / ptc::QM);
+  p.n_mtiles = a.B * ((a.T + ptc::QM - 1) / ptc::QM);
   p.scale_log2 = a.scale_log2;
   p.out = reinterpret_cast<__nv_bfloat16*>(a.out);
   p.dev_err = a.dev_err;

@@ -130,28 +130,17 @@ def test_decode_workspace_reused_many_calls():
 
 
 
-def test_decode_workspace_zeroed_once_stays_ready():
-    """The workspace contract: zeroed once before its first call, then left
-    ready by every call.  The workspace is first filled with NaN bytes and
-    then zeroed, and the cases put fewer cost positions (rows, plus the merge
-    weight of a merged sequence) than the grid has blocks, so some blocks hold
-    no share.  After each call the counters the library keeps in the
-    workspace (its first 4 (1 + 2B) bytes) are zero again."""
+def test_decode_workspace_needs_no_zeroing():
+    """A workspace full of NaN bytes: short sequences leave some blocks of the
+    split-L grid with empty shares inside a split sequence's block range."""
     dims = synth.Dims(H=8, d_h=64, r=256, d_R=32, s=2)
-    for t_prev, merge in (([180], True), ([180, 3, 61], False), ([1, 2, 3, 4], True)):
+    # fewer cost positions (rows, plus the merge weight of a merged sequence)
+    # than the grid's blocks: one merged sequence, then three without merge
+    for t_prev, merge in (([180], True), ([180, 3, 61], False)):
         case = synth.decode_case(dims, t_prev, seed=17, dtype="bf16")
         run = DecodeRun(case)
         run.ws.fill_(0xFF)
-        run.ws.zero_()
-        _check_step(run, merge=merge, what=f"zeroed workspace {t_prev}")
-        n_cnt = 4 * (1 + 2 * case.B)
-        assert int(run.ws[:n_cnt].count_nonzero().item()) == 0, "counters must be left at zero"
-        # a second call on the same workspace (read-only) gives the same outputs
-        first = host(run.out).copy()
-        out2, _ = run.step(case.q_abs, case.q_rope)
-        if not merge:
-            np.testing.assert_array_equal(out2, first)
-        assert int(run.ws[:n_cnt].count_nonzero().item()) == 0
+        _check_step(run, merge=merge, what=f"NaN workspace {t_prev}")
 
 
 def test_decode_device_errors():

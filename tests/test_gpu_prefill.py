@@ -262,3 +262,46 @@ def test_prefill_tensor_core_edges(B, s, T):
         assert_close(host(run.out[b])[idx], ref, "bf16", f"out B={B} s={s} T={T} b={b}")
         assert_close(host(run.cp[b]), Cp, "bf16", f"C_hat' b={b}")
         assert_close(host(run.cache[b]), oracle.compressed_cache(Cp, s), "bf16", f"cache b={b}")
+
+
+@pytest.mark.parametrize("B,s,T", [(2, 2, 17), (3, 3, 33), (2, 1, 23), (2, 2, 5), (1, 8, 1), (1, 2, 4095),
+                                   (1, 2, 4097), (2, 5, 1000)])
+def test_prefill_tensor_core_ragged_prompt(B, s, T):
+    """Prompt lengths that are not a multiple of the 16-query tile stay on the
+    tcgen05 kernel: the last query tile of every sequence is ragged, its rows
+    past T read the next sequence's rows (or the fill past the last one) and
+    must not be stored.  Sampled queries around the tile and group edges vs
+    the oracle; every stored row of C_hat' and the cache is checked, and the
+    output rows of the next sequence are not overwritten."""
+    dims = synth.Dims(H=8, d_h=64, r=256, d_R=32, s=s)
+    case = synth.token_case(dims, B=B, T=T, seed=900 + 7 * s + T, dtype="bf16")
+    run = PrefillRun(dims, "bf16", case.q_abs, case.q_rope, case.c, case.kR, case.lin).run()
+    rng = np.random.default_rng(s * 31 + T)
+    edges = [1, 2, s, s + 1, 15, 16, 17, 32, 33, T - 16, T - 15, T - 1, T]
+    ms = sorted(set(m for m in edges + rng.integers(1, T + 1, size=12).tolist() if 1 <= m <= T))
+    idx = np.array(ms) - 1
+    P = oracle.pe_table(run.J, case.lin["W_p"], case.lin["b_p"])
+    for b in range(B):
+        Cp = oracle.partial_merge_sequence(case.c[b], case.kR[b], case.lin["W_c"], case.lin["b_c"], P, s)
+        ref = np.stack([oracle.masked_forward_query(m, case.q_abs[b, m - 1], case.q_rope[b, m - 1], Cp, s,
+                                                    dims.d_h)[0] for m in ms])
+        got = host(run.out[b])
+        assert np.isfinite(got).all(), "every query of the prompt is written"
+        assert_close(got[idx], ref, "bf16", f"out B={B} s={s} T={T} b={b}")
+        assert_close(host(run.cp[b]), Cp, "bf16", f"C_hat' b={b}")
+        assert_close(host(run.cache[b]), oracle.compressed_cache(Cp, s), "bf16", f"cache b={b}")
+
+
+@pytest.mark.parametrize("T", [5, 17, 100])
+def test_prefill_ragged_prompt_writes_nothing_past_the_end(T):
+    """The output lives inside a larger NaN-filled buffer: the ragged last
+    query tile must not store the rows past the prompt."""
+    dims = synth.Dims(H=8, d_h=64, r=256, d_R=32, s=2)
+    B = 2
+    case = synth.token_case(dims, B=B, T=T, seed=950 + T, dtype="bf16")
+    run = PrefillRun(dims, "bf16", case.q_abs, case.q_rope, case.c, case.kR, case.lin)
+    big = torch.full((B * T + 64, dims.H, dims.r), float("nan"), dtype=torch.bfloat16, device="cuda")
+    run.out = big[:B * T].view(B, T, dims.H, dims.r)
+    run.run()
+    assert torch.isnan(big[B * T:].float()).all(), "rows past the prompt were written"
+    assert torch.isfinite(big[:B * T].float()).all()

@@ -9,7 +9,7 @@ import torch
 
 import mtla_synth as synth
 import temporally_compressed_latent_b200 as mtla
-from gpu_harness import DecodeRun, assert_close, dev, host
+from gpu_harness import DecodeRun, assert_close, dev, host, oracle_decode
 
 pytestmark = pytest.mark.gpu
 
@@ -23,6 +23,9 @@ def _static_step(run: DecodeRun, q_abs, q_rope, c_new=None, kR_new=None):
                  "J_max": run.J_max}
     run._qa = dev(q_abs, run.dtype)
     run._qr = dev(q_rope, run.dtype)
+    torch.cuda.synchronize()
+    # the inputs are on the device: from here on nothing may take device memory
+    run.free_before_call = torch.cuda.mem_get_info()[0]
     mtla.mtla_decode_attn_static(run.md, run.B, run._qa, run._qr, merge, run.cache.buf, run.cache.cache_rows,
                                  run.cache.row_stride, run.cache.offset, run.cache.capacity, run.t, run.cache_len,
                                  run.out, run.lse, run.err)
@@ -44,6 +47,8 @@ def test_static_scratch_matches_workspace_entry():
     # every B the tensor-core path accepts fits the static scratch on this device
     assert mtla.mtla_workspace_bytes(ref.md, 1024) <= mtla.DECODE_STATIC_SCRATCH_BYTES
 
+    rows = [list(np.asarray(r, np.float64)) for r in case.rows]
+    t_prev = case.t_prev.copy()
     for step in range(2):
         qa = synth.cast(rng.standard_normal((case.B, 8, 256)), "bf16")
         qr = synth.cast(rng.standard_normal((case.B, 8, 32)), "bf16")
@@ -51,8 +56,21 @@ def test_static_scratch_matches_workspace_entry():
         kn = synth.cast(rng.standard_normal((case.B, 32)), "bf16")
         o_ref, l_ref = ref.step(qa, qr, cn, kn)
         o_sta, l_sta = _static_step(sta, qa, qr, cn, kn)
+        if step > 0:
+            # after the set-up of the first call (which may load the array: the
+            # driver reserves it when it loads the library's device code, at
+            # first use under lazy loading), a call takes no device memory
+            assert torch.cuda.mem_get_info()[0] == sta.free_before_call
         assert_close(o_sta, o_ref, "bf16", f"step {step} out")
         assert_close(l_sta, l_ref, "bf16", f"step {step} lse")
+        # and both against the fp64 oracle stepping the same tokens
+        o_orc, l_orc, r_orc = oracle_decode(case, ref.J_max, q_abs=qa, q_rope=qr, c_new=cn, kR_new=kn, rows=rows,
+                                            t_prev=t_prev)
+        assert_close(o_sta, np.stack([o_orc[b] for b in range(case.B)]), "bf16", f"step {step} out vs oracle")
+        assert_close(l_sta, np.stack([l_orc[b] for b in range(case.B)]), "bf16", f"step {step} lse vs oracle")
+        # the oracle continues from the device's bf16 cache rows
+        rows = [list(sta.cache.rows(b, len(r_orc[b]))) for b in range(case.B)]
+        t_prev = t_prev + 1
         assert sta.t.cpu().tolist() == ref.t.cpu().tolist()
         assert sta.cache_len.cpu().tolist() == ref.cache_len.cpu().tolist()
         assert int(sta.err.item()) == 0 and int(ref.err.item()) == 0
