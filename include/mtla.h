@@ -206,7 +206,57 @@ mtla_status mtla_prefill_masked_attn(const mtla_dims *dims, int32_t B, int32_t T
                                      void *c_partial, void *cache_out, void *out,
                                      int32_t *dev_err, void *stream);
 
+/*
+ * mtla_project_in — the layer's input maps for one new token per sequence,
+ * with the key map absorbed into the query ([rope]; arXiv 2505.13544 abstract
+ * page, Figure 1: the latent-to-KV maps are absorbed into the query and
+ * output linear layers by associativity).  For every token b:
+ *   [q_abs | q_rope | c_new | kR_new] = x[b] W_in^T, then RoPE at position
+ *   pos[b] on q_rope (each head) and kR_new: channel pair (2k, 2k+1) rotated
+ *   by pos[b] * 10000^(-2k/d_R).
+ *   x      [B, d]       cache dtype (bf16: d a multiple of 64; fp32: of 4)
+ *   W_in   [N_in, d]    cache dtype, row-major (one row per output feature),
+ *          N_in = H (r + d_R) + r + d_R rows in this order:
+ *            H r rows   row h r + i = column i of W_Q^h W_K^h^T (the absorbed
+ *                       query of head h: d_h columns of W_Q^h times the
+ *                       transposed key map of that head)
+ *            H d_R rows row H r + h d_R + k = column k of W_QR^h
+ *            r rows     the latent map W_down (c_t = x W_down)
+ *            d_R rows   the RoPE key map W_KR
+ *   pos    [B] int32    0-based position of each token (t - 1)
+ *   q_abs [B, H, r], q_rope [B, H, d_R], c_new [B, r], kR_new [B, d_R]:
+ *          written in the cache dtype, ready for mtla_decode_attn.
+ *   workspace: mtla_project_workspace_bytes(dims, B, d, MTLA_PROJ_IN) bytes
+ *          (fp32 partial sums; no initialisation needed).
+ * bf16 runs a split-K tensor-core GEMM (tcgen05, batches of up to 256 tokens
+ * per launch) and a finishing kernel; fp32 runs a SIMT kernel.
+ */
+mtla_status mtla_project_in(const mtla_dims *dims, int32_t B, int32_t d, const void *x, const void *W_in,
+                            const int32_t *pos, void *q_abs, void *q_rope, void *c_new, void *kR_new,
+                            void *workspace, size_t workspace_bytes, int32_t *dev_err, void *stream);
+
+/*
+ * mtla_project_out — the layer's output with the value map absorbed into the
+ * output map ([rope]; Figure 1): y[b] = sum_h o[b,h] (W_V^h W_O^h).
+ *   o      [B, H, r]    fp32 (mtla_decode_attn's out); rounded to bf16 for
+ *                       the bf16 tensor-core path
+ *   W_out  [d, H r]     cache dtype, row-major: row n, column h r + i is
+ *                       (W_V^h W_O^h)[i, n]
+ *   y      [B, d]       fp32
+ *   workspace: mtla_project_workspace_bytes(dims, B, d, MTLA_PROJ_OUT) bytes.
+ * bf16: H r a multiple of 64.
+ */
+mtla_status mtla_project_out(const mtla_dims *dims, int32_t B, int32_t d, const float *o, const void *W_out,
+                             float *y, void *workspace, size_t workspace_bytes, int32_t *dev_err, void *stream);
+
 #define MTLA_WS_DECODE 0
+#define MTLA_PROJ_IN 1
+#define MTLA_PROJ_OUT 2
+
+/* Workspace bytes of mtla_project_in (which = MTLA_PROJ_IN) or
+ * mtla_project_out (MTLA_PROJ_OUT) for B tokens and model width d (0 on
+ * unsupported arguments).  Queries the current device. */
+size_t mtla_project_workspace_bytes(const mtla_dims *dims, int32_t B, int32_t d, int32_t which);
 
 /* Bytes of workspace a call needs (0 if none).  Queries the current device. */
 size_t mtla_workspace_bytes(const mtla_dims *dims, int32_t B, int32_t which);

@@ -322,13 +322,15 @@ def rope(v, pos):
     return out
 
 
-def project_inputs(x, W):
+def project_inputs(x, W, pos=None):
     """Hot-path inputs of one sequence from the layer input x [T, d].
 
     Notes, *Overall framework*: Q = X W_Q, latent C = X W_down; Figure 1 and
     the decoupled-RoPE formula: the key map is absorbed into the query,
     q_abs_h = (x W_Q^h)(W_K^h)^T (width r); RoPE query/key from their own maps.
     W: W_Q [d,H,d_h], W_K [H,r,d_h], W_down [d,r], W_QR [d,H,d_R], W_KR [d,d_R].
+    pos: 0-based positions of the T rows for RoPE (default 0..T-1, a whole
+    sequence from its start; a decode step passes its token's t - 1).
     Returns q_abs [T,H,r], q_rope [T,H,d_R], c [T,r], kR [T,d_R]."""
     x = np.asarray(x, dtype=np.float64)
     T = x.shape[0]
@@ -338,7 +340,7 @@ def project_inputs(x, W):
     H = W_Q.shape[1]
     r = W_K.shape[1]
     d_R = W_QR.shape[2]
-    pos = np.arange(T)
+    pos = np.arange(T) if pos is None else np.asarray(pos)
     c = x @ np.asarray(W["W_down"], dtype=np.float64)
     kR = rope(x @ np.asarray(W["W_KR"], dtype=np.float64), pos)
     q_abs = np.zeros((T, H, r))

@@ -16,6 +16,8 @@ from ._abi import (  # noqa: F401
     LIB_PATH,
     MTLA_BF16,
     MTLA_F32,
+    PROJ_IN,
+    PROJ_OUT,
     WS_DECODE,
     MtlaError,
     dims,
@@ -27,6 +29,9 @@ from ._abi import (  # noqa: F401
     mtla_decode_attn_static,
     mtla_merge_append,
     mtla_prefill_masked_attn,
+    mtla_project_in,
+    mtla_project_out,
+    mtla_project_workspace_bytes,
     mtla_status_string,
     mtla_workspace_bytes,
 )

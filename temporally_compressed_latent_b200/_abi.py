@@ -23,6 +23,7 @@ lib = ctypes.CDLL(LIB_PATH)
 
 MTLA_F32, MTLA_BF16 = 0, 1
 WS_DECODE = 0
+PROJ_IN, PROJ_OUT = 1, 2
 DECODE_STATIC_SCRATCH_BYTES = 24 << 20  # MTLA_DECODE_STATIC_SCRATCH_BYTES
 DEVERR_PE_RANGE, DEVERR_CAPACITY, DEVERR_EMPTY, DEVERR_TIMEOUT = 1, 2, 4, 8
 _c = ctypes
@@ -60,6 +61,12 @@ lib.mtla_debug_stride_mask.restype = _c.c_int
 lib.mtla_debug_stride_mask.argtypes = [_I32, _I32, _P]
 lib.mtla_cache_length.restype = _I64
 lib.mtla_cache_length.argtypes = [_I64, _I32]
+lib.mtla_project_in.restype = _c.c_int
+lib.mtla_project_in.argtypes = [_DIMS_P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P]
+lib.mtla_project_out.restype = _c.c_int
+lib.mtla_project_out.argtypes = [_DIMS_P, _I32, _I32, _P, _P, _P, _P, _SZ, _P, _P]
+lib.mtla_project_workspace_bytes.restype = _SZ
+lib.mtla_project_workspace_bytes.argtypes = [_DIMS_P, _I32, _I32, _I32]
 
 
 class MtlaError(RuntimeError):
@@ -133,6 +140,22 @@ def mtla_prefill_masked_attn(d, B, T, q_abs, q_rope, c, kR, W_c, b_c, P, J_max, 
     _check(lib.mtla_prefill_masked_attn(_c.byref(d), B, T, _ptr(q_abs), _ptr(q_rope), _ptr(c), _ptr(kR),
                                         _ptr(W_c), _ptr(b_c), _ptr(P), J_max, _ptr(c_partial), _ptr(cache_out),
                                         _ptr(out), _ptr(dev_err), _stream(stream)), "mtla_prefill_masked_attn")
+
+
+def mtla_project_in(d, B, dm, x, W_in, pos, q_abs, q_rope, c_new, kR_new, workspace, workspace_bytes, dev_err,
+                    stream=None):
+    _check(lib.mtla_project_in(_c.byref(d), B, dm, _ptr(x), _ptr(W_in), _ptr(pos), _ptr(q_abs), _ptr(q_rope),
+                               _ptr(c_new), _ptr(kR_new), _ptr(workspace), workspace_bytes, _ptr(dev_err),
+                               _stream(stream)), "mtla_project_in")
+
+
+def mtla_project_out(d, B, dm, o, W_out, y, workspace, workspace_bytes, dev_err, stream=None):
+    _check(lib.mtla_project_out(_c.byref(d), B, dm, _ptr(o), _ptr(W_out), _ptr(y), _ptr(workspace),
+                                workspace_bytes, _ptr(dev_err), _stream(stream)), "mtla_project_out")
+
+
+def mtla_project_workspace_bytes(d, B, dm, which) -> int:
+    return int(lib.mtla_project_workspace_bytes(_c.byref(d), B, dm, which))
 
 
 def mtla_workspace_bytes(d, B, which=WS_DECODE) -> int:

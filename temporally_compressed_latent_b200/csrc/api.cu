@@ -150,6 +150,36 @@ mtla_status merge_args(const mtla_merge_args* m, MergeArgsDev* md) {
 
 mtla_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MTLA_OK : MTLA_ERR_CUDA; }
 
+int device_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  return sms;
+}
+
+// rows of the input map: H r absorbed-query rows, H d_R RoPE-query rows, r
+// latent rows, d_R RoPE-key rows
+int64_t proj_in_rows(const mtla_dims* d) { return (int64_t)d->H * (d->r + d->d_R) + d->r + d->d_R; }
+
+// workspace of one projection call: the fp32 partial sums of one launch
+size_t proj_ws(const mtla_dims* dims, int32_t B, int32_t d, int32_t which) {
+  if (check_dims(dims) != MTLA_OK || B < 1 || d < 1) return 0;
+  const int64_t N = which == MTLA_PROJ_IN ? proj_in_rows(dims) : d;
+  const int64_t K = which == MTLA_PROJ_IN ? d : (int64_t)dims->H * dims->r;
+  if (dims->dtype != MTLA_BF16) return (size_t)B * N * 4;
+  const int sms = device_sms();
+  if (sms <= 0) return 0;
+  const ProjSplit sp = proj_split(B, (int)K, (int)N, sms);
+  return (size_t)sp.KS * sp.Bp * N * 4;
+}
+
+// 2-D map of a row-major bf16 weight [N rows, K] in boxes of 64 x 128 with the 128-byte swizzle
+bool encode_weight_map(CUtensorMap* map, const void* W, int64_t N, int64_t K) {
+  const cuuint64_t dims2[2] = {(cuuint64_t)K, (cuuint64_t)N}, str[1] = {(cuuint64_t)K * 2};
+  const cuuint32_t box[2] = {64, 128};
+  return encode_bf16_map(map, W, 2, dims2, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 }  // namespace
 
 extern "C" {
@@ -359,6 +389,127 @@ mtla_status mtla_prefill_masked_attn(const mtla_dims* dims, int32_t B, int32_t T
   a.dev_err = dev_err;
   const int tiles = B * ((T + 15) / 16);
   return from_cuda(launch_prefill_tc_args(a, qmap, rmap, smap, kmap, tiles < sms ? tiles : sms, cs));
+}
+
+size_t mtla_project_workspace_bytes(const mtla_dims* dims, int32_t B, int32_t d, int32_t which) {
+  if (which != MTLA_PROJ_IN && which != MTLA_PROJ_OUT) return 0;
+  return proj_ws(dims, B < MAXBP || (dims && dims->dtype != MTLA_BF16) ? B : MAXBP, d, which);
+}
+
+mtla_status mtla_project_in(const mtla_dims* dims, int32_t B, int32_t d, const void* x, const void* W_in,
+                            const int32_t* pos, void* q_abs, void* q_rope, void* c_new, void* kR_new,
+                            void* workspace, size_t workspace_bytes, int32_t* dev_err, void* stream) {
+  mtla_status st = check_dims(dims);
+  if (st != MTLA_OK) return st;
+  if (B < 0 || d < 1) return MTLA_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, W_in, q_abs, q_rope, c_new, kR_new};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return MTLA_ERR_INVALID_ARG;
+  if (!pos || (reinterpret_cast<uintptr_t>(pos) & 3) || !dev_err) return MTLA_ERR_INVALID_ARG;
+  const bool bf = dims->dtype == MTLA_BF16;
+  if (bf ? (d % 64) : (d % 4)) return MTLA_ERR_UNSUPPORTED;
+  if (B == 0) return MTLA_OK;
+  const int64_t N = proj_in_rows(dims);
+  const int sms = device_sms();
+  if (sms <= 0) return MTLA_ERR_CUDA;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < mtla_project_workspace_bytes(dims, B, d, MTLA_PROJ_IN))
+    return MTLA_ERR_WORKSPACE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const size_t es = elem_size(dims->dtype);
+  float* part = static_cast<float*>(workspace);
+  CUtensorMap wmap;
+  if (bf && !encode_weight_map(&wmap, W_in, N, d)) return MTLA_ERR_CUDA;
+  const int chunk = bf ? MAXBP : B;
+  for (int b0 = 0; b0 < B; b0 += chunk) {
+    const int nb = B - b0 < chunk ? B - b0 : chunk;
+    InFinishArgs f;
+    f.part = part;
+    f.B = nb;
+    f.H = dims->H;
+    f.r = dims->r;
+    f.d_R = dims->d_R;
+    f.pos = pos + b0;
+    f.q_abs = static_cast<uint8_t*>(q_abs) + (size_t)b0 * dims->H * dims->r * es;
+    f.q_rope = static_cast<uint8_t*>(q_rope) + (size_t)b0 * dims->H * dims->d_R * es;
+    f.c_new = static_cast<uint8_t*>(c_new) + (size_t)b0 * dims->r * es;
+    f.kR_new = static_cast<uint8_t*>(kR_new) + (size_t)b0 * dims->d_R * es;
+    cudaError_t e;
+    if (bf) {
+      const ProjSplit sp = proj_split(nb, d, (int)N, sms);
+      GemmArgs g;
+      g.x = static_cast<const uint8_t*>(x) + (size_t)b0 * d * es;
+      g.ldx = d;
+      g.B = nb;
+      g.Bp = sp.Bp;
+      g.N = (int)N;
+      g.nkb = sp.nkb;
+      g.kpb = sp.kpb;
+      g.part = part;
+      g.dev_err = dev_err;
+      e = launch_proj_gemm(g, wmap, sp.m_tiles, sp.KS, false, cs);
+      f.KS = sp.KS;
+      f.Bp = sp.Bp;
+    } else {
+      e = launch_proj_simt(static_cast<const float*>(x) + (size_t)b0 * d, d, static_cast<const float*>(W_in), nb, d,
+                           (int)N, part, cs);
+      f.KS = 1;
+      f.Bp = nb;
+    }
+    if (e != cudaSuccess) return MTLA_ERR_CUDA;
+    if ((e = launch_proj_in_finish(f, dims->dtype, cs)) != cudaSuccess) return MTLA_ERR_CUDA;
+  }
+  return MTLA_OK;
+}
+
+mtla_status mtla_project_out(const mtla_dims* dims, int32_t B, int32_t d, const float* o, const void* W_out,
+                             float* y, void* workspace, size_t workspace_bytes, int32_t* dev_err, void* stream) {
+  mtla_status st = check_dims(dims);
+  if (st != MTLA_OK) return st;
+  if (B < 0 || d < 1) return MTLA_ERR_INVALID_ARG;
+  const void* ptrs[] = {o, W_out, y};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return MTLA_ERR_INVALID_ARG;
+  if (!dev_err) return MTLA_ERR_INVALID_ARG;
+  const bool bf = dims->dtype == MTLA_BF16;
+  const int64_t K = (int64_t)dims->H * dims->r;
+  if (bf ? (K % 64) : (K % 4)) return MTLA_ERR_UNSUPPORTED;
+  if (B == 0) return MTLA_OK;
+  const int sms = device_sms();
+  if (sms <= 0) return MTLA_ERR_CUDA;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < mtla_project_workspace_bytes(dims, B, d, MTLA_PROJ_OUT))
+    return MTLA_ERR_WORKSPACE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  float* part = static_cast<float*>(workspace);
+  CUtensorMap wmap;
+  if (bf && !encode_weight_map(&wmap, W_out, d, K)) return MTLA_ERR_CUDA;
+  const int chunk = bf ? MAXBP : B;
+  for (int b0 = 0; b0 < B; b0 += chunk) {
+    const int nb = B - b0 < chunk ? B - b0 : chunk;
+    cudaError_t e;
+    int KS = 1, Bp = nb;
+    if (bf) {
+      const ProjSplit sp = proj_split(nb, (int)K, d, sms);
+      GemmArgs g;
+      g.x = o + (size_t)b0 * K;
+      g.ldx = K;
+      g.B = nb;
+      g.Bp = sp.Bp;
+      g.N = d;
+      g.nkb = sp.nkb;
+      g.kpb = sp.kpb;
+      g.part = part;
+      g.dev_err = dev_err;
+      e = launch_proj_gemm(g, wmap, sp.m_tiles, sp.KS, true, cs);
+      KS = sp.KS;
+      Bp = sp.Bp;
+    } else {
+      e = launch_proj_simt(o + (size_t)b0 * K, K, static_cast<const float*>(W_out), nb, (int)K, d, part, cs);
+    }
+    if (e != cudaSuccess) return MTLA_ERR_CUDA;
+    if ((e = launch_proj_out_finish(part, KS, Bp, nb, d, y + (size_t)b0 * d, cs)) != cudaSuccess)
+      return MTLA_ERR_CUDA;
+  }
+  return MTLA_OK;
 }
 
 }  // extern "C"

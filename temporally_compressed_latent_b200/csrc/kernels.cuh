@@ -120,4 +120,34 @@ cudaError_t launch_prefill_tc_args(const PrefillTcLaunch& a, const CUtensorMap& 
                                    const CUtensorMap& smap, const CUtensorMap& kmap, int grid, cudaStream_t st);
 cudaError_t launch_prefill_simt(const PrefillArgs& p, int B, int dtype, cudaStream_t st);
 
+// The layer's input and output maps with the key / value maps absorbed (proj.cu).
+constexpr int MAXBP = 256;  // tokens per projection launch (MMA N)
+struct GemmArgs {
+  const void* x;   // [B, K] activations (bf16, or fp32 rounded to bf16 when staged)
+  int64_t ldx;     // elements between rows of x
+  int B, Bp, N, nkb, kpb;
+  float* part;     // [KS][Bp][N] fp32 partial sums
+  int32_t* dev_err;
+};
+struct InFinishArgs {
+  const float* part;
+  int KS, Bp, B, H, r, d_R;
+  const int32_t* pos;  // [B] 0-based token positions (RoPE)
+  void* q_abs;
+  void* q_rope;
+  void* c_new;
+  void* kR_new;
+};
+struct ProjSplit {
+  int Bp, KS, kpb, m_tiles, nkb;
+};
+ProjSplit proj_split(int B, int K, int N, int sms);
+size_t proj_smem_bytes();
+cudaError_t launch_proj_gemm(const GemmArgs& a, const CUtensorMap& wmap, int m_tiles, int KS, bool x_f32,
+                             cudaStream_t st);
+cudaError_t launch_proj_simt(const float* x, int64_t ldx, const float* W, int B, int K, int N, float* part,
+                             cudaStream_t st);
+cudaError_t launch_proj_in_finish(const InFinishArgs& a, int dtype, cudaStream_t st);
+cudaError_t launch_proj_out_finish(const float* part, int KS, int Bp, int B, int N, float* y, cudaStream_t st);
+
 }  // namespace mtla

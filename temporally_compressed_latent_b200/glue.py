@@ -65,3 +65,23 @@ def project(x: torch.Tensor, W: dict):
     qR = (x @ W_QR.reshape(d, H * d_R)).reshape(B, T, H, d_R)
     q_rope = rope(qR.permute(0, 2, 1, 3), pos).permute(0, 2, 1, 3)
     return q_abs.contiguous(), q_rope.contiguous(), c.contiguous(), kR.contiguous()
+
+
+def absorbed_weights(W: dict, dtype=torch.bfloat16):
+    """The weight matrices of mtla_project_in / mtla_project_out (row-major,
+    one row per output feature), from the layer's maps W_Q [d,H,d_h],
+    W_K [H,r,d_h], W_V [H,r,d_h], W_O [H*d_h,d], W_down [d,r], W_QR [d,H,d_R],
+    W_KR [d,d_R]:
+      W_in  [H r + H d_R + r + d_R, d]: rows of (W_Q^h W_K^h^T)^T per head,
+            W_QR^h^T per head, W_down^T, W_KR^T;
+      W_out [d, H r]: column block h is (W_V^h W_O^h)^T.
+    The products are formed in float64 and rounded once to `dtype`."""
+    f = lambda t: t.to(torch.float64)
+    W_Q, W_K, W_V, W_O = f(W["W_Q"]), f(W["W_K"]), f(W["W_V"]), f(W["W_O"])
+    H, r, d_h = W_K.shape
+    rows = [(W_Q[:, h, :] @ W_K[h].T).T for h in range(H)]
+    rows += [f(W["W_QR"])[:, h, :].T for h in range(H)]
+    rows += [f(W["W_down"]).T, f(W["W_KR"]).T]
+    W_in = torch.cat(rows, dim=0)
+    W_out = torch.cat([(W_V[h] @ W_O[h * d_h:(h + 1) * d_h, :]).T for h in range(H)], dim=1)
+    return W_in.to(dtype).contiguous(), W_out.to(dtype).contiguous()

@@ -371,3 +371,15 @@ def test_synth_bf16_rounding():
     x = np.random.default_rng(3).standard_normal(10000).astype(np.float32)
     np.testing.assert_array_equal(synth.round_to_bf16(x),
                                   torch.tensor(x).to(torch.bfloat16).to(torch.float32).numpy())
+
+
+def test_project_inputs_at_a_position():
+    """A token projected on its own at position p gives row p of the whole
+    sequence's projections (RoPE depends on the position only)."""
+    mc = synth.tiny_e2e(0)
+    x = mc.x[0]
+    full = oracle.project_inputs(x, mc.W)
+    for p in (0, 5, 63, 79):
+        one = oracle.project_inputs(x[p:p + 1], mc.W, pos=[p])
+        for a, b in zip(one, full):
+            np.testing.assert_allclose(a[0], b[p], rtol=0, atol=1e-12)
