@@ -582,7 +582,107 @@ def run_configs(torch, mtla, glue, dev):
     res["sweep_b64_t16384"] = {"workload": "compression-ratio sweep bf16: B=64, t=16384 processed tokens, H=8, "
                                            "d_h=64, r=256, d_R=32; cache merged from N(0,1) latents with the "
                                            "sigmoid gates", **sweep}
+    res["layer_maps_b32"] = run_layer_maps(torch, mtla, glue, dev, flush, n, warm)
+    res["multi_token_b32_n4"] = run_multi(torch, mtla, glue, dev, flush, n, warm)
     return res
+
+
+def time_calls(torch, call, n, warm, flush):
+    """Median of n single calls (after warm ones), L2 flushed before each."""
+    for _ in range(warm):
+        call()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(n):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        call()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return statistics.median(times)
+
+
+def run_layer_maps(torch, mtla, glue, dev, flush, n, warm):
+    """The absorbed input and output maps of the decode layer at B=32, d=512
+    (mtla_project_in: x -> q_abs, q_rope, c_t, k^R_t with RoPE; mtla_project_out:
+    o -> y): bound by streaming their bf16 weights."""
+    mc = synth.model_case(synth.MAIN, B=32, T=1, d=512, seed=7, dtype="bf16")
+    d = mc.dims
+    B, dm = 32, mc.d
+    W = {k: torch.from_numpy(v).to(dev) for k, v in mc.W.items()}
+    W_in, W_out = glue.absorbed_weights(W, torch.bfloat16)
+    md = mtla.dims(d.H, d.d_h, d.r, d.d_R, d.s, "bf16")
+    x = torch.from_numpy(mc.x[:, 0, :]).to(dev).to(torch.bfloat16)
+    pos = torch.arange(B, dtype=torch.int32, device=dev) * 97
+    qa = torch.empty(B, d.H, d.r, dtype=torch.bfloat16, device=dev)
+    qr = torch.empty(B, d.H, d.d_R, dtype=torch.bfloat16, device=dev)
+    cn = torch.empty(B, d.r, dtype=torch.bfloat16, device=dev)
+    kn = torch.empty(B, d.d_R, dtype=torch.bfloat16, device=dev)
+    o = torch.randn(B, d.H, d.r, device=dev)
+    y = torch.empty(B, dm, dtype=torch.float32, device=dev)
+    wi = mtla.mtla_project_workspace_bytes(md, B, dm, mtla.PROJ_IN)
+    wo = mtla.mtla_project_workspace_bytes(md, B, dm, mtla.PROJ_OUT)
+    ws_i = torch.empty(wi, dtype=torch.uint8, device=dev)
+    ws_o = torch.empty(wo, dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    ms_in = time_calls(torch, lambda: mtla.mtla_project_in(md, B, dm, x, W_in, pos, qa, qr, cn, kn, ws_i, wi, err),
+                       n, warm, flush)
+    ms_out = time_calls(torch, lambda: mtla.mtla_project_out(md, B, dm, o, W_out, y, ws_o, wo, err), n, warm, flush)
+    if int(err.item()):
+        raise RuntimeError(f"device error bits {int(err.item())} in the layer maps")
+    hbm_peak, _, _, kind = measured_peaks()
+    b_in = W_in.numel() * 2 + x.numel() * 2 + B * (d.H * d.D + d.D) * 2
+    b_out = W_out.numel() * 2 + o.numel() * 4 + y.numel() * 4
+    row = lambda ms, by: {"ms": ms, "algorithmic_bytes": by, "achieved_gbs": by / (ms / 1e3) / 1e9,
+                          "frac": by / (ms / 1e3) / 1e9 / hbm_peak}
+    return {"workload": "absorbed layer maps bf16, B=32 tokens, d=512, H=8, r=256, d_R=32 "
+                        f"(W_in {tuple(W_in.shape)}, W_out {tuple(W_out.shape)})",
+            "project_in": row(ms_in, b_in), "project_out": row(ms_out, b_out), "peak_gbs": hbm_peak,
+            "peak_kind": kind, "bound": "hbm (weights streamed once per call)"}
+
+
+def run_multi(torch, mtla, glue, dev, flush, n_calls, warm):
+    """Four new tokens per sequence in one call on the B=32 workload
+    (mtla_decode_attn_multi): 128 queries over the shared rows."""
+    case = synth.decode_uniform(B=32, seed=2)
+    d = case.dims
+    B, n = case.B, 4
+    rng = np.random.default_rng(11)
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(synth.cast(a, "bf16"))).to(dev).to(torch.bfloat16)
+    qa = bf(rng.standard_normal((B, n, d.H, d.r)))
+    qr = bf(rng.standard_normal((B, n, d.H, d.d_R)))
+    cn = bf(rng.standard_normal((B, n, d.r)))
+    kn = bf(rng.standard_normal((B, n, d.d_R)))
+    calls = warm + n_calls
+    st = DecodeState(torch, mtla, glue, dev, d, case.t_prev,
+                     lambda b: torch.from_numpy(case.rows[b]).to(dev).to(torch.bfloat16), case.lin, qa[:, 0],
+                     qr[:, 0], cn[:, 0], kn[:, 0], calls * n + 4)
+    ws_bytes = mtla.mtla_decode_multi_workspace_bytes(st.md, B, n)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    out = torch.empty(B, n, d.H, d.r, dtype=torch.float32, device=dev)
+    merge = dict(st.merge, c_new=cn, kR_new=kn)
+    nbytes = []
+
+    def call():
+        mtla.mtla_decode_attn_multi(st.md, B, n, qa, qr, merge, st.cache, st.cache_rows, d.D, st.offset,
+                                    st.capacity, st.t, st.cache_len, out, None, ws, ws_bytes, st.err)
+        st.t_host += n
+        # unique bytes: every row once, the queries, the new tokens, out
+        rows = int(sum(synth.ceil_div(int(t), d.s) for t in st.t_host))
+        nbytes.append(rows * ROW_BYTES + B * n * (d.H * d.D * 2 + d.D * 2 + d.H * d.r * 4) + B * ROW_BYTES)
+
+    ms = time_calls(torch, call, n_calls, warm, flush)
+    if int(st.err.item()):
+        raise RuntimeError(f"device error bits {int(st.err.item())} in the multi-token decode")
+    hbm_peak, _, _, kind = measured_peaks()
+    by = statistics.median(nbytes)
+    return {"workload": "B=32 decode workload (4096 / 4095 processed tokens, s=2) with n=4 new tokens per "
+                        "sequence in one call", "ms_per_call": ms, "value": B * n / (ms / 1e3), "unit": UNIT,
+            "unique_bytes_per_call": by, "achieved_gbs": by / (ms / 1e3) / 1e9,
+            "frac": by / (ms / 1e3) / 1e9 / hbm_peak, "peak_kind": kind,
+            "note": "query-steps/s counts the B n queries; bytes count every cache row once"}
 
 
 # ---------------------------------------------------------------------------

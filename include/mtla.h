@@ -140,6 +140,42 @@ mtla_status mtla_decode_attn(const mtla_dims *dims, int32_t B,
                              int32_t *dev_err, void *stream);
 
 /*
+ * mtla_decode_attn_multi — n new tokens per sequence in one call (speculative
+ * or beam decode), 1 <= n <= MTLA_MAX_NEW_TOKENS ([merge], [fig2](a)).
+ * Tokens t = t_processed[b] + 1 .. t_processed[b] + n of sequence b are merged
+ * in order exactly as n consecutive mtla_decode_attn calls merge them (the
+ * stored row is rounded to the cache dtype after every token), and query i
+ * attends the cache as it stands after token i: rows 1 .. ceil(t_i / s), the
+ * last one the (possibly partial) row that token i leaves.  Then
+ * t_processed[b] += n and cache_len[b] = ceil(t_processed[b] / s).
+ *   q_abs [B, n, H, r], q_rope [B, n, H, d_R]   cache dtype
+ *   merge (required): c_new [B, n, r], kR_new [B, n, d_R]; W_c, b_c, P, J_max
+ *   out [B, n, H, r] fp32;  lse [B, n, H] fp32 (nullable)
+ *   workspace: mtla_decode_multi_workspace_bytes(dims, B, n) bytes; needs no
+ *   initialisation.
+ * A sequence whose n tokens do not fit its capacity (or P table) merges none
+ * of them (MTLA_DEVERR_CAPACITY / _PE_RANGE) and its queries attend the cache
+ * as it stands.  The attention runs over B n per-query sequences that share
+ * their sequence's rows: on the split-L tensor-core path when B n <= 1024
+ * (bf16, (H, r, d_R) = (8, 256, 32)), else one block per query.
+ */
+#define MTLA_MAX_NEW_TOKENS 16
+
+mtla_status mtla_decode_attn_multi(const mtla_dims *dims, int32_t B, int32_t n,
+                                   const void *q_abs, const void *q_rope,
+                                   const mtla_merge_args *merge,
+                                   void *cache, int64_t cache_rows, int64_t row_stride,
+                                   const int64_t *seq_offset, const int64_t *seq_capacity,
+                                   int32_t *t_processed, int32_t *cache_len,
+                                   float *out, float *lse,
+                                   void *workspace, size_t workspace_bytes,
+                                   int32_t *dev_err, void *stream);
+
+/* Workspace bytes of mtla_decode_attn_multi (0 on unsupported arguments).
+ * Queries the current device. */
+size_t mtla_decode_multi_workspace_bytes(const mtla_dims *dims, int32_t B, int32_t n);
+
+/*
  * mtla_decode_attn_static — mtla_decode_attn with its scratch in a static
  * device array of this library instead of a caller-provided workspace.  The
  * MTLA paper has no counterpart: this is a library convenience, and it

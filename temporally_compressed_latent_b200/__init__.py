@@ -15,6 +15,7 @@ from ._abi import (  # noqa: F401
     DEVERR_TIMEOUT,
     LIB_PATH,
     MTLA_BF16,
+    MAX_NEW_TOKENS,
     MTLA_F32,
     PROJ_IN,
     PROJ_OUT,
@@ -26,6 +27,8 @@ from ._abi import (  # noqa: F401
     mtla_cache_length,
     mtla_debug_stride_mask,
     mtla_decode_attn,
+    mtla_decode_attn_multi,
+    mtla_decode_multi_workspace_bytes,
     mtla_decode_attn_static,
     mtla_merge_append,
     mtla_prefill_masked_attn,

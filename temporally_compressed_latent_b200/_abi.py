@@ -25,6 +25,7 @@ MTLA_F32, MTLA_BF16 = 0, 1
 WS_DECODE = 0
 PROJ_IN, PROJ_OUT = 1, 2
 DECODE_STATIC_SCRATCH_BYTES = 24 << 20  # MTLA_DECODE_STATIC_SCRATCH_BYTES
+MAX_NEW_TOKENS = 16  # MTLA_MAX_NEW_TOKENS
 DEVERR_PE_RANGE, DEVERR_CAPACITY, DEVERR_EMPTY, DEVERR_TIMEOUT = 1, 2, 4, 8
 _c = ctypes
 
@@ -61,6 +62,11 @@ lib.mtla_debug_stride_mask.restype = _c.c_int
 lib.mtla_debug_stride_mask.argtypes = [_I32, _I32, _P]
 lib.mtla_cache_length.restype = _I64
 lib.mtla_cache_length.argtypes = [_I64, _I32]
+lib.mtla_decode_attn_multi.restype = _c.c_int
+lib.mtla_decode_attn_multi.argtypes = [_DIMS_P, _I32, _I32, _P, _P, _MERGE_P, _P, _I64, _I64, _P, _P, _P, _P, _P,
+                                       _P, _P, _SZ, _P, _P]
+lib.mtla_decode_multi_workspace_bytes.restype = _SZ
+lib.mtla_decode_multi_workspace_bytes.argtypes = [_DIMS_P, _I32, _I32]
 lib.mtla_project_in.restype = _c.c_int
 lib.mtla_project_in.argtypes = [_DIMS_P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P]
 lib.mtla_project_out.restype = _c.c_int
@@ -140,6 +146,18 @@ def mtla_prefill_masked_attn(d, B, T, q_abs, q_rope, c, kR, W_c, b_c, P, J_max, 
     _check(lib.mtla_prefill_masked_attn(_c.byref(d), B, T, _ptr(q_abs), _ptr(q_rope), _ptr(c), _ptr(kR),
                                         _ptr(W_c), _ptr(b_c), _ptr(P), J_max, _ptr(c_partial), _ptr(cache_out),
                                         _ptr(out), _ptr(dev_err), _stream(stream)), "mtla_prefill_masked_attn")
+
+
+def mtla_decode_attn_multi(d, B, n, q_abs, q_rope, merge, cache, cache_rows, row_stride, seq_offset, seq_capacity,
+                           t_processed, cache_len, out, lse, workspace, workspace_bytes, dev_err, stream=None):
+    _check(lib.mtla_decode_attn_multi(_c.byref(d), B, n, _ptr(q_abs), _ptr(q_rope), _merge(merge), _ptr(cache),
+                                      cache_rows, row_stride, _ptr(seq_offset), _ptr(seq_capacity),
+                                      _ptr(t_processed), _ptr(cache_len), _ptr(out), _ptr(lse), _ptr(workspace),
+                                      workspace_bytes, _ptr(dev_err), _stream(stream)), "mtla_decode_attn_multi")
+
+
+def mtla_decode_multi_workspace_bytes(d, B, n) -> int:
+    return int(lib.mtla_decode_multi_workspace_bytes(_c.byref(d), B, n))
 
 
 def mtla_project_in(d, B, dm, x, W_in, pos, q_abs, q_rope, c_new, kR_new, workspace, workspace_bytes, dev_err,

@@ -259,6 +259,7 @@ mtla_status mtla_decode_attn(const mtla_dims* dims, int32_t B, const void* q_abs
   o.lse = lse;
   o.scale = (float)(1.0 / sqrt((double)dims->d_h));
   o.H = dims->H;
+  o.tails = nullptr;
 
   if (!tc_decode_dims(dims, B))
     return from_cuda(launch_decode_simt(a, m, merge != nullptr, o, B, dims->dtype, cs));
@@ -284,6 +285,7 @@ mtla_status mtla_decode_attn(const mtla_dims* dims, int32_t B, const void* q_abs
   p.m = m;
   p.o = o;
   p.with_merge = merge != nullptr;
+  p.patch = 0;
   p.B = B;
   p.merge_cost = dtc::MERGE_COST;
   p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->d_h));
@@ -389,6 +391,115 @@ mtla_status mtla_prefill_masked_attn(const mtla_dims* dims, int32_t B, int32_t T
   a.dev_err = dev_err;
   const int tiles = B * ((T + 15) / 16);
   return from_cuda(launch_prefill_tc_args(a, qmap, rmap, smap, kmap, tiles < sms ? tiles : sms, cs));
+}
+
+// Workspace of a call with n new tokens per sequence: the B n virtual
+// sequences' arrays, their tail rows, then the split-L workspace for B n.
+struct MultiLayout {
+  size_t t_v, off_v, cap_v, tails, dec, total;
+};
+static MultiLayout multi_layout(const mtla_dims* dims, int32_t B, int32_t n, size_t dec_bytes) {
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  const size_t Bv = (size_t)B * n;
+  MultiLayout l;
+  l.t_v = 0;
+  l.off_v = up(Bv * 4);
+  l.cap_v = l.off_v + up(Bv * 8);
+  l.tails = l.cap_v + up(Bv * 8);
+  l.dec = l.tails + up(Bv * (dims->r + dims->d_R) * elem_size(dims->dtype));
+  l.total = l.dec + dec_bytes;
+  return l;
+}
+
+size_t mtla_decode_multi_workspace_bytes(const mtla_dims* dims, int32_t B, int32_t n) {
+  if (check_dims(dims) != MTLA_OK || B < 0 || n < 1 || n > MTLA_MAX_NEW_TOKENS) return 0;
+  return multi_layout(dims, B, n, mtla_workspace_bytes(dims, B * n, MTLA_WS_DECODE)).total;
+}
+
+mtla_status mtla_decode_attn_multi(const mtla_dims* dims, int32_t B, int32_t n, const void* q_abs, const void* q_rope,
+                                   const mtla_merge_args* merge, void* cache, int64_t cache_rows, int64_t row_stride,
+                                   const int64_t* seq_offset, const int64_t* seq_capacity, int32_t* t_processed,
+                                   int32_t* cache_len, float* out, float* lse, void* workspace,
+                                   size_t workspace_bytes, int32_t* dev_err, void* stream) {
+  mtla_status st = check_dims(dims);
+  if (st != MTLA_OK) return st;
+  if (B < 0 || n < 1 || n > MTLA_MAX_NEW_TOKENS || (int64_t)B * n > (int64_t(1) << 24)) return MTLA_ERR_INVALID_ARG;
+  SeqArgs a;
+  MergeArgsDev m = {};
+  if ((st = seq_args(dims, cache, cache_rows, row_stride, seq_offset, seq_capacity, t_processed, cache_len, dev_err,
+                     &a)) != MTLA_OK)
+    return st;
+  if ((st = merge_args(merge, &m)) != MTLA_OK) return st;
+  if (!q_abs || !q_rope || !out || !aligned16(q_abs) || !aligned16(q_rope) || !aligned16(out) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3)))
+    return MTLA_ERR_INVALID_ARG;
+  if (B == 0) return MTLA_OK;
+  const int Bv = B * n;
+  const bool tc = tc_decode_dims(dims, Bv);
+  const int grid = tc ? decode_grid() : 0;
+  if (tc && grid <= 0) return MTLA_ERR_CUDA;
+  const size_t dec_bytes = tc ? dtc::workspace_bytes(Bv, grid) : 0;
+  const MultiLayout ml = multi_layout(dims, B, n, dec_bytes);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < ml.total) return MTLA_ERR_WORKSPACE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+
+  // 1. the n tokens of every sequence, merged in order
+  MultiMergeArgs mm;
+  mm.a = a;
+  mm.m = m;
+  mm.n = n;
+  mm.four_part = tc && dims->r == dtc::R && dims->d_R == dtc::DR;  // the tensor-core step's gate order
+  mm.tails = ws + ml.tails;
+  mm.t_v = reinterpret_cast<int32_t*>(ws + ml.t_v);
+  mm.off_v = reinterpret_cast<int64_t*>(ws + ml.off_v);
+  mm.cap_v = reinterpret_cast<int64_t*>(ws + ml.cap_v);
+  if (launch_multi_merge(mm, B, dims->dtype, cs) != cudaSuccess) return MTLA_ERR_CUDA;
+
+  // 2. the attention of the B n queries: virtual sequence b n + i reads b's
+  // rows up to ceil((t0 + i + 1) / s) with its last row from the tails
+  SeqArgs av = a;
+  av.t_processed = mm.t_v;
+  av.seq_offset = mm.off_v;
+  av.seq_capacity = mm.cap_v;
+  av.cache_len = nullptr;
+  DecodeOut o;
+  o.q_abs = q_abs;
+  o.q_rope = q_rope;
+  o.out = out;
+  o.lse = lse;
+  o.scale = (float)(1.0 / sqrt((double)dims->d_h));
+  o.H = dims->H;
+  o.tails = mm.tails;
+  if (!tc) return from_cuda(launch_decode_simt(av, m, false, o, Bv, dims->dtype, cs));
+
+  thread_local CacheMaps maps;
+  if (maps.ptr != cache || maps.rows != cache_rows || maps.stride != row_stride) {
+    if (!encode_cache_map(&maps.m64, cache, cache_rows, row_stride, dtc::UNIT, dtc::D / 32) ||
+        !encode_cache_map(&maps.m8, cache, cache_rows, row_stride, dtc::SUB, 1)) {
+      maps.ptr = nullptr;
+      return MTLA_ERR_CUDA;
+    }
+    maps.ptr = cache;
+    maps.rows = cache_rows;
+    maps.stride = row_stride;
+  }
+  dtc::Params p;
+  p.a = av;
+  p.m = m;
+  p.o = o;
+  p.with_merge = 0;
+  p.patch = 1;
+  p.B = Bv;
+  p.merge_cost = 0;
+  p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->d_h));
+  const dtc::WsLayout wl = dtc::ws_layout(Bv, grid);
+  uint8_t* dws = ws + ml.dec;
+  p.seq_info = reinterpret_cast<int4*>(dws + wl.seq_info);
+  p.tails = reinterpret_cast<__nv_bfloat16*>(mm.tails);
+  p.ws_ml = reinterpret_cast<float*>(dws + wl.ml);
+  p.ws_o = reinterpret_cast<float*>(dws + wl.o);
+  return from_cuda(launch_decode_tc(p, maps.m64, maps.m8, grid, cs));
 }
 
 size_t mtla_project_workspace_bytes(const mtla_dims* dims, int32_t B, int32_t d, int32_t which) {

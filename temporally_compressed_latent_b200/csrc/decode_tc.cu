@@ -243,7 +243,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap map64, const __grid_constan
     for (int b = tid * per; b < B && b < (tid + 1) * per; ++b) {
       const SeqState st = seq_state(p, b, with_merge);
       if (st.err && cta == 0) set_err(p.a.dev_err, st.err);
-      sm.meta[b] = (uint32_t)st.L | (st.merge_ok ? kMetaMergeOk : 0u);
+      // a merged sequence, or (several tokens per call) any sequence with rows:
+      // its last row is patched from the tails buffer
+      const bool patched = st.merge_ok || (p.patch && st.L > 0 && st.err == 0);
+      sm.meta[b] = (uint32_t)st.L | (patched ? kMetaMergeOk : 0u);
       sum += st.L + mcost;
     }
     sm.scan[tid] = sum;

@@ -35,6 +35,7 @@ struct DecodeOut {
   float* lse;
   float scale;  // 1/sqrt(d_h)
   int H;
+  const void* tails;  // nullable [B][D]: replaces every sequence's last row (several tokens per call)
 };
 
 struct PrefillArgs {
@@ -78,6 +79,7 @@ struct Params {
   MergeArgsDev m;
   DecodeOut o;
   int with_merge;
+  int patch;            // 1: every sequence's last row is taken from tails (several tokens per call)
   int B;
   int merge_cost;
   float scale_log2;     // log2(e) / sqrt(d_h)
@@ -119,6 +121,21 @@ struct PrefillTcLaunch {
 cudaError_t launch_prefill_tc_args(const PrefillTcLaunch& a, const CUtensorMap& qmap, const CUtensorMap& rmap,
                                    const CUtensorMap& smap, const CUtensorMap& kmap, int grid, cudaStream_t st);
 cudaError_t launch_prefill_simt(const PrefillArgs& p, int B, int dtype, cudaStream_t st);
+
+// Several new tokens per sequence in one decode call (multi.cu): the merge of
+// the n tokens in order, the tail row as it stands after each token, and the
+// per-query ("virtual") sequence arrays the attention kernels read.
+struct MultiMergeArgs {
+  SeqArgs a;          // the real sequences (B of them)
+  MergeArgsDev m;     // c_new [B, n, r], kR_new [B, n, d_R]
+  int n;
+  int four_part;      // gate sums in four 64-row parts (the tensor-core decode's merge order)
+  void* tails;        // [B n][D] cache dtype: the tail row after token i of sequence b
+  int32_t* t_v;       // [B n] tokens processed after query i's token
+  int64_t* off_v;     // [B n]
+  int64_t* cap_v;     // [B n]
+};
+cudaError_t launch_multi_merge(const MultiMergeArgs& a, int B, int dtype, cudaStream_t st);
 
 // The layer's input and output maps with the key / value maps absorbed (proj.cu).
 constexpr int MAXBP = 256;  // tokens per projection launch (MMA N)

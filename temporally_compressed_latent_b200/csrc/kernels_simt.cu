@@ -165,6 +165,9 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(SeqArgs a, Me
 
   const int64_t L = st.L;
   const T* rows = reinterpret_cast<const T*>(a.cache) + st.off * a.row_stride;
+  // several tokens per call: the last row as it stood after this query's token
+  const T* last = o.tails ? reinterpret_cast<const T*>(o.tails) + (int64_t)b * D : rows + (L - 1) * a.row_stride;
+  auto row_of = [&](int64_t j) { return j == L - 1 ? last : rows + j * a.row_stride; };
   if (L == 0) {
     if (tid == 0) set_err(a.dev_err, MTLA_DEVERR_EMPTY);
     for (int i = tid; i < H * r; i += blockDim.x) o.out[(int64_t)b * H * r + i] = 0.f;
@@ -179,7 +182,7 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(SeqArgs a, Me
       const int64_t j = base + tid;
       float sc = -INFINITY;
       if (j < L) {
-        const T* row = rows + j * a.row_stride;
+        const T* row = row_of(j);
         float dot = 0.f;
         for (int k = 0; k < D; ++k) dot = fmaf(q[k], ld_f32(row + k), dot);
         sc = dot * o.scale;
@@ -197,7 +200,7 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(SeqArgs a, Me
         const int k = tid + c * kSimtThreads;
         if (k < r) {
           float v = acc[c] * alpha;
-          for (int jj = 0; jj < nrows; ++jj) v = fmaf(p_sm[jj], ld_f32(rows + (base + jj) * a.row_stride + k), v);
+          for (int jj = 0; jj < nrows; ++jj) v = fmaf(p_sm[jj], ld_f32(row_of(base + jj) + k), v);
           acc[c] = v;
         }
       }
