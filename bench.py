@@ -311,7 +311,7 @@ def run_ours(args, rank, world, local_rank):
         prefill = run_prefill(torch, mtla, glue, dev)
     configs = None
     if not args.no_configs and rank == 0:
-        configs = run_configs(torch, mtla, glue, dev)
+        configs = run_configs(torch, mtla, glue, dev, set(args.configs.split(",")))
 
     if dist:
         dist.barrier()
@@ -509,6 +509,7 @@ def time_decode_calls(torch, state: DecodeState, n: int, warm: int, flush):
     times, nbytes = [], []
     for _ in range(n):
         flush.zero_()
+        torch.cuda._sleep(100_000)  # the GPU stays busy while the host launches the call
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         state.call()
@@ -527,7 +528,7 @@ def time_decode_calls(torch, state: DecodeState, n: int, warm: int, flush):
             "roofline_ms": by / (hbm_peak * 1e9) * 1e3, "calls": n}
 
 
-def run_configs(torch, mtla, glue, dev):
+def run_configs(torch, mtla, glue, dev, which=("ragged", "sweep", "layer", "multi")):
     """The other decode workloads, one call at a time (L2 flushed before each):
     ragged B=128 (processed lengths uniform in [512, 8192], seed 1) and the
     compression-ratio sweep B=64, T=16384, s in {1, 2, 3, 4, 8}, whose caches
@@ -537,7 +538,20 @@ def run_configs(torch, mtla, glue, dev):
     import dataclasses
     n, warm = 20, 3
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    res = {"timing": f"median of {n} single calls after {warm}, CUDA events, L2 flushed before each call"}
+    res = {"timing": f"median of {n} single calls after {warm}, CUDA events, L2 flushed before each call and a "
+                     "device sleep covering the host's launch"}
+    if "layer" in which:
+        res["layer_maps_b32"] = run_layer_maps(torch, mtla, glue, dev, flush, n, warm)
+    if "multi" in which:
+        res["multi_token_b32_n4"] = run_multi(torch, mtla, glue, dev, flush, n, warm)
+    if "ragged" in which:
+        res["ragged_b128"] = run_ragged(torch, mtla, glue, dev, flush, n, warm)
+    if "sweep" in which:
+        res["sweep_b64_t16384"] = run_sweep(torch, mtla, glue, dev, flush, n, warm)
+    return res
+
+
+def run_ragged(torch, mtla, glue, dev, flush, n, warm):
     case = synth.decode_ragged()
     d = case.dims
     rows_dev = lambda b: torch.from_numpy(case.rows[b]).to(dev).to(torch.bfloat16)
@@ -546,8 +560,11 @@ def run_configs(torch, mtla, glue, dev):
     r = time_decode_calls(torch, st, n, warm, flush)
     r["workload"] = ("ragged decode bf16: B=128, H=8, d_h=64, r=256, d_R=32, s=2, processed lengths uniform in "
                      f"[512, 8192] (seed 1), {int(sum(len(x) for x in case.rows))} cache rows before the calls")
-    res["ragged_b128"] = r
-    del st
+    return r
+
+
+def run_sweep(torch, mtla, glue, dev, flush, n, warm):
+    import dataclasses
     sweep = {}
     B, T = 64, 16384
     for s in (1, 2, 3, 4, 8):
@@ -579,12 +596,8 @@ def run_configs(torch, mtla, glue, dev):
         sweep[f"s={s}"] = r
         del st
         torch.cuda.empty_cache()
-    res["sweep_b64_t16384"] = {"workload": "compression-ratio sweep bf16: B=64, t=16384 processed tokens, H=8, "
-                                           "d_h=64, r=256, d_R=32; cache merged from N(0,1) latents with the "
-                                           "sigmoid gates", **sweep}
-    res["layer_maps_b32"] = run_layer_maps(torch, mtla, glue, dev, flush, n, warm)
-    res["multi_token_b32_n4"] = run_multi(torch, mtla, glue, dev, flush, n, warm)
-    return res
+    return {"workload": "compression-ratio sweep bf16: B=64, t=16384 processed tokens, H=8, d_h=64, r=256, "
+                        "d_R=32; cache merged from N(0,1) latents with the sigmoid gates", **sweep}
 
 
 def time_calls(torch, call, n, warm, flush):
@@ -595,6 +608,7 @@ def time_calls(torch, call, n, warm, flush):
     times = []
     for _ in range(n):
         flush.zero_()
+        torch.cuda._sleep(100_000)  # the GPU stays busy while the host launches the call
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         call()
@@ -859,6 +873,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the ragged and s-sweep decode workloads")
+    ap.add_argument("--configs", default="ragged,sweep,layer,multi",
+                    help="which extra workloads to time (comma-separated: ragged, sweep, layer, multi)")
     ap.add_argument("--cpu-baseline", dest="cpu_baseline", action="store_true", default=True)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=8.0)

@@ -396,7 +396,7 @@ mtla_status mtla_prefill_masked_attn(const mtla_dims* dims, int32_t B, int32_t T
 // Workspace of a call with n new tokens per sequence: the B n virtual
 // sequences' arrays, their tail rows, then the split-L workspace for B n.
 struct MultiLayout {
-  size_t t_v, off_v, cap_v, tails, dec, total;
+  size_t t_v, off_v, cap_v, tails, gates, dec, total;
 };
 static MultiLayout multi_layout(const mtla_dims* dims, int32_t B, int32_t n, size_t dec_bytes) {
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
@@ -406,7 +406,8 @@ static MultiLayout multi_layout(const mtla_dims* dims, int32_t B, int32_t n, siz
   l.off_v = up(Bv * 4);
   l.cap_v = l.off_v + up(Bv * 8);
   l.tails = l.cap_v + up(Bv * 8);
-  l.dec = l.tails + up(Bv * (dims->r + dims->d_R) * elem_size(dims->dtype));
+  l.gates = l.tails + up(Bv * (dims->r + dims->d_R) * elem_size(dims->dtype));
+  l.dec = l.gates + up(Bv * (dims->r + dims->d_R) * 4);
   l.total = l.dec + dec_bytes;
   return l;
 }
@@ -451,6 +452,7 @@ mtla_status mtla_decode_attn_multi(const mtla_dims* dims, int32_t B, int32_t n, 
   mm.n = n;
   mm.four_part = tc && dims->r == dtc::R && dims->d_R == dtc::DR;  // the tensor-core step's gate order
   mm.tails = ws + ml.tails;
+  mm.gates = reinterpret_cast<float*>(ws + ml.gates);
   mm.t_v = reinterpret_cast<int32_t*>(ws + ml.t_v);
   mm.off_v = reinterpret_cast<int64_t*>(ws + ml.off_v);
   mm.cap_v = reinterpret_cast<int64_t*>(ws + ml.cap_v);

@@ -131,6 +131,7 @@ struct MultiMergeArgs {
   int n;
   int four_part;      // gate sums in four 64-row parts (the tensor-core decode's merge order)
   void* tails;        // [B n][D] cache dtype: the tail row after token i of sequence b
+  float* gates;       // [B n][D] fp32: the tokens' gate pre-activations c_t W_c + b_c
   int32_t* t_v;       // [B n] tokens processed after query i's token
   int64_t* off_v;     // [B n]
   int64_t* cap_v;     // [B n]

@@ -36,16 +36,25 @@ constexpr int BK = 64;             // K per block: 128-byte rows
 constexpr int MAXKPB = 4;          // K blocks per CTA
 constexpr int NT = 128;
 constexpr int WTILE = BM * BK * 2;            // 16 KB
-constexpr int XTILE = MAXBP * BK * 2;         // 32 KB (room for Bp = 256)
-constexpr size_t OFF_W = 0;
-constexpr size_t OFF_X = OFF_W + (size_t)MAXKPB * WTILE;
-constexpr size_t OFF_BAR = OFF_X + (size_t)MAXKPB * XTILE;
-constexpr size_t OFF_TMEM = OFF_BAR + (MAXKPB + 1) * 8;
-constexpr size_t SMEM_USED = OFF_TMEM + 16;
-static_assert(OFF_X % 1024 == 0 && XTILE % 1024 == 0 && WTILE % 1024 == 0, "swizzle atoms must be 1024-aligned");
-static_assert(SMEM_USED + 1024 <= 232448, "one block's shared memory (227 KB)");
+// Shared memory of a launch, sized to its K blocks per CTA and padded batch:
+// kpb W tiles, kpb X tiles of Bp rows (each a multiple of 1024 bytes, the
+// swizzle atom), then the barriers and the TMEM address.
+struct Layout {
+  size_t x, xtile, bar, tmem, total;
+};
+__host__ __device__ __forceinline__ Layout layout(int kpb, int Bp) {
+  Layout l;
+  l.xtile = ((size_t)Bp * BK * 2 + 1023) / 1024 * 1024;
+  l.x = (size_t)kpb * WTILE;
+  l.bar = l.x + (size_t)kpb * l.xtile;
+  l.tmem = l.bar + (MAXKPB + 1) * 8;
+  l.total = l.tmem + 16 + 1024;  // + slack to align the base to 1024
+  return l;
+}
+static_assert(WTILE % 1024 == 0, "swizzle atoms must be 1024-aligned");
+static_assert(MAXKPB * (WTILE + MAXBP * BK * 2) + 2048 <= 232448, "one block's shared memory (227 KB)");
 
-size_t smem_bytes() { return SMEM_USED + 1024; }
+size_t smem_bytes() { return layout(MAXKPB, MAXBP).total; }
 
 // mbarrier wait by every lane of a warp with a warp-uniform result (the
 // tcgen05.ld that follow are warp-collective)
@@ -58,9 +67,10 @@ __global__ void __launch_bounds__(NT, 1) proj_gemm_kernel(const __grid_constant_
   // blockIdx.x: 128-row tile of W; blockIdx.y: K split
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* w_full = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+  const Layout L = layout(p.kpb, p.Bp);
+  uint64_t* w_full = reinterpret_cast<uint64_t*>(sm + L.bar);
   uint64_t* mma_done = w_full + MAXKPB;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + L.tmem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int m0 = blockIdx.x * BM, ks = blockIdx.y;
   const int kb0 = ks * p.kpb;
@@ -89,14 +99,14 @@ __global__ void __launch_bounds__(NT, 1) proj_gemm_kernel(const __grid_constant_
   if (tid == 0) {
     for (int i = 0; i < nkb; ++i) {
       mbar_arrive_expect_tx(&w_full[i], WTILE);
-      tma_load_2d(sm + OFF_W + (size_t)i * WTILE, &wmap, (kb0 + i) * BK, m0, &w_full[i]);
+      tma_load_2d(sm + (size_t)i * WTILE, &wmap, (kb0 + i) * BK, m0, &w_full[i]);
     }
   }
   // X: row b of K block i -> eight 16-byte chunks, chunk c at b * 128 +
   // ((c ^ (b % 8)) * 16): the 128-byte swizzle of a K-major operand whose
   // 8-row groups are 1024 bytes apart
   for (int i = 0; i < nkb; ++i) {
-    const uint32_t xbase = smem_u32(sm + OFF_X + (size_t)i * XTILE);
+    const uint32_t xbase = smem_u32(sm + L.x + (size_t)i * L.xtile);
     const int64_t k0 = (int64_t)(kb0 + i) * BK;
     for (int idx = tid; idx < p.Bp * 8; idx += NT) {
       const int b = idx >> 3, c = idx & 7;
@@ -129,8 +139,8 @@ __global__ void __launch_bounds__(NT, 1) proj_gemm_kernel(const __grid_constant_
       if (!warp_wait(&w_full[i], 0)) { ok = false; break; }
       tc_fence_after();
       if (elect_one()) {
-        const uint32_t sW = smem_u32(sm + OFF_W + (size_t)i * WTILE);
-        const uint32_t sX = smem_u32(sm + OFF_X + (size_t)i * XTILE);
+        const uint32_t sW = smem_u32(sm + (size_t)i * WTILE);
+        const uint32_t sX = smem_u32(sm + L.x + (size_t)i * L.xtile);
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
           const uint64_t ad = umma_desc(sW + kk * 32, 16, 1024, 2);
@@ -293,7 +303,7 @@ cudaError_t launch_proj_gemm(const GemmArgs& a, const CUtensorMap& wmap, int m_t
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)m_tiles, (unsigned)KS);
   cfg.blockDim = dim3(prj::NT);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = prj::layout(a.kpb, a.Bp).total;  // several CTAs per SM when the tiles are small
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
