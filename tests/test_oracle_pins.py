@@ -383,3 +383,98 @@ def test_project_inputs_at_a_position():
         one = oracle.project_inputs(x[p:p + 1], mc.W, pos=[p])
         for a, b in zip(one, full):
             np.testing.assert_allclose(a[0], b[p], rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# more planted mistakes: each plausible slip in the oracle fails a pin
+# ---------------------------------------------------------------------------
+
+def test_planted_dropped_rope_term_fails_absorption_pin(monkeypatch):
+    # the score loses its q^R . k^R term in the absorbed forward; the explicit
+    # per-head brute force keeps it
+    real = om.masked_forward
+
+    def planted(q_abs, q_rope, Cp, s, d_h):
+        return real(q_abs, np.zeros_like(np.asarray(q_rope, dtype=np.float64)), Cp, s, d_h)
+
+    monkeypatch.setattr(om, "masked_forward", planted)
+    dims = synth.Dims(H=3, d_h=8, r=32, d_R=4, s=2)
+    T, d = 14, 24
+    mc = synth.model_case(dims, B=1, T=T, d=d, seed=32, dtype="f32")
+    q_abs, q_rope, c, kR = oracle.project_inputs(mc.x[0], mc.W)
+    P = oracle.pe_table(synth.ceil_div(T, 2), mc.lin["W_p"], mc.lin["b_p"])
+    Cp = oracle.partial_merge_sequence(c, kR, mc.lin["W_c"], mc.lin["b_c"], P, 2)
+    y = oracle.absorbed_output(om.masked_forward(q_abs, q_rope, Cp, 2, dims.d_h)[0], mc.W["W_V"], mc.W["W_O"])
+    assert np.abs(y - oracle.unabsorbed_forward(mc.x[0], mc.W, Cp, 2)).max() > 1e-3
+
+
+def test_planted_wrong_sign_fails_worked_example(monkeypatch, golden_dir):
+    # the in-place update subtracts the gated entry instead of adding it
+    def planted(rows, t, s, c_t, kR_t, w):
+        entry = np.asarray(w) * np.concatenate([np.asarray(c_t, np.float64), np.asarray(kR_t, np.float64)])
+        rows = [np.array(r_, dtype=np.float64) for r_ in rows]
+        if om.opens_new_row(t, s):
+            rows.append(entry)
+        else:
+            rows[-1] = rows[-1] - entry
+        return rows
+
+    monkeypatch.setattr(om, "merge_step", planted)
+    monkeypatch.setattr(oracle, "merge_step", planted)
+    with pytest.raises(AssertionError):
+        test_worked_example_merge(golden_dir)
+
+
+def test_planted_off_by_one_group_fails_length_golden(monkeypatch, golden_dir):
+    # j(t) = floor(t/s) + 1 agrees with ceil(t/s) except when s divides t
+    monkeypatch.setattr(om, "group_index", lambda t, s: t // s + 1)
+    monkeypatch.setattr(oracle, "group_index", lambda t, s: t // s + 1)
+    # the golden lengths, or the merge's own check of the row count, fail
+    with pytest.raises((AssertionError, ValueError)):
+        test_cache_lengths_golden(golden_dir)
+
+
+def test_planted_wrong_pe_row_fails_consistency(monkeypatch):
+    # the parallel forward's running merge gates token n with the P row of the
+    # next group (j instead of j - 1); decoding keeps the right row
+    def planted(c, kR, W_c, b_c, P, s):
+        c, kR, P = (np.asarray(a, dtype=np.float64) for a in (c, kR, P))
+        pre = c @ np.asarray(W_c, np.float64) + np.asarray(b_c, np.float64)
+        Cp = np.zeros((c.shape[0], pre.shape[1]))
+        for n in range(1, c.shape[0] + 1):
+            j = om.group_index(n, s)
+            e = om.sigmoid(pre[n - 1] * P[j]) * np.concatenate([c[n - 1], kR[n - 1]])
+            Cp[n - 1] = e if om.opens_new_row(n, s) else Cp[n - 2] + e
+        return Cp
+
+    dims = synth.Dims(H=2, d_h=8, r=16, d_R=4, s=2)
+    case = synth.token_case(dims, B=1, T=10, seed=41, dtype="f32")
+    P = oracle.pe_table(8, case.lin["W_p"], case.lin["b_p"])
+    args = (case.c[0], case.kR[0], case.lin["W_c"], case.lin["b_c"], P, 2)
+    seq = oracle.decode_loop(case.c[0], case.kR[0], case.q_abs[0], case.q_rope[0], case.lin["W_c"], case.lin["b_c"],
+                             P, 2, dims.d_h)
+    good = oracle.masked_forward(case.q_abs[0], case.q_rope[0], oracle.partial_merge_sequence(*args), 2, 8)[0]
+    np.testing.assert_allclose(good, seq["o"], rtol=1e-11, atol=1e-12)
+    monkeypatch.setattr(om, "partial_merge_sequence", planted)
+    bad = oracle.masked_forward(case.q_abs[0], case.q_rope[0], om.partial_merge_sequence(*args), 2, 8)[0]
+    assert np.abs(bad - seq["o"]).max() > 1e-3
+
+
+def test_planted_transposed_value_map_fails_absorption_pin(monkeypatch):
+    # the output side applies W_V^h transposed (square when r == d_h)
+    def planted(o, W_V, W_O):
+        o, W_V, W_O = (np.asarray(a, dtype=np.float64) for a in (o, W_V, W_O))
+        H, d_h = W_V.shape[0], W_V.shape[2]
+        return sum((o[:, h, :] @ W_V[h].T) @ W_O[h * d_h:(h + 1) * d_h, :] for h in range(H))
+
+    dims = synth.Dims(H=2, d_h=8, r=8, d_R=4, s=2)
+    T, d = 12, 16
+    mc = synth.model_case(dims, B=1, T=T, d=d, seed=43, dtype="f32")
+    q_abs, q_rope, c, kR = oracle.project_inputs(mc.x[0], mc.W)
+    P = oracle.pe_table(synth.ceil_div(T, 2), mc.lin["W_p"], mc.lin["b_p"])
+    Cp = oracle.partial_merge_sequence(c, kR, mc.lin["W_c"], mc.lin["b_c"], P, 2)
+    o = oracle.masked_forward(q_abs, q_rope, Cp, 2, dims.d_h)[0]
+    ref = oracle.unabsorbed_forward(mc.x[0], mc.W, Cp, 2)
+    np.testing.assert_allclose(oracle.absorbed_output(o, mc.W["W_V"], mc.W["W_O"]), ref, rtol=1e-11, atol=1e-12)
+    monkeypatch.setattr(om, "absorbed_output", planted)
+    assert np.abs(om.absorbed_output(o, mc.W["W_V"], mc.W["W_O"]) - ref).max() > 1e-3
