@@ -106,11 +106,21 @@ def _stream(stream):
     return stream if isinstance(stream, int) else stream.cuda_stream
 
 
+_MERGE_CACHE: dict = {}
+
+
 def _merge(m):
+    """The merge-argument struct for `m`; the structs of the last few distinct
+    argument sets are kept, so a decode loop does not rebuild one per call."""
     if m is None:
         return None
-    return _c.byref(_Merge(_ptr(m["c_new"]), _ptr(m["kR_new"]), _ptr(m["W_c"]), _ptr(m["b_c"]), _ptr(m["P"]),
-                           int(m["J_max"])))
+    key = (_ptr(m["c_new"]), _ptr(m["kR_new"]), _ptr(m["W_c"]), _ptr(m["b_c"]), _ptr(m["P"]), int(m["J_max"]))
+    st = _MERGE_CACHE.get(key)
+    if st is None:
+        if len(_MERGE_CACHE) >= 64:
+            _MERGE_CACHE.clear()
+        st = _MERGE_CACHE[key] = _Merge(*key)
+    return _c.byref(st)
 
 
 def _check(status: int, where: str):

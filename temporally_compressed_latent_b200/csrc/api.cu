@@ -109,6 +109,28 @@ struct CacheMaps {
   CUtensorMap m64, m8;
 };
 
+// The tensor maps of the last few cache buffers a thread used (a caller
+// that rotates several caches finds each of them encoded), replaced in
+// round-robin order.  Returns nullptr if encoding fails.
+const CacheMaps* cache_maps(void* cache, int64_t cache_rows, int64_t row_stride) {
+  constexpr int kSlots = 32;
+  thread_local CacheMaps slot[kSlots];
+  thread_local int next = 0;
+  for (int i = 0; i < kSlots; ++i)
+    if (slot[i].ptr == cache && slot[i].rows == cache_rows && slot[i].stride == row_stride) return &slot[i];
+  CacheMaps& m = slot[next];
+  next = (next + 1) % kSlots;
+  if (!encode_cache_map(&m.m64, cache, cache_rows, row_stride, dtc::UNIT, dtc::D / 32) ||
+      !encode_cache_map(&m.m8, cache, cache_rows, row_stride, dtc::SUB, 1)) {
+    m.ptr = nullptr;
+    return nullptr;
+  }
+  m.ptr = cache;
+  m.rows = cache_rows;
+  m.stride = row_stride;
+  return &m;
+}
+
 mtla_status seq_args(const mtla_dims* d, void* cache, int64_t cache_rows, int64_t row_stride,
                      const int64_t* seq_offset, const int64_t* seq_capacity, int32_t* t_processed,
                      int32_t* cache_len, int32_t* dev_err, SeqArgs* a) {
@@ -269,17 +291,8 @@ mtla_status mtla_decode_attn(const mtla_dims* dims, int32_t B, const void* q_abs
   const size_t need = dtc::workspace_bytes(B, grid);
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return MTLA_ERR_WORKSPACE;
 
-  thread_local CacheMaps maps;
-  if (maps.ptr != cache || maps.rows != cache_rows || maps.stride != row_stride) {
-    if (!encode_cache_map(&maps.m64, cache, cache_rows, row_stride, dtc::UNIT, dtc::D / 32) ||
-        !encode_cache_map(&maps.m8, cache, cache_rows, row_stride, dtc::SUB, 1)) {
-      maps.ptr = nullptr;
-      return MTLA_ERR_CUDA;
-    }
-    maps.ptr = cache;
-    maps.rows = cache_rows;
-    maps.stride = row_stride;
-  }
+  const CacheMaps* maps = cache_maps(cache, cache_rows, row_stride);
+  if (!maps) return MTLA_ERR_CUDA;
   dtc::Params p;
   p.a = a;
   p.m = m;
@@ -295,7 +308,7 @@ mtla_status mtla_decode_attn(const mtla_dims* dims, int32_t B, const void* q_abs
   p.tails = reinterpret_cast<__nv_bfloat16*>(ws + wl.tails);
   p.ws_ml = reinterpret_cast<float*>(ws + wl.ml);
   p.ws_o = reinterpret_cast<float*>(ws + wl.o);
-  return from_cuda(launch_decode_tc(p, maps.m64, maps.m8, grid, cs));
+  return from_cuda(launch_decode_tc(p, maps->m64, maps->m8, grid, cs));
 }
 
 mtla_status mtla_prefill_masked_attn(const mtla_dims* dims, int32_t B, int32_t T, const void* q_abs,
@@ -475,17 +488,8 @@ mtla_status mtla_decode_attn_multi(const mtla_dims* dims, int32_t B, int32_t n, 
   o.tails = mm.tails;
   if (!tc) return from_cuda(launch_decode_simt(av, m, false, o, Bv, dims->dtype, cs));
 
-  thread_local CacheMaps maps;
-  if (maps.ptr != cache || maps.rows != cache_rows || maps.stride != row_stride) {
-    if (!encode_cache_map(&maps.m64, cache, cache_rows, row_stride, dtc::UNIT, dtc::D / 32) ||
-        !encode_cache_map(&maps.m8, cache, cache_rows, row_stride, dtc::SUB, 1)) {
-      maps.ptr = nullptr;
-      return MTLA_ERR_CUDA;
-    }
-    maps.ptr = cache;
-    maps.rows = cache_rows;
-    maps.stride = row_stride;
-  }
+  const CacheMaps* maps = cache_maps(cache, cache_rows, row_stride);
+  if (!maps) return MTLA_ERR_CUDA;
   dtc::Params p;
   p.a = av;
   p.m = m;
@@ -501,7 +505,7 @@ mtla_status mtla_decode_attn_multi(const mtla_dims* dims, int32_t B, int32_t n, 
   p.tails = reinterpret_cast<__nv_bfloat16*>(mm.tails);
   p.ws_ml = reinterpret_cast<float*>(dws + wl.ml);
   p.ws_o = reinterpret_cast<float*>(dws + wl.o);
-  return from_cuda(launch_decode_tc(p, maps.m64, maps.m8, grid, cs));
+  return from_cuda(launch_decode_tc(p, maps->m64, maps->m8, grid, cs));
 }
 
 size_t mtla_project_workspace_bytes(const mtla_dims* dims, int32_t B, int32_t d, int32_t which) {
