@@ -285,6 +285,39 @@ mtla_status mtla_project_in(const mtla_dims *dims, int32_t B, int32_t d, const v
 mtla_status mtla_project_out(const mtla_dims *dims, int32_t B, int32_t d, const float *o, const void *W_out,
                              float *y, void *workspace, size_t workspace_bytes, int32_t *dev_err, void *stream);
 
+/*
+ * mtla_prefill_kv — the per-head keys and values of a prompt for the
+ * un-absorbed masked forward ([mask], [rope]): for every position n of every
+ * sequence, k[b, n, h] = c_hat'_n W_K^h and v[b, n, h] = c_hat'_n W_V^h, where
+ * c_hat'_n is the latent part of C_hat' (mtla_prefill_masked_attn's c_partial).
+ *   c_partial [B, T, r + d_R] bf16 (row stride r + d_R)
+ *   W_kv      [2 H d_h, r] bf16, row-major: row h d_h + e is column e of W_K^h,
+ *             row H d_h + h d_h + e is column e of W_V^h
+ *   k, v      [B, T, H, d_h] bf16, written
+ * bf16 with d_h = 64, d_R = 32, r a multiple of 64 up to 256, H even (a
+ * tcgen05 GEMM, 128 positions x 256 features per CTA); else UNSUPPORTED.
+ */
+mtla_status mtla_prefill_kv(const mtla_dims *dims, int32_t B, int32_t T, const void *c_partial, const void *W_kv,
+                            void *k, void *v, int32_t *dev_err, void *stream);
+
+/*
+ * mtla_prefill_unabsorbed_attn — the masked parallel forward in its
+ * un-absorbed form ([mask], [rope]): per head, q_h = x W_Q^h (width d_h),
+ *   score_n = (q_h . k_n,h + q_rope_h . k_hat^R'_n) / sqrt(d_h)
+ * over the columns n == m and n = g s (g < ceil(m/s)), and
+ *   out[b, m, h] = sum_n softmax(score)_n v_n,h   (width d_h),
+ * where k_hat^R'_n is the last d_R channels of C_hat'_n.  By associativity
+ * (Figure 1) out[b, m, h] = (the absorbed forward's output) W_V^h; each visible
+ * pair costs 2 (d_h + d_R) + 2 d_h flops instead of 2 (r + d_R) + 2 r.
+ *   q [B, T, H, d_h], q_rope [B, T, H, d_R], k, v [B, T, H, d_h] (from
+ *   mtla_prefill_kv), c_partial [B, T, r + d_R]: bf16, contiguous.
+ *   out [B, T, H, d_h] bf16, written.
+ * Same dims as mtla_prefill_kv; any T >= 1.
+ */
+mtla_status mtla_prefill_unabsorbed_attn(const mtla_dims *dims, int32_t B, int32_t T, const void *q,
+                                         const void *q_rope, const void *k, const void *v, const void *c_partial,
+                                         void *out, int32_t *dev_err, void *stream);
+
 #define MTLA_WS_DECODE 0
 #define MTLA_PROJ_IN 1
 #define MTLA_PROJ_OUT 2

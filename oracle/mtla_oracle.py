@@ -21,7 +21,7 @@ __all__ = [
     "merge_weight", "merge_step", "decode_attention", "decode_step",
     "decode_loop", "partial_merge_sequence", "compressed_cache",
     "masked_forward", "masked_forward_query", "rope", "project_inputs",
-    "absorbed_output", "unabsorbed_forward", "cache_elements_per_token",
+    "absorbed_output", "unabsorbed_forward", "unabsorbed_heads", "cache_elements_per_token",
 ]
 
 
@@ -397,3 +397,34 @@ def unabsorbed_forward(x, W, Cp, s: int):
         E = np.exp(S - S.max(axis=1, keepdims=True))
         heads.append((E / E.sum(axis=1, keepdims=True)) @ V)
     return np.concatenate(heads, axis=1) @ W_O
+
+
+def unabsorbed_heads(x, W, Cp, s: int, pos=None):
+    """Per-head outputs of the masked forward with explicit keys and values
+    (the un-absorbed form the notes page describes before absorbing W_K and
+    W_V, *Key designs: decoupled RoPE with temporal compression*):
+    q_h = x W_Q^h, q^R_h = RoPE(x W_QR^h), K_h = C_hat'_latent W_K^h,
+    V_h = C_hat'_latent W_V^h, K^R = C_hat'_rope;
+    score = (q_h . K_h,n + q^R_h . K^R_n) / sqrt(d_h) under the stride-aware
+    mask; o_h = sum_n softmax(score)_n V_h,n.  Returns [T, H, d_h]."""
+    x = np.asarray(x, dtype=np.float64)
+    Cp = np.asarray(Cp, dtype=np.float64)
+    W_Q = np.asarray(W["W_Q"], dtype=np.float64)
+    W_K = np.asarray(W["W_K"], dtype=np.float64)
+    W_V = np.asarray(W["W_V"], dtype=np.float64)
+    W_QR = np.asarray(W["W_QR"], dtype=np.float64)
+    T = x.shape[0]
+    H, r, d_h = W_K.shape
+    pos = np.arange(T) if pos is None else np.asarray(pos)
+    mask = stride_mask(T, s)
+    out = np.zeros((T, H, d_h))
+    for h in range(H):
+        q = x @ W_Q[:, h, :]
+        qR = rope(x @ W_QR[:, h, :], pos)
+        K = Cp[:, :r] @ W_K[h]
+        V = Cp[:, :r] @ W_V[h]
+        S = (q @ K.T + qR @ Cp[:, r:].T) / math.sqrt(d_h)
+        S = np.where(mask, S, -np.inf)
+        E = np.exp(S - S.max(axis=1, keepdims=True))
+        out[:, h, :] = (E / E.sum(axis=1, keepdims=True)) @ V
+    return out

@@ -31,7 +31,9 @@ from ._abi import (  # noqa: F401
     mtla_decode_multi_workspace_bytes,
     mtla_decode_attn_static,
     mtla_merge_append,
+    mtla_prefill_kv,
     mtla_prefill_masked_attn,
+    mtla_prefill_unabsorbed_attn,
     mtla_project_in,
     mtla_project_out,
     mtla_project_workspace_bytes,

@@ -67,6 +67,10 @@ lib.mtla_decode_attn_multi.argtypes = [_DIMS_P, _I32, _I32, _P, _P, _MERGE_P, _P
                                        _P, _P, _SZ, _P, _P]
 lib.mtla_decode_multi_workspace_bytes.restype = _SZ
 lib.mtla_decode_multi_workspace_bytes.argtypes = [_DIMS_P, _I32, _I32]
+lib.mtla_prefill_kv.restype = _c.c_int
+lib.mtla_prefill_kv.argtypes = [_DIMS_P, _I32, _I32, _P, _P, _P, _P, _P, _P]
+lib.mtla_prefill_unabsorbed_attn.restype = _c.c_int
+lib.mtla_prefill_unabsorbed_attn.argtypes = [_DIMS_P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P]
 lib.mtla_project_in.restype = _c.c_int
 lib.mtla_project_in.argtypes = [_DIMS_P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P]
 lib.mtla_project_out.restype = _c.c_int
@@ -168,6 +172,17 @@ def mtla_decode_attn_multi(d, B, n, q_abs, q_rope, merge, cache, cache_rows, row
 
 def mtla_decode_multi_workspace_bytes(d, B, n) -> int:
     return int(lib.mtla_decode_multi_workspace_bytes(_c.byref(d), B, n))
+
+
+def mtla_prefill_kv(d, B, T, c_partial, W_kv, k, v, dev_err, stream=None):
+    _check(lib.mtla_prefill_kv(_c.byref(d), B, T, _ptr(c_partial), _ptr(W_kv), _ptr(k), _ptr(v), _ptr(dev_err),
+                               _stream(stream)), "mtla_prefill_kv")
+
+
+def mtla_prefill_unabsorbed_attn(d, B, T, q, q_rope, k, v, c_partial, out, dev_err, stream=None):
+    _check(lib.mtla_prefill_unabsorbed_attn(_c.byref(d), B, T, _ptr(q), _ptr(q_rope), _ptr(k), _ptr(v),
+                                            _ptr(c_partial), _ptr(out), _ptr(dev_err), _stream(stream)),
+           "mtla_prefill_unabsorbed_attn")
 
 
 def mtla_project_in(d, B, dm, x, W_in, pos, q_abs, q_rope, c_new, kR_new, workspace, workspace_bytes, dev_err,

@@ -508,6 +508,70 @@ mtla_status mtla_decode_attn_multi(const mtla_dims* dims, int32_t B, int32_t n, 
   return from_cuda(launch_decode_tc(p, maps->m64, maps->m8, grid, cs));
 }
 
+static bool unabs_dims(const mtla_dims* d) {
+  return d->dtype == MTLA_BF16 && d->d_h == 64 && d->d_R == 32 && d->r % 64 == 0 && d->r <= 256 && d->H % 2 == 0;
+}
+
+mtla_status mtla_prefill_kv(const mtla_dims* dims, int32_t B, int32_t T, const void* c_partial, const void* W_kv,
+                            void* k, void* v, int32_t* dev_err, void* stream) {
+  mtla_status st = check_dims(dims);
+  if (st != MTLA_OK) return st;
+  if (!unabs_dims(dims)) return MTLA_ERR_UNSUPPORTED;
+  if (B < 0 || T < 0) return MTLA_ERR_INVALID_ARG;
+  const void* ptrs[] = {c_partial, W_kv, k, v};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return MTLA_ERR_INVALID_ARG;
+  if (!dev_err) return MTLA_ERR_INVALID_ARG;
+  if (B == 0 || T == 0) return MTLA_OK;
+  const int64_t R = (int64_t)B * T, D = dims->r + dims->d_R;
+  if (R >= (int64_t(1) << 31)) return MTLA_ERR_UNSUPPORTED;
+  const int N = 2 * dims->H * dims->d_h;
+  CUtensorMap amap, bmap;
+  {
+    const cuuint64_t d2[2] = {(cuuint64_t)dims->r, (cuuint64_t)R}, str[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, 128};
+    if (!encode_bf16_map(&amap, c_partial, 2, d2, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MTLA_ERR_CUDA;
+  }
+  if (!encode_weight_map(&bmap, W_kv, N, dims->r)) return MTLA_ERR_CUDA;
+  RowsGemmArgs a;
+  a.R = R;
+  a.N = N;
+  a.nkb = dims->r / 64;
+  a.k = static_cast<__nv_bfloat16*>(k);
+  a.v = static_cast<__nv_bfloat16*>(v);
+  a.dev_err = dev_err;
+  return from_cuda(launch_rows_gemm(a, amap, bmap, static_cast<cudaStream_t>(stream)));
+}
+
+mtla_status mtla_prefill_unabsorbed_attn(const mtla_dims* dims, int32_t B, int32_t T, const void* q,
+                                         const void* q_rope, const void* k, const void* v, const void* c_partial,
+                                         void* out, int32_t* dev_err, void* stream) {
+  mtla_status st = check_dims(dims);
+  if (st != MTLA_OK) return st;
+  if (!unabs_dims(dims)) return MTLA_ERR_UNSUPPORTED;
+  if (B < 0 || T < 0) return MTLA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, q_rope, k, v, c_partial, out};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return MTLA_ERR_INVALID_ARG;
+  if (!dev_err) return MTLA_ERR_INVALID_ARG;
+  if (B == 0 || T == 0) return MTLA_OK;
+  if ((int64_t)B * T * dims->H >= (int64_t(1) << 31)) return MTLA_ERR_UNSUPPORTED;
+  UnabsArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.qr = static_cast<const __nv_bfloat16*>(q_rope);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.v = static_cast<const __nv_bfloat16*>(v);
+  a.cp = static_cast<const __nv_bfloat16*>(c_partial);
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.B = B;
+  a.T = T;
+  a.H = dims->H;
+  a.s = dims->s;
+  a.D = dims->r + dims->d_R;
+  a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->d_h));
+  return from_cuda(launch_prefill_unabs(a, static_cast<cudaStream_t>(stream)));
+}
+
 size_t mtla_project_workspace_bytes(const mtla_dims* dims, int32_t B, int32_t d, int32_t which) {
   if (which != MTLA_PROJ_IN && which != MTLA_PROJ_OUT) return 0;
   return proj_ws(dims, B < MAXBP || (dims && dims->dtype != MTLA_BF16) ? B : MAXBP, d, which);

@@ -168,4 +168,31 @@ cudaError_t launch_proj_simt(const float* x, int64_t ldx, const float* W, int B,
 cudaError_t launch_proj_in_finish(const InFinishArgs& a, int dtype, cudaStream_t st);
 cudaError_t launch_proj_out_finish(const float* part, int KS, int Bp, int B, int N, float* y, cudaStream_t st);
 
+// Per-head keys and values of a prompt for the un-absorbed forward (proj.cu):
+// [k | v] [R x N] = C [R x Kd] W^T, R = B T rows, N = 2 H d_h (a multiple of
+// 256), Kd = r <= 256 (a multiple of 64).
+struct RowsGemmArgs {
+  int64_t R;
+  int N, nkb;
+  __nv_bfloat16* k;  // [R, N / 2]
+  __nv_bfloat16* v;  // [R, N / 2]
+  int32_t* dev_err;
+};
+cudaError_t launch_rows_gemm(const RowsGemmArgs& a, const CUtensorMap& amap, const CUtensorMap& bmap,
+                             cudaStream_t st);
+
+// Masked prefill with explicit per-head keys and values (prefill_unabs.cu):
+// bf16, d_h = 64, d_R = 32.
+struct UnabsArgs {
+  const __nv_bfloat16* q;   // [B, T, H, d_h]
+  const __nv_bfloat16* qr;  // [B, T, H, d_R]
+  const __nv_bfloat16* k;   // [B, T, H, d_h]
+  const __nv_bfloat16* v;   // [B, T, H, d_h]
+  const __nv_bfloat16* cp;  // [B, T, D] C_hat' (its last d_R channels are the keys' RoPE part)
+  __nv_bfloat16* out;       // [B, T, H, d_h]
+  int B, T, H, s, D;
+  float scale_log2;
+};
+cudaError_t launch_prefill_unabs(const UnabsArgs& a, cudaStream_t st);
+
 }  // namespace mtla

@@ -344,4 +344,130 @@ cudaError_t launch_proj_out_finish(const float* part, int KS, int Bp, int B, int
   return cudaLaunchKernelEx(&cfg, prj::proj_out_finish_kernel, part, KS, Bp, B, N, y);
 }
 
+// ---------------------------------------------------------------------------
+// Per-head keys and values of a prompt for the un-absorbed forward:
+// [K | V] [R x N] = C [R x Kd] . W^T, C the latent part of C_hat' (row stride
+// ldc), W [N x Kd] = the rows of W_K^h^T then W_V^h^T per head.  One CTA per
+// 128-row x 256-column tile, K <= 256 (four 64-wide blocks, all resident):
+// A = C tile and B = W tile both by TMA (K-major, 128-byte swizzle), D in
+// TMEM (256 columns); thread = row, bf16 stores of 32 consecutive columns.
+// ---------------------------------------------------------------------------
+namespace prj {
+constexpr int RG_BN = 256;
+constexpr int RG_MAXKB = 4;
+constexpr int RG_ATILE = BM * BK * 2;     // 16 KB
+constexpr int RG_BTILE = RG_BN * BK * 2;  // 32 KB
+constexpr size_t RG_OFF_B = (size_t)RG_MAXKB * RG_ATILE;
+constexpr size_t RG_OFF_BAR = RG_OFF_B + (size_t)RG_MAXKB * RG_BTILE;
+constexpr size_t RG_OFF_TMEM = RG_OFF_BAR + (RG_MAXKB + 1) * 8;
+constexpr size_t RG_SMEM = RG_OFF_TMEM + 16 + 1024;
+static_assert(RG_SMEM <= 232448, "one block's shared memory (227 KB)");
+
+__global__ void __launch_bounds__(NT, 1) rows_gemm_kernel(const __grid_constant__ CUtensorMap amap,
+                                                          const __grid_constant__ CUtensorMap bmap, const RowsGemmArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + RG_OFF_BAR);
+  uint64_t* mma_done = full + RG_MAXKB;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + RG_OFF_TMEM);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int m0 = blockIdx.x * BM, n0 = blockIdx.y * RG_BN;
+  if (tid == 0) {
+    for (int i = 0; i < RG_MAXKB; ++i) mbar_init(&full[i], 1);
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+    prefetch_tmap(&amap);
+    prefetch_tmap(&bmap);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_holder, RG_BN);
+    tmem_relinquish();
+  }
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // C_hat' comes from the previous launch
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  if (tid == 0) {
+    for (int i = 0; i < p.nkb; ++i) {
+      mbar_arrive_expect_tx(&full[i], RG_ATILE + RG_BTILE);
+      tma_load_2d(sm + (size_t)i * RG_ATILE, &amap, i * BK, m0, &full[i]);
+      tma_load_2d(sm + RG_OFF_B + (size_t)i * RG_BTILE, &bmap, i * BK, n0, &full[i]);
+      tma_load_2d(sm + RG_OFF_B + (size_t)i * RG_BTILE + RG_BTILE / 2, &bmap, i * BK, n0 + 128, &full[i]);
+    }
+  }
+  bool ok = true;
+  if (warp == 0) {
+    constexpr uint32_t idesc = umma_idesc_bf16(BM, RG_BN, false, false);
+    for (int i = 0; i < p.nkb && ok; ++i) {
+      if (!warp_wait(&full[i], 0)) { ok = false; break; }
+      tc_fence_after();
+      if (elect_one()) {
+        const uint32_t sA = smem_u32(sm + (size_t)i * RG_ATILE);
+        const uint32_t sB = smem_u32(sm + RG_OFF_B + (size_t)i * RG_BTILE);
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
+          umma_bf16(tmem, umma_desc(sA + kk * 32, 16, 1024, 2), umma_desc(sB + kk * 32, 16, 1024, 2), idesc,
+                    (i > 0 || kk > 0) ? 1u : 0u);
+      }
+      __syncwarp();
+    }
+    if (elect_one()) umma_commit(mma_done);
+    __syncwarp();
+  }
+  if (!warp_wait(mma_done, 0)) ok = false;
+  tc_fence_after();
+  const int64_t row = m0 + 32 * warp + lane;
+  for (int c0 = 0; c0 < RG_BN; c0 += 32) {
+    uint32_t v[32];
+    tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)c0, v);
+    tmem_wait_ld();
+    if (row < p.R && n0 + c0 < p.N) {
+      uint4 o[4];
+      uint32_t* w = reinterpret_cast<uint32_t*>(o);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+      // columns n0 + c0 .. + 31 of the row: keys below N / 2, values above
+      const int n = n0 + c0;
+      __nv_bfloat16* dst = n < p.N / 2 ? p.k + row * (int64_t)(p.N / 2) + n : p.v + row * (int64_t)(p.N / 2) + (n - p.N / 2);
+      uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) d4[j] = o[j];
+    }
+  }
+  if (!ok && tid == 0) set_err(p.dev_err, MTLA_DEVERR_TIMEOUT);
+  if (tid == 0)
+    for (int i = 0; i < p.nkb; ++i) mbar_wait(&full[i], 0);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, RG_BN);
+  }
+}
+}  // namespace prj
+
+cudaError_t launch_rows_gemm(const RowsGemmArgs& a, const CUtensorMap& amap, const CUtensorMap& bmap,
+                             cudaStream_t st) {
+  static uint64_t done_mask = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64 || !(done_mask & (1ull << dev))) {
+    e = cudaFuncSetAttribute(prj::rows_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prj::RG_SMEM);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) done_mask |= 1ull << dev;
+  }
+  cudaLaunchAttribute attr[1] = {pdl_attr()};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((a.R + prj::BM - 1) / prj::BM), (unsigned)(a.N / prj::RG_BN));
+  cfg.blockDim = dim3(prj::NT);
+  cfg.dynamicSmemBytes = prj::RG_SMEM;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, prj::rows_gemm_kernel, amap, bmap, a);
+}
+
 }  // namespace mtla

@@ -85,3 +85,19 @@ def absorbed_weights(W: dict, dtype=torch.bfloat16):
     W_in = torch.cat(rows, dim=0)
     W_out = torch.cat([(W_V[h] @ W_O[h * d_h:(h + 1) * d_h, :]).T for h in range(H)], dim=1)
     return W_in.to(dtype).contiguous(), W_out.to(dtype).contiguous()
+
+
+def query_heads(x: torch.Tensor, W: dict) -> torch.Tensor:
+    """q_h = x W_Q^h for the un-absorbed forward: x [B, T, d] -> [B, T, H, d_h] (fp32)."""
+    W_Q = W["W_Q"].to(torch.float32)
+    d, H, d_h = W_Q.shape
+    return (x.to(torch.float32) @ W_Q.reshape(d, H * d_h)).reshape(*x.shape[:-1], H, d_h).contiguous()
+
+
+def kv_weights(W: dict, dtype=torch.bfloat16) -> torch.Tensor:
+    """W_kv [2 H d_h, r] of mtla_prefill_kv: row h d_h + e is column e of
+    W_K^h, row H d_h + h d_h + e is column e of W_V^h."""
+    W_K, W_V = W["W_K"], W["W_V"]
+    H, r, d_h = W_K.shape
+    rows = [W_K[h].T for h in range(H)] + [W_V[h].T for h in range(H)]
+    return torch.cat(rows, dim=0).to(dtype).contiguous()

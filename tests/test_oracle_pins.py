@@ -478,3 +478,23 @@ def test_planted_transposed_value_map_fails_absorption_pin(monkeypatch):
     np.testing.assert_allclose(oracle.absorbed_output(o, mc.W["W_V"], mc.W["W_O"]), ref, rtol=1e-11, atol=1e-12)
     monkeypatch.setattr(om, "absorbed_output", planted)
     assert np.abs(om.absorbed_output(o, mc.W["W_V"], mc.W["W_O"]) - ref).max() > 1e-3
+
+
+
+@pytest.mark.parametrize("s", [1, 2, 3])
+def test_unabsorbed_heads_equal_absorbed_times_value_map(s):
+    """Figure 1 per head: the explicit-key form's o_h equals the absorbed
+    form's o_h (width r) times W_V^h, and concatenated through W_O it is the
+    brute-force layer output."""
+    dims = synth.Dims(H=3, d_h=8, r=32, d_R=4, s=s)
+    T, d = 13, 24
+    mc = synth.model_case(dims, B=1, T=T, d=d, seed=50 + s, dtype="f32")
+    q_abs, q_rope, c, kR = oracle.project_inputs(mc.x[0], mc.W)
+    P = oracle.pe_table(synth.ceil_div(T, s), mc.lin["W_p"], mc.lin["b_p"])
+    Cp = oracle.partial_merge_sequence(c, kR, mc.lin["W_c"], mc.lin["b_c"], P, s)
+    heads = oracle.unabsorbed_heads(mc.x[0], mc.W, Cp, s)
+    o_abs, _ = oracle.masked_forward(q_abs, q_rope, Cp, s, dims.d_h)
+    for h in range(dims.H):
+        np.testing.assert_allclose(heads[:, h, :], o_abs[:, h, :] @ mc.W["W_V"][h], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(heads.reshape(T, -1) @ mc.W["W_O"], oracle.unabsorbed_forward(mc.x[0], mc.W, Cp, s),
+                               rtol=1e-11, atol=1e-12)
