@@ -440,6 +440,7 @@ def run_prefill(torch, mtla, glue, dev):
     ms_merge = timed(False)  # cache-only call: the running-merge kernel alone
     if int(err.item()):
         raise RuntimeError(f"device error bits {int(err.item())} in the prefill")
+    unabs = run_unabsorbed(torch, mtla, glue, dev, mc, W, qr, cp, md, err, flush, timed_call=time_calls)
     ms_attn = ms - ms_merge
     # algorithmic work: every visible (query, head, column) pair, one score of
     # length D and one value row of length r, 2 flops per multiply-add
@@ -454,7 +455,41 @@ def run_prefill(torch, mtla, glue, dev):
                          "frac": attn_tflops / tflops_peak, "kernel": "mtla::ptc::prefill_tc_kernel",
                          "peak_kind": f"{kind} cuBLAS bf16 (burst)"},
             "note": "attention time = full call - cache-only call (the running merge alone); "
-                    "L2 flushed before each call"}
+                    "L2 flushed before each call",
+            "unabsorbed": unabs}
+
+
+def run_unabsorbed(torch, mtla, glue, dev, mc, W, qr, cp, md, err, flush, timed_call):
+    """The same prefill in the un-absorbed form on the running merge's C_hat':
+    mtla_prefill_kv (k, v = C_hat' W_K^h, C_hat' W_V^h) and
+    mtla_prefill_unabsorbed_attn (d_h = 64 keys plus the d_R = 32 RoPE keys)."""
+    d = mc.dims
+    B, T = cp.shape[0], cp.shape[1]
+    q = glue.query_heads(torch.from_numpy(mc.x).to(dev), W).to(torch.bfloat16).contiguous()
+    W_kv = glue.kv_weights(W)
+    k = torch.empty(B, T, d.H, d.d_h, dtype=torch.bfloat16, device=dev)
+    v = torch.empty_like(k)
+    out = torch.empty_like(k)
+    ms_kv = timed_call(torch, lambda: mtla.mtla_prefill_kv(md, B, T, cp, W_kv, k, v, err), 7, 3, flush)
+    ms_at = timed_call(torch, lambda: mtla.mtla_prefill_unabsorbed_attn(md, B, T, q, qr, k, v, cp, out, err),
+                       7, 3, flush)
+    if int(err.item()):
+        raise RuntimeError(f"device error bits {int(err.item())} in the un-absorbed prefill")
+    hbm_peak, tflops_peak, _, kind = measured_peaks()
+    pairs = B * d.H * sum(math.ceil(m / d.s) for m in range(1, T + 1))
+    flops = pairs * (2 * (d.d_h + d.d_R) + 2 * d.d_h)
+    kv_flops = 2 * B * T * d.r * 2 * d.H * d.d_h
+    kv_bytes = B * T * (d.D * 2 + 2 * d.H * d.d_h * 2) + W_kv.numel() * 2
+    at = flops / (ms_at / 1e3) / 1e12
+    return {"ms_kv": ms_kv, "ms_attention": ms_at, "algorithmic_tflop": flops / 1e12,
+            "kv": {"algorithmic_bytes": kv_bytes, "algorithmic_tflop": kv_flops / 1e12,
+                   "achieved_gbs": kv_bytes / (ms_kv / 1e3) / 1e9,
+                   "frac_hbm": kv_bytes / (ms_kv / 1e3) / 1e9 / hbm_peak},
+            "roofline": {"bound": "tensor", "achieved": at, "peak": tflops_peak, "unit": "TFLOP/s",
+                         "frac": at / tflops_peak, "kernel": "mtla::pua::prefill_unabs_kernel",
+                         "peak_kind": f"{kind} cuBLAS bf16 (burst)"},
+            "note": "320 flop per visible (query, head, column): 2 (d_h + d_R) for the score, 2 d_h for the "
+                    "value; median of 7 calls, L2 flushed before each"}
 
 
 class DecodeState:

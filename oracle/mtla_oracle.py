@@ -22,6 +22,8 @@ __all__ = [
     "decode_loop", "partial_merge_sequence", "compressed_cache",
     "masked_forward", "masked_forward_query", "rope", "project_inputs",
     "absorbed_output", "unabsorbed_forward", "unabsorbed_heads", "cache_elements_per_token",
+    "latent_partial_merge", "shortcut_attention", "shortcut_attention_backward", "kv_backward",
+    "latent_merge_backward",
 ]
 
 
@@ -428,3 +430,135 @@ def unabsorbed_heads(x, W, Cp, s: int, pos=None):
         E = np.exp(S - S.max(axis=1, keepdims=True))
         out[:, h, :] = (E / E.sum(axis=1, keepdims=True)) @ V
     return out
+
+
+# ---------------------------------------------------------------------------
+# training path: the uncompressed-RoPE-key shortcut and its backward pass
+# ---------------------------------------------------------------------------
+
+def latent_partial_merge(c, W_c, b_c, P, s: int) -> np.ndarray:
+    """C_hat'_latent [T, r]: the latent channels of the running merge.
+
+    Notes, *Key designs: stride-aware causal mask* (C_hat') and *hyper-network
+    temporal merging* (the gate): C_hat'_n = sum_{i=(j(n)-1)s+1}^{n} w_i[:r] ⊙ c_i
+    with w_i = Sigmoid(Linear(c_i) ⊙ P[j(i)-1]).  Under the training shortcut
+    (*decoupled RoPE with temporal compression*: training may take the
+    uncompressed K^R in place of K_hat^R) only these channels feed the
+    attention, so gate channels r.. play no part."""
+    c = np.asarray(c, dtype=np.float64)
+    W_c = np.asarray(W_c, dtype=np.float64)
+    b_c = np.asarray(b_c, dtype=np.float64)
+    P = np.asarray(P, dtype=np.float64)
+    T, r = c.shape
+    gate_pre = c @ W_c[:, :r] + b_c[:r]
+    Cp = np.zeros((T, r))
+    for n in range(1, T + 1):
+        j = group_index(n, s)
+        entry = sigmoid(gate_pre[n - 1] * P[j - 1, :r]) * c[n - 1]
+        Cp[n - 1] = entry if opens_new_row(n, s) else Cp[n - 2] + entry
+    return Cp
+
+
+def shortcut_attention(q, q_rope, k, v, kR, s: int):
+    """Masked attention with explicit per-head keys and values and the
+    uncompressed RoPE keys (the training shortcut).
+
+    Notes, *Key designs: decoupled RoPE with temporal compression* (training
+    may use K^R itself instead of the merged K_hat^R) and *stride-aware causal
+    mask*: per head h, score_{m,n} = (q_{m,h} . k_{n,h} + q^R_{m,h} . k^R_n) /
+    sqrt(d_h) for n == m or (n < m and n mod s == 0), p = softmax over n,
+    o_{m,h} = sum_n p_{m,n} v_{n,h}.  q, k, v [T, H, d_h], q_rope [T, H, d_R],
+    kR [T, d_R].  Returns (o [T, H, d_h], lse [T, H]), lse the natural log of
+    sum_n exp(score_{m,n})."""
+    q, q_rope, k, v, kR = (np.asarray(a, dtype=np.float64) for a in (q, q_rope, k, v, kR))
+    T, H, d_h = q.shape
+    mask = stride_mask(T, s)
+    o = np.zeros((T, H, d_h))
+    lse = np.zeros((T, H))
+    for h in range(H):
+        S = (q[:, h] @ k[:, h].T + q_rope[:, h] @ kR.T) / math.sqrt(d_h)
+        S = np.where(mask, S, -np.inf)
+        mx = S.max(axis=1, keepdims=True)
+        E = np.exp(S - mx)
+        denom = E.sum(axis=1, keepdims=True)
+        o[:, h] = (E / denom) @ v[:, h]
+        lse[:, h] = mx[:, 0] + np.log(denom[:, 0])
+    return o, lse
+
+
+def shortcut_attention_backward(q, q_rope, k, v, kR, s: int, d_out):
+    """Gradients of a loss through ``shortcut_attention``, given d_out = dL/do.
+
+    The chain rule through score -> softmax -> weighted sum, per head:
+    dP = d_out V^T; dS = P ⊙ (dP - rowsum(P ⊙ dP)) (the softmax Jacobian);
+    dq = dS K / sqrt(d_h), dq^R = dS K^R / sqrt(d_h), dk = dS^T q / sqrt(d_h),
+    dv = P^T d_out, dk^R = sum_h dS^T q^R_h / sqrt(d_h) (K^R is shared by
+    every head).  Returns (dq, dq_rope, dk, dv, dkR) shaped like the inputs."""
+    q, q_rope, k, v, kR, d_out = (np.asarray(a, dtype=np.float64) for a in (q, q_rope, k, v, kR, d_out))
+    T, H, d_h = q.shape
+    mask = stride_mask(T, s)
+    sc = 1.0 / math.sqrt(d_h)
+    dq, dq_rope, dk, dv = (np.zeros_like(a) for a in (q, q_rope, k, v))
+    dkR = np.zeros_like(kR)
+    for h in range(H):
+        S = (q[:, h] @ k[:, h].T + q_rope[:, h] @ kR.T) * sc
+        S = np.where(mask, S, -np.inf)
+        E = np.exp(S - S.max(axis=1, keepdims=True))
+        Pm = E / E.sum(axis=1, keepdims=True)
+        dP = d_out[:, h] @ v[:, h].T
+        dS = Pm * (dP - (Pm * dP).sum(axis=1, keepdims=True))
+        dq[:, h] = dS @ k[:, h] * sc
+        dq_rope[:, h] = dS @ kR * sc
+        dk[:, h] = dS.T @ q[:, h] * sc
+        dv[:, h] = Pm.T @ d_out[:, h]
+        dkR += dS.T @ q_rope[:, h] * sc
+    return dq, dq_rope, dk, dv, dkR
+
+
+def kv_backward(dk, dv, W_K, W_V) -> np.ndarray:
+    """dL/dC_hat'_latent through k_h = C_hat'_latent W_K^h and v_h = C_hat'_latent W_V^h
+    (the un-absorbed key and value maps, Figure 1): sum_h dk_h (W_K^h)^T + dv_h (W_V^h)^T.
+    dk, dv [T, H, d_h]; W_K, W_V [H, r, d_h].  Returns [T, r]."""
+    dk, dv, W_K, W_V = (np.asarray(a, dtype=np.float64) for a in (dk, dv, W_K, W_V))
+    H = W_K.shape[0]
+    return sum(dk[:, h] @ W_K[h].T + dv[:, h] @ W_V[h].T for h in range(H))
+
+
+def latent_merge_backward(c, W_c, b_c, P, s: int, dCp):
+    """Gradients of a loss through ``latent_partial_merge``, given dCp = dL/dC_hat'_latent.
+
+    Chain rule in the order of the forward (Notes, *hyper-network temporal
+    merging*):
+    - de_i = sum of dCp_n over the positions n >= i of token i's group
+      (C_hat'_n sums the gated entries e_i of its group up to n);
+    - e_i = w_i ⊙ c_i gives dw_i = de_i ⊙ c_i and a direct dc_i = de_i ⊙ w_i;
+    - w_i = Sigmoid(z_i) gives dz_i = dw_i ⊙ w_i ⊙ (1 - w_i);
+    - z_i = g_i ⊙ P[j(i)-1] gives dg_i = dz_i ⊙ P[j(i)-1] and dP[j(i)-1] += dz_i ⊙ g_i;
+    - g_i = c_i W_c + b_c gives dc_i += dg_i W_c^T, dW_c += c_i^T dg_i, db_c += dg_i.
+    Only the first r gate channels reach C_hat'_latent; the other channels of
+    dW_c, db_c and dP are zero.  Returns (dc [T, r], dW_c, db_c, dP) shaped
+    like c, W_c, b_c and P."""
+    c, W_c, b_c, P, dCp = (np.asarray(a, dtype=np.float64) for a in (c, W_c, b_c, P, dCp))
+    T, r = c.shape
+    g = c @ W_c[:, :r] + b_c[:r]
+    de = np.zeros((T, r))
+    for i in range(T, 0, -1):
+        de[i - 1] = dCp[i - 1]
+        if i < T and not opens_new_row(i + 1, s):
+            de[i - 1] += de[i]
+    dc = np.zeros((T, r))
+    dW_c = np.zeros_like(W_c)
+    db_c = np.zeros_like(b_c)
+    dP = np.zeros_like(P)
+    for i in range(1, T + 1):
+        j = group_index(i, s)
+        u = P[j - 1, :r]
+        w = sigmoid(g[i - 1] * u)
+        dw = de[i - 1] * c[i - 1]
+        dz = dw * w * (1.0 - w)
+        dg = dz * u
+        dP[j - 1, :r] += dz * g[i - 1]
+        dc[i - 1] = de[i - 1] * w + W_c[:, :r] @ dg
+        dW_c[:, :r] += np.outer(c[i - 1], dg)
+        db_c[:r] += dg
+    return dc, dW_c, db_c, dP
