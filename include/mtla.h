@@ -5,8 +5,9 @@
  * KV cache compressed twice: in feature width (a latent c of width r plus a
  * decoupled-RoPE key of width d_R) and in time (every s adjacent steps are
  * merged by a sigmoid-gated hyper-network).  This library runs the inference
- * hot path (merge/append + absorbed decode attention) and the parallel
- * training/prefill forward under the stride-aware causal mask.
+ * hot path (merge/append + absorbed decode attention), the parallel
+ * training/prefill forward under the stride-aware causal mask, and the
+ * training shortcut's backward pass.
  *
  * Sources (page title, section):
  *   [merge]   MTLA paper notes, "Key designs: hyper-network temporal merging":
@@ -20,6 +21,9 @@
  *   [fig2]    arXiv 2505.13544 abstract page, Figure 2: (a) incremental
  *             inference attends a temporary c_hat'_j at steps 1, 3, 5 (s = 2);
  *             (c) training with the stride-aware mask.
+ *   [train]   MTLA paper notes, "Key designs: decoupled RoPE with temporal
+ *             compression": training may take the uncompressed K^R in place
+ *             of the merged K_hat^R (the training shortcut).
  *
  * Conventions for every call
  *   - Time is 1-indexed as on the pages: token t of a sequence belongs to group
@@ -317,6 +321,85 @@ mtla_status mtla_prefill_kv(const mtla_dims *dims, int32_t B, int32_t T, const v
 mtla_status mtla_prefill_unabsorbed_attn(const mtla_dims *dims, int32_t B, int32_t T, const void *q,
                                          const void *q_rope, const void *k, const void *v, const void *c_partial,
                                          void *out, int32_t *dev_err, void *stream);
+
+/*
+ * Training path ([train], [mask], [merge]).  The forward is
+ *   mtla_prefill_masked_attn (cache-only: C_hat') -> mtla_prefill_kv (k, v)
+ *   -> mtla_train_attn_fwd (out, lse);
+ * the backward, given d_out = dL/dout, runs the same chain in reverse:
+ *   mtla_train_attn_bwd (dq, dq_rope, dk, dv, dkR) -> mtla_train_kv_bwd
+ *   (dL/dC_hat'_latent) -> mtla_train_merge_bwd (dc, dW_c, db_c, dP).
+ * Under the shortcut only the latent channels of C_hat' reach the attention;
+ * the RoPE key gradient dkR goes to the caller's K^R directly.  Gradients of
+ * the caller's own maps (W_Q, W_K, W_V, the projections) are plain GEMMs on
+ * these outputs and are left to the caller.  All three backward calls need
+ * bf16, d_h = 64, d_R = 32, r = 256.
+ */
+
+/*
+ * mtla_train_attn_fwd — the masked forward with explicit keys and values and
+ * the uncompressed RoPE keys: per head,
+ *   score_n = (q_h . k_n,h + q_rope_h . kR_n) / sqrt(d_h)
+ * over the columns n == m and n = g s < m ([mask]), out = softmax(score) v.
+ *   q, k, v [B, T, H, d_h], q_rope [B, T, H, d_R], kR [B, T, d_R] (RoPE
+ *   applied): bf16, contiguous.
+ *   out [B, T, H, d_h] bf16 and lse [B, T, H] fp32 (natural log of each
+ *   softmax denominator, for mtla_train_attn_bwd): written.
+ * Dims as mtla_prefill_unabsorbed_attn; any T >= 1.
+ */
+mtla_status mtla_train_attn_fwd(const mtla_dims *dims, int32_t B, int32_t T, const void *q, const void *q_rope,
+                                const void *k, const void *v, const void *kR, void *out, float *lse,
+                                int32_t *dev_err, void *stream);
+
+#define MTLA_TRAIN_ATTN_BWD 1
+#define MTLA_TRAIN_KV_BWD 2
+#define MTLA_TRAIN_MERGE_BWD 3
+
+/* Workspace bytes of the training backward call `which` (MTLA_TRAIN_*) for B
+ * sequences of T tokens (0 on unsupported arguments). */
+size_t mtla_train_workspace_bytes(const mtla_dims *dims, int32_t B, int32_t T, int32_t which);
+
+/*
+ * mtla_train_attn_bwd — gradients through mtla_train_attn_fwd given
+ * d_out = dL/dout (softmax Jacobian: dS = P (d_out v^T - rowsum(d_out out))):
+ *   dq, dk, dv [B, T, H, d_h] and dq_rope [B, T, H, d_R]: bf16, written;
+ *   dkR [B, T, d_R] fp32, written: summed over heads (every head reads the
+ *   same K^R).
+ * Inputs as mtla_train_attn_fwd plus its out and lse, and d_out [B, T, H, d_h]
+ * bf16.  Every output element is written by exactly one block in a fixed
+ * order: the results do not depend on scheduling.
+ */
+mtla_status mtla_train_attn_bwd(const mtla_dims *dims, int32_t B, int32_t T, const void *q, const void *q_rope,
+                                const void *k, const void *v, const void *kR, const void *out, const float *lse,
+                                const void *d_out, void *dq, void *dq_rope, void *dk, void *dv, float *dkR,
+                                void *workspace, size_t workspace_bytes, int32_t *dev_err, void *stream);
+
+/*
+ * mtla_train_kv_bwd — dL/dC_hat'_latent through k = C_hat'_latent W_K^h and
+ * v = C_hat'_latent W_V^h: dC[b, n] = sum_h dk[b,n,h] (W_K^h)^T + dv[b,n,h] (W_V^h)^T.
+ *   dk, dv [B, T, H, d_h] bf16; W_kv as in mtla_prefill_kv.
+ *   dC [B, T, r] fp32, written.  One tensor-core GEMM (K = 2 H d_h).
+ */
+mtla_status mtla_train_kv_bwd(const mtla_dims *dims, int32_t B, int32_t T, const void *dk, const void *dv,
+                              const void *W_kv, float *dC, void *workspace, size_t workspace_bytes,
+                              int32_t *dev_err, void *stream);
+
+/*
+ * mtla_train_merge_bwd — gradients through the latent channels of the running
+ * merge ([merge], [mask]): C_hat'_n = sum over tokens i <= n of n's group of
+ * w_i ⊙ c_i, w_i = Sigmoid((c_i W_c + b_c) ⊙ P[j(i)-1]), given dC = dL/dC_hat'.
+ *   c [B, T, r] bf16 (the latents given to the forward); W_c [r, D], b_c [D],
+ *   P [J_max, D] fp32 as in mtla_merge_args; dC [B, T, r] fp32.
+ *   dc [B, T, r], dW_c [r, D], db_c [D], dP [J_max, D] fp32: written in full
+ *   (entries the latent merge does not reach, the RoPE gate channels and the
+ *   groups past T, are zero).  J_max >= ceil(T/s).
+ * The gate pre-activations are recomputed from bf16 c and W_c on the tensor
+ * cores; the chain rule runs in fp32.
+ */
+mtla_status mtla_train_merge_bwd(const mtla_dims *dims, int32_t B, int32_t T, const void *c, const float *W_c,
+                                 const float *b_c, const float *P, int32_t J_max, const float *dC, float *dc,
+                                 float *dW_c, float *db_c, float *dP, void *workspace, size_t workspace_bytes,
+                                 int32_t *dev_err, void *stream);
 
 #define MTLA_WS_DECODE 0
 #define MTLA_PROJ_IN 1

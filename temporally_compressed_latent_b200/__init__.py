@@ -19,6 +19,9 @@ from ._abi import (  # noqa: F401
     MTLA_F32,
     PROJ_IN,
     PROJ_OUT,
+    TRAIN_ATTN_BWD,
+    TRAIN_KV_BWD,
+    TRAIN_MERGE_BWD,
     WS_DECODE,
     MtlaError,
     dims,
@@ -38,5 +41,10 @@ from ._abi import (  # noqa: F401
     mtla_project_out,
     mtla_project_workspace_bytes,
     mtla_status_string,
+    mtla_train_attn_bwd,
+    mtla_train_attn_fwd,
+    mtla_train_kv_bwd,
+    mtla_train_merge_bwd,
+    mtla_train_workspace_bytes,
     mtla_workspace_bytes,
 )

@@ -24,6 +24,7 @@ lib = ctypes.CDLL(LIB_PATH)
 MTLA_F32, MTLA_BF16 = 0, 1
 WS_DECODE = 0
 PROJ_IN, PROJ_OUT = 1, 2
+TRAIN_ATTN_BWD, TRAIN_KV_BWD, TRAIN_MERGE_BWD = 1, 2, 3  # MTLA_TRAIN_*
 DECODE_STATIC_SCRATCH_BYTES = 24 << 20  # MTLA_DECODE_STATIC_SCRATCH_BYTES
 MAX_NEW_TOKENS = 16  # MTLA_MAX_NEW_TOKENS
 DEVERR_PE_RANGE, DEVERR_CAPACITY, DEVERR_EMPTY, DEVERR_TIMEOUT = 1, 2, 4, 8
@@ -77,6 +78,17 @@ lib.mtla_project_out.restype = _c.c_int
 lib.mtla_project_out.argtypes = [_DIMS_P, _I32, _I32, _P, _P, _P, _P, _SZ, _P, _P]
 lib.mtla_project_workspace_bytes.restype = _SZ
 lib.mtla_project_workspace_bytes.argtypes = [_DIMS_P, _I32, _I32, _I32]
+lib.mtla_train_attn_fwd.restype = _c.c_int
+lib.mtla_train_attn_fwd.argtypes = [_DIMS_P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _P]
+lib.mtla_train_workspace_bytes.restype = _SZ
+lib.mtla_train_workspace_bytes.argtypes = [_DIMS_P, _I32, _I32, _I32]
+lib.mtla_train_attn_bwd.restype = _c.c_int
+lib.mtla_train_attn_bwd.argtypes = [_DIMS_P, _I32, _I32] + [_P] * 14 + [_SZ, _P, _P]
+lib.mtla_train_kv_bwd.restype = _c.c_int
+lib.mtla_train_kv_bwd.argtypes = [_DIMS_P, _I32, _I32, _P, _P, _P, _P, _P, _SZ, _P, _P]
+lib.mtla_train_merge_bwd.restype = _c.c_int
+lib.mtla_train_merge_bwd.argtypes = [_DIMS_P, _I32, _I32, _P, _P, _P, _P, _I32, _P, _P, _P, _P, _P, _P, _SZ, _P,
+                                     _P]
 
 
 class MtlaError(RuntimeError):
@@ -183,6 +195,35 @@ def mtla_prefill_unabsorbed_attn(d, B, T, q, q_rope, k, v, c_partial, out, dev_e
     _check(lib.mtla_prefill_unabsorbed_attn(_c.byref(d), B, T, _ptr(q), _ptr(q_rope), _ptr(k), _ptr(v),
                                             _ptr(c_partial), _ptr(out), _ptr(dev_err), _stream(stream)),
            "mtla_prefill_unabsorbed_attn")
+
+
+def mtla_train_attn_fwd(d, B, T, q, q_rope, k, v, kR, out, lse, dev_err, stream=None):
+    _check(lib.mtla_train_attn_fwd(_c.byref(d), B, T, _ptr(q), _ptr(q_rope), _ptr(k), _ptr(v), _ptr(kR), _ptr(out),
+                                   _ptr(lse), _ptr(dev_err), _stream(stream)), "mtla_train_attn_fwd")
+
+
+def mtla_train_workspace_bytes(d, B, T, which) -> int:
+    return int(lib.mtla_train_workspace_bytes(_c.byref(d), B, T, which))
+
+
+def mtla_train_attn_bwd(d, B, T, q, q_rope, k, v, kR, out, lse, d_out, dq, dq_rope, dk, dv, dkR, workspace,
+                        workspace_bytes, dev_err, stream=None):
+    _check(lib.mtla_train_attn_bwd(_c.byref(d), B, T, _ptr(q), _ptr(q_rope), _ptr(k), _ptr(v), _ptr(kR), _ptr(out),
+                                   _ptr(lse), _ptr(d_out), _ptr(dq), _ptr(dq_rope), _ptr(dk), _ptr(dv), _ptr(dkR),
+                                   _ptr(workspace), workspace_bytes, _ptr(dev_err), _stream(stream)),
+           "mtla_train_attn_bwd")
+
+
+def mtla_train_kv_bwd(d, B, T, dk, dv, W_kv, dC, workspace, workspace_bytes, dev_err, stream=None):
+    _check(lib.mtla_train_kv_bwd(_c.byref(d), B, T, _ptr(dk), _ptr(dv), _ptr(W_kv), _ptr(dC), _ptr(workspace),
+                                 workspace_bytes, _ptr(dev_err), _stream(stream)), "mtla_train_kv_bwd")
+
+
+def mtla_train_merge_bwd(d, B, T, c, W_c, b_c, P, J_max, dC, dc, dW_c, db_c, dP, workspace, workspace_bytes, dev_err,
+                         stream=None):
+    _check(lib.mtla_train_merge_bwd(_c.byref(d), B, T, _ptr(c), _ptr(W_c), _ptr(b_c), _ptr(P), J_max, _ptr(dC),
+                                    _ptr(dc), _ptr(dW_c), _ptr(db_c), _ptr(dP), _ptr(workspace), workspace_bytes,
+                                    _ptr(dev_err), _stream(stream)), "mtla_train_merge_bwd")
 
 
 def mtla_project_in(d, B, dm, x, W_in, pos, q_abs, q_rope, c_new, kR_new, workspace, workspace_bytes, dev_err,

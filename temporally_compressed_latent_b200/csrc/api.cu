@@ -561,13 +561,14 @@ mtla_status mtla_prefill_unabsorbed_attn(const mtla_dims* dims, int32_t B, int32
   a.qr = static_cast<const __nv_bfloat16*>(q_rope);
   a.k = static_cast<const __nv_bfloat16*>(k);
   a.v = static_cast<const __nv_bfloat16*>(v);
-  a.cp = static_cast<const __nv_bfloat16*>(c_partial);
+  a.kr = static_cast<const __nv_bfloat16*>(c_partial) + dims->r;
+  a.kr_stride = dims->r + dims->d_R;
   a.out = static_cast<__nv_bfloat16*>(out);
+  a.lse = nullptr;
   a.B = B;
   a.T = T;
   a.H = dims->H;
   a.s = dims->s;
-  a.D = dims->r + dims->d_R;
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->d_h));
   return from_cuda(launch_prefill_unabs(a, static_cast<cudaStream_t>(stream)));
 }
@@ -691,6 +692,271 @@ mtla_status mtla_project_out(const mtla_dims* dims, int32_t B, int32_t d, const 
       return MTLA_ERR_CUDA;
   }
   return MTLA_OK;
+}
+
+
+// ---------------------------------------------------------------------------
+// training path: the uncompressed-RoPE-key shortcut and its backward pass
+
+static bool train_dims(const mtla_dims* d) {
+  return d->dtype == MTLA_BF16 && d->d_h == 64 && d->d_R == 32 && d->r == 256;
+}
+
+static size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct MergeBwdLayout {
+  int64_t BT, BTp;
+  int J, splits, kb_per;
+  size_t wcT, wc, G, dg, cT, dgT, dbp, dwp, total;
+};
+
+static MergeBwdLayout merge_bwd_layout(const mtla_dims* d, int32_t B, int32_t T) {
+  MergeBwdLayout L = {};
+  const int64_t r = d->r;
+  L.BT = (int64_t)B * T;
+  L.BTp = (L.BT + 63) / 64 * 64;  // K of the dW_c GEMM, padded with zero columns
+  L.J = (int)((T + d->s - 1) / d->s);
+  const int64_t nkb = L.BTp / 64;
+  int sms = device_sms();
+  if (sms < 2) sms = 2;
+  const int64_t want = sms / 2;  // two 128-row tiles of dW_c per K slice: one wave
+  L.kb_per = (int)((nkb + (want < nkb ? want : nkb) - 1) / (want < nkb ? want : nkb));
+  L.splits = (int)((nkb + L.kb_per - 1) / L.kb_per);
+  size_t o = 0;
+  L.wcT = o; o = up256(o + (size_t)r * r * 2);
+  L.wc = o;  o = up256(o + (size_t)r * r * 2);
+  L.G = o;   o = up256(o + (size_t)L.BT * r * 4);
+  L.dg = o;  o = up256(o + (size_t)L.BT * r * 2);
+  L.cT = o;  o = up256(o + (size_t)r * L.BTp * 2);
+  L.dgT = o; o = up256(o + (size_t)r * L.BTp * 2);
+  L.dbp = o; o = up256(o + (size_t)L.J * r * 4);
+  L.dwp = o; o = up256(o + (size_t)L.splits * r * r * 4);
+  L.total = o;
+  return L;
+}
+
+static size_t attn_bwd_bytes(const mtla_dims* d, int32_t B, int32_t T, size_t* off_delta, size_t* off_dkrh) {
+  const size_t n = (size_t)B * T * d->H;
+  const size_t a = up256(n * 4);
+  if (off_delta) *off_delta = a;
+  if (off_dkrh) *off_dkrh = 2 * a;
+  return 2 * a + up256(n * 32 * 4);
+}
+
+size_t mtla_train_workspace_bytes(const mtla_dims* dims, int32_t B, int32_t T, int32_t which) {
+  if (check_dims(dims) != MTLA_OK || !train_dims(dims) || B < 1 || T < 1) return 0;
+  if (which == MTLA_TRAIN_ATTN_BWD) return attn_bwd_bytes(dims, B, T, nullptr, nullptr);
+  if (which == MTLA_TRAIN_KV_BWD) return (size_t)dims->r * 2 * dims->H * dims->d_h * 2;
+  if (which == MTLA_TRAIN_MERGE_BWD) return merge_bwd_layout(dims, B, T).total;
+  return 0;
+}
+
+mtla_status mtla_train_attn_fwd(const mtla_dims* dims, int32_t B, int32_t T, const void* q, const void* q_rope,
+                                const void* k, const void* v, const void* kR, void* out, float* lse,
+                                int32_t* dev_err, void* stream) {
+  mtla_status st = check_dims(dims);
+  if (st != MTLA_OK) return st;
+  if (!unabs_dims(dims)) return MTLA_ERR_UNSUPPORTED;
+  if (B < 0 || T < 0) return MTLA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, q_rope, k, v, kR, out, lse};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return MTLA_ERR_INVALID_ARG;
+  if (!dev_err) return MTLA_ERR_INVALID_ARG;
+  if (B == 0 || T == 0) return MTLA_OK;
+  if ((int64_t)B * T * dims->H >= (int64_t(1) << 31)) return MTLA_ERR_UNSUPPORTED;
+  UnabsArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.qr = static_cast<const __nv_bfloat16*>(q_rope);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.v = static_cast<const __nv_bfloat16*>(v);
+  a.kr = static_cast<const __nv_bfloat16*>(kR);
+  a.kr_stride = dims->d_R;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.lse = lse;
+  a.B = B;
+  a.T = T;
+  a.H = dims->H;
+  a.s = dims->s;
+  a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->d_h));
+  return from_cuda(launch_prefill_unabs(a, static_cast<cudaStream_t>(stream)));
+}
+
+mtla_status mtla_train_attn_bwd(const mtla_dims* dims, int32_t B, int32_t T, const void* q, const void* q_rope,
+                                const void* k, const void* v, const void* kR, const void* out, const float* lse,
+                                const void* d_out, void* dq, void* dq_rope, void* dk, void* dv, float* dkR,
+                                void* workspace, size_t workspace_bytes, int32_t* dev_err, void* stream) {
+  mtla_status st = check_dims(dims);
+  if (st != MTLA_OK) return st;
+  if (!train_dims(dims)) return MTLA_ERR_UNSUPPORTED;
+  if (B < 0 || T < 0) return MTLA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, q_rope, k, v, kR, out, lse, d_out, dq, dq_rope, dk, dv, dkR};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return MTLA_ERR_INVALID_ARG;
+  if (!dev_err) return MTLA_ERR_INVALID_ARG;
+  if (B == 0 || T == 0) return MTLA_OK;
+  if ((int64_t)B * T * dims->H * 32 >= (int64_t(1) << 31)) return MTLA_ERR_UNSUPPORTED;
+  size_t off_delta = 0, off_dkrh = 0;
+  const size_t need = attn_bwd_bytes(dims, B, T, &off_delta, &off_dkrh);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < need) return MTLA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  BwdArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.qr = static_cast<const __nv_bfloat16*>(q_rope);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.v = static_cast<const __nv_bfloat16*>(v);
+  a.kr = static_cast<const __nv_bfloat16*>(kR);
+  a.o = static_cast<const __nv_bfloat16*>(out);
+  a.dout = static_cast<const __nv_bfloat16*>(d_out);
+  a.lse = lse;
+  a.dq = static_cast<__nv_bfloat16*>(dq);
+  a.dqr = static_cast<__nv_bfloat16*>(dq_rope);
+  a.dk = static_cast<__nv_bfloat16*>(dk);
+  a.dv = static_cast<__nv_bfloat16*>(dv);
+  a.dkr = dkR;
+  a.ws_lse2 = reinterpret_cast<float*>(ws);
+  a.ws_delta = reinterpret_cast<float*>(ws + off_delta);
+  a.ws_dkrh = reinterpret_cast<float*>(ws + off_dkrh);
+  a.B = B;
+  a.T = T;
+  a.H = dims->H;
+  a.s = dims->s;
+  a.scale = (float)(1.0 / sqrt((double)dims->d_h));
+  a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->d_h));
+  return from_cuda(launch_attn_bwd(a, static_cast<cudaStream_t>(stream)));
+}
+
+// 2-D map of a row-major bf16 matrix [rows, cols] (row stride ld elements) in
+// boxes of 64 columns x 128 rows with the 128-byte swizzle: a K-major GEMM operand
+static bool encode_operand_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld) {
+  const cuuint64_t d2[2] = {(cuuint64_t)cols, (cuuint64_t)rows}, str[1] = {(cuuint64_t)ld * 2};
+  const cuuint32_t box[2] = {64, 128};
+  return encode_bf16_map(map, base, 2, d2, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+mtla_status mtla_train_kv_bwd(const mtla_dims* dims, int32_t B, int32_t T, const void* dk, const void* dv,
+                              const void* W_kv, float* dC, void* workspace, size_t workspace_bytes,
+                              int32_t* dev_err, void* stream) {
+  mtla_status st = check_dims(dims);
+  if (st != MTLA_OK) return st;
+  if (!train_dims(dims)) return MTLA_ERR_UNSUPPORTED;
+  if (B < 0 || T < 0) return MTLA_ERR_INVALID_ARG;
+  const void* ptrs[] = {dk, dv, W_kv, dC};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return MTLA_ERR_INVALID_ARG;
+  if (!dev_err) return MTLA_ERR_INVALID_ARG;
+  if (B == 0 || T == 0) return MTLA_OK;
+  const int64_t BT = (int64_t)B * T;
+  if (BT >= (int64_t(1) << 31)) return MTLA_ERR_UNSUPPORTED;
+  const int r = dims->r, Hd = dims->H * dims->d_h;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < (size_t)r * 2 * Hd * 2) return MTLA_ERR_WORKSPACE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  __nv_bfloat16* wkvT = static_cast<__nv_bfloat16*>(workspace);  // [r, 2 H d_h]: W_kv transposed
+  if (launch_transpose_bf16(static_cast<const __nv_bfloat16*>(W_kv), 2 * Hd, r, r, wkvT, 2 * Hd, cs) != cudaSuccess)
+    return MTLA_ERR_CUDA;
+  CUtensorMap a0, a1, bm;
+  if (!encode_operand_map(&a0, dk, BT, Hd, Hd) || !encode_operand_map(&a1, dv, BT, Hd, Hd) ||
+      !encode_operand_map(&bm, wkvT, r, 2 * Hd, 2 * Hd))
+    return MTLA_ERR_CUDA;
+  GemmBtArgs g;
+  g.M = BT;
+  g.N = r;
+  g.K = 2 * Hd;
+  g.ka_split = Hd;
+  g.kb_per_split = (2 * Hd + 63) / 64;
+  g.C = dC;
+  g.ldc = r;
+  g.split_stride = 0;
+  g.accumulate = 0;
+  g.dev_err = dev_err;
+  return from_cuda(launch_gemm_bt(g, a0, a1, bm, 1, cs));
+}
+
+mtla_status mtla_train_merge_bwd(const mtla_dims* dims, int32_t B, int32_t T, const void* c, const float* W_c,
+                                 const float* b_c, const float* P, int32_t J_max, const float* dC, float* dc,
+                                 float* dW_c, float* db_c, float* dP, void* workspace, size_t workspace_bytes,
+                                 int32_t* dev_err, void* stream) {
+  mtla_status st = check_dims(dims);
+  if (st != MTLA_OK) return st;
+  if (!train_dims(dims)) return MTLA_ERR_UNSUPPORTED;
+  if (B < 0 || T < 0 || J_max < 0) return MTLA_ERR_INVALID_ARG;
+  const void* ptrs[] = {c, W_c, b_c, P, dC, dc, dW_c, db_c, dP};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return MTLA_ERR_INVALID_ARG;
+  if (!dev_err) return MTLA_ERR_INVALID_ARG;
+  if (B == 0 || T == 0) return MTLA_OK;
+  const int r = dims->r, D = dims->r + dims->d_R;
+  if ((int64_t)J_max < (T + (int64_t)dims->s - 1) / dims->s) return MTLA_ERR_INVALID_ARG;
+  if ((int64_t)B * T * r >= (int64_t(1) << 31) || (int64_t)J_max * D >= (int64_t(1) << 31))
+    return MTLA_ERR_UNSUPPORTED;
+  const MergeBwdLayout L = merge_bwd_layout(dims, B, T);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < L.total) return MTLA_ERR_WORKSPACE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  __nv_bfloat16* wcT = reinterpret_cast<__nv_bfloat16*>(ws + L.wcT);  // [k][i] = W_c[i][k], k < r
+  __nv_bfloat16* wc = reinterpret_cast<__nv_bfloat16*>(ws + L.wc);    // [i][k] = W_c[i][k], k < r
+  float* G = reinterpret_cast<float*>(ws + L.G);
+  __nv_bfloat16* dg = reinterpret_cast<__nv_bfloat16*>(ws + L.dg);
+  __nv_bfloat16* cT = reinterpret_cast<__nv_bfloat16*>(ws + L.cT);
+  __nv_bfloat16* dgT = reinterpret_cast<__nv_bfloat16*>(ws + L.dgT);
+  float* dbp = reinterpret_cast<float*>(ws + L.dbp);
+  float* dwp = reinterpret_cast<float*>(ws + L.dwp);
+  const __nv_bfloat16* cb = static_cast<const __nv_bfloat16*>(c);
+  cudaError_t e;
+  if ((e = launch_transpose_f32_bf16(W_c, r, r, D, wcT, r, cs)) != cudaSuccess) return MTLA_ERR_CUDA;
+  if ((e = launch_convert_bf16(W_c, r, r, D, wc, r, cs)) != cudaSuccess) return MTLA_ERR_CUDA;
+  CUtensorMap mc, mwcT, mwc, mdg, mcT, mdgT;
+  if (!encode_operand_map(&mc, cb, L.BT, r, r) || !encode_operand_map(&mwcT, wcT, r, r, r) ||
+      !encode_operand_map(&mwc, wc, r, r, r) || !encode_operand_map(&mdg, dg, L.BT, r, r) ||
+      !encode_operand_map(&mcT, cT, r, L.BTp, L.BTp) || !encode_operand_map(&mdgT, dgT, r, L.BTp, L.BTp))
+    return MTLA_ERR_CUDA;
+  GemmBtArgs g;
+  g.N = r;
+  g.dev_err = dev_err;
+  g.split_stride = 0;
+  // G = c W_c[:, :r]: the gate pre-activations without the bias
+  g.M = L.BT;
+  g.K = r;
+  g.ka_split = r;
+  g.kb_per_split = r / 64;
+  g.C = G;
+  g.ldc = r;
+  g.accumulate = 0;
+  if ((e = launch_gemm_bt(g, mc, mc, mwcT, 1, cs)) != cudaSuccess) return MTLA_ERR_CUDA;
+  MergeBwdArgs m;
+  m.c = cb;
+  m.G = G;
+  m.b_c = b_c;
+  m.P = P;
+  m.dC = dC;
+  m.dc = dc;
+  m.dg = dg;
+  m.dP = dP;
+  m.db_part = dbp;
+  m.B = B;
+  m.T = T;
+  m.r = r;
+  m.D = D;
+  m.s = dims->s;
+  m.J_max = J_max;
+  if ((e = launch_merge_bwd(m, cs)) != cudaSuccess) return MTLA_ERR_CUDA;
+  // dc += dg W_c[:, :r]^T
+  g.C = dc;
+  g.accumulate = 1;
+  if ((e = launch_gemm_bt(g, mdg, mdg, mwc, 1, cs)) != cudaSuccess) return MTLA_ERR_CUDA;
+  // dW_c[:, :r] = c^T dg, split over the tokens, then the slices summed
+  if ((e = launch_transpose_bf16(cb, L.BT, r, r, cT, L.BTp, cs)) != cudaSuccess) return MTLA_ERR_CUDA;
+  if ((e = launch_transpose_bf16(dg, L.BT, r, r, dgT, L.BTp, cs)) != cudaSuccess) return MTLA_ERR_CUDA;
+  g.M = r;
+  g.K = (int)L.BTp;
+  g.ka_split = (int)L.BTp;
+  g.kb_per_split = L.kb_per;
+  g.C = dwp;
+  g.ldc = r;
+  g.split_stride = (int64_t)r * r;
+  g.accumulate = 0;
+  if ((e = launch_gemm_bt(g, mcT, mcT, mdgT, L.splits, cs)) != cudaSuccess) return MTLA_ERR_CUDA;
+  if ((e = launch_sum_slices(dwp, r, r, D, L.splits, (int64_t)r * r, dW_c, cs)) != cudaSuccess) return MTLA_ERR_CUDA;
+  return from_cuda(launch_db_reduce(dbp, L.J, r, D, db_c, cs));
 }
 
 }  // extern "C"

@@ -188,11 +188,78 @@ struct UnabsArgs {
   const __nv_bfloat16* qr;  // [B, T, H, d_R]
   const __nv_bfloat16* k;   // [B, T, H, d_h]
   const __nv_bfloat16* v;   // [B, T, H, d_h]
-  const __nv_bfloat16* cp;  // [B, T, D] C_hat' (its last d_R channels are the keys' RoPE part)
+  const __nv_bfloat16* kr;  // RoPE part of the keys: row n at kr + n * kr_stride (d_R wide); the last d_R
+                            // channels of C_hat' (stride D), or the uncompressed K^R of the training
+                            // shortcut (stride d_R)
+  int64_t kr_stride;
   __nv_bfloat16* out;       // [B, T, H, d_h]
-  int B, T, H, s, D;
+  float* lse;               // nullable [B, T, H]: natural log of each softmax denominator
+  int B, T, H, s;
   float scale_log2;
 };
 cudaError_t launch_prefill_unabs(const UnabsArgs& a, cudaStream_t st);
+
+// Backward of the masked attention with explicit keys and values and the
+// uncompressed RoPE keys (training shortcut): bf16, d_h = 64, d_R = 32.
+struct BwdArgs {
+  const __nv_bfloat16 *q, *qr, *k, *v, *kr;  // [B,T,H,64], [B,T,H,32], [B,T,H,64] x 2, [B,T,32]
+  const __nv_bfloat16 *o, *dout;             // [B,T,H,64]
+  const float* lse;                          // [B,T,H] natural log
+  __nv_bfloat16 *dq, *dqr, *dk, *dv;         // like q, qr, k, v
+  float* dkr;                                // [B,T,32], summed over heads
+  float* ws_lse2;                            // [B,H,T] lse in log2 units of the scaled score
+  float* ws_delta;                           // [B,H,T] rowsum(dO * O)
+  float* ws_dkrh;                            // [B,T,H,32] per-head RoPE key gradients
+  int B, T, H, s;
+  float scale, scale_log2;
+};
+cudaError_t launch_attn_bwd(const BwdArgs& a, cudaStream_t st);
+
+// C[M, N] (fp32) = A[M, K] B[N, K]^T, A and B bf16 K-major through TMA
+// (boxes of 64 x 128, 128-byte swizzle); A from amap0 for k < ka_split, from
+// amap1 beyond; N a multiple of 256.  grid.z > 1 splits K into slices of
+// kb_per_split blocks, slice z written to C + z * split_stride.
+struct GemmBtArgs {
+  int64_t M;
+  int N, K, ka_split, kb_per_split;
+  float* C;
+  int64_t ldc, split_stride;
+  int accumulate;  // C += A B^T (one slice only)
+  int32_t* dev_err;
+};
+cudaError_t launch_gemm_bt(const GemmBtArgs& a, const CUtensorMap& amap0, const CUtensorMap& amap1,
+                           const CUtensorMap& bmap, int splits, cudaStream_t st);
+size_t gemm_bt_smem_bytes();
+
+// out[r * ld_out + c] = sum over the n slices z of src[z * stride + r * cols + c]
+// (c < cols; columns cols .. ld_out - 1 written as zeros)
+cudaError_t launch_sum_slices(const float* src, int64_t rows, int cols, int64_t ld_out, int n, int64_t stride,
+                              float* out, cudaStream_t st);
+
+// out[c][r] = bf16(in[r][c]) for a [rows, cols] matrix with row stride ld_in;
+// out has row stride ld_out >= rows, columns rows .. ld_out - 1 zero-filled.
+cudaError_t launch_transpose_bf16(const __nv_bfloat16* in, int64_t rows, int cols, int64_t ld_in,
+                                  __nv_bfloat16* out, int64_t ld_out, cudaStream_t st);
+cudaError_t launch_transpose_f32_bf16(const float* in, int64_t rows, int cols, int64_t ld_in,
+                                      __nv_bfloat16* out, int64_t ld_out, cudaStream_t st);
+// out[r][c] = bf16(in[r][c]), r < rows, c < cols (row strides ld_in, ld_out)
+cudaError_t launch_convert_bf16(const float* in, int64_t rows, int cols, int64_t ld_in, __nv_bfloat16* out,
+                                int64_t ld_out, cudaStream_t st);
+
+// The gate part of the merge backward (latent channels, training shortcut).
+struct MergeBwdArgs {
+  const __nv_bfloat16* c;  // [B, T, r]
+  const float* G;          // [B, T, r] c W_c[:, :r] (bias not included)
+  const float *b_c, *P;    // [D], [J_max, D]
+  const float* dC;         // [B, T, r]
+  float* dc;               // [B, T, r] out: the direct term de * w
+  __nv_bfloat16* dg;       // [B, T, r] out: gate pre-activation gradient (bf16, for the GEMMs)
+  float* dP;               // [J_max, D] out (all rows and channels written)
+  float* db_part;          // [ceil(T/s), r] per-group partial sums of dg
+  int B, T, r, D, s, J_max;
+};
+cudaError_t launch_merge_bwd(const MergeBwdArgs& a, cudaStream_t st);
+// db[k] = sum_j part[j][k] for k < r, zero for r <= k < D
+cudaError_t launch_db_reduce(const float* part, int J, int r, int D, float* db, cudaStream_t st);
 
 }  // namespace mtla

@@ -5,7 +5,8 @@
 // and "decoupled RoPE with temporal compression"): for query m (1-based) of
 // sequence b and head h, with q_h = x W_Q^h, K_h = C_hat'_latent W_K^h,
 // V_h = C_hat'_latent W_V^h and the merged RoPE keys k_hat^R' (the last d_R
-// channels of C_hat'),
+// channels of C_hat'; the training shortcut of "decoupled RoPE with temporal
+// compression" passes the uncompressed K^R instead),
 //   score_n = (q_h . K_h,n + q^R_h . k_hat^R'_n) / sqrt(d_h),
 //   o_h = sum_{n visible} softmax(score)_n V_h,n
 // over the columns n == m and n = g s (g < ceil(m/s)).  Equal to the absorbed
@@ -19,7 +20,8 @@
 // shared memory with cp.async, double-buffered.  The own column n = m is
 // taken first, from a shared-memory copy of the CTA's own rows, and seeds the
 // online softmax.  Tiles past the staircase are never visited; columns past a
-// row's last visible group are masked.  CTAs run heaviest first.
+// row's last visible group are masked.  CTAs run heaviest first.  The log of
+// each softmax denominator is written on request, for the backward pass.
 #include "kernels.cuh"
 
 namespace mtla {
@@ -52,7 +54,7 @@ __global__ void __launch_bounds__(NT) prefill_unabs_kernel(const UnabsArgs p) {
   __nv_bfloat16* Vo = Ko + QB * KS;              // [QB][VS] own rows' values
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, q = lane & 3;
-  const int T = p.T, H = p.H, s = p.s, D = p.D;
+  const int T = p.T, H = p.H, s = p.s;
   const int nqb = (T + QB - 1) / QB;
   // heaviest first: the last query blocks of every (sequence, head) come first
   const int qb = nqb - 1 - (int)(blockIdx.x / (p.B * H));
@@ -74,11 +76,11 @@ __global__ void __launch_bounds__(NT) prefill_unabs_kernel(const UnabsArgs p) {
       const int r = i / 20, c = i % 20;
       const int grp = kt * KB + r;
       const bool valid = grp < n_groups;
-      const int64_t pos = row0 + (int64_t)(valid ? grp + 1 : 1) * s - 1;  // 0-based position of column n
+      const int64_t pos = row0 + (valid ? (int64_t)(grp + 1) * s - 1 : 0);  // column n; a row of the sequence even when not read
       if (c < 8) {
         cp_async16(kb + (uint32_t)(r * KS + c * 8) * 2, p.k + (pos * H + h) * DH + c * 8, valid);
       } else if (c < 12) {
-        cp_async16(kb + (uint32_t)(r * KS + DH + (c - 8) * 8) * 2, p.cp + pos * D + (D - DR) + (c - 8) * 8, valid);
+        cp_async16(kb + (uint32_t)(r * KS + DH + (c - 8) * 8) * 2, p.kr + pos * p.kr_stride + (c - 8) * 8, valid);
       } else {
         cp_async16(vb + (uint32_t)(r * VS + (c - 12) * 8) * 2, p.v + (pos * H + h) * DH + (c - 12) * 8, valid);
       }
@@ -93,7 +95,7 @@ __global__ void __launch_bounds__(NT) prefill_unabs_kernel(const UnabsArgs p) {
       const int64_t pos = row0 + (valid ? m0 - 1 + r : 0);
       if (c < 8) cp_async16(kb + (uint32_t)(r * KS + c * 8) * 2, p.k + (pos * H + h) * DH + c * 8, valid);
       else if (c < 12)
-        cp_async16(kb + (uint32_t)(r * KS + DH + (c - 8) * 8) * 2, p.cp + pos * D + (D - DR) + (c - 8) * 8, valid);
+        cp_async16(kb + (uint32_t)(r * KS + DH + (c - 8) * 8) * 2, p.kr + pos * p.kr_stride + (c - 8) * 8, valid);
       else cp_async16(vb + (uint32_t)(r * VS + (c - 12) * 8) * 2, p.v + (pos * H + h) * DH + (c - 12) * 8, valid);
     }
     cp_commit();
@@ -269,6 +271,11 @@ __global__ void __launch_bounds__(NT) prefill_unabs_kernel(const UnabsArgs p) {
   lB += __shfl_xor_sync(0xffffffffu, lB, 1);
   lB += __shfl_xor_sync(0xffffffffu, lB, 2);
   const float iA = 1.f / lA, iB = 1.f / lB;
+  if (p.lse && q == 0) {
+    // natural log of the denominator: the running max and sum are in log2 units of the scaled score
+    if (va) p.lse[(row0 + ma - 1) * H + h] = (mA + log2f(lA)) * 0.69314718055994531f;
+    if (vbq) p.lse[(row0 + mb - 1) * H + h] = (mB + log2f(lB)) * 0.69314718055994531f;
+  }
   __nv_bfloat16* oA = p.out + ((row0 + ma - 1) * H + h) * DH;
   __nv_bfloat16* oB = p.out + ((row0 + mb - 1) * H + h) * DH;
 #pragma unroll

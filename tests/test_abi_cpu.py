@@ -81,3 +81,28 @@ def test_binding_raises_on_error_status():
         mtla.mtla_merge_append(d, 1, {"c_new": p, "kR_new": p, "W_c": p, "b_c": p, "P": p, "J_max": 3},
                                p, 10, 288, p, p, p, p, p, stream=0)
     assert ei.value.status == 1
+
+
+def test_training_calls_check_arguments_on_the_host():
+    keep, p = _fake()
+    d = mtla.dims(8, 64, 256, 32, 2, "bf16")
+    other = mtla.dims(8, 32, 256, 32, 2, "bf16")  # d_h = 32: no training kernels
+    L = mtla.lib
+    ws = mtla.mtla_train_workspace_bytes(d, 2, 100, mtla.TRAIN_ATTN_BWD)
+    # two fp32 [B, H, T] arrays and the per-head RoPE key gradients
+    assert ws >= 2 * 2 * 8 * 100 * 4 + 2 * 100 * 8 * 32 * 4
+    assert mtla.mtla_train_workspace_bytes(d, 2, 100, mtla.TRAIN_KV_BWD) == 256 * 2 * 8 * 64 * 2
+    assert mtla.mtla_train_workspace_bytes(d, 2, 100, mtla.TRAIN_MERGE_BWD) > 2 * 100 * 256 * 4
+    assert mtla.mtla_train_workspace_bytes(other, 2, 100, mtla.TRAIN_ATTN_BWD) == 0
+    assert mtla.mtla_train_workspace_bytes(d, 2, 100, 9) == 0
+    bwd = lambda dims, B, T, wsb: L.mtla_train_attn_bwd(ctypes.byref(dims), B, T, *([p] * 13), p, wsb, p, None)
+    assert bwd(other, 2, 100, ws) == 2                      # unsupported dims
+    assert bwd(d, 2, 100, ws - 1) == 3                      # workspace too small
+    assert bwd(d, 0, 100, 0) == 0                           # empty batch: nothing to do
+    assert L.mtla_train_attn_bwd(ctypes.byref(d), 2, 100, *([p] * 12), None, p, ws, p, None) == 1  # null dkR
+    # merge backward: the P table must cover ceil(T / s) groups
+    wm = mtla.mtla_train_workspace_bytes(d, 2, 100, mtla.TRAIN_MERGE_BWD)
+    assert L.mtla_train_merge_bwd(ctypes.byref(d), 2, 100, p, p, p, p, 49, p, p, p, p, p, p, wm, p, None) == 1
+    assert L.mtla_train_merge_bwd(ctypes.byref(d), 2, 100, p, p, p, p, 50, p, p, p, p, p, p, wm - 1, p, None) == 3
+    assert L.mtla_train_kv_bwd(ctypes.byref(d), 2, 100, p, p, p, p, p, 100, p, None) == 3
+    assert L.mtla_train_attn_fwd(ctypes.byref(other), 2, 100, p, p, p, p, p, p, p, p, None) == 2
