@@ -441,6 +441,7 @@ def run_prefill(torch, mtla, glue, dev):
     if int(err.item()):
         raise RuntimeError(f"device error bits {int(err.item())} in the prefill")
     unabs = run_unabsorbed(torch, mtla, glue, dev, mc, W, qr, cp, md, err, flush, timed_call=time_calls)
+    train = run_train(torch, mtla, glue, dev, mc, W, qr, c, kR, cp, md, err, flush, P, W_c, b_c, J)
     ms_attn = ms - ms_merge
     # algorithmic work: every visible (query, head, column) pair, one score of
     # length D and one value row of length r, 2 flops per multiply-add
@@ -456,7 +457,66 @@ def run_prefill(torch, mtla, glue, dev):
                          "peak_kind": f"{kind} cuBLAS bf16 (burst)"},
             "note": "attention time = full call - cache-only call (the running merge alone); "
                     "L2 flushed before each call",
-            "unabsorbed": unabs}
+            "unabsorbed": unabs, "training": train}
+
+
+def run_train(torch, mtla, glue, dev, mc, W, qr, c, kR, cp, md, err, flush, P, W_c, b_c, J):
+    """One training step of the shortcut on the prefill workload (B=8, T=4096,
+    s=2): the forward on the uncompressed RoPE keys and the backward chain
+    attention -> key/value maps -> merge, each call timed alone."""
+    d = mc.dims
+    B, T = c.shape[0], c.shape[1]
+    q = glue.query_heads(torch.from_numpy(mc.x).to(dev), W).to(torch.bfloat16).contiguous()
+    W_kv = glue.kv_weights(W)
+    k = torch.empty(B, T, d.H, d.d_h, dtype=torch.bfloat16, device=dev)
+    v, out, dO, dq, dk, dv = (torch.empty_like(k) for _ in range(6))
+    dO.normal_(generator=torch.Generator(device=dev).manual_seed(5))
+    dqr = torch.empty_like(qr)
+    lse = torch.empty(B, T, d.H, device=dev)
+    dkR = torch.empty(B, T, d.d_R, device=dev)
+    dC = torch.empty(B, T, d.r, device=dev)
+    dc = torch.empty(B, T, d.r, device=dev)
+    dW = torch.empty(d.r, d.D, device=dev)
+    db = torch.empty(d.D, device=dev)
+    dP = torch.empty(J, d.D, device=dev)
+    mtla.mtla_prefill_kv(md, B, T, cp, W_kv, k, v, err)
+    wa, wk, wm = (mtla.mtla_train_workspace_bytes(md, B, T, w)
+                  for w in (mtla.TRAIN_ATTN_BWD, mtla.TRAIN_KV_BWD, mtla.TRAIN_MERGE_BWD))
+    ws = torch.empty(max(wa, wk, wm), dtype=torch.uint8, device=dev)
+    ms_fwd = time_calls(torch, lambda: mtla.mtla_train_attn_fwd(md, B, T, q, qr, k, v, kR, out, lse, err), 7, 3, flush)
+    ms_bwd = time_calls(torch, lambda: mtla.mtla_train_attn_bwd(md, B, T, q, qr, k, v, kR, out, lse, dO, dq, dqr, dk, dv,
+                                                               dkR, ws, wa, err), 7, 3, flush)
+    ms_kv = time_calls(torch, lambda: mtla.mtla_train_kv_bwd(md, B, T, dk, dv, W_kv, dC, ws, wk, err), 7, 3, flush)
+    ms_merge = time_calls(torch, lambda: mtla.mtla_train_merge_bwd(md, B, T, c, W_c, b_c, P, J, dC, dc, dW, db, dP, ws,
+                                                                   wm, err), 7, 3, flush)
+    if int(err.item()):
+        raise RuntimeError(f"device error bits {int(err.item())} in the training step")
+    hbm_peak, tflops_peak, _, kind = measured_peaks()
+    pairs = B * d.H * sum(math.ceil(m / d.s) for m in range(1, T + 1))
+    f_fwd = pairs * (2 * (d.d_h + d.d_R) + 2 * d.d_h)
+    # backward per visible pair: score recompute 2 (d_h + d_R), dP 2 d_h, dv 2 d_h, [dk | dk^R] and
+    # [dq | dq^R] 2 (d_h + d_R) each
+    f_bwd = pairs * (3 * 2 * (d.d_h + d.d_R) + 2 * 2 * d.d_h)
+    BT = B * T
+    kv_bytes = 2 * BT * d.H * d.d_h * 2 + BT * d.r * 4 + W_kv.numel() * 2
+    merge_bytes = BT * d.r * 2 + 2 * BT * d.r * 4  # c and dC read, dc written
+    tf = lambda f, ms: f / (ms / 1e3) / 1e12
+    gb = lambda by, ms: by / (ms / 1e3) / 1e9
+    return {"workload": "training step of the shortcut (uncompressed K^R), B=8, T=4096, H=8, d_h=64, r=256, "
+                        "d_R=32, s=2; d_out drawn N(0, 1)",
+            "ms_forward": ms_fwd, "ms_attn_backward": ms_bwd, "ms_kv_backward": ms_kv, "ms_merge_backward": ms_merge,
+            "ms_total": ms_fwd + ms_bwd + ms_kv + ms_merge,
+            "attn_forward": {"algorithmic_tflop": f_fwd / 1e12, "tflops": tf(f_fwd, ms_fwd),
+                             "frac": tf(f_fwd, ms_fwd) / tflops_peak},
+            "roofline": {"bound": "tensor", "achieved": tf(f_bwd, ms_bwd), "peak": tflops_peak, "unit": "TFLOP/s",
+                         "frac": tf(f_bwd, ms_bwd) / tflops_peak, "kernel": "mtla::bwt::dkv::bwd_dkv_tc_kernel + mtla::bwt::dq::bwd_dq_tc_kernel",
+                         "algorithmic_tflop": f_bwd / 1e12, "peak_kind": f"{kind} cuBLAS bf16 (burst)"},
+            "kv_backward": {"algorithmic_bytes": kv_bytes, "achieved_gbs": gb(kv_bytes, ms_kv),
+                            "frac_hbm": gb(kv_bytes, ms_kv) / hbm_peak},
+            "merge_backward": {"algorithmic_bytes": merge_bytes, "achieved_gbs": gb(merge_bytes, ms_merge),
+                               "frac_hbm": gb(merge_bytes, ms_merge) / hbm_peak},
+            "note": "each call alone, median of 7 after 3, L2 flushed before each; the backward's flops count "
+                    "each product once (the kernels recompute the scores in both the dq and dk/dv passes)"}
 
 
 def run_unabsorbed(torch, mtla, glue, dev, mc, W, qr, cp, md, err, flush, timed_call):
@@ -486,7 +546,7 @@ def run_unabsorbed(torch, mtla, glue, dev, mc, W, qr, cp, md, err, flush, timed_
                    "achieved_gbs": kv_bytes / (ms_kv / 1e3) / 1e9,
                    "frac_hbm": kv_bytes / (ms_kv / 1e3) / 1e9 / hbm_peak},
             "roofline": {"bound": "tensor", "achieved": at, "peak": tflops_peak, "unit": "TFLOP/s",
-                         "frac": at / tflops_peak, "kernel": "mtla::pua::prefill_unabs_kernel",
+                         "frac": at / tflops_peak, "kernel": "mtla::utc::prefill_unabs_tc_kernel",
                          "peak_kind": f"{kind} cuBLAS bf16 (burst)"},
             "note": "320 flop per visible (query, head, column): 2 (d_h + d_R) for the score, 2 d_h for the "
                     "value; median of 7 calls, L2 flushed before each"}

@@ -512,6 +512,82 @@ static bool unabs_dims(const mtla_dims* d) {
   return d->dtype == MTLA_BF16 && d->d_h == 64 && d->d_R == 32 && d->r % 64 == 0 && d->r <= 256 && d->H % 2 == 0;
 }
 
+// Tensor maps of the un-absorbed attention's bf16 operands, 64-byte swizzle,
+// boxes 32 elements wide: a 64-wide row lands as two [rows x 64 B] planes.
+// Rows of a [B T, H, 64] tensor for one head: 4-D {32, H, B T, 2 planes}.
+static bool map_head_rows(CUtensorMap* m, const void* base, int H, int64_t BT, uint32_t rows) {
+  const cuuint64_t d[4] = {32, (cuuint64_t)H, (cuuint64_t)BT, 2}, st[3] = {128, (cuuint64_t)H * 128, 64};
+  const cuuint32_t box[4] = {32, 1, rows, 2};
+  return encode_bf16_map(m, base, 4, d, st, box);
+}
+// Rows of a [B T, H, 32] tensor (q^R) for one head: 3-D {32, H, B T}.
+static bool map_head_rope(CUtensorMap* m, const void* base, int H, int64_t BT, uint32_t rows) {
+  const cuuint64_t d[3] = {32, (cuuint64_t)H, (cuuint64_t)BT}, st[2] = {64, (cuuint64_t)H * 64};
+  const cuuint32_t box[3] = {32, 1, rows};
+  return encode_bf16_map(m, base, 3, d, st, box);
+}
+// Rows of the RoPE keys (row n at kr + n kr_stride): 2-D {32, B T}.
+static bool map_key_rope(CUtensorMap* m, const void* kr, int64_t kr_stride, int64_t BT, uint32_t rows) {
+  const cuuint64_t d[2] = {32, (cuuint64_t)BT}, st[1] = {(cuuint64_t)kr_stride * 2};
+  const cuuint32_t box[2] = {32, rows};
+  return encode_bf16_map(m, kr, 2, d, st, box);
+}
+// The group columns n = g s (0-based rows s - 1, 2 s - 1, ...) of each
+// sequence; G = T / s of them (a sequence with none still gets a valid map,
+// never read).  [B T, H, 64] tensors: 5-D {32, H, G, B, 2 planes}.
+static bool map_group_rows(CUtensorMap* m, const void* base, int H, int s, int T, int B, uint32_t groups) {
+  const int64_t G = T / s, Gm = G > 0 ? G : 1, off = G > 0 ? s - 1 : 0;
+  const cuuint64_t d[5] = {32, (cuuint64_t)H, (cuuint64_t)Gm, (cuuint64_t)B, 2};
+  const cuuint64_t st[4] = {128, (cuuint64_t)s * H * 128, (cuuint64_t)T * H * 128, 64};
+  const cuuint32_t box[5] = {32, 1, groups, 1, 2};
+  return encode_bf16_map(m, static_cast<const __nv_bfloat16*>(base) + off * H * 64, 5, d, st, box);
+}
+// [B T, H, 32] tensors (q^R) at the group columns: 4-D {32, H, G, B}.
+static bool map_group_rope(CUtensorMap* m, const void* base, int H, int s, int T, int B, uint32_t groups) {
+  const int64_t G = T / s, Gm = G > 0 ? G : 1, off = G > 0 ? s - 1 : 0;
+  const cuuint64_t d[4] = {32, (cuuint64_t)H, (cuuint64_t)Gm, (cuuint64_t)B};
+  const cuuint64_t st[3] = {64, (cuuint64_t)s * H * 64, (cuuint64_t)T * H * 64};
+  const cuuint32_t box[4] = {32, 1, groups, 1};
+  return encode_bf16_map(m, static_cast<const __nv_bfloat16*>(base) + off * H * 32, 4, d, st, box);
+}
+// The RoPE keys at the group columns: 3-D {32, G, B}.
+static bool map_group_key_rope(CUtensorMap* m, const void* kr, int64_t kr_stride, int s, int T, int B,
+                               uint32_t groups) {
+  const int64_t G = T / s, Gm = G > 0 ? G : 1, off = G > 0 ? s - 1 : 0;
+  const cuuint64_t d[3] = {32, (cuuint64_t)Gm, (cuuint64_t)B};
+  const cuuint64_t st[2] = {(cuuint64_t)s * kr_stride * 2, (cuuint64_t)T * kr_stride * 2};
+  const cuuint32_t box[3] = {32, groups, 1};
+  return encode_bf16_map(m, static_cast<const __nv_bfloat16*>(kr) + off * kr_stride, 3, d, st, box);
+}
+
+// The un-absorbed attention on the tensor cores: the tensor maps of q, q^R,
+// k, v and the RoPE keys (row n at kr + n kr_stride), then a persistent grid.
+static mtla_status launch_unabs_attn(const mtla_dims* dims, int32_t B, int32_t T, const void* q, const void* q_rope,
+                                     const void* k, const void* v, const void* kr, int64_t kr_stride, void* out,
+                                     float* lse, int32_t* dev_err, void* stream) {
+  const int H = dims->H, s = dims->s;
+  const int64_t BT = (int64_t)B * T;
+  UnabsTcLaunch a;
+  if (!map_head_rows(&a.q, q, H, BT, 128) || !map_head_rows(&a.k_own, k, H, BT, 128) ||
+      !map_head_rows(&a.v_own, v, H, BT, 128) || !map_head_rope(&a.qr, q_rope, H, BT, 128) ||
+      !map_key_rope(&a.kr_own, kr, kr_stride, BT, 128) || !map_group_rows(&a.k_grp, k, H, s, T, B, 64) ||
+      !map_group_rows(&a.v_grp, v, H, s, T, B, 64) || !map_group_key_rope(&a.kr_grp, kr, kr_stride, s, T, B, 64))
+    return MTLA_ERR_CUDA;
+  a.B = B;
+  a.T = T;
+  a.H = H;
+  a.s = s;
+  a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->d_h));
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.lse = lse;
+  a.dev_err = dev_err;
+  const int64_t tiles = (int64_t)B * H * ((T + 127) / 128);
+  const int sms = device_sms();
+  if (sms <= 0) return MTLA_ERR_CUDA;
+  const int grid = (int)(tiles < sms ? tiles : sms);
+  return from_cuda(launch_prefill_unabs_tc(a, grid, static_cast<cudaStream_t>(stream)));
+}
+
 mtla_status mtla_prefill_kv(const mtla_dims* dims, int32_t B, int32_t T, const void* c_partial, const void* W_kv,
                             void* k, void* v, int32_t* dev_err, void* stream) {
   mtla_status st = check_dims(dims);
@@ -556,21 +632,8 @@ mtla_status mtla_prefill_unabsorbed_attn(const mtla_dims* dims, int32_t B, int32
   if (!dev_err) return MTLA_ERR_INVALID_ARG;
   if (B == 0 || T == 0) return MTLA_OK;
   if ((int64_t)B * T * dims->H >= (int64_t(1) << 31)) return MTLA_ERR_UNSUPPORTED;
-  UnabsArgs a;
-  a.q = static_cast<const __nv_bfloat16*>(q);
-  a.qr = static_cast<const __nv_bfloat16*>(q_rope);
-  a.k = static_cast<const __nv_bfloat16*>(k);
-  a.v = static_cast<const __nv_bfloat16*>(v);
-  a.kr = static_cast<const __nv_bfloat16*>(c_partial) + dims->r;
-  a.kr_stride = dims->r + dims->d_R;
-  a.out = static_cast<__nv_bfloat16*>(out);
-  a.lse = nullptr;
-  a.B = B;
-  a.T = T;
-  a.H = dims->H;
-  a.s = dims->s;
-  a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->d_h));
-  return from_cuda(launch_prefill_unabs(a, static_cast<cudaStream_t>(stream)));
+  return launch_unabs_attn(dims, B, T, q, q_rope, k, v, static_cast<const __nv_bfloat16*>(c_partial) + dims->r,
+                           dims->r + dims->d_R, out, nullptr, dev_err, stream);
 }
 
 size_t mtla_project_workspace_bytes(const mtla_dims* dims, int32_t B, int32_t d, int32_t which) {
@@ -735,12 +798,14 @@ static MergeBwdLayout merge_bwd_layout(const mtla_dims* d, int32_t B, int32_t T)
   return L;
 }
 
+// lse2 and Delta [B, H, Tp] (Tp = T rounded up to 64), then the per-head RoPE
+// key gradients [B, T, H, d_R]
 static size_t attn_bwd_bytes(const mtla_dims* d, int32_t B, int32_t T, size_t* off_delta, size_t* off_dkrh) {
-  const size_t n = (size_t)B * T * d->H;
-  const size_t a = up256(n * 4);
+  const size_t Tp = ((size_t)T + 63) / 64 * 64;
+  const size_t a = up256((size_t)B * d->H * Tp * 4);
   if (off_delta) *off_delta = a;
   if (off_dkrh) *off_dkrh = 2 * a;
-  return 2 * a + up256(n * 32 * 4);
+  return 2 * a + up256((size_t)B * T * d->H * 32 * 4);
 }
 
 size_t mtla_train_workspace_bytes(const mtla_dims* dims, int32_t B, int32_t T, int32_t which) {
@@ -764,21 +829,7 @@ mtla_status mtla_train_attn_fwd(const mtla_dims* dims, int32_t B, int32_t T, con
   if (!dev_err) return MTLA_ERR_INVALID_ARG;
   if (B == 0 || T == 0) return MTLA_OK;
   if ((int64_t)B * T * dims->H >= (int64_t(1) << 31)) return MTLA_ERR_UNSUPPORTED;
-  UnabsArgs a;
-  a.q = static_cast<const __nv_bfloat16*>(q);
-  a.qr = static_cast<const __nv_bfloat16*>(q_rope);
-  a.k = static_cast<const __nv_bfloat16*>(k);
-  a.v = static_cast<const __nv_bfloat16*>(v);
-  a.kr = static_cast<const __nv_bfloat16*>(kR);
-  a.kr_stride = dims->d_R;
-  a.out = static_cast<__nv_bfloat16*>(out);
-  a.lse = lse;
-  a.B = B;
-  a.T = T;
-  a.H = dims->H;
-  a.s = dims->s;
-  a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->d_h));
-  return from_cuda(launch_prefill_unabs(a, static_cast<cudaStream_t>(stream)));
+  return launch_unabs_attn(dims, B, T, q, q_rope, k, v, kR, dims->d_R, out, lse, dev_err, stream);
 }
 
 mtla_status mtla_train_attn_bwd(const mtla_dims* dims, int32_t B, int32_t T, const void* q, const void* q_rope,
@@ -820,9 +871,50 @@ mtla_status mtla_train_attn_bwd(const mtla_dims* dims, int32_t B, int32_t T, con
   a.T = T;
   a.H = dims->H;
   a.s = dims->s;
+  a.Tp = (T + 63) / 64 * 64;
   a.scale = (float)(1.0 / sqrt((double)dims->d_h));
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->d_h));
-  return from_cuda(launch_attn_bwd(a, static_cast<cudaStream_t>(stream)));
+  const int H = dims->H, s = dims->s;
+  const int64_t BT = (int64_t)B * T;
+  TrainBwdMaps mq;
+  TrainBwdKvMaps mk;
+  if (!map_head_rows(&mq.q128, q, H, BT, 128) || !map_head_rope(&mq.qr128, q_rope, H, BT, 128) ||
+      !map_head_rows(&mq.do128, d_out, H, BT, 128) || !map_head_rows(&mq.k128, k, H, BT, 128) ||
+      !map_key_rope(&mq.kr128, kR, dims->d_R, BT, 128) || !map_head_rows(&mq.v128, v, H, BT, 128) ||
+      !map_group_rows(&mq.k_g64, k, H, s, T, B, 64) || !map_group_key_rope(&mq.kr_g64, kR, dims->d_R, s, T, B, 64) ||
+      !map_group_rows(&mq.v_g64, v, H, s, T, B, 64))
+    return MTLA_ERR_CUDA;
+  if (!map_group_rows(&mk.k_g, k, H, s, T, B, 128) || !map_group_key_rope(&mk.kr_g, kR, dims->d_R, s, T, B, 128) ||
+      !map_group_rows(&mk.v_g, v, H, s, T, B, 128) || !map_group_rows(&mk.q_g, q, H, s, T, B, 128) ||
+      !map_group_rope(&mk.qr_g, q_rope, H, s, T, B, 128) || !map_group_rows(&mk.do_g, d_out, H, s, T, B, 128) ||
+      !map_head_rows(&mk.q64, q, H, BT, 64) || !map_head_rope(&mk.qr64, q_rope, H, BT, 64) ||
+      !map_head_rows(&mk.do64, d_out, H, BT, 64))
+    return MTLA_ERR_CUDA;
+  TrainBwdTc t;
+  t.B = B;
+  t.T = T;
+  t.H = H;
+  t.s = s;
+  t.Tp = a.Tp;
+  t.scale = a.scale;
+  t.scale_log2 = a.scale_log2;
+  t.lse2 = a.ws_lse2;
+  t.delta = a.ws_delta;
+  t.dq = a.dq;
+  t.dqr = a.dqr;
+  t.dk = a.dk;
+  t.dv = a.dv;
+  t.dkrh = a.ws_dkrh;
+  t.dev_err = dev_err;
+  const int sms = device_sms();
+  if (sms <= 0) return MTLA_ERR_CUDA;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (launch_bwd_prep(a, cs) != cudaSuccess) return MTLA_ERR_CUDA;
+  const int64_t q_tiles = (int64_t)B * H * ((T + 127) / 128);
+  if (launch_bwd_dq_tc(mq, t, (int)(q_tiles < sms ? q_tiles : sms), cs) != cudaSuccess) return MTLA_ERR_CUDA;
+  const int64_t items = (int64_t)B * H * ((T / s + 127) / 128);
+  if (items > 0 && launch_bwd_dkv_tc(mk, t, (int)(items < sms ? items : sms), cs) != cudaSuccess) return MTLA_ERR_CUDA;
+  return from_cuda(launch_dkr_reduce(a, cs));
 }
 
 // 2-D map of a row-major bf16 matrix [rows, cols] (row stride ld elements) in

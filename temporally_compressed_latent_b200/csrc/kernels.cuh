@@ -181,23 +181,25 @@ struct RowsGemmArgs {
 cudaError_t launch_rows_gemm(const RowsGemmArgs& a, const CUtensorMap& amap, const CUtensorMap& bmap,
                              cudaStream_t st);
 
-// Masked prefill with explicit per-head keys and values (prefill_unabs.cu):
-// bf16, d_h = 64, d_R = 32.
-struct UnabsArgs {
-  const __nv_bfloat16* q;   // [B, T, H, d_h]
-  const __nv_bfloat16* qr;  // [B, T, H, d_R]
-  const __nv_bfloat16* k;   // [B, T, H, d_h]
-  const __nv_bfloat16* v;   // [B, T, H, d_h]
-  const __nv_bfloat16* kr;  // RoPE part of the keys: row n at kr + n * kr_stride (d_R wide); the last d_R
-                            // channels of C_hat' (stride D), or the uncompressed K^R of the training
-                            // shortcut (stride d_R)
-  int64_t kr_stride;
-  __nv_bfloat16* out;       // [B, T, H, d_h]
-  float* lse;               // nullable [B, T, H]: natural log of each softmax denominator
+// Masked attention with explicit per-head keys and values (the un-absorbed
+// prefill, and the training shortcut's forward) on the tensor cores (tcgen05
+// + TMEM): tensor maps of the inputs (bf16, 64-byte swizzle, 32-element
+// boxes) and the sizes.  The RoPE keys are the last d_R channels of C_hat'
+// (row stride D) or the uncompressed K^R (row stride d_R).
+struct UnabsTcLaunch {
+  CUtensorMap q, qr;          // q: 4-D {32, H, B T, 2 planes}, box {32, 1, 128, 2}; q^R: 3-D {32, H, B T}, box {32, 1, 128}
+  CUtensorMap k_own, v_own;   // like q, on k and v
+  CUtensorMap kr_own;         // 2-D {32, B T}, box {32, 128}
+  CUtensorMap k_grp, v_grp;   // 5-D {32, H, T / s groups, B, 2 planes} from row s - 1, box {32, 1, 64, 1, 2}
+  CUtensorMap kr_grp;         // 3-D {32, T / s groups, B} from row s - 1, box {32, 64, 1}
   int B, T, H, s;
   float scale_log2;
+  __nv_bfloat16* out;
+  float* lse;
+  int32_t* dev_err;
 };
-cudaError_t launch_prefill_unabs(const UnabsArgs& a, cudaStream_t st);
+size_t prefill_unabs_tc_smem();
+cudaError_t launch_prefill_unabs_tc(const UnabsTcLaunch& a, int grid, cudaStream_t st);
 
 // Backward of the masked attention with explicit keys and values and the
 // uncompressed RoPE keys (training shortcut): bf16, d_h = 64, d_R = 32.
@@ -207,13 +209,42 @@ struct BwdArgs {
   const float* lse;                          // [B,T,H] natural log
   __nv_bfloat16 *dq, *dqr, *dk, *dv;         // like q, qr, k, v
   float* dkr;                                // [B,T,32], summed over heads
-  float* ws_lse2;                            // [B,H,T] lse in log2 units of the scaled score
-  float* ws_delta;                           // [B,H,T] rowsum(dO * O)
+  float* ws_lse2;                            // [B,H,Tp] lse in log2 units of the scaled score
+  float* ws_delta;                           // [B,H,Tp] rowsum(dO * O)
   float* ws_dkrh;                            // [B,T,H,32] per-head RoPE key gradients
-  int B, T, H, s;
+  int B, T, H, s, Tp;                        // Tp: T rounded up to 64
   float scale, scale_log2;
 };
-cudaError_t launch_attn_bwd(const BwdArgs& a, cudaStream_t st);
+// Delta and lse2 per (sequence, head, query), then (after the gradient
+// kernels) dk^R summed over heads.
+cudaError_t launch_bwd_prep(const BwdArgs& a, cudaStream_t st);
+cudaError_t launch_dkr_reduce(const BwdArgs& a, cudaStream_t st);
+
+// The gradient kernels on the tensor cores (train_bwd_tc.cu).
+struct TrainBwdTc {
+  int B, T, H, s, Tp;
+  float scale, scale_log2;
+  const float *lse2, *delta;           // [B, H, Tp]
+  __nv_bfloat16 *dq, *dqr, *dk, *dv;   // [B, T, H, 64] (dqr: 32)
+  float* dkrh;                         // [B, T, H, 32]
+  int32_t* dev_err;
+};
+// dq kernel: 128-query tiles and 64-column key tiles (bf16, 64-byte swizzle)
+struct TrainBwdMaps {
+  CUtensorMap q128, qr128, do128;   // q, dO: 4-D {32, H, B T, 2 planes} box {32, 1, 128, 2}; q^R 3-D box {32, 1, 128}
+  CUtensorMap k128, kr128, v128;    // the tile's own rows: k, v like q; k^R 2-D {32, B T} box {32, 128}
+  CUtensorMap k_g64, kr_g64, v_g64; // group columns: k, v 5-D {32, H, T / s, B, 2} box {32, 1, 64, 1, 2}; k^R 3-D
+};
+// dk / dv kernel: 128 group columns per item and 64-query tiles
+struct TrainBwdKvMaps {
+  CUtensorMap k_g, kr_g, v_g;       // group columns, boxes of 128
+  CUtensorMap q_g, qr_g, do_g;      // the query rows at the group columns' positions (q^R: 4-D {32, H, T / s, B})
+  CUtensorMap q64, qr64, do64;      // query tiles, boxes of 64 rows
+};
+size_t bwd_dq_tc_smem();
+size_t bwd_dkv_tc_smem();
+cudaError_t launch_bwd_dq_tc(const TrainBwdMaps& mp, const TrainBwdTc& p, int grid, cudaStream_t st);
+cudaError_t launch_bwd_dkv_tc(const TrainBwdKvMaps& mp, const TrainBwdTc& p, int grid, cudaStream_t st);
 
 // C[M, N] (fp32) = A[M, K] B[N, K]^T, A and B bf16 K-major through TMA
 // (boxes of 64 x 128, 128-byte swizzle); A from amap0 for k < ka_split, from
