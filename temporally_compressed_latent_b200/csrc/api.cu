@@ -770,7 +770,7 @@ static size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 struct MergeBwdLayout {
   int64_t BT, BTp;
   int J, splits, kb_per;
-  size_t wcT, wc, G, dg, cT, dgT, dbp, dwp, total;
+  size_t wcT, wc, G, dg, cT, dgT, dbp, dbs, dwp, total;
 };
 
 static MergeBwdLayout merge_bwd_layout(const mtla_dims* d, int32_t B, int32_t T) {
@@ -793,6 +793,7 @@ static MergeBwdLayout merge_bwd_layout(const mtla_dims* d, int32_t B, int32_t T)
   L.cT = o;  o = up256(o + (size_t)r * L.BTp * 2);
   L.dgT = o; o = up256(o + (size_t)r * L.BTp * 2);
   L.dbp = o; o = up256(o + (size_t)L.J * r * 4);
+  L.dbs = o; o = up256(o + (size_t)DB_SLICE_COUNT * r * 4);
   L.dwp = o; o = up256(o + (size_t)L.splits * r * r * 4);
   L.total = o;
   return L;
@@ -1048,7 +1049,7 @@ mtla_status mtla_train_merge_bwd(const mtla_dims* dims, int32_t B, int32_t T, co
   g.accumulate = 0;
   if ((e = launch_gemm_bt(g, mcT, mcT, mdgT, L.splits, cs)) != cudaSuccess) return MTLA_ERR_CUDA;
   if ((e = launch_sum_slices(dwp, r, r, D, L.splits, (int64_t)r * r, dW_c, cs)) != cudaSuccess) return MTLA_ERR_CUDA;
-  return from_cuda(launch_db_reduce(dbp, L.J, r, D, db_c, cs));
+  return from_cuda(launch_db_reduce(dbp, L.J, r, D, reinterpret_cast<float*>(ws + L.dbs), db_c, cs));
 }
 
 }  // extern "C"

@@ -290,7 +290,9 @@ struct MergeBwdArgs {
   int B, T, r, D, s, J_max;
 };
 cudaError_t launch_merge_bwd(const MergeBwdArgs& a, cudaStream_t st);
-// db[k] = sum_j part[j][k] for k < r, zero for r <= k < D
-cudaError_t launch_db_reduce(const float* part, int J, int r, int D, float* db, cudaStream_t st);
+// db[k] = sum_j part[j][k] for k < r, zero for r <= k < D, through 64 partial
+// slices [64, r] in `slices` (fixed order)
+constexpr int DB_SLICE_COUNT = 64;
+cudaError_t launch_db_reduce(const float* part, int J, int r, int D, float* slices, float* db, cudaStream_t st);
 
 }  // namespace mtla

@@ -208,40 +208,58 @@ __global__ void __launch_bounds__(256) merge_bwd_kernel(const MergeBwdArgs p) {
   const float u = p.P[idx], bc = p.b_c[k];
   const int i0 = j * p.s, i1 = i0 + p.s < p.T ? i0 + p.s : p.T;  // 0-based tokens i0 .. i1 - 1
   float dP = 0.f, db = 0.f;
-  for (int b = 0; b < p.B; ++b) {
-    float de = 0.f;
+  // four sequences at a time: their loads are independent, so they are in
+  // flight together; dP and db are summed in a fixed order (blocks of four
+  // sequences, tokens last to first, sequences within a block)
+  for (int b0 = 0; b0 < p.B; b0 += 4) {
+    const int nb = p.B - b0 < 4 ? p.B - b0 : 4;
+    float de[4] = {0.f, 0.f, 0.f, 0.f};
     for (int i = i1 - 1; i >= i0; --i) {
-      const int64_t e = ((int64_t)b * p.T + i) * p.r + k;
-      de += p.dC[e];
-      const float g = p.G[e] + bc;
-      const float w = sigmoidf_(g * u);
-      const float cv = __bfloat162float(p.c[e]);
-      const float dz = de * cv * w * (1.f - w);
-      const float dg = dz * u;
-      dP += dz * g;
-      db += dg;
-      p.dc[e] = de * w;
-      p.dg[e] = __float2bfloat16_rn(dg);
+      float dCv[4], gv[4], cv[4];
+#pragma unroll
+      for (int u4 = 0; u4 < 4; ++u4) {
+        const int64_t e = ((int64_t)(b0 + (u4 < nb ? u4 : 0)) * p.T + i) * p.r + k;
+        dCv[u4] = p.dC[e];
+        gv[u4] = p.G[e];
+        cv[u4] = __bfloat162float(p.c[e]);
+      }
+#pragma unroll
+      for (int u4 = 0; u4 < 4; ++u4) {
+        if (u4 >= nb) break;
+        const int64_t e = ((int64_t)(b0 + u4) * p.T + i) * p.r + k;
+        de[u4] += dCv[u4];
+        const float g = gv[u4] + bc;
+        const float w = sigmoidf_(g * u);
+        const float dz = de[u4] * cv[u4] * w * (1.f - w);
+        const float dg = dz * u;
+        dP += dz * g;
+        db += dg;
+        p.dc[e] = de[u4] * w;
+        p.dg[e] = __float2bfloat16_rn(dg);
+      }
     }
   }
   p.dP[idx] = dP;
   p.db_part[(int64_t)j * p.r + k] = db;
 }
 
-// db[k] = sum_j part[j][k] in a fixed order: block = 32 channels x 8 lanes of j
-__global__ void __launch_bounds__(256) db_reduce_kernel(const float* part, int J, int r, int D, float* db) {
+// First pass of db[k] = sum_j part[j][k] in a fixed order: block (x, z) sums
+// channels 32 x .. 32 x + 31 over groups j = z, z + DB_SLICES, ... (8 lanes of
+// j, then the lanes in order) into out[z][k]; the slices are summed after.
+constexpr int DB_SLICES = 64;
+__global__ void __launch_bounds__(256) db_partial_kernel(const float* part, int J, int r, float* out) {
   __shared__ float red[8][33];
   const int kx = threadIdx.x & 31, jl = threadIdx.x >> 5;
-  const int k = blockIdx.x * 32 + kx;
+  const int k = blockIdx.x * 32 + kx, z = blockIdx.y;
   float acc = 0.f;
   if (k < r)
-    for (int j = jl; j < J; j += 8) acc += part[(int64_t)j * r + k];
+    for (int j = z + jl * DB_SLICES; j < J; j += 8 * DB_SLICES) acc += part[(int64_t)j * r + k];
   red[jl][kx] = acc;
   __syncthreads();
-  if (jl == 0 && k < D) {
+  if (jl == 0 && k < r) {
     float t = 0.f;
     for (int i = 0; i < 8; ++i) t += red[i][kx];
-    db[k] = k < r ? t : 0.f;
+    out[(int64_t)z * r + k] = t;
   }
 }
 
@@ -299,9 +317,11 @@ cudaError_t launch_merge_bwd(const MergeBwdArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_db_reduce(const float* part, int J, int r, int D, float* db, cudaStream_t st) {
-  tgm::db_reduce_kernel<<<(unsigned)((D + 31) / 32), 256, 0, st>>>(part, J, r, D, db);
-  return cudaGetLastError();
+cudaError_t launch_db_reduce(const float* part, int J, int r, int D, float* slices, float* db, cudaStream_t st) {
+  tgm::db_partial_kernel<<<dim3((unsigned)((r + 31) / 32), tgm::DB_SLICES), 256, 0, st>>>(part, J, r, slices);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_sum_slices(slices, 1, r, D, tgm::DB_SLICES, r, db, st);
 }
 
 }  // namespace mtla
