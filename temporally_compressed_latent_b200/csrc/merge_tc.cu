@@ -143,14 +143,28 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
   if (warp == TMA_WARP && lane == 0) prefetch_tmap(&cmap);
 
   // this CTA's half of W_c -> bf16 hi + lo, K-major with the 128-byte swizzle:
-  // output channel n, latents k = kb*64 + ch*8 .. +7 form one 16-byte chunk
-  for (int it = tid; it < KB * 8 * NH; it += NT) {
+  // output channel n, latents k = kb*64 + ch*8 .. +7 form one 16-byte chunk.
+  // Each thread first loads all of its chunks (at most 11, 88 values), so the
+  // L2 round trips overlap instead of following one another.
+  constexpr int NIT = (KB * 8 * NH + NT - 1) / NT;
+  float wv[NIT][8];
+#pragma unroll
+  for (int u = 0; u < NIT; ++u) {
+    const int it = tid + u * NT;
+    if (it < KB * 8 * NH) {
+      const int n = it % NH, kc = it / NH;
+      const float* src = p.W_c + (size_t)((kc >> 3) * 64 + (kc & 7) * 8) * D + half * NH + n;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) wv[u][e] = __ldg(src + (size_t)e * D);
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < NIT; ++u) {
+    const int it = tid + u * NT;
+    if (it >= KB * 8 * NH) break;
     const int n = it % NH, kc = it / NH;
     const int kb = kc >> 3, ch = kc & 7;
-    const float* src = p.W_c + (size_t)(kb * 64 + ch * 8) * D + half * NH + n;
-    float v[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] = __ldg(src + (size_t)e * D);
+    const float* v = wv[u];
     uint32_t hi[4], lo[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
