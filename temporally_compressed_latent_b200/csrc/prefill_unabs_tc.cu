@@ -24,9 +24,11 @@
 //    K 64) are tcgen05.mma ops with fp32 accumulators in TMEM (four 64-column
 //    S / P buffers and the 64 columns of O).  A score warp and a value warp
 //    issue them, each as soon as its inputs are ready.
-//  * Eight softmax warps, two per TMEM lane quarter, split each tile's 64
-//    columns; the pair agrees on the running max through shared memory and
-//    rescales O in TMEM only when the max grows by more than 2^8.  bf16 P is
+//  * Eight softmax warps, two per TMEM lane quarter: one takes the even key
+//    tiles, the other the odd ones, all 64 columns each, with its own running
+//    max and sum and its own O accumulator in TMEM (d_h = 64 makes a second
+//    O cheap), rescaled only when the max grows by more than 2^8; the two
+//    never wait for each other, and the epilogue merges them.  bf16 P is
 //    written back over the tile's S columns, where the value MMA reads it.
 //    A dot warp takes the own-column scores while the key tiles run; four
 //    epilogue warps fold the own column in, normalise, and write out and lse.
@@ -53,7 +55,7 @@ constexpr int TMA_WARP = SMW, SMMA_WARP = SMW + 1, PMMA_WARP = SMW + 2, DOT_WARP
 static_assert(EPI_WARP0 % 4 == 0, "epilogue warp e reads TMEM lane quarter e");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int NSB = 4;                 // S / P buffers in TMEM (64 columns each)
-constexpr uint32_t O_COL = 256;
+constexpr uint32_t O_COL = 256;         // two O accumulators: even tiles at O_COL, odd tiles at O_COL + 64
 __host__ __device__ constexpr uint32_t s_col(int b) { return 64u * (uint32_t)b; }
 constexpr uint32_t IDESC_S = umma_idesc_bf16(BM, BN, false, false);
 constexpr uint32_t IDESC_O = umma_idesc_bf16(BM, DH, false, true);
@@ -94,6 +96,14 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr) : "memory");
+}
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
@@ -169,10 +179,9 @@ __global__ void __launch_bounds__(NT, 1) prefill_unabs_tc_kernel(const __grid_co
   uint64_t* const o_empty = o_full + 1;
   uint64_t* const mma_done = o_full + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
-  float* xmax = reinterpret_cast<float*>(sm + OFF_XCH);                 // [2 parity][2 halves][BM]
-  float* xl = reinterpret_cast<float*>(sm + OFF_XCH + 4 * BM * 4);      // [2 parity][2 halves][BM]: row sums
-  float* xdot = reinterpret_cast<float*>(sm + OFF_XCH + 8 * BM * 4);    // [2 parity][BM]: own-column scores
-  float* xm = reinterpret_cast<float*>(sm + OFF_XCH + 10 * BM * 4);     // [2 parity][BM]: final row maxima
+  float* xm = reinterpret_cast<float*>(sm + OFF_XCH);                   // [2 M-tile parity][2 tile parity][BM]: maxima
+  float* xl = reinterpret_cast<float*>(sm + OFF_XCH + 4 * BM * 4);      // [2][2][BM]: row sums
+  float* xdot = reinterpret_cast<float*>(sm + OFF_XCH + 8 * BM * 4);    // [2 M-tile parity][BM]: own-column scores
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
@@ -192,7 +201,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_unabs_tc_kernel(const __grid_co
     }
     for (int i = 0; i < NSB; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], SMW);
+      mbar_init(&p_full[i], SMW / 2);  // the four warps of the tile's parity
       mbar_init(&p_empty[i], 1);
     }
     mbar_init(o_full, 1);
@@ -350,7 +359,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_unabs_tc_kernel(const __grid_co
             for (int kk = 0; kk < BN / 16; ++kk) {
               const uint32_t pa = tmem + s_col(pb) + 8 * kk;  // two bf16 per column: 8 columns per K step
               const uint64_t bd = dv0 + (uint64_t)((st * STAGE + kk * 16 * 64) >> 4);
-              umma_bf16_ts(tmem + O_COL, pa, bd, IDESC_O, (kt > 0 || kk > 0) ? 1u : 0u);
+              umma_bf16_ts(tmem + O_COL + 64 * (kt & 1), pa, bd, IDESC_O, (kt > 1 || kk > 0) ? 1u : 0u);
             }
             umma_commit(&k_empty[st]);
             umma_commit(&p_empty[pb]);
@@ -387,71 +396,70 @@ __global__ void __launch_bounds__(NT, 1) prefill_unabs_tc_kernel(const __grid_co
       if (ok && !warp_wait(&stat_full[sb2], (tc >> 1) & 1)) ok = false;
       if (ok && !warp_wait(&dot_full[sb2], (tc >> 1) & 1)) ok = false;
       if (ok && !warp_wait(&own_full[sb2], (tc >> 1) & 1)) ok = false;
-      const float m_run = xm[sb2 * BM + i];
-      const float lt = xl[(sb2 * 2 + 0) * BM + i] + xl[(sb2 * 2 + 1) * BM + i];
+      // the even and the odd tiles' running max and sum, merged with the own column
+      const float m_e = xm[(sb2 * 2 + 0) * BM + i], m_o = xm[(sb2 * 2 + 1) * BM + i];
+      const float l_e = xl[(sb2 * 2 + 0) * BM + i], l_o = xl[(sb2 * 2 + 1) * BM + i];
       const float xs = xdot[sb2 * BM + i] * sl2;
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&stat_empty[sb2]);
         mbar_arrive(&dot_empty[sb2]);
       }
-      const float mf = fmaxf(m_run, xs);
-      const float alpha = m_run == -INFINITY ? 0.f : exp2f(m_run - mf);
+      const float mf = fmaxf(fmaxf(m_e, m_o), xs);
+      const float a_e = m_e == -INFINITY ? 0.f : exp2f(m_e - mf);
+      const float a_o = m_o == -INFINITY ? 0.f : exp2f(m_o - mf);
       const float pown = exp2f(xs - mf);
-      const float den = lt * alpha + pown;
+      const float den = l_e * a_e + l_o * a_o + pown;
       const float inv = 1.f / den;
       if (ok && !warp_wait(o_full, tc & 1)) ok = false;
       tc_fence_after();
-      uint32_t ov[64];
-      if (t.nkt > 0) {
-        tmem_ld32(lane_base + O_COL, *reinterpret_cast<uint32_t(*)[32]>(&ov[0]));
-        tmem_ld32(lane_base + O_COL + 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[32]));
+      const int m = t.m0 + i;  // this row's query (1-based)
+      const uint32_t vown = sOwn + sb2 * OWNB + 3 * QPL;
+      const size_t row = ((size_t)t.b * p.T + (m <= p.T ? m - 1 : 0)) * p.H + t.h;
+      uint4* dst = reinterpret_cast<uint4*>(p.out + row * DH);
+#pragma unroll 1
+      for (int c2 = 0; c2 < 2; ++c2) {  // 32 channels at a time
+        uint32_t oe[32], oo[32];
+        if (t.nkt > 0) tmem_ld32(lane_base + O_COL + 32 * c2, oe);
+        if (t.nkt > 1) tmem_ld32(lane_base + O_COL + 64 + 32 * c2, oo);
         tmem_wait_ld();
-      } else {
 #pragma unroll
-        for (int e = 0; e < 64; ++e) ov[e] = 0u;
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t cv[4], res[4];
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(cv[0]), "=r"(cv[1]), "=r"(cv[2]), "=r"(cv[3])
+                       : "r"(vown + plane_off(BM, i, 4 * c2 + ch)));
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cv[e]));
+            const int k = ch * 8 + e * 2;
+            // (an accumulator the M tile never wrote counts as zero)
+            const float e0 = t.nkt > 0 ? __uint_as_float(oe[k]) : 0.f, e1 = t.nkt > 0 ? __uint_as_float(oe[k + 1]) : 0.f;
+            const float o0 = t.nkt > 1 ? __uint_as_float(oo[k]) : 0.f, o1 = t.nkt > 1 ? __uint_as_float(oo[k + 1]) : 0.f;
+            res[e] = pack_bf16x2((e0 * a_e + o0 * a_o + pown * c.x) * inv, (e1 * a_e + o1 * a_o + pown * c.y) * inv);
+          }
+          if (m <= p.T) dst[4 * c2 + ch] = make_uint4(res[0], res[1], res[2], res[3]);
+        }
       }
       // the last read of O in TMEM: the next M tile's value MMAs may start
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(o_empty);
-      const int m = t.m0 + i;  // this row's query (1-based)
-      const uint32_t vown = sOwn + sb2 * OWNB + 3 * QPL;
-      uint32_t res[32];
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        uint32_t cv[4];
-        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(cv[0]), "=r"(cv[1]), "=r"(cv[2]), "=r"(cv[3])
-                     : "r"(vown + plane_off(BM, i, ch)));
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cv[e]));
-          const int k = ch * 8 + e * 2;
-          res[ch * 4 + e] = pack_bf16x2((__uint_as_float(ov[k]) * alpha + pown * c.x) * inv,
-                                        (__uint_as_float(ov[k + 1]) * alpha + pown * c.y) * inv);
-        }
+      if (lane == 0) {
+        mbar_arrive(o_empty);
+        mbar_arrive(&own_empty[sb2]);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&own_empty[sb2]);
-      if (m <= p.T) {
-        const size_t row = ((size_t)t.b * p.T + (m - 1)) * p.H + t.h;
-        uint4* dst = reinterpret_cast<uint4*>(p.out + row * DH);
-#pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4) dst[c4] = make_uint4(res[4 * c4], res[4 * c4 + 1], res[4 * c4 + 2], res[4 * c4 + 3]);
-        if (p.lse) p.lse[row] = (mf + log2f(den)) * 0.69314718055994531f;
-      }
+      if (m <= p.T && p.lse) p.lse[row] = (mf + log2f(den)) * 0.69314718055994531f;
     }
     if (!ok && lane == 0) set_err(p.dev_err, MTLA_DEVERR_TIMEOUT);
   } else {
     // ======================= softmax warps =======================
-    // warp w: TMEM lane quarter w % 4 and half w / 4 of the key tile's 64
-    // columns and of O's 64 columns.  Warps w and w + 4 agree on the running
-    // max every tile (64-thread named barrier per pair; exchange buffers
-    // alternate with the tile).  A wait that times out only stops further
-    // waiting: every warp still takes every pair barrier.
-    const int qw = warp & 3, hf = warp >> 2;
+    // warp w: TMEM lane quarter w % 4 and the key tiles of parity w / 4, all
+    // 64 columns of each, with its own running max and sum and its own O
+    // accumulator (columns O_COL + 64 (w / 4)); the epilogue merges the two.
+    // The two warps of a lane quarter never wait for each other.
+    const int qw = warp & 3, par = warp >> 2;
     const int i = qw * 32 + lane;              // row of the M tile = TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
+    const uint32_t ocol = O_COL + 64 * par;
     const float sl2 = p.scale_log2;
     uint32_t tc = 0, kc = 0;
     for (int o; (o = tile_index(tc, blockIdx.x, G)) < p.n_mtiles; ++tc) {
@@ -459,58 +467,61 @@ __global__ void __launch_bounds__(NT, 1) prefill_unabs_tc_kernel(const __grid_co
       const int m = t.m0 + i;
       const int vis = (int)group_of(m, p.s) - 1;  // completed groups the query sees
       float m_run = -INFINITY, l = 0.f;
-      for (int kt = 0; kt < t.nkt; ++kt) {
+      for (int kt = par; kt < t.nkt; kt += 2) {
         const uint32_t j = kc + kt;
-        const int sb = j % NSB, xb = j & 1;
+        const int sb = j % NSB;
         if (ok && !warp_wait(&s_full[sb], (j / NSB) & 1)) ok = false;
         tc_fence_after();
-        uint32_t sr[32];
-        tmem_ld32(lane_base + s_col(sb) + 32 * hf, sr);
+        uint32_t sr[64];  // the tile's 64 scores, both loads in flight
+        tmem_ld32(lane_base + s_col(sb), *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(lane_base + s_col(sb) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
         tmem_wait_ld();
-        const int nvis = vis - kt * BN - 32 * hf;
-        float x[32];
+        const int nvis = vis - kt * BN;
         float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          x[c] = c < nvis ? __uint_as_float(sr[c]) * sl2 : -INFINITY;
-          mq[c & 3] = fmaxf(mq[c & 3], x[c]);
+        for (int c = 0; c < 64; ++c) {  // masked and scaled in place
+          const float xc = c < nvis ? __uint_as_float(sr[c]) * sl2 : -INFINITY;
+          sr[c] = __float_as_uint(xc);
+          mq[c & 3] = fmaxf(mq[c & 3], xc);
         }
         const float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
-        xmax[(xb * 2 + hf) * BM + i] = mx;
-        tc_fence_before();
-        named_bar(1 + qw, 64);
-        tc_fence_after();
-        const float rmx = fmaxf(mx, xmax[(xb * 2 + (hf ^ 1)) * BM + i]);
-        const bool grow = rmx > m_run + 8.f;
+        const bool grow = mx > m_run + 8.f;
         const bool resc = grow && m_run != -INFINITY;
-        if (kt > 0 && __any_sync(0xffffffffu, resc)) {
-          // rescale this half of O once the previous value MMA has landed
-          const uint32_t jp = j - 1;
+        if (kt >= 2 && __any_sync(0xffffffffu, resc)) {
+          // rescale this parity's O once its previous value MMA (tile j - 2) has landed
+          const uint32_t jp = j - 2;
           if (ok && !warp_wait(&p_empty[jp % NSB], (jp / NSB) & 1)) ok = false;
           tc_fence_after();
-          const float a = resc ? exp2f(m_run - rmx) : 1.f;
-          uint32_t ov[32];
-          tmem_ld32(lane_base + O_COL + 32 * hf, ov);
-          tmem_wait_ld();
+          const float a = resc ? exp2f(m_run - mx) : 1.f;
+#pragma unroll 1
+          for (int c4 = 0; c4 < 4; ++c4) {  // 16 columns at a time (the scores stay live)
+            uint32_t ov[16];
+            tmem_ld16(lane_base + ocol + 16 * c4, ov);
+            tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * a);
-          tmem_st32(lane_base + O_COL + 32 * hf, ov);
+            for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * a);
+            tmem_st16(lane_base + ocol + 16 * c4, ov);
+          }
           tmem_wait_st();
           l *= a;
         }
-        if (grow) m_run = rmx;
+        if (grow) m_run = mx;
         const float mref = m_run == -INFINITY ? 0.f : m_run;
-        uint32_t pk[16];
         float lq[4] = {0.f, 0.f, 0.f, 0.f};
+        // bf16 P over the tile's first 32 S columns (this warp alone read them)
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          const float p0 = ex2_approx(x[c] - mref);
-          const float p1 = ex2_approx(x[c + 1] - mref);
-          lq[(c >> 1) & 3] += p0 + p1;
-          pk[c >> 1] = pack_bf16x2(p0, p1);
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float p0 = ex2_approx(__uint_as_float(sr[32 * h2 + c]) - mref);
+            const float p1 = ex2_approx(__uint_as_float(sr[32 * h2 + c + 1]) - mref);
+            lq[(c >> 1) & 3] += p0 + p1;
+            pk[c >> 1] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(lane_base + s_col(sb) + 16 * h2, pk);
         }
         l += (lq[0] + lq[1]) + (lq[2] + lq[3]);
-        tmem_st16(lane_base + s_col(sb) + 16 * hf, pk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -518,8 +529,8 @@ __global__ void __launch_bounds__(NT, 1) prefill_unabs_tc_kernel(const __grid_co
       }
       const int sb2 = tc & 1;
       if (ok && tc >= 2 && !warp_wait(&stat_empty[sb2], ((tc >> 1) & 1) ^ 1)) ok = false;
-      xl[(sb2 * 2 + hf) * BM + i] = l;
-      if (hf == 0) xm[sb2 * BM + i] = m_run;
+      xl[(sb2 * 2 + par) * BM + i] = l;
+      xm[(sb2 * 2 + par) * BM + i] = m_run;
       __syncwarp();
       if (lane == 0) mbar_arrive(&stat_full[sb2]);
       kc += t.nkt;
