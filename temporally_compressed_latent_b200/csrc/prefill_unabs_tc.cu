@@ -359,7 +359,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_unabs_tc_kernel(const __grid_co
             for (int kk = 0; kk < BN / 16; ++kk) {
               const uint32_t pa = tmem + s_col(pb) + 8 * kk;  // two bf16 per column: 8 columns per K step
               const uint64_t bd = dv0 + (uint64_t)((st * STAGE + kk * 16 * 64) >> 4);
-              umma_bf16_ts(tmem + O_COL + 64 * (kt & 1), pa, bd, IDESC_O, (kt > 1 || kk > 0) ? 1u : 0u);
+              umma_bf16_ts(tmem + O_COL + 64 * (j & 1), pa, bd, IDESC_O, (kt > 1 || kk > 0) ? 1u : 0u);
             }
             umma_commit(&k_empty[st]);
             umma_commit(&p_empty[pb]);
@@ -389,14 +389,18 @@ __global__ void __launch_bounds__(NT, 1) prefill_unabs_tc_kernel(const __grid_co
     const int i = qe * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(qe * 32) << 16);
     const float sl2 = p.scale_log2;
-    uint32_t tc = 0;
+    uint32_t tc = 0, kc = 0;
     for (int o; (o = tile_index(tc, blockIdx.x, G)) < p.n_mtiles; ++tc) {
       const Tile t = tile_of(p, o);
       const int sb2 = tc & 1;
+      // O accumulator q was written by this M tile iff one of its key tiles j has j mod 2 == q
+      const bool w0 = t.nkt >= 2 || (t.nkt == 1 && (kc & 1) == 0);
+      const bool w1 = t.nkt >= 2 || (t.nkt == 1 && (kc & 1) == 1);
+      kc += t.nkt;
       if (ok && !warp_wait(&stat_full[sb2], (tc >> 1) & 1)) ok = false;
       if (ok && !warp_wait(&dot_full[sb2], (tc >> 1) & 1)) ok = false;
       if (ok && !warp_wait(&own_full[sb2], (tc >> 1) & 1)) ok = false;
-      // the even and the odd tiles' running max and sum, merged with the own column
+      // the two groups' running max and sum (even and odd j), merged with the own column
       const float m_e = xm[(sb2 * 2 + 0) * BM + i], m_o = xm[(sb2 * 2 + 1) * BM + i];
       const float l_e = xl[(sb2 * 2 + 0) * BM + i], l_o = xl[(sb2 * 2 + 1) * BM + i];
       const float xs = xdot[sb2 * BM + i] * sl2;
@@ -420,8 +424,8 @@ __global__ void __launch_bounds__(NT, 1) prefill_unabs_tc_kernel(const __grid_co
 #pragma unroll 1
       for (int c2 = 0; c2 < 2; ++c2) {  // 32 channels at a time
         uint32_t oe[32], oo[32];
-        if (t.nkt > 0) tmem_ld32(lane_base + O_COL + 32 * c2, oe);
-        if (t.nkt > 1) tmem_ld32(lane_base + O_COL + 64 + 32 * c2, oo);
+        if (w0) tmem_ld32(lane_base + O_COL + 32 * c2, oe);
+        if (w1) tmem_ld32(lane_base + O_COL + 64 + 32 * c2, oo);
         tmem_wait_ld();
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
@@ -433,8 +437,8 @@ __global__ void __launch_bounds__(NT, 1) prefill_unabs_tc_kernel(const __grid_co
             const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cv[e]));
             const int k = ch * 8 + e * 2;
             // (an accumulator the M tile never wrote counts as zero)
-            const float e0 = t.nkt > 0 ? __uint_as_float(oe[k]) : 0.f, e1 = t.nkt > 0 ? __uint_as_float(oe[k + 1]) : 0.f;
-            const float o0 = t.nkt > 1 ? __uint_as_float(oo[k]) : 0.f, o1 = t.nkt > 1 ? __uint_as_float(oo[k + 1]) : 0.f;
+            const float e0 = w0 ? __uint_as_float(oe[k]) : 0.f, e1 = w0 ? __uint_as_float(oe[k + 1]) : 0.f;
+            const float o0 = w1 ? __uint_as_float(oo[k]) : 0.f, o1 = w1 ? __uint_as_float(oo[k + 1]) : 0.f;
             res[e] = pack_bf16x2((e0 * a_e + o0 * a_o + pown * c.x) * inv, (e1 * a_e + o1 * a_o + pown * c.y) * inv);
           }
           if (m <= p.T) dst[4 * c2 + ch] = make_uint4(res[0], res[1], res[2], res[3]);
@@ -452,10 +456,12 @@ __global__ void __launch_bounds__(NT, 1) prefill_unabs_tc_kernel(const __grid_co
     if (!ok && lane == 0) set_err(p.dev_err, MTLA_DEVERR_TIMEOUT);
   } else {
     // ======================= softmax warps =======================
-    // warp w: TMEM lane quarter w % 4 and the key tiles of parity w / 4, all
-    // 64 columns of each, with its own running max and sum and its own O
-    // accumulator (columns O_COL + 64 (w / 4)); the epilogue merges the two.
-    // The two warps of a lane quarter never wait for each other.
+    // warp w: TMEM lane quarter w % 4 and the key tiles j (counted over the
+    // block's whole run) with j mod 2 == w / 4, all 64 columns of each, with
+    // its own running max and sum and its own O accumulator (columns O_COL +
+    // 64 (w / 4)); the epilogue merges the two.  The two warps of a lane
+    // quarter never wait for each other; buffer j mod 4 is always used by the
+    // same warps, so they take its mbarrier phases in order.
     const int qw = warp & 3, par = warp >> 2;
     const int i = qw * 32 + lane;              // row of the M tile = TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
@@ -467,8 +473,10 @@ __global__ void __launch_bounds__(NT, 1) prefill_unabs_tc_kernel(const __grid_co
       const int m = t.m0 + i;
       const int vis = (int)group_of(m, p.s) - 1;  // completed groups the query sees
       float m_run = -INFINITY, l = 0.f;
-      for (int kt = par; kt < t.nkt; kt += 2) {
+      bool first = true;  // this warp's first key tile of the M tile
+      for (int kt = 0; kt < t.nkt; ++kt) {
         const uint32_t j = kc + kt;
+        if ((int)(j & 1) != par) continue;
         const int sb = j % NSB;
         if (ok && !warp_wait(&s_full[sb], (j / NSB) & 1)) ok = false;
         tc_fence_after();
@@ -487,7 +495,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_unabs_tc_kernel(const __grid_co
         const float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
         const bool grow = mx > m_run + 8.f;
         const bool resc = grow && m_run != -INFINITY;
-        if (kt >= 2 && __any_sync(0xffffffffu, resc)) {
+        if (!first && __any_sync(0xffffffffu, resc)) {
           // rescale this parity's O once its previous value MMA (tile j - 2) has landed
           const uint32_t jp = j - 2;
           if (ok && !warp_wait(&p_empty[jp % NSB], (jp / NSB) & 1)) ok = false;
@@ -506,6 +514,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_unabs_tc_kernel(const __grid_co
           l *= a;
         }
         if (grow) m_run = mx;
+        first = false;
         const float mref = m_run == -INFINITY ? 0.f : m_run;
         float lq[4] = {0.f, 0.f, 0.f, 0.f};
         // bf16 P over the tile's first 32 S columns (this warp alone read them)
