@@ -377,8 +377,9 @@ mtla_status mtla_train_attn_bwd(const mtla_dims *dims, int32_t B, int32_t T, con
 /*
  * mtla_train_kv_bwd — dL/dC_hat'_latent through k = C_hat'_latent W_K^h and
  * v = C_hat'_latent W_V^h: dC[b, n] = sum_h dk[b,n,h] (W_K^h)^T + dv[b,n,h] (W_V^h)^T.
- *   dk, dv [B, T, H, d_h] bf16; W_kv as in mtla_prefill_kv.
+ *   dk, dv [B, T, H, d_h] bf16; W_kv as in mtla_prefill_kv (read as stored).
  *   dC [B, T, r] fp32, written.  One tensor-core GEMM (K = 2 H d_h).
+ *   Needs no workspace (mtla_train_workspace_bytes returns 0; NULL is fine).
  */
 mtla_status mtla_train_kv_bwd(const mtla_dims *dims, int32_t B, int32_t T, const void *dk, const void *dv,
                               const void *W_kv, float *dC, void *workspace, size_t workspace_bytes,

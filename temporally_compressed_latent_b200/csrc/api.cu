@@ -768,30 +768,26 @@ static bool train_dims(const mtla_dims* d) {
 static size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct MergeBwdLayout {
-  int64_t BT, BTp;
+  int64_t BT;
   int J, splits, kb_per;
-  size_t wcT, wc, G, dg, cT, dgT, dbp, dbs, dwp, total;
+  size_t wc, G, dg, dbp, dbs, dwp, total;
 };
 
 static MergeBwdLayout merge_bwd_layout(const mtla_dims* d, int32_t B, int32_t T) {
   MergeBwdLayout L = {};
   const int64_t r = d->r;
   L.BT = (int64_t)B * T;
-  L.BTp = (L.BT + 63) / 64 * 64;  // K of the dW_c GEMM, padded with zero columns
   L.J = (int)((T + d->s - 1) / d->s);
-  const int64_t nkb = L.BTp / 64;
+  const int64_t nkb = (L.BT + 63) / 64;  // K blocks of the dW_c GEMM (K = the tokens)
   int sms = device_sms();
   if (sms < 2) sms = 2;
   const int64_t want = sms / 2;  // two 128-row tiles of dW_c per K slice: one wave
   L.kb_per = (int)((nkb + (want < nkb ? want : nkb) - 1) / (want < nkb ? want : nkb));
   L.splits = (int)((nkb + L.kb_per - 1) / L.kb_per);
   size_t o = 0;
-  L.wcT = o; o = up256(o + (size_t)r * r * 2);
   L.wc = o;  o = up256(o + (size_t)r * r * 2);
   L.G = o;   o = up256(o + (size_t)L.BT * r * 4);
   L.dg = o;  o = up256(o + (size_t)L.BT * r * 2);
-  L.cT = o;  o = up256(o + (size_t)r * L.BTp * 2);
-  L.dgT = o; o = up256(o + (size_t)r * L.BTp * 2);
   L.dbp = o; o = up256(o + (size_t)L.J * r * 4);
   L.dbs = o; o = up256(o + (size_t)DB_SLICE_COUNT * r * 4);
   L.dwp = o; o = up256(o + (size_t)L.splits * r * r * 4);
@@ -812,7 +808,7 @@ static size_t attn_bwd_bytes(const mtla_dims* d, int32_t B, int32_t T, size_t* o
 size_t mtla_train_workspace_bytes(const mtla_dims* dims, int32_t B, int32_t T, int32_t which) {
   if (check_dims(dims) != MTLA_OK || !train_dims(dims) || B < 1 || T < 1) return 0;
   if (which == MTLA_TRAIN_ATTN_BWD) return attn_bwd_bytes(dims, B, T, nullptr, nullptr);
-  if (which == MTLA_TRAIN_KV_BWD) return (size_t)dims->r * 2 * dims->H * dims->d_h * 2;
+  if (which == MTLA_TRAIN_KV_BWD) return 0;  // no workspace: W_kv is read as stored
   if (which == MTLA_TRAIN_MERGE_BWD) return merge_bwd_layout(dims, B, T).total;
   return 0;
 }
@@ -925,6 +921,13 @@ static bool encode_operand_map(CUtensorMap* map, const void* base, int64_t rows,
   const cuuint32_t box[2] = {64, 128};
   return encode_bf16_map(map, base, 2, d2, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
+// The same matrix as an MN-major operand whose K runs along the rows: boxes of
+// 64 columns x 64 rows with the 128-byte swizzle
+static bool encode_mn_operand_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld) {
+  const cuuint64_t d2[2] = {(cuuint64_t)cols, (cuuint64_t)rows}, str[1] = {(cuuint64_t)ld * 2};
+  const cuuint32_t box[2] = {64, 64};
+  return encode_bf16_map(map, base, 2, d2, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
 
 mtla_status mtla_train_kv_bwd(const mtla_dims* dims, int32_t B, int32_t T, const void* dk, const void* dv,
                               const void* W_kv, float* dC, void* workspace, size_t workspace_bytes,
@@ -941,14 +944,13 @@ mtla_status mtla_train_kv_bwd(const mtla_dims* dims, int32_t B, int32_t T, const
   const int64_t BT = (int64_t)B * T;
   if (BT >= (int64_t(1) << 31)) return MTLA_ERR_UNSUPPORTED;
   const int r = dims->r, Hd = dims->H * dims->d_h;
-  if (!workspace || !aligned16(workspace) || workspace_bytes < (size_t)r * 2 * Hd * 2) return MTLA_ERR_WORKSPACE;
+  (void)workspace;
+  (void)workspace_bytes;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  __nv_bfloat16* wkvT = static_cast<__nv_bfloat16*>(workspace);  // [r, 2 H d_h]: W_kv transposed
-  if (launch_transpose_bf16(static_cast<const __nv_bfloat16*>(W_kv), 2 * Hd, r, r, wkvT, 2 * Hd, cs) != cudaSuccess)
-    return MTLA_ERR_CUDA;
+  // W_kv [2 H d_h, r] as stored is the MN-major B of dC = [dk | dv] W_kv
   CUtensorMap a0, a1, bm;
   if (!encode_operand_map(&a0, dk, BT, Hd, Hd) || !encode_operand_map(&a1, dv, BT, Hd, Hd) ||
-      !encode_operand_map(&bm, wkvT, r, 2 * Hd, 2 * Hd))
+      !encode_mn_operand_map(&bm, W_kv, 2 * Hd, r, r))
     return MTLA_ERR_CUDA;
   GemmBtArgs g;
   g.M = BT;
@@ -960,6 +962,8 @@ mtla_status mtla_train_kv_bwd(const mtla_dims* dims, int32_t B, int32_t T, const
   g.ldc = r;
   g.split_stride = 0;
   g.accumulate = 0;
+  g.a_mn = 0;
+  g.b_mn = 1;
   g.dev_err = dev_err;
   return from_cuda(launch_gemm_bt(g, a0, a1, bm, 1, cs));
 }
@@ -985,27 +989,26 @@ mtla_status mtla_train_merge_bwd(const mtla_dims* dims, int32_t B, int32_t T, co
   if (!workspace || !aligned16(workspace) || workspace_bytes < L.total) return MTLA_ERR_WORKSPACE;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  __nv_bfloat16* wcT = reinterpret_cast<__nv_bfloat16*>(ws + L.wcT);  // [k][i] = W_c[i][k], k < r
   __nv_bfloat16* wc = reinterpret_cast<__nv_bfloat16*>(ws + L.wc);    // [i][k] = W_c[i][k], k < r
   float* G = reinterpret_cast<float*>(ws + L.G);
   __nv_bfloat16* dg = reinterpret_cast<__nv_bfloat16*>(ws + L.dg);
-  __nv_bfloat16* cT = reinterpret_cast<__nv_bfloat16*>(ws + L.cT);
-  __nv_bfloat16* dgT = reinterpret_cast<__nv_bfloat16*>(ws + L.dgT);
   float* dbp = reinterpret_cast<float*>(ws + L.dbp);
   float* dwp = reinterpret_cast<float*>(ws + L.dwp);
   const __nv_bfloat16* cb = static_cast<const __nv_bfloat16*>(c);
   cudaError_t e;
-  if ((e = launch_transpose_f32_bf16(W_c, r, r, D, wcT, r, cs)) != cudaSuccess) return MTLA_ERR_CUDA;
   if ((e = launch_convert_bf16(W_c, r, r, D, wc, r, cs)) != cudaSuccess) return MTLA_ERR_CUDA;
-  CUtensorMap mc, mwcT, mwc, mdg, mcT, mdgT;
-  if (!encode_operand_map(&mc, cb, L.BT, r, r) || !encode_operand_map(&mwcT, wcT, r, r, r) ||
+  // wc [i][k] is K-major for dc += dg W_c^T (K = k) and MN-major for G = c W_c (K = i)
+  CUtensorMap mc, mwcm, mwc, mdg, mcm, mdgm;
+  if (!encode_operand_map(&mc, cb, L.BT, r, r) || !encode_mn_operand_map(&mwcm, wc, r, r, r) ||
       !encode_operand_map(&mwc, wc, r, r, r) || !encode_operand_map(&mdg, dg, L.BT, r, r) ||
-      !encode_operand_map(&mcT, cT, r, L.BTp, L.BTp) || !encode_operand_map(&mdgT, dgT, r, L.BTp, L.BTp))
+      !encode_mn_operand_map(&mcm, cb, L.BT, r, r) || !encode_mn_operand_map(&mdgm, dg, L.BT, r, r))
     return MTLA_ERR_CUDA;
   GemmBtArgs g;
   g.N = r;
   g.dev_err = dev_err;
   g.split_stride = 0;
+  g.a_mn = 0;
+  g.b_mn = 0;
   // G = c W_c[:, :r]: the gate pre-activations without the bias
   g.M = L.BT;
   g.K = r;
@@ -1014,7 +1017,9 @@ mtla_status mtla_train_merge_bwd(const mtla_dims* dims, int32_t B, int32_t T, co
   g.C = G;
   g.ldc = r;
   g.accumulate = 0;
-  if ((e = launch_gemm_bt(g, mc, mc, mwcT, 1, cs)) != cudaSuccess) return MTLA_ERR_CUDA;
+  g.b_mn = 1;
+  if ((e = launch_gemm_bt(g, mc, mc, mwcm, 1, cs)) != cudaSuccess) return MTLA_ERR_CUDA;
+  g.b_mn = 0;
   MergeBwdArgs m;
   m.c = cb;
   m.G = G;
@@ -1036,18 +1041,20 @@ mtla_status mtla_train_merge_bwd(const mtla_dims* dims, int32_t B, int32_t T, co
   g.C = dc;
   g.accumulate = 1;
   if ((e = launch_gemm_bt(g, mdg, mdg, mwc, 1, cs)) != cudaSuccess) return MTLA_ERR_CUDA;
-  // dW_c[:, :r] = c^T dg, split over the tokens, then the slices summed
-  if ((e = launch_transpose_bf16(cb, L.BT, r, r, cT, L.BTp, cs)) != cudaSuccess) return MTLA_ERR_CUDA;
-  if ((e = launch_transpose_bf16(dg, L.BT, r, r, dgT, L.BTp, cs)) != cudaSuccess) return MTLA_ERR_CUDA;
+  // dW_c[:, :r] = c^T dg: a contraction over the tokens, the rows of both
+  // c and dg (MN-major operands, no transposed copies), split over the
+  // tokens, then the slices summed
   g.M = r;
-  g.K = (int)L.BTp;
-  g.ka_split = (int)L.BTp;
+  g.K = (int)L.BT;
+  g.ka_split = (int)L.BT;
   g.kb_per_split = L.kb_per;
   g.C = dwp;
   g.ldc = r;
   g.split_stride = (int64_t)r * r;
   g.accumulate = 0;
-  if ((e = launch_gemm_bt(g, mcT, mcT, mdgT, L.splits, cs)) != cudaSuccess) return MTLA_ERR_CUDA;
+  g.a_mn = 1;
+  g.b_mn = 1;
+  if ((e = launch_gemm_bt(g, mcm, mcm, mdgm, L.splits, cs)) != cudaSuccess) return MTLA_ERR_CUDA;
   if ((e = launch_sum_slices(dwp, r, r, D, L.splits, (int64_t)r * r, dW_c, cs)) != cudaSuccess) return MTLA_ERR_CUDA;
   return from_cuda(launch_db_reduce(dbp, L.J, r, D, reinterpret_cast<float*>(ws + L.dbs), db_c, cs));
 }

@@ -256,6 +256,10 @@ struct GemmBtArgs {
   float* C;
   int64_t ldc, split_stride;
   int accumulate;  // C += A B^T (one slice only)
+  // MN-major operands: A stored [K, M] (maps {M, K}, boxes of 64 x 64) and B
+  // stored [K, N], so that C = A^T-as-stored B-as-stored: a contraction over
+  // the rows of both (K-major: boxes of 64 K x 128 rows)
+  int a_mn, b_mn;
   int32_t* dev_err;
 };
 cudaError_t launch_gemm_bt(const GemmBtArgs& a, const CUtensorMap& amap0, const CUtensorMap& amap1,
@@ -267,12 +271,6 @@ size_t gemm_bt_smem_bytes();
 cudaError_t launch_sum_slices(const float* src, int64_t rows, int cols, int64_t ld_out, int n, int64_t stride,
                               float* out, cudaStream_t st);
 
-// out[c][r] = bf16(in[r][c]) for a [rows, cols] matrix with row stride ld_in;
-// out has row stride ld_out >= rows, columns rows .. ld_out - 1 zero-filled.
-cudaError_t launch_transpose_bf16(const __nv_bfloat16* in, int64_t rows, int cols, int64_t ld_in,
-                                  __nv_bfloat16* out, int64_t ld_out, cudaStream_t st);
-cudaError_t launch_transpose_f32_bf16(const float* in, int64_t rows, int cols, int64_t ld_in,
-                                      __nv_bfloat16* out, int64_t ld_out, cudaStream_t st);
 // out[r][c] = bf16(in[r][c]), r < rows, c < cols (row strides ld_in, ld_out)
 cudaError_t launch_convert_bf16(const float* in, int64_t rows, int cols, int64_t ld_in, __nv_bfloat16* out,
                                 int64_t ld_out, cudaStream_t st);

@@ -4,13 +4,14 @@
 //
 // - gemm_bt: C[M, N] = A[M, K] B[N, K]^T on the tensor cores (tcgen05, TMEM
 //   accumulator, a four-stage TMA ring of 128 x 64 A and 256 x 64 B tiles),
-//   fp32 out, optionally accumulated into C or split over K.  It carries
+//   fp32 out, optionally accumulated into C or split over K; each operand
+//   K-major or MN-major (as stored, no transposed copies).  It carries
 //     dC_hat' = [dk | dv] W_kv (K = 2 H d_h),  G = c W_c (the gate
 //     pre-activations, recomputed), dc += dg W_c^T and dW_c = c^T dg;
 // - merge_bwd: per group and latent channel, the reverse scan over the
 //   group's tokens and the gate's chain rule (de, w, dz, dg, dP, the direct
 //   dc = de w), in a fixed order;
-// - small helpers: transposes and conversions to bf16 operands, slice sums.
+// - small helpers: the conversion of W_c to a bf16 operand, slice sums.
 #include "kernels.cuh"
 
 namespace mtla {
@@ -75,16 +76,28 @@ __global__ void __launch_bounds__(NT, 1) gemm_bt_kernel(const __grid_constant__ 
         mbar_arrive_expect_tx(&full[st], STAGE);
         const int kc = (kb0 + i) * BK;
         uint8_t* a = sm + (size_t)st * STAGE;
-        if (kc < p.ka_split) tma_load_2d(a, &amap0, kc, (int32_t)m0, &full[st]);
-        else tma_load_2d(a, &amap1, kc - p.ka_split, (int32_t)m0, &full[st]);
-        tma_load_2d(a + ATILE, &bmap, kc, n0, &full[st]);
-        tma_load_2d(a + ATILE + BTILE / 2, &bmap, kc, n0 + 128, &full[st]);
+        if (p.a_mn) {
+          // [64 K rows x 64 M] boxes, two along M
+          tma_load_2d(a, &amap0, (int32_t)m0, kc, &full[st]);
+          tma_load_2d(a + ATILE / 2, &amap0, (int32_t)m0 + 64, kc, &full[st]);
+        } else if (kc < p.ka_split) {
+          tma_load_2d(a, &amap0, kc, (int32_t)m0, &full[st]);
+        } else {
+          tma_load_2d(a, &amap1, kc - p.ka_split, (int32_t)m0, &full[st]);
+        }
+        if (p.b_mn) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) tma_load_2d(a + ATILE + u * (BTILE / 4), &bmap, n0 + 64 * u, kc, &full[st]);
+        } else {
+          tma_load_2d(a + ATILE, &bmap, kc, n0, &full[st]);
+          tma_load_2d(a + ATILE + BTILE / 2, &bmap, kc, n0 + 128, &full[st]);
+        }
         issued = i + 1;
       }
     }
     __syncwarp();
   } else if (warp == 1) {  // MMA issue: one elected lane
-    constexpr uint32_t idesc = umma_idesc_bf16(BM, BN, false, false);
+    const uint32_t idesc = umma_idesc_bf16(BM, BN, p.a_mn != 0, p.b_mn != 0);
     for (int i = 0; i < nk; ++i) {
       const int st = i % STAGES;
       if (!warp_wait(&full[st], (i / STAGES) & 1)) {
@@ -94,10 +107,16 @@ __global__ void __launch_bounds__(NT, 1) gemm_bt_kernel(const __grid_constant__ 
       tc_fence_after();
       if (elect_one()) {
         const uint32_t sA = smem_u32(sm + (size_t)st * STAGE), sB = sA + ATILE;
+        // K-major: a K step of 16 is 32 bytes along each 128-byte row.
+        // MN-major (128-byte swizzle): 64-element chunks along M / N are 8 KB
+        // apart (one box each), 8-row groups along K 1 KB apart, and a K step
+        // of 16 is 16 rows = 2 KB.
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk)
-          umma_bf16(tmem, umma_desc(sA + kk * 32, 16, 1024, 2), umma_desc(sB + kk * 32, 16, 1024, 2), idesc,
-                    (i > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          const uint64_t ad = p.a_mn ? umma_desc(sA + kk * 2048, ATILE / 2, 1024, 2) : umma_desc(sA + kk * 32, 16, 1024, 2);
+          const uint64_t bd = p.b_mn ? umma_desc(sB + kk * 2048, BTILE / 4, 1024, 2) : umma_desc(sB + kk * 32, 16, 1024, 2);
+          umma_bf16(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        }
         umma_commit(&empty[st]);  // the stage is free once these MMAs have read it
       }
       __syncwarp();
@@ -154,28 +173,6 @@ __global__ void __launch_bounds__(256) sum_slices_kernel(const float* src, int64
   if (c < cols)
     for (int z = 0; z < n; ++z) acc += src[z * stride + r * cols + c];
   out[idx] = acc;
-}
-
-// 32 x 32 tiles through shared memory: out[c][r] = bf16(in[r][c]); columns
-// rows .. ld_out - 1 of out are written as zeros
-template <typename TI>
-__global__ void __launch_bounds__(256) transpose_kernel(const TI* in, int64_t rows, int cols, int64_t ld_in,
-                                                        __nv_bfloat16* out, int64_t ld_out) {
-  __shared__ float tile[32][33];
-  const int64_t r0 = (int64_t)blockIdx.x * 32;
-  const int c0 = blockIdx.y * 32;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  for (int i = ty; i < 32; i += 8) {
-    const int64_t r = r0 + i;
-    const int c = c0 + tx;
-    tile[i][tx] = r < rows && c < cols ? ld_f32(in + r * ld_in + c) : 0.f;
-  }
-  __syncthreads();
-  for (int i = ty; i < 32; i += 8) {
-    const int c = c0 + i;
-    const int64_t r = r0 + tx;
-    if (c < cols && r < ld_out) out[(int64_t)c * ld_out + r] = __float2bfloat16_rn(tile[tx][i]);
-  }
 }
 
 __global__ void __launch_bounds__(256) convert_kernel(const float* in, int64_t rows, int cols, int64_t ld_in,
@@ -287,20 +284,6 @@ cudaError_t launch_sum_slices(const float* src, int64_t rows, int cols, int64_t 
                               float* out, cudaStream_t st) {
   const int64_t nth = rows * ld_out;
   tgm::sum_slices_kernel<<<(unsigned)((nth + 255) / 256), 256, 0, st>>>(src, rows, cols, ld_out, n, stride, out);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_transpose_bf16(const __nv_bfloat16* in, int64_t rows, int cols, int64_t ld_in,
-                                  __nv_bfloat16* out, int64_t ld_out, cudaStream_t st) {
-  const dim3 grid((unsigned)((ld_out + 31) / 32), (unsigned)((cols + 31) / 32));
-  tgm::transpose_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(in, rows, cols, ld_in, out, ld_out);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_transpose_f32_bf16(const float* in, int64_t rows, int cols, int64_t ld_in, __nv_bfloat16* out,
-                                      int64_t ld_out, cudaStream_t st) {
-  const dim3 grid((unsigned)((ld_out + 31) / 32), (unsigned)((cols + 31) / 32));
-  tgm::transpose_kernel<float><<<grid, 256, 0, st>>>(in, rows, cols, ld_in, out, ld_out);
   return cudaGetLastError();
 }
 

@@ -91,7 +91,7 @@ def test_training_calls_check_arguments_on_the_host():
     ws = mtla.mtla_train_workspace_bytes(d, 2, 100, mtla.TRAIN_ATTN_BWD)
     # two fp32 [B, H, T] arrays and the per-head RoPE key gradients
     assert ws >= 2 * 2 * 8 * 100 * 4 + 2 * 100 * 8 * 32 * 4
-    assert mtla.mtla_train_workspace_bytes(d, 2, 100, mtla.TRAIN_KV_BWD) == 256 * 2 * 8 * 64 * 2
+    assert mtla.mtla_train_workspace_bytes(d, 2, 100, mtla.TRAIN_KV_BWD) == 0  # W_kv is read as stored
     assert mtla.mtla_train_workspace_bytes(d, 2, 100, mtla.TRAIN_MERGE_BWD) > 2 * 100 * 256 * 4
     assert mtla.mtla_train_workspace_bytes(other, 2, 100, mtla.TRAIN_ATTN_BWD) == 0
     assert mtla.mtla_train_workspace_bytes(d, 2, 100, 9) == 0
@@ -104,5 +104,5 @@ def test_training_calls_check_arguments_on_the_host():
     wm = mtla.mtla_train_workspace_bytes(d, 2, 100, mtla.TRAIN_MERGE_BWD)
     assert L.mtla_train_merge_bwd(ctypes.byref(d), 2, 100, p, p, p, p, 49, p, p, p, p, p, p, wm, p, None) == 1
     assert L.mtla_train_merge_bwd(ctypes.byref(d), 2, 100, p, p, p, p, 50, p, p, p, p, p, p, wm - 1, p, None) == 3
-    assert L.mtla_train_kv_bwd(ctypes.byref(d), 2, 100, p, p, p, p, p, 100, p, None) == 3
+    assert L.mtla_train_kv_bwd(ctypes.byref(other), 2, 100, p, p, p, p, None, 0, p, None) == 2
     assert L.mtla_train_attn_fwd(ctypes.byref(other), 2, 100, p, p, p, p, p, p, p, p, None) == 2
