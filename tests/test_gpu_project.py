@@ -61,10 +61,11 @@ def _oracle_in(mc, x, pos):
     return [np.concatenate([o[i] for o in outs]) for i in range(4)]
 
 
-@pytest.mark.parametrize("B", [1, 32, 300])
+@pytest.mark.parametrize("B", [1, 17, 32, 33, 300])
 def test_project_in_bf16(B):
     """d = 512, H = 8, r = 256, d_R = 32: absorbed query, RoPE query and key,
-    latent; positions up to 16k.  B = 300 runs two launches (256 + 44)."""
+    latent; positions up to 16k.  B = 17 and 33 leave ragged token tiles;
+    B = 300 runs two launches (256 + 44)."""
     mc = synth.model_case(synth.MAIN, B=B, T=1, d=512, seed=1100 + B, dtype="bf16")
     x = mc.x[:, 0, :]
     pos = np.random.default_rng(B).integers(0, 16384, size=B)
@@ -77,7 +78,7 @@ def test_project_in_bf16(B):
         assert_close(host(g), r, "bf16", f"{name} B={B}")
 
 
-@pytest.mark.parametrize("B", [1, 32, 257])
+@pytest.mark.parametrize("B", [1, 17, 32, 33, 257])
 def test_project_out_bf16(B):
     mc = synth.model_case(synth.MAIN, B=B, T=1, d=512, seed=1200 + B, dtype="bf16")
     rng = np.random.default_rng(1300 + B)
