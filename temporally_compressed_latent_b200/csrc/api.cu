@@ -7,11 +7,6 @@
 
 #include "kernels.cuh"
 
-namespace mtla {
-// tensor-core running merge (merge_tc.cu)
-cudaError_t launch_merge_tc(const PrefillArgs& a, int B, const CUtensorMap& cmap, int sms, cudaStream_t st);
-}  // namespace mtla
-
 namespace {
 
 using namespace mtla;
@@ -82,14 +77,18 @@ bool encode_cache_map(CUtensorMap* map, void* cache, int64_t cache_rows, int64_t
 }
 
 // Generic tiled map of a bf16 tensor with the 64-byte swizzle (dims innermost first).
-bool encode_bf16_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
-                     const cuuint32_t* box, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_64B) {
+bool encode_map(CUtensorMap* map, CUtensorMapDataType type, const void* base, int rank, const cuuint64_t* dims,
+                const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle swizzle) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims, strides, box, estr,
+  return fn(map, type, (cuuint32_t)rank, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+bool encode_bf16_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+                     const cuuint32_t* box, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_64B) {
+  return encode_map(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rank, dims, strides, box, swizzle);
 }
 
 // the running merge on the tensor cores: bf16, r = 256, d_R = 32, s <= 32
@@ -353,13 +352,44 @@ mtla_status mtla_prefill_masked_attn(const mtla_dims* dims, int32_t B, int32_t T
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return MTLA_ERR_CUDA;
   cudaError_t e;
-  if (tc_merge_dims(dims, B, T)) {
-    // latents as [B*T rows, 256], boxes of 64 latents x 32 rows, 128-byte swizzle
-    CUtensorMap cmap;
-    const cuuint64_t dims2[2] = {256, (cuuint64_t)B * T}, str[1] = {512};
-    const cuuint32_t box[2] = {64, 32};
-    if (!encode_bf16_map(&cmap, c, 2, dims2, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MTLA_ERR_CUDA;
-    e = launch_merge_tc(p, B, cmap, sms, cs);
+  if (tc_merge_dims(dims, B, T) && aligned16(c) && aligned16(kR) && aligned16(P) && aligned16(c_partial) &&
+      (!cache_out || aligned16(cache_out))) {
+    // latents as [B*T rows, 256], boxes of 64 latents x 128 rows, 128-byte
+    // swizzle; RoPE keys [B*T rows, 32], boxes of 128 rows; P [J rows, 288]
+    // fp32, boxes of one channel tile (96) x one tile's groups; C_hat' as
+    // [B][T][288] and the cache rows as [B][groups][288], boxes of one
+    // channel tile x one token tile (or its groups)
+    const int s = dims->s, tt = (128 / s) * s;
+    const int64_t ng = cdiv(T, s);
+    MergeMaps mm;
+    const CUtensorMapSwizzle none = CU_TENSOR_MAP_SWIZZLE_NONE;
+    {
+      const cuuint64_t dims2[2] = {256, (cuuint64_t)B * T}, str[1] = {512};
+      const cuuint32_t box[2] = {64, 128};
+      if (!encode_bf16_map(&mm.c, c, 2, dims2, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MTLA_ERR_CUDA;
+    }
+    {
+      const cuuint64_t dims2[2] = {32, (cuuint64_t)B * T}, str[1] = {64};
+      const cuuint32_t box[2] = {32, 128};
+      if (!encode_bf16_map(&mm.kr, kR, 2, dims2, str, box, none)) return MTLA_ERR_CUDA;
+    }
+    {
+      const cuuint64_t dims2[2] = {288, (cuuint64_t)J_max}, str[1] = {288 * 4};
+      const cuuint32_t box[2] = {96, (cuuint32_t)(tt / s)};
+      if (!encode_map(&mm.p, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, P, 2, dims2, str, box, none)) return MTLA_ERR_CUDA;
+    }
+    {
+      const cuuint64_t dims3[3] = {288, (cuuint64_t)T, (cuuint64_t)B}, str[2] = {576, (cuuint64_t)T * 576};
+      const cuuint32_t box[3] = {96, (cuuint32_t)tt, 1};
+      if (!encode_bf16_map(&mm.out, c_partial, 3, dims3, str, box, none)) return MTLA_ERR_CUDA;
+    }
+    mm.cache = mm.out;
+    if (cache_out) {
+      const cuuint64_t dims3[3] = {288, (cuuint64_t)ng, (cuuint64_t)B}, str[2] = {576, (cuuint64_t)ng * 576};
+      const cuuint32_t box[3] = {96, (cuuint32_t)(tt / s), 1};
+      if (!encode_bf16_map(&mm.cache, cache_out, 3, dims3, str, box, none)) return MTLA_ERR_CUDA;
+    }
+    e = launch_merge_tc(p, B, mm, sms, cs);
   } else {
     e = launch_partial_merge(p, B, dims->dtype, cs);
   }

@@ -107,6 +107,13 @@ cudaError_t launch_decode_tc(const dtc::Params& p, const CUtensorMap& map64, con
                              cudaStream_t st);
 cudaError_t launch_partial_merge(const PrefillArgs& p, int B, int dtype, cudaStream_t st);
 
+// Running merge on tcgen05 (merge_tc.cu): the tensor maps it reads and writes
+// (latents, RoPE keys, P rows; C_hat' and the cache rows).
+struct MergeMaps {
+  CUtensorMap c, kr, p, out, cache;
+};
+cudaError_t launch_merge_tc(const PrefillArgs& a, int B, const MergeMaps& m, int sms, cudaStream_t st);
+
 // Masked prefill on tcgen05 (bf16, H = 8, r = 256, d_R = 32, any T >= 1).
 namespace ptc {
 struct Params;

@@ -10,69 +10,86 @@
 // also writes its C'_n as compressed-cache row j - 1.
 //
 // Design (B200):
-//  * The gate pre-activations are a dense contraction (tokens x 256 x 288), so
-//    they run as tcgen05.mma with fp32 accumulators in TMEM.  W_c stays
-//    near-fp32: each CTA splits its half of W_c (144 output channels) into
-//    bf16 hi + lo parts once, keeps both resident in shared memory (K-major,
-//    128-byte swizzle) and issues two MMAs per K step; the latents are bf16
-//    already, so the products are exact and only the lo part's rounding
-//    (2^-17 relative) remains.  The two channel halves of a token tile run in
-//    neighbouring CTAs, so the second read of the latent tile hits L2.
-//  * An MMA tile is 128 rows = 4 warp blocks of 32.  A warp block holds
-//    floor(32 / s) * s consecutive tokens that start on a group boundary, so
-//    no group crosses a warp: the running merge inside a group is a
-//    Hillis-Steele scan over lanes of ceil(log2 s) shuffle steps, with no
-//    carry between warps or tiles.  TMA loads the four 32-row boxes of a K
-//    block (64 latents, 128 B per row) into one pipeline stage.
-//  * Roles: one TMA warp, one MMA warp (one elected lane issues), twelve
-//    epilogue warps (three per TMEM lane quarter, 48 of the 144 channels
-//    each: the epilogue is latency-bound, so more warps overlap more of it).
-//    The accumulator is
-//    double-buffered in TMEM so a tile's epilogue overlaps the next tile's
-//    MMAs.  The epilogue reads each token's P row, b_c and its own latent /
-//    RoPE key (just loaded, so L2-resident), forms the gate and the gated
-//    entry in fp32 with non-contracted multiplies, scans, and stores bf16.
+//  * The gate pre-activations are a dense contraction (256 latents in, 288
+//    channels out per token), so they run as tcgen05.mma with fp32
+//    accumulators in TMEM, transposed: D[channel, token] = W_c^T c^T.  The
+//    channels sit on the TMEM lanes, so an epilogue thread owns one channel;
+//    the running merge inside a group is a sum along the thread's own
+//    columns.
+//  * The 288 channels form three tiles of 96, one per CTA (MMA rows 96..127
+//    are padding).  Each CTA rounds its 96 columns of W_c to bf16 once, the
+//    cache's own precision, and keeps them in TMEM as the MMA's A operand
+//    (two bf16 of K per column); the latents are bf16 already and the sums
+//    are fp32.  The TMA warp streams the first tiles while W_c is placed.
+//  * A token tile is floor(128 / s) * s tokens of one sequence, so groups
+//    never cross tiles.  Every input of the epilogue arrives by TMA: the
+//    latent tile (four K blocks of 128 rows x 64 latents, 128-byte swizzle,
+//    eight stages: two tiles in flight), which the MMA reads and the
+//    epilogue reads again for the gated entries before releasing it; the
+//    RoPE keys of the tile (RoPE channel tile only, two buffers); the P rows
+//    of the tile's groups for the CTA's channels (one buffer).  A CTA takes a
+//    contiguous range of tiles ordered by position, then sequence, so
+//    consecutive tiles mostly share their P rows and P is loaded again only
+//    when the position changes.  The three channel tiles of a token tile run
+//    in neighbouring CTAs, so the second and third reads of the latent tile
+//    hit L2.
+//  * The epilogue stages C_hat' rows and the closing rows in shared memory;
+//    the three warps that share a quarter of the tokens then write their
+//    rows with 16-byte stores (contiguous 192-byte row segments), so the
+//    quarters never wait for one another.
+//  * Roles (16 warps, four per SM sub-partition): twelve epilogue warps, four
+//    per live TMEM lane quarter, each over a group-aligned quarter of the
+//    tile's tokens; the padding quarter's warps take the TMA producer and the
+//    MMA issuer (one elected lane issues).  The accumulator is double-buffered
+//    in TMEM so a tile's epilogue overlaps the next tile's MMAs.  Per chunk of
+//    16 tokens the epilogue loads everything first, then forms the gates and
+//    gated entries (independent across tokens), then the group sums and the
+//    staged stores.  Strides 1, 2, 4, 8 and 16 have their own instances, in
+//    which every chunk starts a group and the positions are constants.
 #include "kernels.cuh"
 
 namespace mtla {
 namespace mtc {
 
 constexpr int R = 256, DR = 32, D = R + DR;
-constexpr int NH = D / 2;            // output channels per CTA (one half): 144
-constexpr int KB = R / 64;           // K blocks of 64 latents (128-byte rows): 4
-constexpr int ROWS = 128;            // MMA rows: 4 warp blocks of 32
-constexpr int WROWS = 32;            // rows of one warp block / one TMA box
-constexpr int ABLK = ROWS * 128;     // one K block of the latent tile: 16384 B
-constexpr int KS = 4;                // latent-tile stages
-constexpr int WKB = NH * 128;        // one K block of a W part: 18432 B
-constexpr int WBYTES = KB * WKB;     // one W part (hi or lo): 73728 B
-constexpr int NEPI = 12;             // epilogue warps: three per TMEM lane quarter, three chunks each
-constexpr int TMA_WARP = NEPI, MMA_WARP = NEPI + 1, NT = 32 * (NEPI + 2);
-constexpr int NCH = NH / 16;         // 16-column chunks per half: 9
-constexpr uint32_t TMEM_COLS = 512, ACC_STRIDE = 256;
-constexpr uint32_t IDESC = umma_idesc_bf16(ROWS, NH, false, false);
+constexpr int CT = 3;                 // channel tiles
+constexpr int NCT = D / CT;           // channels per tile: 96
+constexpr int M = 128;                // MMA rows: the tile's channels, then padding
+constexpr int NTOK = 128;             // MMA columns: token slots per tile
+constexpr int KB = R / 64;            // K blocks of 64 latents (128-byte rows): 4
+constexpr int BBLK = NTOK * 128;      // one K block of the latent tile: 16384 B
+constexpr int KS = 2 * KB;            // latent stages: two tiles
+constexpr int KRBLK = NTOK * DR * 2;  // one tile of RoPE keys: 8192 B
+constexpr int NWARPS = 16, NT = 32 * NWARPS;
+constexpr int NEPI = 4 * (NCT / 32);  // epilogue warps: four per live lane quarter (12)
+constexpr int TMA_WARP = 3, MMA_WARP = 7;  // warps of the padding quarter
+constexpr uint32_t TMEM_COLS = 512, ACC_STRIDE = 128, W_COL = 256;  // W^T: 128 columns (K / 2)
+constexpr uint32_t IDESC = umma_idesc_bf16(M, NTOK, false, false);
+constexpr int PROW = NCT * 4;                    // one staged P row (fp32): 384 B
+constexpr int OROW = NCT * 2;                    // one staged output row (bf16): 192 B
+constexpr int P_BYTES_MAX = NTOK * PROW;         // P rows of a tile at s = 1: 49152 B
+constexpr int P_BYTES_S2 = (NTOK / 2) * PROW;    // at s >= 2 (at most 64 groups): 24576 B
 
-constexpr size_t OFF_WHI = 0;
-constexpr size_t OFF_WLO = OFF_WHI + WBYTES;
-constexpr size_t OFF_A = OFF_WLO + WBYTES;
-constexpr size_t OFF_BAR = OFF_A + (size_t)KS * ABLK;
-constexpr int NBAR = 2 * KS + 2 + 2 + 1;
+constexpr size_t OFF_B = 0;
+constexpr size_t OFF_KR = OFF_B + (size_t)KS * BBLK;
+constexpr size_t OFF_X = OFF_KR + 2 * (size_t)KRBLK;  // P rows; at s >= 2 the closing rows follow them
+constexpr size_t OFF_OUT = OFF_X + P_BYTES_MAX;
+constexpr size_t OFF_BAR = OFF_OUT + (size_t)NTOK * OROW;
+constexpr int NBAR = 2 * KS + 2 + 2 + 2 + 2 + 2 + 1;
 constexpr size_t OFF_TMEM = OFF_BAR + NBAR * 8;
-constexpr size_t OFF_BC = OFF_TMEM + 16;             // this CTA's half of b_c (fp32)
-constexpr size_t SMEM_USED = OFF_BC + NH * 4;
-static_assert(OFF_WLO % 1024 == 0 && OFF_A % 1024 == 0 && WKB % 1024 == 0, "swizzle atoms must be 1024-aligned");
-static_assert(NH % 16 == 0 && NH <= 256, "N of one MMA");
+constexpr size_t SMEM_USED = OFF_TMEM + 16;
+static_assert(BBLK % 1024 == 0 && OFF_KR % 1024 == 0 && OFF_X % 1024 == 0 && OFF_OUT % 1024 == 0,
+              "stage and staging alignment");
+static_assert(P_BYTES_S2 + (NTOK / 2) * OROW <= P_BYTES_MAX, "closing rows fit beside the P rows");
+static_assert(NCT * CT == D && NCT <= M && NCT % 32 == 0 && OROW % 16 == 0 && PROW % 16 == 0, "channel tiles");
 
 size_t smem_bytes() { return SMEM_USED + 1024; }
 
 struct Params {
-  int B, s, tpw, tiles_per_seq, n_tiles;
+  int B, s, tt, tiles_per_seq, n_tiles;
   int64_t T, n_groups;
-  const __nv_bfloat16* c;
-  const __nv_bfloat16* kR;
   const float* W_c;
   const float* b_c;
-  const float* P;
   __nv_bfloat16* cp;
   __nv_bfloat16* cache;
   int32_t* dev_err;
@@ -99,17 +116,18 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 // the fp32 paths of the library keep the correctly rounded form.
 __device__ __forceinline__ float gate_sigmoid(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
 
-__device__ __forceinline__ void unpack8(const uint4& u, float* f) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
-    f[2 * i] = v.x;
-    f[2 * i + 1] = v.y;
-  }
+// first column of part `part` (0..4) of a tile of tt tokens: group-aligned quarters
+__device__ __forceinline__ int part_start(int part, int tt, int s) { return part >= 4 ? tt : ((part * tt / 4) / s) * s; }
+
+// Tile u of the ordering by position, then sequence: (sequence, tile in it).
+__device__ __forceinline__ void tile_of(int u, int B, int& b, int& tb) {
+  tb = u / B;
+  b = u - tb * B;
 }
 
-__global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__ CUtensorMap cmap, const Params p) {
+// S: the stride when it divides 16 (positions fold to constants), else 0
+template <int S>
+__global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__ MergeMaps mp, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
@@ -117,22 +135,33 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
   uint64_t* const k_empty = bar + KS;          // [KS]
   uint64_t* const acc_full = bar + 2 * KS;     // [2]
   uint64_t* const acc_empty = bar + 2 * KS + 2;  // [2]
-  uint64_t* const mma_done = bar + 2 * KS + 4;
+  uint64_t* const kr_full = bar + 2 * KS + 4;    // [2]
+  uint64_t* const kr_empty = bar + 2 * KS + 6;   // [2]
+  uint64_t* const p_full = bar + 2 * KS + 8;
+  uint64_t* const p_empty = bar + 2 * KS + 9;
+  uint64_t* const mma_done = bar + 2 * KS + 10;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + OFF_TMEM);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int half = blockIdx.x & 1;
-  const int G2 = gridDim.x >> 1;
-  const int first = blockIdx.x >> 1;
+  const int ct = blockIdx.x % CT;              // channel tile
+  const int G = gridDim.x / CT;                // CTAs per channel tile
+  const int j = blockIdx.x / CT;
+  const int u_beg = (int)((int64_t)j * p.n_tiles / G), u_end = (int)((int64_t)(j + 1) * p.n_tiles / G);
+  const bool has_rope = (ct + 1) * NCT > R;    // this channel tile holds the RoPE channels
+  const int s = S > 0 ? S : p.s, tt = p.tt, gpt = tt / s;  // groups per tile
 
   if (tid == 0) {
     for (int i = 0; i < KS; ++i) {
       mbar_init(&k_full[i], 1);
-      mbar_init(&k_empty[i], 1);
+      mbar_init(&k_empty[i], NEPI);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], NEPI);
+      mbar_init(&kr_full[i], 1);
+      mbar_init(&kr_empty[i], 4);              // the four warps of the RoPE lane quarter
     }
+    mbar_init(p_full, 1);
+    mbar_init(p_empty, NEPI);
     mbar_init(mma_done, 1);
     fence_mbar_init();
   }
@@ -140,85 +169,69 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
     tmem_alloc(tmem_holder, TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == TMA_WARP && lane == 0) prefetch_tmap(&cmap);
-
-  // this CTA's half of W_c -> bf16 hi + lo, K-major with the 128-byte swizzle:
-  // output channel n, latents k = kb*64 + ch*8 .. +7 form one 16-byte chunk.
-  // Each thread first loads all of its chunks (at most 11, 88 values), so the
-  // L2 round trips overlap instead of following one another.
-  constexpr int NIT = (KB * 8 * NH + NT - 1) / NT;
-  float wv[NIT][8];
-#pragma unroll
-  for (int u = 0; u < NIT; ++u) {
-    const int it = tid + u * NT;
-    if (it < KB * 8 * NH) {
-      const int n = it % NH, kc = it / NH;
-      const float* src = p.W_c + (size_t)((kc >> 3) * 64 + (kc & 7) * 8) * D + half * NH + n;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) wv[u][e] = __ldg(src + (size_t)e * D);
-    }
+  if (warp == TMA_WARP && lane == 0) {
+    prefetch_tmap(&mp.c);
+    prefetch_tmap(&mp.kr);
+    prefetch_tmap(&mp.p);
   }
-#pragma unroll
-  for (int u = 0; u < NIT; ++u) {
-    const int it = tid + u * NT;
-    if (it >= KB * 8 * NH) break;
-    const int n = it % NH, kc = it / NH;
-    const int kb = kc >> 3, ch = kc & 7;
-    const float* v = wv[u];
-    uint32_t hi[4], lo[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float h0 = __bfloat162float(__float2bfloat16_rn(v[2 * e]));
-      const float h1 = __bfloat162float(__float2bfloat16_rn(v[2 * e + 1]));
-      hi[e] = pack_bf16x2(h0, h1);
-      lo[e] = pack_bf16x2(v[2 * e] - h0, v[2 * e + 1] - h1);
-    }
-    const uint32_t off = (uint32_t)(kb * WKB + (n >> 3) * 1024 + (n & 7) * 128 + ((ch ^ (n & 7)) << 4));
-    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(sm + OFF_WHI + off)), "r"(hi[0]),
-                 "r"(hi[1]), "r"(hi[2]), "r"(hi[3]) : "memory");
-    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(sm + OFF_WLO + off)), "r"(lo[0]),
-                 "r"(lo[1]), "r"(lo[2]), "r"(lo[3]) : "memory");
-  }
-  float* const bc_s = reinterpret_cast<float*>(sm + OFF_BC);
-  for (int n = tid; n < NH; n += NT) bc_s[n] = __ldg(p.b_c + half * NH + n);
-  fence_proxy_async_smem();  // the tensor core reads what the threads wrote
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  const int q = warp & 3, part = warp >> 2;    // TMEM lane quarter; quarter of the tile's tokens
   bool ok = true;
 
   if (warp == TMA_WARP) {
-    // ======================= TMA producer =======================
+    // ======================= TMA producer (starts at once) =======================
     if (lane == 0) {
-      uint32_t kc = 0;
-      for (int it = first; it < p.n_tiles && ok; it += G2) {
-        const int b = it / p.tiles_per_seq, tb = it % p.tiles_per_seq;
-        const int64_t row_base = (int64_t)b * p.T;
+      uint32_t kc = 0, tc = 0, np = 0, kr_n = 0;
+      int prev_tb = -1;
+      for (int u = u_beg; u < u_end && ok; ++u, ++tc) {
+        int b, tb;
+        tile_of(u, p.B, b, tb);
+        const int32_t row = (int32_t)((int64_t)b * p.T + (int64_t)tb * tt);
+        // the latent stages first (the MMA waits on them), then the RoPE
+        // keys, then the P rows when the position changes (their buffer is
+        // free only once the epilogue has finished the previous tile)
         for (int kb = 0; kb < KB; ++kb, ++kc) {
           const int st = kc % KS;
           if (kc >= KS && !mbar_wait(&k_empty[st], ((kc / KS) & 1) ^ 1)) { ok = false; break; }
-          mbar_arrive_expect_tx(&k_full[st], ABLK);
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            // a warp block past the prompt's end loads rows it never uses
-            const int64_t n0 = ((int64_t)tb * 4 + w) * p.tpw;
-            tma_load_2d(sm + OFF_A + st * ABLK + w * (WROWS * 128), &cmap, kb * 64, (int32_t)(row_base + n0),
-                        &k_full[st]);
-          }
+          mbar_arrive_expect_tx(&k_full[st], BBLK);
+          // slots past the tile's tokens load rows that are never used
+          tma_load_2d(sm + OFF_B + st * BBLK, &mp.c, kb * 64, row, &k_full[st]);
+        }
+        if (!ok) break;
+        if (has_rope) {
+          const int kb2 = tc & 1;
+          if (tc >= 2 && !mbar_wait(&kr_empty[kb2], ((tc >> 1) & 1) ^ 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(&kr_full[kb2], KRBLK);
+          tma_load_2d(sm + OFF_KR + kb2 * KRBLK, &mp.kr, 0, row, &kr_full[kb2]);
+          ++kr_n;
+        }
+        if (tb != prev_tb) {  // the P rows of this position's groups
+          if (np > 0 && !mbar_wait(p_empty, (np - 1) & 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(p_full, (uint32_t)(gpt * PROW));
+          tma_load_2d(sm + OFF_X, &mp.p, ct * NCT, tb * gpt, p_full);
+          ++np;
+          prev_tb = tb;
         }
       }
       if (!ok) set_err(p.dev_err, MTLA_DEVERR_TIMEOUT);
       // drain: no copy may still be writing shared memory when the block exits
-      for (uint32_t j = kc > (uint32_t)KS ? kc - KS : 0; j < kc; ++j) mbar_wait(&k_full[j % KS], (j / KS) & 1);
+      for (uint32_t i = kc > (uint32_t)KS ? kc - KS : 0; i < kc; ++i) mbar_wait(&k_full[i % KS], (i / KS) & 1);
+      for (uint32_t i = kr_n > 2u ? kr_n - 2 : 0; i < kr_n; ++i) mbar_wait(&kr_full[i & 1], (i >> 1) & 1);
+      if (np > 0) mbar_wait(p_full, (np - 1) & 1);
     }
   } else if (warp == MMA_WARP) {
     // ======================= MMA issuer =======================
     // The whole warp runs the loop (warp-uniform operands); one elected lane
-    // issues the MMAs and the commits that track them.
-    const uint32_t sA = smem_u32(sm + OFF_A), sHi = smem_u32(sm + OFF_WHI), sLo = smem_u32(sm + OFF_WLO);
+    // issues the MMAs and the commits that track them.  The epilogue releases
+    // the latent stages (it reads them too).
+    named_bar(1, 32 * (NEPI + 1));  // W^T is in TMEM
+    tc_fence_after();
+    const uint32_t sB = smem_u32(sm + OFF_B);
     uint32_t kc = 0, tc = 0;
-    for (int it = first; it < p.n_tiles && ok; it += G2, ++tc) {
+    for (int u = u_beg; u < u_end && ok; ++u, ++tc) {
       const int ab = tc & 1;
       if (tc >= 2 && !warp_wait(&acc_empty[ab], ((tc >> 1) & 1) ^ 1)) { ok = false; break; }
       tc_fence_after();
@@ -230,13 +243,9 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = umma_desc(sA + st * ABLK + kk * 32, 16, 1024, 2);
-            const uint64_t bh = umma_desc(sHi + kb * WKB + kk * 32, 16, 1024, 2);
-            const uint64_t bl = umma_desc(sLo + kb * WKB + kk * 32, 16, 1024, 2);
-            umma_bf16(dcol, ad, bh, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
-            umma_bf16(dcol, ad, bl, IDESC, 1u);
+            const uint64_t bd = umma_desc(sB + st * BBLK + kk * 32, 16, 1024, 2);
+            umma_bf16_ts(dcol, tmem + W_COL + (kb * 4 + kk) * 8, bd, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
           }
-          umma_commit(&k_empty[st]);
         }
         __syncwarp();
       }
@@ -249,98 +258,183 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
     if (elect_one()) umma_commit(mma_done);
     __syncwarp();
     warp_wait(mma_done, 0);
-  } else {
-    // ======================= epilogue: gate, gated entry, group scan =======================
-    const int q = warp & 3;                            // TMEM lane quarter = warp block
-    const int cbeg = (warp >> 2) * (NCH / 3), cend = cbeg + NCH / 3;
+  } else if (q * 32 < NCT) {
+    // ================= epilogue: gate, gated entry, group sums =================
+    const int chl = q * 32 + lane;                   // this thread's channel inside the tile
+    const int ch = ct * NCT + chl;                   // and in the row of D channels
+    const bool rope = ch >= R;                       // warp-uniform
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
-    const int s = p.s;
-    const int pos = lane % s;                          // position inside the token's group
-    uint32_t tc = 0;
-    for (int it = first; it < p.n_tiles && ok; it += G2, ++tc) {
-      const int ab = tc & 1;
-      const int b = it / p.tiles_per_seq, tb = it % p.tiles_per_seq;
-      const int64_t n = ((int64_t)tb * 4 + q) * p.tpw + lane;  // 0-based token of sequence b
-      const bool valid = lane < p.tpw && n < p.T;
-      const int64_t nn = valid ? n : 0;
-      const int64_t tok = (int64_t)b * p.T + nn;
-      const int64_t grp = nn / s;                       // 0-based group = P row = cache row
-      const bool closes = valid && (pos == s - 1 || n == p.T - 1);
-      // a chunk's inputs (the token's latent or RoPE key, its group's P row)
-      // do not depend on the accumulator: the first chunk's are requested
-      // before the wait, every next chunk's while the current one is processed
-      uint4 vin_c[2], vin_n[2];
-      float4 pr_c[4], pr_n[4];
-      auto fetch = [&](int c16, uint4 (&vi)[2], float4 (&pr)[4]) {
-        if (!valid || c16 >= cend) return;
-        const int ch0 = half * NH + c16 * 16;
-        const __nv_bfloat16* vin = ch0 < R ? p.c + tok * R + ch0 : p.kR + tok * DR + (ch0 - R);
-        vi[0] = __ldg(reinterpret_cast<const uint4*>(vin));
-        vi[1] = __ldg(reinterpret_cast<const uint4*>(vin) + 1);
-        const float4* Pr = reinterpret_cast<const float4*>(p.P + grp * D + ch0);
+    {
+      // W^T into TMEM: this warp's 32 columns (latents 64 part .. +63, two
+      // per column) of its quarter's lanes, all 64 loads in flight at once
+      float wv[64];
 #pragma unroll
-        for (int e4 = 0; e4 < 4; ++e4) pr[e4] = __ldg(Pr + e4);
-      };
-      fetch(cbeg, vin_c, pr_c);
-      if (!warp_wait(&acc_full[ab], (tc >> 1) & 1)) { ok = false; break; }
+      for (int k = 0; k < 64; ++k) wv[k] = __ldg(p.W_c + (size_t)(64 * part + k) * D + ch);
+      uint32_t wp[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) wp[k] = pack_bf16x2(wv[2 * k], wv[2 * k + 1]);
+      tmem_st32(lane_base + W_COL + 32 * part, wp);
+      tmem_wait_st();
+      tc_fence_before();
+    }
+    named_bar(1, 32 * (NEPI + 1));
+
+    const float bc = __ldg(p.b_c + ch);
+    const int cb = part_start(part, tt, s), ce = part_start(part + 1, tt, s);
+    const uint32_t sB = smem_u32(sm + OFF_B);
+    // this channel's byte inside a swizzled 128-byte latent row (K block ch / 64)
+    const uint32_t c_kb = (uint32_t)(ch >> 6), c_chunk = (uint32_t)((ch & 63) >> 3), c_in = (uint32_t)(ch & 7) * 2;
+    const uint32_t p_addr = smem_u32(sm + OFF_X) + (uint32_t)chl * 4;
+    const uint32_t o_base = smem_u32(sm + OFF_OUT), g_base = smem_u32(sm + OFF_X + P_BYTES_S2);
+    const uint32_t o_addr = o_base + (uint32_t)chl * 2, g_addr = g_base + (uint32_t)chl * 2;
+    const int ptid = q * 32 + lane;                  // thread of this quarter of the tokens (0..95)
+    uint32_t tc = 0, np = 0;
+    int prev_tb = -1;
+    for (int u = u_beg; u < u_end && ok; ++u, ++tc) {
+      const int ab = tc & 1, sb = (tc & 1) * KB;      // accumulator; the tile's first stage
+      int b, tb;
+      tile_of(u, p.B, b, tb);
+      int nb, ntb = -1;                               // the next tile's position (P still needed?)
+      if (u + 1 < u_end) tile_of(u + 1, p.B, nb, ntb);
+      const int64_t n0 = (int64_t)tb * tt;           // first token of the tile (a group start)
+      const int64_t left = p.T - n0;
+      const int hi = (int)(left < ce ? left : ce);   // this warp's columns: [cb, hi)
+      const uint32_t par = (tc >> 1) & 1;
+      if (tb != prev_tb) {
+        ++np;
+        prev_tb = tb;
+      }
+      // the accumulator; the P rows; the stage holding this channel's K
+      // block (latent channels) or the tile's RoPE keys
+      ok = warp_wait(&acc_full[ab], par) && warp_wait(p_full, (np - 1) & 1) &&
+           (rope ? warp_wait(&kr_full[tc & 1], par) : warp_wait(&k_full[sb + c_kb], par));
       tc_fence_after();
-      for (int c16 = cbeg; c16 < cend; ++c16) {
-        fetch(c16 + 1, vin_n, pr_n);
+      const uint32_t crow = rope ? smem_u32(sm + OFF_KR + (tc & 1) * KRBLK) + (uint32_t)(ch - R) * 2
+                                 : sB + (sb + c_kb) * BBLK + c_in;
+      float run = 0.f, pe = 0.f;
+      for (int cc = (cb / 16) * 16; cc < hi && ok; cc += 16) {
+        // pass 1: the chunk's accumulators, entries and P values (loads only)
         uint32_t g[16];
-        tmem_ld16(lane_base + ab * ACC_STRIDE + c16 * 16, g);
+        tmem_ld16(lane_base + ab * ACC_STRIDE + cc, g);
+        float v[16], pc[16];
+        const int pos0 = (S > 0 && 16 % S == 0) ? 0 : cc % s, gl0 = cc / s;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const int col = cc + k;  // < 128: inside the stage
+          uint16_t raw;
+          const uint32_t a = rope ? crow + (uint32_t)col * (DR * 2)
+                                  : crow + (uint32_t)(col >> 3) * 1024 + (uint32_t)(col & 7) * 128 +
+                                        ((c_chunk ^ (uint32_t)(col & 7)) << 4);
+          asm volatile("ld.shared.u16 %0, [%1];" : "=h"(raw) : "r"(a));
+          v[k] = __bfloat162float(__ushort_as_bfloat16(raw));
+        }
+        {
+          // the P entry of each column's group (rows past the tile's groups
+          // hold the TMA's zero fill or an earlier tile's rows: unused)
+          int pos = pos0, gl = gl0;
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            if (pos == 0) asm volatile("ld.shared.f32 %0, [%1];" : "=f"(pe) : "r"(p_addr + (uint32_t)(gl < gpt ? gl : 0) * PROW));
+            pc[k] = pe;
+            if (++pos == s) {
+              pos = 0;
+              ++gl;
+            }
+          }
+        }
         tmem_wait_ld();
-        const int ch0 = half * NH + c16 * 16;
-        float x[16];
-        if (valid) {
-          float v[16];
-          unpack8(vin_c[0], v);
-          unpack8(vin_c[1], v + 8);
+        // pass 2: the gate and the gated entry, independent across columns
 #pragma unroll
-          for (int e4 = 0; e4 < 4; ++e4) {
-            const float pe[4] = {pr_c[e4].x, pr_c[e4].y, pr_c[e4].z, pr_c[e4].w};
+        for (int k = 0; k < 16; ++k) {
+          const float gate = __fadd_rn(__uint_as_float(g[k]), bc);
+          v[k] = __fmul_rn(gate_sigmoid(__fmul_rn(gate, pc[k])), v[k]);
+        }
+        // pass 3: the running sums inside groups and the staged stores; a
+        // chunk inside this warp's columns that does not hold the prompt's
+        // last token needs no per-column checks
+        int pos = pos0, gl = gl0;
+        if (cc >= cb && cc + 16 <= hi && cc + 16 < left) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int k = 4 * e4 + e;
-              const float gate = __fadd_rn(__uint_as_float(g[k]), bc_s[c16 * 16 + k]);
-              const float w = gate_sigmoid(__fmul_rn(gate, pe[e]));
-              x[k] = __fmul_rn(w, v[k]);
+          for (int k = 0; k < 16; ++k) {
+            run = pos == 0 ? v[k] : __fadd_rn(run, v[k]);
+            const unsigned short o = __bfloat16_as_ushort(__float2bfloat16_rn(run));
+            asm volatile("st.shared.u16 [%0], %1;" ::"r"(o_addr + (uint32_t)(cc + k) * OROW), "h"(o));
+            if (s > 1 && pos == s - 1)
+              asm volatile("st.shared.u16 [%0], %1;" ::"r"(g_addr + (uint32_t)gl * OROW), "h"(o));
+            if (++pos == s) {
+              pos = 0;
+              ++gl;
             }
           }
         } else {
 #pragma unroll
-          for (int k = 0; k < 16; ++k) x[k] = 0.f;
-        }
-        vin_c[0] = vin_n[0];
-        vin_c[1] = vin_n[1];
-#pragma unroll
-        for (int e4 = 0; e4 < 4; ++e4) pr_c[e4] = pr_n[e4];
-        // running merge inside the group: groups start at lanes that are multiples of s
-        for (int d = 1; d < s; d <<= 1) {
-#pragma unroll
           for (int k = 0; k < 16; ++k) {
-            const float y = __shfl_up_sync(0xffffffffu, x[k], d);
-            if (pos >= d) x[k] = __fadd_rn(x[k], y);
-          }
-        }
-        if (valid) {
-          uint4 o[2];
-          o[0] = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
-                            pack_bf16x2(x[6], x[7]));
-          o[1] = make_uint4(pack_bf16x2(x[8], x[9]), pack_bf16x2(x[10], x[11]), pack_bf16x2(x[12], x[13]),
-                            pack_bf16x2(x[14], x[15]));
-          uint4* dst = reinterpret_cast<uint4*>(p.cp + tok * D + ch0);
-          dst[0] = o[0];
-          dst[1] = o[1];
-          if (closes && p.cache) {
-            uint4* cdst = reinterpret_cast<uint4*>(p.cache + ((int64_t)b * p.n_groups + grp) * D + ch0);
-            cdst[0] = o[0];
-            cdst[1] = o[1];
+            const int col = cc + k;
+            run = pos == 0 ? v[k] : __fadd_rn(run, v[k]);
+            if (col >= cb && col < hi) {
+              const unsigned short o = __bfloat16_as_ushort(__float2bfloat16_rn(run));
+              asm volatile("st.shared.u16 [%0], %1;" ::"r"(o_addr + (uint32_t)col * OROW), "h"(o));
+              if (s > 1 && (pos == s - 1 || col == left - 1))
+                asm volatile("st.shared.u16 [%0], %1;" ::"r"(g_addr + (uint32_t)gl * OROW), "h"(o));
+            }
+            if (++pos == s) {
+              pos = 0;
+              ++gl;
+            }
           }
         }
       }
+      // the accumulator and this tile's stages have been read; the P rows
+      // too when the next tile needs others
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[ab]);
+      if (lane == 0) {
+        mbar_arrive(&acc_empty[ab]);
+        for (int kb = 0; kb < KB; ++kb) mbar_arrive(&k_empty[sb + kb]);
+        if (rope) mbar_arrive(&kr_empty[tc & 1]);
+        if (ntb >= 0 && ntb != tb) mbar_arrive(p_empty);
+      }
+      // the three warps of this quarter of the tokens write its staged rows
+      // [cb, hi) (and their closing rows) with 16-byte stores: 12 per row
+      named_bar(4 + part, 96);
+      {
+        const int64_t row0 = (int64_t)b * p.T + n0;
+        const int nrow = hi > cb ? hi - cb : 0;
+        for (int i = ptid; i < nrow * 12; i += 96) {
+          const int r = cb + i / 12, c16 = i % 12;
+          uint4 w;
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w)
+                       : "r"(o_base + (uint32_t)r * OROW + c16 * 16));
+          *reinterpret_cast<uint4*>(p.cp + (row0 + r) * D + ct * NCT + c16 * 8) = w;
+        }
+        if (p.cache && nrow > 0) {
+          // closing rows: the groups of columns cb .. hi-1 (a partial last
+          // group closes at the prompt's last token)
+          const int gb = cb / s, ge = (hi - 1) / s + 1;
+          const uint32_t src = s == 1 ? o_base : g_base;
+          const int64_t grow0 = (int64_t)b * p.n_groups + n0 / s;
+          for (int i = ptid; i < (ge - gb) * 12; i += 96) {
+            const int r = gb + i / 12, c16 = i % 12;
+            uint4 w;
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w)
+                         : "r"(src + (uint32_t)r * OROW + c16 * 16));
+            *reinterpret_cast<uint4*>(p.cache + (grow0 + r) * D + ct * NCT + c16 * 8) = w;
+          }
+        }
+      }
+      // the next tile writes the staged rows again only after this barrier;
+      // it also ORs the three warps' failed waits, so they leave the loop
+      // at the same tile
+      uint32_t failed;
+      asm volatile(
+          "{\n .reg .pred f;\n setp.eq.u32 f, %1, 0;\n bar.red.or.pred f, %2, 96, f;\n selp.u32 %0, 1, 0, f;\n}"
+          : "=r"(failed) : "r"(ok ? 1u : 0u), "r"(4 + part) : "memory");
+      if (failed) {
+        ok = false;
+        break;
+      }
     }
     if (!ok && lane == 0) set_err(p.dev_err, MTLA_DEVERR_TIMEOUT);
   }
@@ -355,38 +449,45 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
 
 }  // namespace mtc
 
-cudaError_t launch_merge_tc(const PrefillArgs& a, int B, const CUtensorMap& cmap, int sms, cudaStream_t st) {
+cudaError_t launch_merge_tc(const PrefillArgs& a, int B, const MergeMaps& m, int sms, cudaStream_t st) {
   mtc::Params p;
   p.B = B;
   p.T = a.T;
   p.s = a.s;
-  p.tpw = (mtc::WROWS / a.s) * a.s;
-  const int64_t wblocks = cdiv(a.T, p.tpw);
-  p.tiles_per_seq = (int)cdiv(wblocks, 4);
+  p.tt = (mtc::NTOK / a.s) * a.s;
+  p.tiles_per_seq = (int)cdiv(a.T, p.tt);
   p.n_tiles = B * p.tiles_per_seq;
   p.n_groups = cdiv(a.T, a.s);
-  p.c = static_cast<const __nv_bfloat16*>(a.c);
-  p.kR = static_cast<const __nv_bfloat16*>(a.kR);
   p.W_c = a.W_c;
   p.b_c = a.b_c;
-  p.P = a.P;
   p.cp = static_cast<__nv_bfloat16*>(a.c_partial);
   p.cache = static_cast<__nv_bfloat16*>(a.cache_out);
   p.dev_err = a.dev_err;
   const size_t smem = mtc::smem_bytes();
-  static uint64_t done_mask = 0;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev >= 64 || !(done_mask & (1ull << dev))) {
-    e = cudaFuncSetAttribute(mtc::merge_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  int per_tile = sms / mtc::CT > 0 ? sms / mtc::CT : 1;  // CTAs per channel tile
+  if (p.n_tiles < per_tile) per_tile = p.n_tiles;
+  auto go = [&](auto kernel, int slot) -> cudaError_t {
+    // the shared-memory opt-in, once per instance and device
+    static uint64_t done_mask[6] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 64) done_mask |= 1ull << dev;
+    if (dev >= 64 || !(done_mask[slot] & (1ull << dev))) {
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      if (dev < 64) done_mask[slot] |= 1ull << dev;
+    }
+    kernel<<<mtc::CT * per_tile, mtc::NT, smem, st>>>(m, p);
+    return cudaGetLastError();
+  };
+  switch (a.s) {
+    case 1: return go(mtc::merge_tc_kernel<1>, 1);
+    case 2: return go(mtc::merge_tc_kernel<2>, 2);
+    case 4: return go(mtc::merge_tc_kernel<4>, 3);
+    case 8: return go(mtc::merge_tc_kernel<8>, 4);
+    case 16: return go(mtc::merge_tc_kernel<16>, 5);
+    default: return go(mtc::merge_tc_kernel<0>, 0);
   }
-  int pairs = sms / 2 > 0 ? sms / 2 : 1;
-  if (p.n_tiles < pairs) pairs = p.n_tiles;
-  mtc::merge_tc_kernel<<<2 * pairs, mtc::NT, smem, st>>>(cmap, p);
-  return cudaGetLastError();
 }
 
 }  // namespace mtla

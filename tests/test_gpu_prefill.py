@@ -216,8 +216,11 @@ def test_prefill_tensor_core_rising_scores(s, T):
     qa = synth.cast(case.q_abs * head, "bf16")
     qr = synth.cast(case.q_rope * head, "bf16")
     run = PrefillRun(dims, "bf16", qa, qr, c, kR, case.lin).run()
+    # the bf16 running merge takes W_c at bf16 (fp32 sums), so the C_hat' it
+    # stores is the oracle's for the bf16-rounded weights
+    lin16 = dict(case.lin, W_c=synth.round_to_bf16(case.lin["W_c"]))
     for b in range(2):
-        Cp, _ = _oracle_seq(case.lin, c[b], kR[b], qa[b], qr[b], dims, with_out=False)
+        Cp, _ = _oracle_seq(lin16, c[b], kR[b], qa[b], qr[b], dims, with_out=False)
         # scores reach ~50 here, so the bf16 storage of C_hat' alone moves the
         # fp64 answer by ~4e-2 of its range; the oracle therefore attends over
         # its own C_hat' rounded to the cache's storage type
