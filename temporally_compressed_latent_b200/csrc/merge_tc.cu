@@ -148,6 +148,19 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
   const int u_beg = (int)((int64_t)j * p.n_tiles / G), u_end = (int)((int64_t)(j + 1) * p.n_tiles / G);
   const bool has_rope = (ct + 1) * NCT > R;    // this channel tile holds the RoPE channels
   const int s = S > 0 ? S : p.s, tt = p.tt, gpt = tt / s;  // groups per tile
+  const int q = warp & 3, part = warp >> 2;    // TMEM lane quarter; quarter of the tile's tokens
+  const bool epi = q * 32 < NCT;               // an epilogue warp
+  const int chl = q * 32 + lane;               // its channel inside the tile
+  const int ch = ct * NCT + chl;               // and in the row of D channels
+
+  // W^T, this warp's 32 TMEM columns (latents 64 part .. +63, two per
+  // column) of its quarter's lanes: requested before anything else, while
+  // the memory system is idle (all 64 loads in flight at once)
+  float wv[64];
+  if (epi) {
+#pragma unroll
+    for (int k = 0; k < 64; ++k) wv[k] = __ldg(p.W_c + (size_t)(64 * part + k) * D + ch);
+  }
 
   if (tid == 0) {
     for (int i = 0; i < KS; ++i) {
@@ -178,7 +191,6 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const int q = warp & 3, part = warp >> 2;    // TMEM lane quarter; quarter of the tile's tokens
   bool ok = true;
 
   if (warp == TMA_WARP) {
@@ -258,18 +270,12 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
     if (elect_one()) umma_commit(mma_done);
     __syncwarp();
     warp_wait(mma_done, 0);
-  } else if (q * 32 < NCT) {
+  } else if (epi) {
     // ================= epilogue: gate, gated entry, group sums =================
-    const int chl = q * 32 + lane;                   // this thread's channel inside the tile
-    const int ch = ct * NCT + chl;                   // and in the row of D channels
     const bool rope = ch >= R;                       // warp-uniform
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     {
-      // W^T into TMEM: this warp's 32 columns (latents 64 part .. +63, two
-      // per column) of its quarter's lanes, all 64 loads in flight at once
-      float wv[64];
-#pragma unroll
-      for (int k = 0; k < 64; ++k) wv[k] = __ldg(p.W_c + (size_t)(64 * part + k) * D + ch);
+      // W^T into TMEM (its loads were issued at the kernel's start)
       uint32_t wp[32];
 #pragma unroll
       for (int k = 0; k < 32; ++k) wp[k] = pack_bf16x2(wv[2 * k], wv[2 * k + 1]);
@@ -400,8 +406,9 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
       {
         const int64_t row0 = (int64_t)b * p.T + n0;
         const int nrow = hi > cb ? hi - cb : 0;
-        for (int i = ptid; i < nrow * 12; i += 96) {
-          const int r = cb + i / 12, c16 = i % 12;
+        // thread ptid takes the 16-byte piece ptid % 12 of every eighth row
+        const int c16 = ptid % 12, r_first = ptid / 12;
+        for (int r = cb + r_first; r < hi; r += 8) {
           uint4 w;
           asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                        : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w)
@@ -414,8 +421,7 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
           const int gb = cb / s, ge = (hi - 1) / s + 1;
           const uint32_t src = s == 1 ? o_base : g_base;
           const int64_t grow0 = (int64_t)b * p.n_groups + n0 / s;
-          for (int i = ptid; i < (ge - gb) * 12; i += 96) {
-            const int r = gb + i / 12, c16 = i % 12;
+          for (int r = gb + r_first; r < ge; r += 8) {
             uint4 w;
             asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                          : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w)
