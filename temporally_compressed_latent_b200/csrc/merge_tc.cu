@@ -111,10 +111,19 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr) : "memory");
 }
 
-// The gate's sigmoid with the hardware exponential and divide: a few fp32 ulp
-// (relative error near 1e-6), far below the bf16 rounding of what it scales;
-// the fp32 paths of the library keep the correctly rounded form.
-__device__ __forceinline__ float gate_sigmoid(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
+// The gated entry v * sigmoid(z) = v / (1 + 2^(-z log2 e)).  The caller
+// passes y = -z log2 e, formed as one fused multiply-add of the accumulator
+// with -P log2 e and (b_c P)(-log2 e) (both once per group); the base-2
+// exponential and the reciprocal are the hardware approximations (relative
+// error near 2^-22 each), far below the bf16 rounding of what they scale.
+// The fp32 paths of the library keep the correctly rounded sigmoid.
+__device__ __forceinline__ float gated(float v, float y) {
+  float e, r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(y));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.f + e));
+  return v * r;
+}
+constexpr float kNegLog2e = -1.4426950408889634f;
 
 // first column of part `part` (0..4) of a tile of tt tokens: group-aligned quarters
 __device__ __forceinline__ int part_start(int part, int tt, int s) { return part >= 4 ? tt : ((part * tt / 4) / s) * s; }
@@ -290,6 +299,11 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
     const uint32_t sB = smem_u32(sm + OFF_B);
     // this channel's byte inside a swizzled 128-byte latent row (K block ch / 64)
     const uint32_t c_kb = (uint32_t)(ch >> 6), c_chunk = (uint32_t)((ch & 63) >> 3), c_in = (uint32_t)(ch & 7) * 2;
+    // byte of this channel's 16-byte piece in a latent row r of an 8-row
+    // swizzle atom: (c_chunk ^ r) * 16, for r = 0..7
+    uint32_t xo[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) xo[r] = (c_chunk ^ (uint32_t)r) << 4;
     const uint32_t p_addr = smem_u32(sm + OFF_X) + (uint32_t)chl * 4;
     const uint32_t o_base = smem_u32(sm + OFF_OUT), g_base = smem_u32(sm + OFF_X + P_BYTES_S2);
     const uint32_t o_addr = o_base + (uint32_t)chl * 2, g_addr = g_base + (uint32_t)chl * 2;
@@ -324,13 +338,14 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
         tmem_ld16(lane_base + ab * ACC_STRIDE + cc, g);
         float v[16], pc[16];
         const int pos0 = (S > 0 && 16 % S == 0) ? 0 : cc % s, gl0 = cc / s;
+        // chunks start at multiples of 16 columns, so column cc + k sits in
+        // row k & 7 of swizzle atom cc / 8 + k / 8
+        const uint32_t cbase = rope ? crow + (uint32_t)cc * (DR * 2) : crow + (uint32_t)(cc >> 3) * 1024;
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-          const int col = cc + k;  // < 128: inside the stage
           uint16_t raw;
-          const uint32_t a = rope ? crow + (uint32_t)col * (DR * 2)
-                                  : crow + (uint32_t)(col >> 3) * 1024 + (uint32_t)(col & 7) * 128 +
-                                        ((c_chunk ^ (uint32_t)(col & 7)) << 4);
+          const uint32_t a = rope ? cbase + (uint32_t)k * (DR * 2)
+                                  : cbase + (uint32_t)(k >> 3) * 1024 + (uint32_t)(k & 7) * 128 + xo[k & 7];
           asm volatile("ld.shared.u16 %0, [%1];" : "=h"(raw) : "r"(a));
           v[k] = __bfloat162float(__ushort_as_bfloat16(raw));
         }
@@ -350,10 +365,19 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
         }
         tmem_wait_ld();
         // pass 2: the gate and the gated entry, independent across columns
+        // (the group's two factors are formed at its first column)
+        {
+          int pos = pos0;
+          float pa = 0.f, pb = 0.f;
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const float gate = __fadd_rn(__uint_as_float(g[k]), bc);
-          v[k] = __fmul_rn(gate_sigmoid(__fmul_rn(gate, pc[k])), v[k]);
+          for (int k = 0; k < 16; ++k) {
+            if (k == 0 || pos == 0) {
+              pa = pc[k] * kNegLog2e;
+              pb = bc * pa;
+            }
+            v[k] = gated(v[k], fmaf(__uint_as_float(g[k]), pa, pb));
+            if (++pos == s) pos = 0;
+          }
         }
         // pass 3: the running sums inside groups and the staged stores; a
         // chunk inside this warp's columns that does not hold the prompt's
