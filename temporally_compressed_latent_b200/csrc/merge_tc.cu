@@ -33,9 +33,11 @@
 //    when the position changes.  The three channel tiles of a token tile run
 //    in neighbouring CTAs, so the second and third reads of the latent tile
 //    hit L2.
-//  * The epilogue stages C_hat' rows and the closing rows in shared memory;
-//    the three warps that share a quarter of the tokens then write their
-//    rows with 16-byte stores (contiguous 192-byte row segments), so the
+//  * The epilogue stages C_hat' rows and the closing rows in shared memory.
+//    With a stride that divides 16 each quarter of the tokens is 32 rows and
+//    leaves by TMA stores (maps [B][T][D] and [B][groups][D], clipping rows
+//    past the prompt's end) as soon as its three warps are done; otherwise
+//    the three warps write their rows with 16-byte stores.  Either way the
 //    quarters never wait for one another.
 //  * Roles (16 warps, four per SM sub-partition): twelve epilogue warps, four
 //    per live TMEM lane quarter, each over a group-aligned quarter of the
@@ -308,6 +310,11 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
     const uint32_t o_base = smem_u32(sm + OFF_OUT), g_base = smem_u32(sm + OFF_X + P_BYTES_S2);
     const uint32_t o_addr = o_base + (uint32_t)chl * 2, g_addr = g_base + (uint32_t)chl * 2;
     const int ptid = q * 32 + lane;                  // thread of this quarter of the tokens (0..95)
+    // With a stride that divides 16 every quarter of a tile is 32 rows, so
+    // its rows leave by one TMA store each (C_hat' and the closing rows),
+    // issued by the quarter's first thread; otherwise its threads store them.
+    constexpr bool kTmaRows = S > 0;
+    const bool st_leader = q == 0 && lane == 0;
     uint32_t tc = 0, np = 0;
     int prev_tb = -1;
     for (int u = u_beg; u < u_end && ok; ++u, ++tc) {
@@ -332,6 +339,11 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
       const uint32_t crow = rope ? smem_u32(sm + OFF_KR + (tc & 1) * KRBLK) + (uint32_t)(ch - R) * 2
                                  : sB + (sb + c_kb) * BBLK + c_in;
       float run = 0.f, pe = 0.f;
+      // (TMA rows) the staged rows of this quarter are written again only
+      // after the stores issued at the previous tile have read them: waited
+      // for just before the first staged write, after that chunk's loads
+      // and gate math
+      bool need_free = kTmaRows && tc > 0;
       for (int cc = (cb / 16) * 16; cc < hi && ok; cc += 16) {
         // pass 1: the chunk's accumulators, entries and P values (loads only)
         uint32_t g[16];
@@ -379,6 +391,11 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
             if (++pos == s) pos = 0;
           }
         }
+        if (need_free) {
+          if (st_leader) bulk_wait_read_all();
+          named_bar(4 + part, 96);
+          need_free = false;
+        }
         // pass 3: the running sums inside groups and the staged stores; a
         // chunk inside this warp's columns that does not hold the prompt's
         // last token needs no per-column checks
@@ -424,10 +441,35 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
         if (rope) mbar_arrive(&kr_empty[tc & 1]);
         if (ntb >= 0 && ntb != tb) mbar_arrive(p_empty);
       }
-      // the three warps of this quarter of the tokens write its staged rows
-      // [cb, hi) (and their closing rows) with 16-byte stores: 12 per row
-      named_bar(4 + part, 96);
-      {
+      if (need_free) {  // a quarter without columns in this tile keeps the count
+        if (st_leader) bulk_wait_read_all();
+        named_bar(4 + part, 96);
+      }
+      if constexpr (kTmaRows) {
+        // the quarter's staged rows are complete (the barrier also ORs the
+        // three warps' failed waits, so they leave the loop at the same
+        // tile); its first thread sends them, the map clipping rows past
+        // the prompt's end
+        fence_proxy_async_smem();
+        uint32_t failed;
+        asm volatile(
+            "{\n .reg .pred f;\n setp.eq.u32 f, %1, 0;\n bar.red.or.pred f, %2, 96, f;\n selp.u32 %0, 1, 0, f;\n}"
+            : "=r"(failed) : "r"(ok ? 1u : 0u), "r"(4 + part) : "memory");
+        if (failed) {
+          ok = false;
+          break;
+        }
+        if (st_leader && hi > cb) {
+          tma_store_3d(&mp.out, sm + OFF_OUT + cb * OROW, ct * NCT, (int32_t)(n0 + cb), b);
+          if (p.cache)
+            tma_store_3d(&mp.cache, s == 1 ? sm + OFF_OUT + cb * OROW : sm + OFF_X + P_BYTES_S2 + (cb / s) * OROW,
+                         ct * NCT, (int32_t)((n0 + cb) / s), b);
+          bulk_commit();
+        }
+      } else {
+        // the three warps of this quarter of the tokens write its staged rows
+        // [cb, hi) (and their closing rows) with 16-byte stores: 12 per row
+        named_bar(4 + part, 96);
         const int64_t row0 = (int64_t)b * p.T + n0;
         const int nrow = hi > cb ? hi - cb : 0;
         // thread ptid takes the 16-byte piece ptid % 12 of every eighth row
@@ -453,19 +495,20 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
             *reinterpret_cast<uint4*>(p.cache + (grow0 + r) * D + ct * NCT + c16 * 8) = w;
           }
         }
-      }
-      // the next tile writes the staged rows again only after this barrier;
-      // it also ORs the three warps' failed waits, so they leave the loop
-      // at the same tile
-      uint32_t failed;
-      asm volatile(
-          "{\n .reg .pred f;\n setp.eq.u32 f, %1, 0;\n bar.red.or.pred f, %2, 96, f;\n selp.u32 %0, 1, 0, f;\n}"
-          : "=r"(failed) : "r"(ok ? 1u : 0u), "r"(4 + part) : "memory");
-      if (failed) {
-        ok = false;
-        break;
+        // the next tile writes the staged rows again only after this
+        // barrier; it also ORs the three warps' failed waits, so they leave
+        // the loop at the same tile
+        uint32_t failed;
+        asm volatile(
+            "{\n .reg .pred f;\n setp.eq.u32 f, %1, 0;\n bar.red.or.pred f, %2, 96, f;\n selp.u32 %0, 1, 0, f;\n}"
+            : "=r"(failed) : "r"(ok ? 1u : 0u), "r"(4 + part) : "memory");
+        if (failed) {
+          ok = false;
+          break;
+        }
       }
     }
+    if (kTmaRows && st_leader) bulk_wait_all();  // no store may still read shared memory at exit
     if (!ok && lane == 0) set_err(p.dev_err, MTLA_DEVERR_TIMEOUT);
   }
 
