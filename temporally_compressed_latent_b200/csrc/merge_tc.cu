@@ -139,6 +139,11 @@ __device__ __forceinline__ void tile_of(int u, int B, int& b, int& tb) {
 // S: the stride when it divides 16 (positions fold to constants), else 0
 template <int S>
 __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__ MergeMaps mp, const Params p) {
+  // a tiled TMA store reads shared memory from a 128-byte aligned address:
+  // each quarter's staged rows and closing rows must start on one
+  static_assert(S == 0 || (((NTOK / 4) * OROW) % 128 == 0 && ((NTOK / 4 / (S > 0 ? S : 1)) * OROW) % 128 == 0 &&
+                           OFF_OUT % 128 == 0 && (OFF_X + P_BYTES_S2) % 128 == 0),
+                "TMA store sources of the token quarters");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
