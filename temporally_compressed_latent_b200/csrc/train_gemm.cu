@@ -162,7 +162,10 @@ __global__ void __launch_bounds__(NT, 1) gemm_bt_kernel(const __grid_constant__ 
   }
 }
 
-// out[r * ld_out + c] = sum_z src[z * stride + r * cols + c] for c < cols, zero for cols <= c < ld_out
+// out[r * ld_out + c] = sum_z src[z * stride + r * cols + c] for c < cols, zero for cols <= c < ld_out.
+// Slice z goes to partial sum z % 8 and the eight are added in a fixed tree,
+// so eight loads are in flight per thread and the result does not depend on
+// scheduling.
 __global__ void __launch_bounds__(256) sum_slices_kernel(const float* src, int64_t rows, int cols, int64_t ld_out,
                                                          int n, int64_t stride, float* out) {
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -170,8 +173,24 @@ __global__ void __launch_bounds__(256) sum_slices_kernel(const float* src, int64
   const int64_t r = idx / ld_out;
   const int c = (int)(idx % ld_out);
   float acc = 0.f;
-  if (c < cols)
-    for (int z = 0; z < n; ++z) acc += src[z * stride + r * cols + c];
+  if (c < cols) {
+    const float* q = src + r * cols + c;
+    float a[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) a[u] = 0.f;
+    int z = 0;
+    for (; z + 8 <= n; z += 8) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldg(q + (int64_t)(z + u) * stride);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) a[u] += v[u];
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (z + u < n) a[u] += __ldg(q + (int64_t)(z + u) * stride);
+    acc = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+  }
   out[idx] = acc;
 }
 
