@@ -46,8 +46,9 @@
 //    in TMEM so a tile's epilogue overlaps the next tile's MMAs.  Per chunk of
 //    16 tokens the epilogue loads everything first, then forms the gates and
 //    gated entries (independent across tokens), then the group sums and the
-//    staged stores.  Strides 1, 2, 4, 8 and 16 have their own instances, in
-//    which every chunk starts a group and the positions are constants.
+//    staged stores.  Strides 1, 2, 3, 4, 8 and 16 have their own instances,
+//    in which the positions and divisions are constants (and, for the
+//    strides that divide 16, every chunk starts a group).
 #include "kernels.cuh"
 
 namespace mtla {
@@ -136,12 +137,13 @@ __device__ __forceinline__ void tile_of(int u, int B, int& b, int& tb) {
   b = u - tb * B;
 }
 
-// S: the stride when it divides 16 (positions fold to constants), else 0
+// S: the stride when it has its own instance (1, 2, 3, 4, 8, 16: positions
+// and divisions fold to constants), else 0
 template <int S>
 __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__ MergeMaps mp, const Params p) {
   // a tiled TMA store reads shared memory from a 128-byte aligned address:
   // each quarter's staged rows and closing rows must start on one
-  static_assert(S == 0 || (((NTOK / 4) * OROW) % 128 == 0 && ((NTOK / 4 / (S > 0 ? S : 1)) * OROW) % 128 == 0 &&
+  static_assert(S == 0 || 16 % S != 0 || (((NTOK / 4) * OROW) % 128 == 0 && ((NTOK / 4 / S) * OROW) % 128 == 0 &&
                            OFF_OUT % 128 == 0 && (OFF_X + P_BYTES_S2) % 128 == 0),
                 "TMA store sources of the token quarters");
   extern __shared__ uint8_t smem_raw[];
@@ -318,7 +320,7 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
     // With a stride that divides 16 every quarter of a tile is 32 rows, so
     // its rows leave by one TMA store each (C_hat' and the closing rows),
     // issued by the quarter's first thread; otherwise its threads store them.
-    constexpr bool kTmaRows = S > 0;
+    constexpr bool kTmaRows = S > 0 && 16 % S == 0;
     const bool st_leader = q == 0 && lane == 0;
     uint32_t tc = 0, np = 0;
     int prev_tb = -1;
@@ -546,7 +548,7 @@ cudaError_t launch_merge_tc(const PrefillArgs& a, int B, const MergeMaps& m, int
   if (p.n_tiles < per_tile) per_tile = p.n_tiles;
   auto go = [&](auto kernel, int slot) -> cudaError_t {
     // the shared-memory opt-in, once per instance and device
-    static uint64_t done_mask[6] = {};
+    static uint64_t done_mask[7] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -564,6 +566,7 @@ cudaError_t launch_merge_tc(const PrefillArgs& a, int B, const MergeMaps& m, int
     case 4: return go(mtc::merge_tc_kernel<4>, 3);
     case 8: return go(mtc::merge_tc_kernel<8>, 4);
     case 16: return go(mtc::merge_tc_kernel<16>, 5);
+    case 3: return go(mtc::merge_tc_kernel<3>, 6);
     default: return go(mtc::merge_tc_kernel<0>, 0);
   }
 }
