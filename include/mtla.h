@@ -236,7 +236,11 @@ mtla_status mtla_decode_attn_static(const mtla_dims *dims, int32_t B,
  *   (J_max >= ceil(T/s)); c_partial [B, T, D], cache_out [B, ceil(T/s), D],
  *   out [B, T, H, r] all cache dtype, contiguous, written by the call.
  * Kernels: bf16 with (H, r, d_R) = (8, 256, 32) runs the tcgen05/TMEM
- * tensor-core kernel; other supported dims run a SIMT kernel.
+ * tensor-core kernel; other supported dims run a SIMT kernel.  The running
+ * merge of bf16 prompts with r = 256, d_R = 32, s <= 32 runs on the tensor
+ * cores with W_c rounded to bf16 (fp32 sums; an error near the bf16 rounding
+ * of C_hat' itself) when c, kR, P, c_partial and cache_out are 16-byte
+ * aligned; other cases keep fp32 W_c.
  */
 mtla_status mtla_prefill_masked_attn(const mtla_dims *dims, int32_t B, int32_t T,
                                      const void *q_abs, const void *q_rope,
