@@ -239,8 +239,8 @@ mtla_status mtla_decode_attn_static(const mtla_dims *dims, int32_t B,
  * tensor-core kernel; other supported dims run a SIMT kernel.  The running
  * merge of bf16 prompts with r = 256, d_R = 32, s <= 32 runs on the tensor
  * cores with W_c rounded to bf16 (fp32 sums; an error near the bf16 rounding
- * of C_hat' itself) when c, kR, P, c_partial and cache_out are 16-byte
- * aligned; other cases keep fp32 W_c.
+ * of C_hat' itself); other dims and strides keep fp32 W_c.  Every pointer
+ * must be 16-byte aligned (MTLA_ERR_INVALID_ARG otherwise).
  */
 mtla_status mtla_prefill_masked_attn(const mtla_dims *dims, int32_t B, int32_t T,
                                      const void *q_abs, const void *q_rope,

@@ -69,6 +69,12 @@ def test_host_argument_errors_need_no_gpu():
     # prefill: P table shorter than ceil(T/s)
     assert L.mtla_prefill_masked_attn(ctypes.byref(d), 1, 10, p, p, p, p, p, p, p, 4, p, None, p, p, None) == 1
     assert L.mtla_prefill_masked_attn(ctypes.byref(d), 0, 10, p, p, p, p, p, p, p, 4, p, None, p, p, None) == 0
+    # prefill: C_hat' or the cache rows off a 16-byte boundary (the running
+    # merge's TMA maps and stores need it) are refused before any launch
+    assert L.mtla_prefill_masked_attn(ctypes.byref(d), 1, 10, None, None, p, p, p, p, p, 8, p + 2, p, None, p,
+                                      None) == 1
+    assert L.mtla_prefill_masked_attn(ctypes.byref(d), 1, 10, None, None, p, p, p, p, p, 8, p, p + 2, None, p,
+                                      None) == 1
     # merge arguments: J_max must be positive
     m = mtla._abi._Merge(p, p, p, p, p, 0)
     assert L.mtla_merge_append(ctypes.byref(d), 1, ctypes.byref(m), p, 10, 288, p, p, p, p, p, None) == 1
