@@ -374,15 +374,17 @@ def run_e2e(torch, mtla, md, case, reps, W_c, b_c, P, J_max, ws, ws_bytes, err, 
     h2d = sum(sizes)
     d2h = h_out.numel() * 4
 
+    merge = {"c_new": cn, "kR_new": kn, "W_c": W_c, "b_c": b_c, "P": P, "J_max": J_max}
+    handle = stream.cuda_stream  # the calls' stream (current inside the block below)
+
     def one(i):
         rep = reps[i % N_REPLICAS]
         d_in.copy_(h_in, non_blocking=True)
-        merge = {"c_new": cn, "kR_new": kn, "W_c": W_c, "b_c": b_c, "P": P, "J_max": J_max}
         mtla.mtla_decode_attn(md, B, qa, qr, merge, rep.cache, rep.cache_rows, d.D, rep.offset,
                               rep.capacity, rep.t, rep.cache_len, rep.out, rep.lse, ws, ws_bytes, err,
-                              stream=torch.cuda.current_stream())
+                              stream=handle)
         h_out.copy_(rep.out, non_blocking=True)
-        torch.cuda.current_stream().synchronize()
+        stream.synchronize()
 
     # the replicas may run out of spare rows: e2e reuses at most n steps
     with torch.cuda.stream(stream):
