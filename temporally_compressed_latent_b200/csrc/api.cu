@@ -357,7 +357,7 @@ mtla_status mtla_prefill_masked_attn(const mtla_dims* dims, int32_t B, int32_t T
     // swizzle; RoPE keys [B*T rows, 32], boxes of 128 rows; P [J rows, 288]
     // fp32, boxes of one channel tile (96) x one tile's groups; C_hat' as
     // [B][T][288] and the cache rows as [B][groups][288], boxes of one
-    // channel tile x a quarter of a 128-token tile (or its groups)
+    // warp's 32 channels x a quarter of a 128-token tile (or its groups)
     const int s = dims->s, tt = (128 / s) * s;
     const int64_t ng = cdiv(T, s);
     MergeMaps mm;
@@ -379,13 +379,13 @@ mtla_status mtla_prefill_masked_attn(const mtla_dims* dims, int32_t B, int32_t T
     }
     {
       const cuuint64_t dims3[3] = {288, (cuuint64_t)T, (cuuint64_t)B}, str[2] = {576, (cuuint64_t)T * 576};
-      const cuuint32_t box[3] = {96, 32, 1};  // one quarter of a 128-token tile
+      const cuuint32_t box[3] = {32, 32, 1};  // one warp's channels x a quarter of a 128-token tile
       if (!encode_bf16_map(&mm.out, c_partial, 3, dims3, str, box, none)) return MTLA_ERR_CUDA;
     }
     mm.cache = mm.out;
     if (cache_out) {
       const cuuint64_t dims3[3] = {288, (cuuint64_t)ng, (cuuint64_t)B}, str[2] = {576, (cuuint64_t)ng * 576};
-      const cuuint32_t box[3] = {96, (cuuint32_t)(s <= 32 ? 32 / s : 1), 1};  // the groups of a quarter
+      const cuuint32_t box[3] = {32, (cuuint32_t)(s <= 32 ? 32 / s : 1), 1};  // the groups of a quarter
       if (!encode_bf16_map(&mm.cache, cache_out, 3, dims3, str, box, none)) return MTLA_ERR_CUDA;
     }
     e = launch_merge_tc(p, B, mm, sms, cs);

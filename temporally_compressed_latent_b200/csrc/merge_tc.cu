@@ -34,11 +34,11 @@
 //    in neighbouring CTAs, so the second and third reads of the latent tile
 //    hit L2.
 //  * The epilogue stages C_hat' rows and the closing rows in shared memory.
-//    With a stride that divides 16 each quarter of the tokens is 32 rows and
-//    leaves by TMA stores (maps [B][T][D] and [B][groups][D], clipping rows
-//    past the prompt's end) as soon as its three warps are done; otherwise
-//    the three warps write their rows with 16-byte stores.  Either way the
-//    quarters never wait for one another.
+//    With a stride that divides 16 each warp stages its own 32 channels of
+//    its 32 rows and sends them by TMA stores (maps [B][T][D] and
+//    [B][groups][D], clipping rows past the prompt's end), so no warp waits
+//    for another; otherwise a quarter's three warps stage its rows together
+//    and write them with 16-byte stores after a barrier.
 //  * Roles (16 warps, four per SM sub-partition): twelve epilogue warps, four
 //    per live TMEM lane quarter, each over a group-aligned quarter of the
 //    tile's tokens; the padding quarter's warps take the TMA producer and the
@@ -142,10 +142,13 @@ __device__ __forceinline__ void tile_of(int u, int B, int& b, int& tb) {
 template <int S>
 __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__ MergeMaps mp, const Params p) {
   // a tiled TMA store reads shared memory from a 128-byte aligned address:
-  // each quarter's staged rows and closing rows must start on one
-  static_assert(S == 0 || 16 % S != 0 || (((NTOK / 4) * OROW) % 128 == 0 && ((NTOK / 4 / S) * OROW) % 128 == 0 &&
-                           OFF_OUT % 128 == 0 && (OFF_X + P_BYTES_S2) % 128 == 0),
-                "TMA store sources of the token quarters");
+  // each warp's staged rows (2 KB) and closing rows ((32 / S) x 64 B) must
+  // start on one, and twelve of each fit the staging regions
+  static_assert(S == 0 || 16 % S != 0 ||
+                    (NTOK == 128 && OFF_OUT % 128 == 0 && (OFF_X + P_BYTES_S2) % 128 == 0 &&
+                     ((32 / S) * 64) % 128 == 0 && 12 * 2048 <= NTOK * OROW &&
+                     12 * (32 / S) * 64 <= P_BYTES_MAX - P_BYTES_S2),
+                "TMA store sources of the warps");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
@@ -315,13 +318,23 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
     for (int r = 0; r < 8; ++r) xo[r] = (c_chunk ^ (uint32_t)r) << 4;
     const uint32_t p_addr = smem_u32(sm + OFF_X) + (uint32_t)chl * 4;
     const uint32_t o_base = smem_u32(sm + OFF_OUT), g_base = smem_u32(sm + OFF_X + P_BYTES_S2);
-    const uint32_t o_addr = o_base + (uint32_t)chl * 2, g_addr = g_base + (uint32_t)chl * 2;
     const int ptid = q * 32 + lane;                  // thread of this quarter of the tokens (0..95)
-    // With a stride that divides 16 every quarter of a tile is 32 rows, so
-    // its rows leave by one TMA store each (C_hat' and the closing rows),
-    // issued by the quarter's first thread; otherwise its threads store them.
+    // With a stride that divides 16 every quarter of a tile is 32 rows, and
+    // each warp stages its own 32 channels of them ([32 rows][32 channels],
+    // 2 KB; the closing rows likewise) and sends them with its own TMA
+    // stores: no warp waits for another.  Otherwise the quarter's three warps
+    // stage [rows][96 channels] together and store the rows with 16-byte
+    // stores after a barrier.
     constexpr bool kTmaRows = S > 0 && 16 % S == 0;
-    const bool st_leader = q == 0 && lane == 0;
+    constexpr uint32_t o_pitch = kTmaRows ? 64u : (uint32_t)OROW;  // bytes per staged row
+    const int ew = part * 3 + q;                     // epilogue warp index, 0..11
+    const int cb0 = part_start(part, tt, s);         // the quarter's first column
+    const uint32_t o_w = o_base + (uint32_t)ew * 2048u;
+    const uint32_t g_w = g_base + (uint32_t)ew * (uint32_t)((32 / s) * 64);
+    // staged element of column col (group gl) for this thread's channel
+    const uint32_t o_row0 = kTmaRows ? o_w - (uint32_t)cb0 * 64u + (uint32_t)lane * 2u : o_base + (uint32_t)chl * 2u;
+    const uint32_t g_row0 =
+        kTmaRows ? g_w - (uint32_t)(cb0 / s) * 64u + (uint32_t)lane * 2u : g_base + (uint32_t)chl * 2u;
     uint32_t tc = 0, np = 0;
     int prev_tb = -1;
     for (int u = u_beg; u < u_end && ok; ++u, ++tc) {
@@ -399,8 +412,8 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
           }
         }
         if (need_free) {
-          if (st_leader) bulk_wait_read_all();
-          named_bar(4 + part, 96);
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
           need_free = false;
         }
         // pass 3: the running sums inside groups and the staged stores; a
@@ -412,9 +425,9 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
           for (int k = 0; k < 16; ++k) {
             run = pos == 0 ? v[k] : __fadd_rn(run, v[k]);
             const unsigned short o = __bfloat16_as_ushort(__float2bfloat16_rn(run));
-            asm volatile("st.shared.u16 [%0], %1;" ::"r"(o_addr + (uint32_t)(cc + k) * OROW), "h"(o));
+            asm volatile("st.shared.u16 [%0], %1;" ::"r"(o_row0 + (uint32_t)(cc + k) * o_pitch), "h"(o));
             if (s > 1 && pos == s - 1)
-              asm volatile("st.shared.u16 [%0], %1;" ::"r"(g_addr + (uint32_t)gl * OROW), "h"(o));
+              asm volatile("st.shared.u16 [%0], %1;" ::"r"(g_row0 + (uint32_t)gl * o_pitch), "h"(o));
             if (++pos == s) {
               pos = 0;
               ++gl;
@@ -427,9 +440,9 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
             run = pos == 0 ? v[k] : __fadd_rn(run, v[k]);
             if (col >= cb && col < hi) {
               const unsigned short o = __bfloat16_as_ushort(__float2bfloat16_rn(run));
-              asm volatile("st.shared.u16 [%0], %1;" ::"r"(o_addr + (uint32_t)col * OROW), "h"(o));
+              asm volatile("st.shared.u16 [%0], %1;" ::"r"(o_row0 + (uint32_t)col * o_pitch), "h"(o));
               if (s > 1 && (pos == s - 1 || col == left - 1))
-                asm volatile("st.shared.u16 [%0], %1;" ::"r"(g_addr + (uint32_t)gl * OROW), "h"(o));
+                asm volatile("st.shared.u16 [%0], %1;" ::"r"(g_row0 + (uint32_t)gl * o_pitch), "h"(o));
             }
             if (++pos == s) {
               pos = 0;
@@ -448,31 +461,24 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
         if (rope) mbar_arrive(&kr_empty[tc & 1]);
         if (ntb >= 0 && ntb != tb) mbar_arrive(p_empty);
       }
-      if (need_free) {  // a quarter without columns in this tile keeps the count
-        if (st_leader) bulk_wait_read_all();
-        named_bar(4 + part, 96);
+      if (need_free) {  // a warp without columns in this tile
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
       }
       if constexpr (kTmaRows) {
-        // the quarter's staged rows are complete (the barrier also ORs the
-        // three warps' failed waits, so they leave the loop at the same
-        // tile); its first thread sends them, the map clipping rows past
-        // the prompt's end
+        // this warp's staged rows are complete: its first lane sends them
+        // (the maps clip rows past the prompt's end); a failed wait ends
+        // only this warp's loop (the others' waits are bounded)
         fence_proxy_async_smem();
-        uint32_t failed;
-        asm volatile(
-            "{\n .reg .pred f;\n setp.eq.u32 f, %1, 0;\n bar.red.or.pred f, %2, 96, f;\n selp.u32 %0, 1, 0, f;\n}"
-            : "=r"(failed) : "r"(ok ? 1u : 0u), "r"(4 + part) : "memory");
-        if (failed) {
-          ok = false;
-          break;
-        }
-        if (st_leader && hi > cb) {
-          tma_store_3d(&mp.out, sm + OFF_OUT + cb * OROW, ct * NCT, (int32_t)(n0 + cb), b);
+        __syncwarp();
+        if (lane == 0 && ok && hi > cb) {
+          tma_store_3d(&mp.out, sm + OFF_OUT + ew * 2048, ct * NCT + q * 32, (int32_t)(n0 + cb), b);
           if (p.cache)
-            tma_store_3d(&mp.cache, s == 1 ? sm + OFF_OUT + cb * OROW : sm + OFF_X + P_BYTES_S2 + (cb / s) * OROW,
-                         ct * NCT, (int32_t)((n0 + cb) / s), b);
+            tma_store_3d(&mp.cache, s == 1 ? sm + OFF_OUT + ew * 2048 : sm + OFF_X + P_BYTES_S2 + ew * ((32 / s) * 64),
+                         ct * NCT + q * 32, (int32_t)((n0 + cb) / s), b);
           bulk_commit();
         }
+        if (!ok) break;
       } else {
         // the three warps of this quarter of the tokens write its staged rows
         // [cb, hi) (and their closing rows) with 16-byte stores: 12 per row
@@ -515,7 +521,7 @@ __global__ void __launch_bounds__(NT, 1) merge_tc_kernel(const __grid_constant__
         }
       }
     }
-    if (kTmaRows && st_leader) bulk_wait_all();  // no store may still read shared memory at exit
+    if (kTmaRows && lane == 0) bulk_wait_all();  // no store may still read shared memory at exit
     if (!ok && lane == 0) set_err(p.dev_err, MTLA_DEVERR_TIMEOUT);
   }
 
