@@ -13,10 +13,25 @@ import bench  # noqa: E402
 def test_committed_decode_profile_is_plausible():
     # when the committed capture matches the decode sources, its DRAM bytes
     # per launch are at least the cache rows the step streams (37.76 MB) and
-    # close to the step's algorithmic bytes (39.40 MB)
+    # close to the step's algorithmic bytes (38.54 MB)
     traffic = bench.profiled_traffic()
     if traffic is not None:
-        assert 37.76e6 <= traffic <= 1.1 * 39.40e6
+        assert 37.76e6 <= traffic <= 1.1 * 38.54e6
+
+
+def test_decode_step_bytes_of_the_b32_workload():
+    # 16 sequences with 4097 tokens after the step (2049 rows at s = 2) and 16
+    # with 4096 (2048 rows): the cache rows once, plus the per-sequence and
+    # per-step terms the roofline counts
+    import mtla_synth as synth
+    d = synth.MAIN
+    B = 32
+    t_after = [4097 if b % 2 == 0 else 4096 for b in range(B)]
+    rows = 16 * 2049 + 16 * 2048
+    D = d.r + d.d_R
+    expect = (rows * D * 2 + B * D * 2 + B * d.H * D * 2 + B * D * 2 + B * d.H * d.r * 4 + B * d.H * 4 +
+              d.r * D * 4 + D * 4 + B * D * 4)
+    assert bench.decode_step_bytes(t_after, d) == expect == 38538368
 
 
 def test_traffic_is_dropped_when_the_source_changed(tmp_path, monkeypatch):
